@@ -1,0 +1,258 @@
+// dcattn.cu -- host side of libdcattn: argument checks, kernel selection,
+// launches and the device status word.  One translation unit holds every
+// kernel so the status word needs no relocatable device code.
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+#include <string.h>
+
+#include "dcattn.h"
+#include "common.cuh"
+#include "simt.cuh"
+#include "tc_host.cuh"
+
+namespace {
+
+thread_local int32_t t_launches = 0;
+
+struct Checked {
+    dc::Shape s;
+    int dtype;
+    int impl;   // resolved: DC_IMPL_SIMT or DC_IMPL_TCGEN05
+};
+
+bool aligned16(const void *p) { return ((uintptr_t)p & 15u) == 0; }
+
+// Host-side argument check; fills `out` and returns DC_OK or an error.
+dc_status_t check_params(const dc_attn_params *p, Checked *out) {
+    if (!p) return DC_ERR_INVALID_ARG;
+    if (p->dtype != DC_F32 && p->dtype != DC_BF16) return DC_ERR_INVALID_ARG;
+    if (p->impl != DC_IMPL_AUTO && p->impl != DC_IMPL_SIMT && p->impl != DC_IMPL_TCGEN05)
+        return DC_ERR_INVALID_ARG;
+    if (p->reserved != 0) return DC_ERR_INVALID_ARG;
+    if (p->total_tokens < 0 || p->total_tokens > (int64_t)INT32_MAX) return DC_ERR_INVALID_ARG;
+    if (p->num_heads < 1 || p->num_heads > dc::simt::kMaxHeads) return DC_ERR_INVALID_ARG;
+    if (p->head_dim < 1 || p->window < 1) return DC_ERR_INVALID_ARG;
+    if (p->total_tokens > 0 && (p->num_docs < 1 || p->num_docs > p->total_tokens + 1 || !p->cu_seqlens))
+        return DC_ERR_INVALID_ARG;
+    if (!(p->softmax_scale == p->softmax_scale)) return DC_ERR_INVALID_ARG;   // NaN
+    if (p->head_dim % 32 != 0 || p->head_dim > 128) return DC_ERR_UNSUPPORTED;
+    if (p->window > 4096) return DC_ERR_UNSUPPORTED;
+    out->s.N = p->total_tokens;
+    out->s.num_docs = p->num_docs;
+    out->s.H = p->num_heads;
+    out->s.d = p->head_dim;
+    out->s.W = p->window;
+    out->s.scale = p->softmax_scale;
+    out->s.cu = p->cu_seqlens;
+    out->dtype = p->dtype;
+    const bool tc_ok = p->dtype == DC_BF16 && dc::tc::supports(out->s);
+    if (p->impl == DC_IMPL_TCGEN05) {
+        if (!tc_ok) return DC_ERR_UNSUPPORTED;
+        out->impl = DC_IMPL_TCGEN05;
+    } else if (p->impl == DC_IMPL_SIMT) {
+        out->impl = DC_IMPL_SIMT;
+    } else {
+        out->impl = tc_ok ? DC_IMPL_TCGEN05 : DC_IMPL_SIMT;
+    }
+    return DC_OK;
+}
+
+dc_status_t ptrs_ok(std::initializer_list<const void *> required, std::initializer_list<const void *> optional) {
+    for (const void *x : required)
+        if (!x || !aligned16(x)) return DC_ERR_INVALID_ARG;
+    for (const void *x : optional)
+        if (x && !aligned16(x)) return DC_ERR_INVALID_ARG;
+    return DC_OK;
+}
+
+dc_status_t cuda_status(cudaError_t e) {
+    if (e != cudaSuccess) {
+        (void)cudaGetLastError();
+        return DC_ERR_CUDA;
+    }
+    return DC_OK;
+}
+
+// --------------------------------------------------------------------------
+// SIMT launches
+// --------------------------------------------------------------------------
+
+template <typename K>
+cudaError_t launch_warps(K kernel, const dc::Shape &s, size_t per_warp, cudaStream_t st, auto &&...args) {
+    int wpb = (int)((96 * 1024) / (per_warp > 0 ? per_warp : 1));
+    if (wpb > 8) wpb = 8;
+    if (wpb < 1) wpb = 1;
+    const size_t smem = per_warp * wpb;
+    cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    const int64_t blocks = (s.N + wpb - 1) / wpb;
+    kernel<<<(unsigned)blocks, 32 * wpb, smem, st>>>(s, args...);
+    ++t_launches;
+    return cudaGetLastError();
+}
+
+template <typename T, int DPL>
+cudaError_t simt_fwd(const dc::Shape &s, const void *q, const void *k, const void *v, const float *c,
+                     const float *g, void *o, float *lse, void *pmap, cudaStream_t st) {
+    return launch_warps(dc::simt::fwd_kernel<T, DPL>, s, dc::simt::fwd_smem_per_warp(s.H, s.d, s.W), st,
+                        (const T *)q, (const T *)k, (const T *)v, c, g, (T *)o, lse, (T *)pmap, 1);
+}
+
+template <typename T, int DPL>
+cudaError_t simt_bwd_query(const dc::Shape &s, const void *q, const void *k, const void *v, const float *c,
+                           const float *g, const void *dO, const float *lse, const void *pmap, void *dq,
+                           float *dc_, float *dg, float *band, cudaStream_t st) {
+    return launch_warps(dc::simt::bwd_query_kernel<T, DPL>, s, dc::simt::bwdq_smem_per_warp(s.H, s.d, s.W), st,
+                        (const T *)q, (const T *)k, (const T *)v, c, g, (const T *)dO, lse, (const T *)pmap,
+                        (T *)dq, dc_, dg, band, 1);
+}
+
+template <typename T, int DPL>
+cudaError_t simt_bwd_key(const dc::Shape &s, const void *q, const void *k, const float *c, const float *g,
+                         const void *dO, const float *lse, const void *pmap, const float *dc_,
+                         const float *band, void *dk, void *dv, cudaStream_t st) {
+    return launch_warps(dc::simt::bwd_key_kernel<T, DPL>, s, dc::simt::bwdk_smem_per_warp(s.H, s.d, s.W), st,
+                        (const T *)q, (const T *)k, c, g, (const T *)dO, lse, (const T *)pmap, dc_, band,
+                        (T *)dk, (T *)dv);
+}
+
+// Calls F<T, DPL>::run(args...) for the runtime dtype and d = 32 * DPL.
+#define DC_DISPATCH(FN, dtype, d, ...)                                              \
+    [&]() -> cudaError_t {                                                          \
+        if ((dtype) == DC_F32) {                                                    \
+            switch ((d) / 32) {                                                     \
+                case 1: return FN<float, 1>(__VA_ARGS__);                           \
+                case 2: return FN<float, 2>(__VA_ARGS__);                           \
+                case 3: return FN<float, 3>(__VA_ARGS__);                           \
+                default: return FN<float, 4>(__VA_ARGS__);                          \
+            }                                                                       \
+        }                                                                           \
+        switch ((d) / 32) {                                                         \
+            case 1: return FN<__nv_bfloat16, 1>(__VA_ARGS__);                       \
+            case 2: return FN<__nv_bfloat16, 2>(__VA_ARGS__);                       \
+            case 3: return FN<__nv_bfloat16, 3>(__VA_ARGS__);                       \
+            default: return FN<__nv_bfloat16, 4>(__VA_ARGS__);                      \
+        }                                                                           \
+    }()
+
+size_t band_bytes(const dc::Shape &s) { return sizeof(float) * (size_t)s.N * (size_t)s.W; }
+
+}  // namespace
+
+extern "C" {
+
+dc_status_t dc_attn_fwd(const dc_attn_params *params, const void *q, const void *k, const void *v,
+                        const float *c, const float *g, void *o, float *lse, void *pmap, void *stream) {
+    Checked ck;
+    dc_status_t r = check_params(params, &ck);
+    if (r != DC_OK) return r;
+    t_launches = 0;
+    if (ck.s.N == 0) return DC_OK;
+    r = ptrs_ok({q, k, v, c, g, o}, {lse, pmap});
+    if (r != DC_OK) return r;
+    cudaStream_t st = (cudaStream_t)stream;
+    if (ck.impl == DC_IMPL_TCGEN05)
+        return cuda_status(dc::tc::fwd(ck.s, q, k, v, c, g, o, lse, pmap, st, &t_launches));
+    return cuda_status(DC_DISPATCH(simt_fwd, ck.dtype, ck.s.d, ck.s, q, k, v, c, g, o, lse, pmap, st));
+}
+
+size_t dc_attn_bwd_workspace_size(const dc_attn_params *params) {
+    Checked ck;
+    if (check_params(params, &ck) != DC_OK) return 0;
+    return band_bytes(ck.s);
+}
+
+dc_status_t dc_attn_bwd_query(const dc_attn_params *params, const void *q, const void *k, const void *v,
+                              const float *c, const float *g, const void *dO, const float *lse,
+                              const void *pmap, void *dq, float *dc_, float *dg, void *workspace,
+                              size_t workspace_bytes, void *stream) {
+    Checked ck;
+    dc_status_t r = check_params(params, &ck);
+    if (r != DC_OK) return r;
+    t_launches = 0;
+    if (ck.s.N == 0) return DC_OK;
+    r = ptrs_ok({q, k, v, c, g, dO, lse, pmap, dq, dc_, dg, workspace}, {});
+    if (r != DC_OK) return r;
+    if (workspace_bytes < band_bytes(ck.s)) return DC_ERR_INVALID_ARG;
+    cudaStream_t st = (cudaStream_t)stream;
+    float *band = (float *)workspace;
+    if (ck.impl == DC_IMPL_TCGEN05)
+        return cuda_status(dc::tc::bwd_query(ck.s, q, k, v, c, g, dO, lse, pmap, dq, dc_, dg, band, st,
+                                             &t_launches));
+    return cuda_status(DC_DISPATCH(simt_bwd_query, ck.dtype, ck.s.d, ck.s, q, k, v, c, g, dO, lse, pmap, dq,
+                                   dc_, dg, band, st));
+}
+
+dc_status_t dc_attn_bwd_key(const dc_attn_params *params, const void *q, const void *k, const float *c,
+                            const float *g, const void *dO, const float *lse, const void *pmap,
+                            const float *dc_, void *dk, void *dv, const void *workspace,
+                            size_t workspace_bytes, void *stream) {
+    Checked ck;
+    dc_status_t r = check_params(params, &ck);
+    if (r != DC_OK) return r;
+    t_launches = 0;
+    if (ck.s.N == 0) return DC_OK;
+    r = ptrs_ok({q, k, c, g, dO, lse, pmap, dc_, dk, dv, workspace}, {});
+    if (r != DC_OK) return r;
+    if (workspace_bytes < band_bytes(ck.s)) return DC_ERR_INVALID_ARG;
+    cudaStream_t st = (cudaStream_t)stream;
+    const float *band = (const float *)workspace;
+    if (ck.impl == DC_IMPL_TCGEN05)
+        return cuda_status(dc::tc::bwd_key(ck.s, q, k, c, g, dO, lse, pmap, dc_, band, dk, dv, st,
+                                           &t_launches));
+    return cuda_status(DC_DISPATCH(simt_bwd_key, ck.dtype, ck.s.d, ck.s, q, k, c, g, dO, lse, pmap, dc_, band,
+                                   dk, dv, st));
+}
+
+dc_status_t dc_attn_bwd(const dc_attn_params *params, const void *q, const void *k, const void *v,
+                        const float *c, const float *g, const void *dO, const float *lse, const void *pmap,
+                        void *dq, void *dk, void *dv, float *dc_, float *dg, void *workspace,
+                        size_t workspace_bytes, void *stream) {
+    dc_status_t r = dc_attn_bwd_query(params, q, k, v, c, g, dO, lse, pmap, dq, dc_, dg, workspace,
+                                      workspace_bytes, stream);
+    if (r != DC_OK) return r;
+    const int32_t n1 = t_launches;
+    r = dc_attn_bwd_key(params, q, k, c, g, dO, lse, pmap, dc_, dk, dv, workspace, workspace_bytes, stream);
+    t_launches += n1;
+    return r;
+}
+
+int32_t dc_attn_resolve_impl(const dc_attn_params *params) {
+    Checked ck;
+    if (check_params(params, &ck) != DC_OK) return -1;
+    return ck.impl;
+}
+
+dc_status_t dc_attn_device_status(void *stream, uint32_t *status_out, int32_t reset) {
+    if (!status_out) return DC_ERR_INVALID_ARG;
+    cudaStream_t st = (cudaStream_t)stream;
+    unsigned int v = 0;
+    cudaError_t e = cudaStreamSynchronize(st);
+    if (e == cudaSuccess) e = cudaMemcpyFromSymbol(&v, dc::g_status, sizeof(v));
+    if (e == cudaSuccess && reset) {
+        const unsigned int zero = 0;
+        e = cudaMemcpyToSymbol(dc::g_status, &zero, sizeof(zero));
+    }
+    if (e != cudaSuccess) {
+        (void)cudaGetLastError();
+        return DC_ERR_CUDA;
+    }
+    *status_out = v;
+    return DC_OK;
+}
+
+const char *dc_attn_status_string(dc_status_t status) {
+    switch (status) {
+        case DC_OK: return "ok";
+        case DC_ERR_INVALID_ARG: return "invalid argument";
+        case DC_ERR_UNSUPPORTED: return "unsupported shape or type";
+        case DC_ERR_CUDA: return "CUDA error";
+        case DC_ERR_DEVICE: return "device status word holds an error";
+    }
+    return "unknown status";
+}
+
+int32_t dc_attn_last_launch_count(void) { return t_launches; }
+
+}  // extern "C"

@@ -1,0 +1,254 @@
+// simt.cuh -- CUDA-core kernels for Lightweight DC attention (fp32 arithmetic).
+//
+// One warp per query token (forward, backward query side) or per key token
+// (backward key side), all heads of that token in the warp.  These kernels
+// cover every supported shape and both storage types; they are the fp32 path
+// (tensor cores cannot meet an fp32 tolerance) and the path for bf16 shapes
+// the tcgen05 kernels do not take.  Arithmetic is fp32 with expf/logf.
+#pragma once
+
+#include "common.cuh"
+
+namespace dc {
+namespace simt {
+
+constexpr int kMaxHeads = 16;
+
+// Bytes of shared memory one warp needs in each kernel.
+inline size_t fwd_smem_per_warp(int H, int d, int W) { return sizeof(float) * ((size_t)H * d + kMaxHeads + W); }
+inline size_t bwdq_smem_per_warp(int H, int d, int W) { return sizeof(float) * (2 * (size_t)H * d + 3 * (size_t)W); }
+inline size_t bwdk_smem_per_warp(int H, int d, int W) { return sizeof(float) * ((size_t)H * d); }
+
+template <typename T, int DPL>
+__device__ __forceinline__ float dot_row(const float *xs, const T *row) {
+    // <xs, row> over d = 32*DPL elements; xs is in shared memory (broadcast read).
+    float acc = 0.f;
+#pragma unroll 8
+    for (int e = 0; e < 32 * DPL; ++e) acc = fmaf(xs[e], ldf<T>(row + e), acc);
+    return acc;
+}
+
+// Forward: lse per head (pass 1), composed map P over the window (pass 2),
+// o_h = g_h * sum_j P(j) v_h(j) (pass 3).
+template <typename T, int DPL>
+__global__ void fwd_kernel(Shape s, const T *__restrict__ q, const T *__restrict__ k,
+                           const T *__restrict__ v, const float *__restrict__ c,
+                           const float *__restrict__ g, T *__restrict__ o,
+                           float *__restrict__ lse, T *__restrict__ pmap, int check_seqlens) {
+    constexpr int d = 32 * DPL;
+    extern __shared__ float smem[];
+    if (check_seqlens) validate_seqlens(s);
+    const int H = s.H, W = s.W;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int64_t t = (int64_t)blockIdx.x * (blockDim.x >> 5) + warp;
+    if (t >= s.N) return;
+    float *qs = smem + (size_t)warp * (H * d + kMaxHeads + W);
+    float *ls = qs + H * d;
+    float *Pw = ls + kMaxHeads;
+
+    for (int i = lane; i < H * d; i += 32) qs[i] = ldf<T>(q + t * H * d + i);
+    __syncwarp();
+    const int64_t lo = window_lo(s, t);
+    const int n = (int)(t - lo + 1);
+
+    for (int h = 0; h < H; ++h) {
+        float m = -INFINITY, z = 0.f;
+        for (int jj = lane; jj < n; jj += 32) {
+            float x = s.scale * dot_row<T, DPL>(qs + h * d, k + ((lo + jj) * H + h) * d);
+            if (x > m) {
+                z = z * expf(m - x) + 1.f;
+                m = x;
+            } else {
+                z += expf(x - m);
+            }
+        }
+        const float M = warp_max(m);
+        z = (m == -INFINITY) ? 0.f : z * expf(m - M);
+        const float Z = warp_sum(z);
+        const float l = M + logf(Z);
+        if (lane == 0) {
+            ls[h] = l;
+            if (lse) lse[t * H + h] = l;
+        }
+    }
+    __syncwarp();
+    for (int jj = lane; jj < n; jj += 32) {
+        float P = 0.f;
+        for (int h = 0; h < H; ++h) {
+            float x = s.scale * dot_row<T, DPL>(qs + h * d, k + ((lo + jj) * H + h) * d);
+            P = fmaf(__ldg(c + t * H + h), expf(x - ls[h]), P);
+        }
+        Pw[jj] = P;
+    }
+    __syncwarp();
+    if (pmap) {
+        const int64_t w0 = lo - (t - W + 1);   // band index of key lo
+        for (int w = lane; w < W; w += 32) stf<T>(pmap + t * W + w, (w >= w0) ? Pw[w - w0] : 0.f);
+    }
+    for (int h = 0; h < H; ++h) {
+        float acc[DPL];
+#pragma unroll
+        for (int i = 0; i < DPL; ++i) acc[i] = 0.f;
+        for (int jj = 0; jj < n; ++jj) {
+            const float P = Pw[jj];
+            const T *vr = v + ((lo + jj) * H + h) * d;
+#pragma unroll
+            for (int i = 0; i < DPL; ++i) acc[i] = fmaf(P, ldf<T>(vr + lane + 32 * i), acc[i]);
+        }
+        const float gh = __ldg(g + t * H + h);
+#pragma unroll
+        for (int i = 0; i < DPL; ++i) stf<T>(o + (t * H + h) * d + lane + 32 * i, gh * acc[i]);
+    }
+}
+
+// Backward, query side.  Pass 1 over the window: E_h(j) = <dO_h, v_h(j)>,
+// dP(j) = sum_h g_h E_h(j) (stored to the workspace band), dg_h = sum_j P(j) E_h(j).
+// Pass 2 per head: p_h(j) from lse, dc_h = sum_j dP(j) p_h(j),
+// ds_h(j) = c_h p_h(j) (dP(j) - dc_h), dq_h = sigma sum_j ds_h(j) k_h(j).
+template <typename T, int DPL>
+__global__ void bwd_query_kernel(Shape s, const T *__restrict__ q, const T *__restrict__ k,
+                                 const T *__restrict__ v, const float *__restrict__ c,
+                                 const float *__restrict__ g, const T *__restrict__ dO,
+                                 const float *__restrict__ lse, const T *__restrict__ pmap,
+                                 T *__restrict__ dq, float *__restrict__ dc, float *__restrict__ dg,
+                                 float *__restrict__ dPband, int check_seqlens) {
+    constexpr int d = 32 * DPL;
+    extern __shared__ float smem[];
+    if (check_seqlens) validate_seqlens(s);
+    const int H = s.H, W = s.W;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int64_t t = (int64_t)blockIdx.x * (blockDim.x >> 5) + warp;
+    if (t >= s.N) return;
+    float *qs = smem + (size_t)warp * (2 * H * d + 3 * W);
+    float *dos = qs + H * d;
+    float *Pw = dos + H * d;
+    float *dPw = Pw + W;
+    float *sw = dPw + W;
+
+    for (int i = lane; i < H * d; i += 32) {
+        qs[i] = ldf<T>(q + t * H * d + i);
+        dos[i] = ldf<T>(dO + t * H * d + i);
+    }
+    const int64_t lo = window_lo(s, t);
+    const int n = (int)(t - lo + 1);
+    const int w0 = (int)(lo - (t - W + 1));
+    for (int jj = lane; jj < n; jj += 32) Pw[jj] = ldf<T>(pmap + t * W + w0 + jj);
+    for (int w = lane; w < w0; w += 32) dPband[t * W + w] = 0.f;
+    __syncwarp();
+
+    float dgp[kMaxHeads];
+#pragma unroll
+    for (int h = 0; h < kMaxHeads; ++h) dgp[h] = 0.f;
+    for (int jj = lane; jj < n; jj += 32) {
+        float dP = 0.f;
+#pragma unroll
+        for (int h = 0; h < kMaxHeads; ++h) {
+            if (h < H) {
+                const float E = dot_row<T, DPL>(dos + h * d, v + ((lo + jj) * H + h) * d);
+                dP = fmaf(__ldg(g + t * H + h), E, dP);
+                dgp[h] = fmaf(Pw[jj], E, dgp[h]);
+            }
+        }
+        dPw[jj] = dP;
+        dPband[t * W + w0 + jj] = dP;
+    }
+#pragma unroll
+    for (int h = 0; h < kMaxHeads; ++h) {
+        if (h < H) {
+            const float x = warp_sum(dgp[h]);
+            if (lane == 0) dg[t * H + h] = x;
+        }
+    }
+    __syncwarp();
+
+    for (int h = 0; h < H; ++h) {
+        const float l = __ldg(lse + t * H + h);
+        float dcp = 0.f;
+        for (int jj = lane; jj < n; jj += 32) {
+            const float x = s.scale * dot_row<T, DPL>(qs + h * d, k + ((lo + jj) * H + h) * d);
+            const float p = expf(x - l);
+            sw[jj] = p;
+            dcp = fmaf(dPw[jj], p, dcp);
+        }
+        const float dch = warp_sum(dcp);
+        if (lane == 0) dc[t * H + h] = dch;
+        const float ch = __ldg(c + t * H + h);
+        for (int jj = lane; jj < n; jj += 32) sw[jj] = ch * sw[jj] * (dPw[jj] - dch);
+        __syncwarp();
+        float acc[DPL];
+#pragma unroll
+        for (int i = 0; i < DPL; ++i) acc[i] = 0.f;
+        for (int jj = 0; jj < n; ++jj) {
+            const float ds = sw[jj];
+            const T *kr = k + ((lo + jj) * H + h) * d;
+#pragma unroll
+            for (int i = 0; i < DPL; ++i) acc[i] = fmaf(ds, ldf<T>(kr + lane + 32 * i), acc[i]);
+        }
+#pragma unroll
+        for (int i = 0; i < DPL; ++i) stf<T>(dq + (t * H + h) * d + lane + 32 * i, s.scale * acc[i]);
+        __syncwarp();
+    }
+}
+
+// Backward, key side: for key j and the queries t whose window holds it,
+// ds_h(t,j) = c[t,h] p_h(t,j) (dP(t,j) - dc[t,h]) with p_h from lse and dP from
+// the workspace band, dk_h(j) = sigma sum_t ds_h q_h(t), dv_h(j) = sum_t P g_h dO_h(t).
+template <typename T, int DPL>
+__global__ void bwd_key_kernel(Shape s, const T *__restrict__ q, const T *__restrict__ k,
+                               const float *__restrict__ c, const float *__restrict__ g,
+                               const T *__restrict__ dO, const float *__restrict__ lse,
+                               const T *__restrict__ pmap, const float *__restrict__ dc,
+                               const float *__restrict__ dPband, T *__restrict__ dk,
+                               T *__restrict__ dv) {
+    constexpr int d = 32 * DPL;
+    extern __shared__ float smem[];
+    const int H = s.H, W = s.W;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int64_t j = (int64_t)blockIdx.x * (blockDim.x >> 5) + warp;
+    if (j >= s.N) return;
+    float *ks = smem + (size_t)warp * (H * d);
+    for (int i = lane; i < H * d; i += 32) ks[i] = ldf<T>(k + j * H * d + i);
+    __syncwarp();
+    int64_t hi = j + W - 1;
+    const int64_t b = doc_end(s, j);
+    if (hi > b - 1) hi = b - 1;
+    const int n = (int)(hi - j + 1);
+
+    for (int h = 0; h < H; ++h) {
+        float ak[DPL], av[DPL];
+#pragma unroll
+        for (int i = 0; i < DPL; ++i) ak[i] = av[i] = 0.f;
+        for (int base = 0; base < n; base += 32) {
+            float ds = 0.f, pg = 0.f;
+            if (base + lane < n) {
+                const int64_t t = j + base + lane;
+                const int64_t w = j - (t - W + 1);
+                const float x = s.scale * dot_row<T, DPL>(ks + h * d, q + (t * H + h) * d);
+                const float p = expf(x - __ldg(lse + t * H + h));
+                ds = __ldg(c + t * H + h) * p * (__ldg(dPband + t * W + w) - __ldg(dc + t * H + h));
+                pg = ldf<T>(pmap + t * W + w) * __ldg(g + t * H + h);
+            }
+            const int cnt = min(32, n - base);
+            for (int l = 0; l < cnt; ++l) {
+                const float dsl = __shfl_sync(0xffffffffu, ds, l);
+                const float pgl = __shfl_sync(0xffffffffu, pg, l);
+                const int64_t t = j + base + l;
+                const T *qr = q + (t * H + h) * d;
+                const T *dr = dO + (t * H + h) * d;
+#pragma unroll
+                for (int i = 0; i < DPL; ++i) {
+                    ak[i] = fmaf(dsl, ldf<T>(qr + lane + 32 * i), ak[i]);
+                    av[i] = fmaf(pgl, ldf<T>(dr + lane + 32 * i), av[i]);
+                }
+            }
+        }
+#pragma unroll
+        for (int i = 0; i < DPL; ++i) {
+            stf<T>(dk + (j * H + h) * d + lane + 32 * i, s.scale * ak[i]);
+            stf<T>(dv + (j * H + h) * d + lane + 32 * i, av[i]);
+        }
+    }
+}
+
+}  // namespace simt
+}  // namespace dc

@@ -1,0 +1,229 @@
+"""Python binding of libdcattn (ctypes).  Argument marshalling only: every step
+of the computation runs in the CUDA kernels behind include/dcattn.h.
+
+Functions carry the C entry points' names and take torch CUDA tensors; torch is
+used for device memory and the current stream, nothing else.  There is no CPU
+path: a missing library or a CPU tensor raises.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libdcattn.so")
+
+DC_OK, DC_ERR_INVALID_ARG, DC_ERR_UNSUPPORTED, DC_ERR_CUDA, DC_ERR_DEVICE = range(5)
+DC_F32, DC_BF16 = 0, 1
+IMPLS = {"auto": 0, "simt": 1, "tcgen05": 2}
+IMPL_NAMES = {v: k for k, v in IMPLS.items()}
+DC_DEVERR_SEQLENS = 0x1
+DC_DEVERR_TIMEOUT = 0x2
+
+EXPORTED = ("dc_attn_fwd", "dc_attn_bwd_workspace_size", "dc_attn_bwd_query", "dc_attn_bwd_key",
+            "dc_attn_bwd", "dc_attn_resolve_impl", "dc_attn_device_status", "dc_attn_status_string",
+            "dc_attn_last_launch_count")
+
+
+class DCAttnError(RuntimeError):
+    def __init__(self, fn: str, code: int, msg: str):
+        super().__init__(f"{fn} failed: {msg} (status {code})")
+        self.code = code
+
+
+class Params(ctypes.Structure):
+    _fields_ = [("dtype", ctypes.c_int32), ("impl", ctypes.c_int32), ("total_tokens", ctypes.c_int64),
+                ("num_docs", ctypes.c_int32), ("num_heads", ctypes.c_int32), ("head_dim", ctypes.c_int32),
+                ("window", ctypes.c_int32), ("softmax_scale", ctypes.c_float), ("reserved", ctypes.c_int32),
+                ("cu_seqlens", ctypes.c_void_p)]
+
+
+_lib = None
+
+
+def load_library(path: str = LIB_PATH):
+    """Load libdcattn.so and declare its signatures.  Raises if it is not built."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(path):
+        raise RuntimeError(f"libdcattn.so is not built ({path}); run `python -m cross_head_dynamic_b200.build`")
+    lib = ctypes.CDLL(path)
+    P = ctypes.POINTER(Params)
+    vp = ctypes.c_void_p
+    st = ctypes.c_int
+    lib.dc_attn_fwd.argtypes = [P] + [vp] * 9
+    lib.dc_attn_fwd.restype = st
+    lib.dc_attn_bwd_workspace_size.argtypes = [P]
+    lib.dc_attn_bwd_workspace_size.restype = ctypes.c_size_t
+    lib.dc_attn_bwd_query.argtypes = [P] + [vp] * 12 + [ctypes.c_size_t, vp]
+    lib.dc_attn_bwd_query.restype = st
+    lib.dc_attn_bwd_key.argtypes = [P] + [vp] * 11 + [ctypes.c_size_t, vp]
+    lib.dc_attn_bwd_key.restype = st
+    lib.dc_attn_bwd.argtypes = [P] + [vp] * 14 + [ctypes.c_size_t, vp]
+    lib.dc_attn_bwd.restype = st
+    lib.dc_attn_resolve_impl.argtypes = [P]
+    lib.dc_attn_resolve_impl.restype = ctypes.c_int32
+    lib.dc_attn_device_status.argtypes = [vp, ctypes.POINTER(ctypes.c_uint32), ctypes.c_int32]
+    lib.dc_attn_device_status.restype = st
+    lib.dc_attn_status_string.argtypes = [st]
+    lib.dc_attn_status_string.restype = ctypes.c_char_p
+    lib.dc_attn_last_launch_count.argtypes = []
+    lib.dc_attn_last_launch_count.restype = ctypes.c_int32
+    _lib = lib
+    return lib
+
+
+def _check(fn: str, code: int):
+    if code != DC_OK:
+        msg = load_library().dc_attn_status_string(code).decode()
+        raise DCAttnError(fn, code, msg)
+
+
+def _stream_handle(stream) -> int:
+    s = torch.cuda.current_stream() if stream is None else stream
+    return s.cuda_stream
+
+
+def _dev(x: torch.Tensor, name: str, dtype=None):
+    if not isinstance(x, torch.Tensor):
+        raise TypeError(f"{name} must be a torch tensor")
+    if not x.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor (libdcattn has no CPU path)")
+    if not x.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if dtype is not None and x.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype}, got {x.dtype}")
+    return x.data_ptr()
+
+
+def _opt(x, name, dtype=None):
+    return None if x is None else _dev(x, name, dtype)
+
+
+def make_params(q: torch.Tensor, cu_seqlens: torch.Tensor, window: int, scale: float,
+                impl: str = "auto") -> Params:
+    if q.dim() != 3:
+        raise ValueError("q must be [N, H, d]")
+    N, H, d = q.shape
+    if q.dtype == torch.float32:
+        dt = DC_F32
+    elif q.dtype == torch.bfloat16:
+        dt = DC_BF16
+    else:
+        raise TypeError(f"unsupported dtype {q.dtype}")
+    return Params(dtype=dt, impl=IMPLS[impl], total_tokens=N, num_docs=cu_seqlens.numel() - 1,
+                  num_heads=H, head_dim=d, window=int(window), softmax_scale=float(scale), reserved=0,
+                  cu_seqlens=_dev(cu_seqlens, "cu_seqlens", torch.int32))
+
+
+def dc_attn_resolve_impl(q, cu_seqlens, window, scale, impl="auto") -> str:
+    p = make_params(q, cu_seqlens, window, scale, impl)
+    r = load_library().dc_attn_resolve_impl(ctypes.byref(p))
+    if r < 0:
+        raise DCAttnError("dc_attn_resolve_impl", DC_ERR_INVALID_ARG, "invalid parameters")
+    return IMPL_NAMES[r]
+
+
+def dc_attn_fwd(q, k, v, c, g, cu_seqlens, window: int, scale: float, *, o=None, lse=None, pmap=None,
+                need_backward: bool = True, impl: str = "auto", stream=None):
+    """Forward pass; returns (o, lse, pmap).  lse/pmap are None when need_backward
+    is False and none were passed in."""
+    p = make_params(q, cu_seqlens, window, scale, impl)
+    N, H, d = q.shape
+    if o is None:
+        o = torch.empty_like(q)
+    if need_backward:
+        if lse is None:
+            lse = torch.empty(N, H, device=q.device, dtype=torch.float32)
+        if pmap is None:
+            pmap = torch.empty(N, int(window), device=q.device, dtype=q.dtype)
+    code = load_library().dc_attn_fwd(
+        ctypes.byref(p), _dev(q, "q", q.dtype), _dev(k, "k", q.dtype), _dev(v, "v", q.dtype),
+        _dev(c, "c", torch.float32), _dev(g, "g", torch.float32), _dev(o, "o", q.dtype),
+        _opt(lse, "lse", torch.float32), _opt(pmap, "pmap", q.dtype), _stream_handle(stream))
+    _check("dc_attn_fwd", code)
+    return o, lse, pmap
+
+
+def dc_attn_bwd_workspace_size(q, cu_seqlens, window, scale, impl="auto") -> int:
+    p = make_params(q, cu_seqlens, window, scale, impl)
+    return int(load_library().dc_attn_bwd_workspace_size(ctypes.byref(p)))
+
+
+def _workspace(q, cu_seqlens, window, scale, impl, workspace):
+    need = dc_attn_bwd_workspace_size(q, cu_seqlens, window, scale, impl)
+    if workspace is None:
+        workspace = torch.empty(max(need, 16), device=q.device, dtype=torch.uint8)
+    return workspace
+
+
+def dc_attn_bwd_query(q, k, v, c, g, dO, lse, pmap, cu_seqlens, window, scale, *, dq=None, dc=None,
+                      dg=None, workspace=None, impl="auto", stream=None):
+    """Query side of the backward; returns (dq, dc, dg, workspace)."""
+    p = make_params(q, cu_seqlens, window, scale, impl)
+    N, H, d = q.shape
+    dq = torch.empty_like(q) if dq is None else dq
+    dc = torch.empty(N, H, device=q.device, dtype=torch.float32) if dc is None else dc
+    dg = torch.empty(N, H, device=q.device, dtype=torch.float32) if dg is None else dg
+    workspace = _workspace(q, cu_seqlens, window, scale, impl, workspace)
+    code = load_library().dc_attn_bwd_query(
+        ctypes.byref(p), _dev(q, "q", q.dtype), _dev(k, "k", q.dtype), _dev(v, "v", q.dtype),
+        _dev(c, "c", torch.float32), _dev(g, "g", torch.float32), _dev(dO, "dO", q.dtype),
+        _dev(lse, "lse", torch.float32), _dev(pmap, "pmap", q.dtype), _dev(dq, "dq", q.dtype),
+        _dev(dc, "dc", torch.float32), _dev(dg, "dg", torch.float32), _dev(workspace, "workspace"),
+        workspace.numel() * workspace.element_size(), _stream_handle(stream))
+    _check("dc_attn_bwd_query", code)
+    return dq, dc, dg, workspace
+
+
+def dc_attn_bwd_key(q, k, c, g, dO, lse, pmap, dc, workspace, cu_seqlens, window, scale, *, dk=None, dv=None,
+                    impl="auto", stream=None):
+    """Key side of the backward (after dc_attn_bwd_query); returns (dk, dv)."""
+    p = make_params(q, cu_seqlens, window, scale, impl)
+    dk = torch.empty_like(q) if dk is None else dk
+    dv = torch.empty_like(q) if dv is None else dv
+    code = load_library().dc_attn_bwd_key(
+        ctypes.byref(p), _dev(q, "q", q.dtype), _dev(k, "k", q.dtype), _dev(c, "c", torch.float32),
+        _dev(g, "g", torch.float32), _dev(dO, "dO", q.dtype), _dev(lse, "lse", torch.float32),
+        _dev(pmap, "pmap", q.dtype), _dev(dc, "dc", torch.float32), _dev(dk, "dk", q.dtype),
+        _dev(dv, "dv", q.dtype), _dev(workspace, "workspace"), workspace.numel() * workspace.element_size(),
+        _stream_handle(stream))
+    _check("dc_attn_bwd_key", code)
+    return dk, dv
+
+
+def dc_attn_bwd(q, k, v, c, g, dO, lse, pmap, cu_seqlens, window, scale, *, dq=None, dk=None, dv=None,
+                dc=None, dg=None, workspace=None, impl="auto", stream=None):
+    """Full backward; returns (dq, dk, dv, dc, dg)."""
+    p = make_params(q, cu_seqlens, window, scale, impl)
+    N, H, d = q.shape
+    dq = torch.empty_like(q) if dq is None else dq
+    dk = torch.empty_like(q) if dk is None else dk
+    dv = torch.empty_like(q) if dv is None else dv
+    dc = torch.empty(N, H, device=q.device, dtype=torch.float32) if dc is None else dc
+    dg = torch.empty(N, H, device=q.device, dtype=torch.float32) if dg is None else dg
+    workspace = _workspace(q, cu_seqlens, window, scale, impl, workspace)
+    code = load_library().dc_attn_bwd(
+        ctypes.byref(p), _dev(q, "q", q.dtype), _dev(k, "k", q.dtype), _dev(v, "v", q.dtype),
+        _dev(c, "c", torch.float32), _dev(g, "g", torch.float32), _dev(dO, "dO", q.dtype),
+        _dev(lse, "lse", torch.float32), _dev(pmap, "pmap", q.dtype), _dev(dq, "dq", q.dtype),
+        _dev(dk, "dk", q.dtype), _dev(dv, "dv", q.dtype), _dev(dc, "dc", torch.float32),
+        _dev(dg, "dg", torch.float32), _dev(workspace, "workspace"),
+        workspace.numel() * workspace.element_size(), _stream_handle(stream))
+    _check("dc_attn_bwd", code)
+    return dq, dk, dv, dc, dg
+
+
+def dc_attn_device_status(reset: bool = True, stream=None) -> int:
+    """Synchronize and return the device status word (DC_DEVERR_* bits)."""
+    out = ctypes.c_uint32(0)
+    code = load_library().dc_attn_device_status(_stream_handle(stream), ctypes.byref(out), int(reset))
+    _check("dc_attn_device_status", code)
+    return int(out.value)
+
+
+def dc_attn_last_launch_count() -> int:
+    return int(load_library().dc_attn_last_launch_count())

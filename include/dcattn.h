@@ -1,0 +1,149 @@
+/*
+ * dcattn.h -- C ABI of libdcattn, Lightweight DC attention on NVIDIA B200 (sm_100a).
+ *
+ * The operation (the "Lightweight DC" paragraph of the m.aitntnews.com blog
+ * post on the NanoGPT speedrun, section "第二刀-砍层内"): the layer's existing
+ * Q and K are reused for an extra causal local window of W keys (112 there);
+ * every head takes a softmax over its window scores; the H per-head maps are
+ * merged with per-token, input-dependent weights into one shared map; the
+ * shared map is applied to each head's V with a per-head scale.  For query
+ * token t in document [a, b) and head h:
+ *
+ *   window(t) = { j : max(a, t-W+1) <= j <= t }
+ *   p_h(t,j)  = softmax over window(t) of  sigma * <q_h(t), k_h(j)>
+ *   P(t,j)    = sum_h c[t,h] * p_h(t,j)           (c: signed, per token)
+ *   o_h(t)    = g[t,h] * sum_j P(t,j) * v_h(j)     (g: per-token head scale)
+ *
+ * Conventions shared by every entry point
+ * ---------------------------------------
+ * - Tokens are packed: N = total_tokens rows, documents given by cu_seqlens
+ *   (device, int32, num_docs + 1 entries, 0 = cu[0] <= ... <= cu[num_docs] = N;
+ *   empty documents are allowed).  No key of another document is ever used.
+ * - q, k, v, o, dO, dq, dk, dv: contiguous [N][H][d] in `dtype` (fp32 or bf16).
+ *   c, g, lse, dc, dg: contiguous [N][H] fp32.
+ *   pmap: contiguous [N][W] in `dtype`; pmap[t][w] = P(t, t-W+1+w), 0 outside
+ *   window(t).  It is the one composed map per token (the H per-head maps are
+ *   never written to memory); the forward produces it, the backward reads it.
+ * - Every pointer is caller-owned DEVICE memory, 16-byte aligned.  The library
+ *   never allocates, frees or synchronizes (except dc_attn_device_status).
+ *   Outputs are overwritten, never accumulated into.  Inputs are not modified.
+ * - Calls are asynchronous on `stream` (a cudaStream_t; NULL = legacy default
+ *   stream).  Argument errors are detected on the host and returned before
+ *   anything is launched.  Errors found on the device (malformed cu_seqlens, a
+ *   bounded wait that gave up) are recorded in a per-device status word read by
+ *   dc_attn_device_status(); kernels never trap.  Malformed cu_seqlens cannot
+ *   make a kernel read or write out of bounds; they only make results undefined.
+ * - The library is compiled for sm_100a only.
+ */
+#ifndef DCATTN_H
+#define DCATTN_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    DC_OK = 0,
+    DC_ERR_INVALID_ARG = 1,   /* null/misaligned pointer, bad size, bad enum   */
+    DC_ERR_UNSUPPORTED = 2,   /* valid request outside what this build covers  */
+    DC_ERR_CUDA = 3,          /* a CUDA runtime/driver call failed             */
+    DC_ERR_DEVICE = 4         /* the device status word holds an error         */
+} dc_status_t;
+
+typedef enum { DC_F32 = 0, DC_BF16 = 1 } dc_dtype_t;
+
+/* Kernel family.  AUTO picks the tcgen05/TMA path when the shape allows it
+ * (bf16, d in {64,128}, W <= 193) and the SIMT path otherwise.  SIMT is the
+ * fp32-accumulating CUDA-core path used for fp32 tensors and any shape. */
+typedef enum { DC_IMPL_AUTO = 0, DC_IMPL_SIMT = 1, DC_IMPL_TCGEN05 = 2 } dc_impl_t;
+
+/* Bits of the device status word. */
+#define DC_DEVERR_SEQLENS 0x1u   /* cu_seqlens not 0-based, non-decreasing, ending at N */
+#define DC_DEVERR_TIMEOUT 0x2u   /* a bounded wait inside a kernel gave up              */
+
+typedef struct {
+    int32_t dtype;              /* dc_dtype_t: type of q,k,v,o,dO,dq,dk,dv,pmap           */
+    int32_t impl;               /* dc_impl_t                                              */
+    int64_t total_tokens;       /* N >= 0; N == 0 is a no-op                              */
+    int32_t num_docs;           /* >= 1 when N > 0                                        */
+    int32_t num_heads;          /* H in [1, 16]                                           */
+    int32_t head_dim;           /* d in {32, 64, 96, 128} (tcgen05 path: {64, 128})        */
+    int32_t window;             /* W in [1, 4096]: keys t-W+1 .. t (query included)       */
+    float softmax_scale;        /* sigma, usually 1/sqrt(d); 1 when q is pre-scaled        */
+    int32_t reserved;           /* must be 0                                              */
+    const int32_t *cu_seqlens;  /* device pointer, num_docs + 1 entries                   */
+} dc_attn_params;
+
+/* Forward pass.
+ * In : q, k, v [N][H][d]; c, g [N][H] fp32.
+ * Out: o [N][H][d]; lse [N][H] fp32, lse_h(t) = log sum_j exp(sigma<q_h(t),k_h(j)>)
+ *      (natural log); pmap [N][W].  lse and pmap may be NULL when no backward
+ *      pass will follow; the backward needs both. */
+dc_status_t dc_attn_fwd(const dc_attn_params *params,
+                        const void *q, const void *k, const void *v,
+                        const float *c, const float *g,
+                        void *o, float *lse, void *pmap, void *stream);
+
+/* Bytes of device scratch the backward entry points need (the composed-map
+ * gradient dP(t, .) handed from the query pass to the key pass, fp32 [N][W]).
+ * 0 when N == 0. */
+size_t dc_attn_bwd_workspace_size(const dc_attn_params *params);
+
+/* Backward, query side: dq [N][H][d], dc [N][H], dg [N][H] fp32, and dP into
+ * the workspace.  Needs lse and pmap from dc_attn_fwd with the same inputs.
+ *   dg[t,h]   = sum_j P(t,j) <dO_h(t), v_h(j)>
+ *   dP(t,j)   = sum_h g[t,h] <dO_h(t), v_h(j)>
+ *   dc[t,h]   = sum_j dP(t,j) p_h(t,j)
+ *   ds_h(t,j) = c[t,h] p_h(t,j) (dP(t,j) - dc[t,h])
+ *   dq_h(t)   = sigma sum_j ds_h(t,j) k_h(j)
+ * (chain rule of the definition above; the page states no backward pass). */
+dc_status_t dc_attn_bwd_query(const dc_attn_params *params,
+                              const void *q, const void *k, const void *v,
+                              const float *c, const float *g, const void *dO,
+                              const float *lse, const void *pmap,
+                              void *dq, float *dc, float *dg,
+                              void *workspace, size_t workspace_bytes, void *stream);
+
+/* Backward, key side: dk, dv [N][H][d].  Must follow dc_attn_bwd_query on the
+ * same stream with the same workspace (it reads dc and the stored dP).
+ *   dk_h(j) = sigma sum_{t: j in window(t)} ds_h(t,j) q_h(t)
+ *   dv_h(j) = sum_{t: j in window(t)} P(t,j) g[t,h] dO_h(t) */
+dc_status_t dc_attn_bwd_key(const dc_attn_params *params,
+                            const void *q, const void *k,
+                            const float *c, const float *g, const void *dO,
+                            const float *lse, const void *pmap, const float *dc,
+                            void *dk, void *dv,
+                            const void *workspace, size_t workspace_bytes, void *stream);
+
+/* Full backward: dc_attn_bwd_query followed by dc_attn_bwd_key. */
+dc_status_t dc_attn_bwd(const dc_attn_params *params,
+                        const void *q, const void *k, const void *v,
+                        const float *c, const float *g, const void *dO,
+                        const float *lse, const void *pmap,
+                        void *dq, void *dk, void *dv, float *dc, float *dg,
+                        void *workspace, size_t workspace_bytes, void *stream);
+
+/* Which kernel family AUTO resolves to for these params (DC_IMPL_SIMT or
+ * DC_IMPL_TCGEN05), or -1 if the params are invalid. */
+int32_t dc_attn_resolve_impl(const dc_attn_params *params);
+
+/* Synchronizes `stream`, stores the current device's status word (DC_DEVERR_*
+ * bits, 0 = no error) into *status_out and clears it when `reset` != 0.
+ * Returns DC_ERR_CUDA if the synchronization itself failed. */
+dc_status_t dc_attn_device_status(void *stream, uint32_t *status_out, int32_t reset);
+
+/* Static, human-readable name of a status code. */
+const char *dc_attn_status_string(dc_status_t status);
+
+/* Number of kernel launches the last successful call on this host thread made
+ * (used to report launches per step). */
+int32_t dc_attn_last_launch_count(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* DCATTN_H */

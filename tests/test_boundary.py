@@ -1,0 +1,122 @@
+"""Host-side checks of the C ABI: the library builds/loads, exports every
+function include/dcattn.h declares, and rejects bad arguments on the host
+before any CUDA call (so these run without a GPU)."""
+import ctypes
+import os
+import re
+import subprocess
+
+import pytest
+
+from cross_head_dynamic_b200 import build as dcbuild
+from cross_head_dynamic_b200 import dcattn
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "dcattn.h")
+
+
+@pytest.fixture(scope="module")
+def lib():
+    dcbuild.build()
+    return dcattn.load_library()
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(dc_attn_\w+)\s*\(", text)))
+
+
+def test_header_declares_expected_api():
+    names = declared_functions()
+    assert set(dcattn.EXPORTED) <= set(names), names
+    assert set(names) <= set(dcattn.EXPORTED) | {"dc_attn_fwd_noalloc"}, names
+
+
+def test_library_exports_every_declared_symbol(lib):
+    out = subprocess.check_output(["nm", "-D", "--defined-only", dcattn.LIB_PATH]).decode()
+    exported = set(re.findall(r"\bT (dc_attn_\w+)$", out, flags=re.M))
+    for name in declared_functions():
+        assert name in exported, name
+        assert hasattr(lib, name)
+
+
+def test_library_has_no_oracle_dependency(lib):
+    out = subprocess.check_output(["nm", "-D", dcattn.LIB_PATH]).decode()
+    assert "dc_oracle" not in out
+    ldd = subprocess.check_output(["ldd", dcattn.LIB_PATH]).decode()
+    assert "dcoracle" not in ldd
+
+
+def test_status_strings(lib):
+    for code in range(5):
+        assert lib.dc_attn_status_string(code)
+    assert lib.dc_attn_status_string(99) == b"unknown status"
+
+
+def _params(**kw):
+    base = dict(dtype=dcattn.DC_BF16, impl=0, total_tokens=256, num_docs=1, num_heads=6, head_dim=128,
+                window=112, softmax_scale=0.088, reserved=0, cu_seqlens=0x1000)
+    base.update(kw)
+    return dcattn.Params(**base)
+
+
+def _fwd(lib, p, ptr=0x2000):
+    return lib.dc_attn_fwd(ctypes.byref(p), ptr, ptr, ptr, ptr, ptr, ptr, None, None, None)
+
+
+@pytest.mark.parametrize("kw,expect", [
+    (dict(dtype=7), dcattn.DC_ERR_INVALID_ARG),
+    (dict(impl=9), dcattn.DC_ERR_INVALID_ARG),
+    (dict(reserved=1), dcattn.DC_ERR_INVALID_ARG),
+    (dict(total_tokens=-1), dcattn.DC_ERR_INVALID_ARG),
+    (dict(num_heads=0), dcattn.DC_ERR_INVALID_ARG),
+    (dict(num_heads=17), dcattn.DC_ERR_INVALID_ARG),
+    (dict(window=0), dcattn.DC_ERR_INVALID_ARG),
+    (dict(num_docs=0), dcattn.DC_ERR_INVALID_ARG),
+    (dict(num_docs=258), dcattn.DC_ERR_INVALID_ARG),
+    (dict(cu_seqlens=0), dcattn.DC_ERR_INVALID_ARG),
+    (dict(softmax_scale=float("nan")), dcattn.DC_ERR_INVALID_ARG),
+    (dict(head_dim=48), dcattn.DC_ERR_UNSUPPORTED),
+    (dict(head_dim=256), dcattn.DC_ERR_UNSUPPORTED),
+    (dict(window=5000), dcattn.DC_ERR_UNSUPPORTED),
+    (dict(dtype=dcattn.DC_F32, impl=2), dcattn.DC_ERR_UNSUPPORTED),
+])
+def test_bad_params_rejected_on_host(lib, kw, expect):
+    assert _fwd(lib, _params(**kw)) == expect
+
+
+def test_null_and_misaligned_pointers_rejected(lib):
+    p = _params(dtype=dcattn.DC_F32)
+    assert _fwd(lib, p, ptr=0) == dcattn.DC_ERR_INVALID_ARG
+    assert _fwd(lib, p, ptr=0x2008) == dcattn.DC_ERR_INVALID_ARG
+
+
+def test_empty_problem_is_a_noop(lib):
+    p = _params(total_tokens=0, num_docs=0, cu_seqlens=0)
+    assert _fwd(lib, p, ptr=0) == dcattn.DC_OK
+    assert lib.dc_attn_bwd_workspace_size(ctypes.byref(p)) == 0
+
+
+def test_workspace_size_and_check(lib):
+    p = _params(dtype=dcattn.DC_F32, total_tokens=1000, num_docs=3, window=112)
+    need = lib.dc_attn_bwd_workspace_size(ctypes.byref(p))
+    assert need == 4 * 1000 * 112
+    a = 0x4000
+    args = [a] * 12
+    rc = lib.dc_attn_bwd_query(ctypes.byref(p), *args, need - 1, None)
+    assert rc == dcattn.DC_ERR_INVALID_ARG
+
+
+def test_resolve_impl(lib):
+    assert lib.dc_attn_resolve_impl(ctypes.byref(_params(dtype=dcattn.DC_F32))) == 1
+    assert lib.dc_attn_resolve_impl(ctypes.byref(_params(impl=1))) == 1
+    assert lib.dc_attn_resolve_impl(ctypes.byref(_params(window=0))) == -1
+
+
+def test_binding_refuses_cpu_tensors():
+    import torch
+    q = torch.zeros(4, 1, 32)
+    with pytest.raises(ValueError):
+        dcattn.dc_attn_fwd(q, q, q, torch.zeros(4, 1), torch.zeros(4, 1), torch.tensor([0, 4], dtype=torch.int32),
+                           4, 1.0)
