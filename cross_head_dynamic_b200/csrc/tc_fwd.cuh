@@ -1,0 +1,343 @@
+// tc_fwd.cuh -- tcgen05 forward kernel of Lightweight DC attention (bf16 in,
+// fp32 accumulate).
+//
+// One CTA per block of BM (<= 128) consecutive packed query tokens, all heads.
+// Keys of the block live in one tile of span = round16(BM + W - 1) rows that
+// starts W - 1 tokens before the block; tile column c is key kbase + c.
+//
+// Phase 1, per head h (double-buffered Q/K tiles in smem):
+//   TMA     Q_h [128 x d], K_h [span x d]          (128-byte swizzle)
+//   MMA     S_h = Q_h K_h^T  -> TMEM columns [0, span) fp32
+//   SIMT    pull the row band of S_h into registers (which frees the S columns
+//           for the next head's MMA), mask to the causal window inside the
+//           document, softmax per row, P += c[t,h] * p_h with P accumulated in
+//           TMEM columns [256, 256 + span) (the H maps never leave the chip)
+// Phase 2:
+//   SIMT    P -> bf16 tile in smem (K-major, swizzled), band copy -> pmap
+//   per head: TMA V_h [span x d]; MMA U_h = P V_h -> TMEM [128 x d];
+//           SIMT o_h = g[t,h] * U_h -> bf16 -> global
+//
+// Warps 0-7 do the SIMT work: warp w reads TMEM lanes 32*(w%4).. (rows of
+// the tile) and half (w/4) of its quarter's column band.  Warp 8 lane 0
+// issues every TMA and MMA.  All waits are bounded (see wait_bar).
+#pragma once
+
+#include "tc_common.cuh"
+
+namespace dc {
+namespace tc {
+
+template <int D>
+struct FwdLayout {
+    static constexpr uint32_t kQBytes = 128u * D * 2;        // Q_h tile: D/64 boxes of 128 rows x 128 B
+    static constexpr uint32_t kKHalf = 256u * 128;           // one 64-column box of a K/V tile (<= 256 rows)
+    static constexpr uint32_t kKBytes = (D / 64) * kKHalf;   // K_h or V_h tile
+    static constexpr uint32_t kPBytes = 4u * 16384;          // P tile: 4 blocks of 64 columns x 128 rows
+    static constexpr uint32_t kQ0 = 0;
+    static constexpr uint32_t kQ1 = kQBytes;
+    static constexpr uint32_t kK0 = 2 * kQBytes;
+    static constexpr uint32_t kK1 = kK0 + kKBytes;
+    // the P tile reuses the Q buffers when they are large enough (free after the last S MMA)
+    static constexpr uint32_t kP = (2 * kQBytes >= kPBytes) ? 0u : kK1 + kKBytes;
+    static constexpr uint32_t kRed = (kP == 0 ? kK1 + kKBytes : kP + kPBytes);
+    static constexpr uint32_t kBars = kRed + 2 * 2 * 128 * 4;
+    static constexpr uint32_t kBytes = kBars + 256;
+    static constexpr uint32_t kAlloc = kBytes + 1024;        // slack to align the base to 1 KiB
+};
+
+struct FwdArgs {
+    Shape s;
+    int BM;
+    int span;
+    const float *c;
+    const float *g;
+    __nv_bfloat16 *o;
+    float *lse;
+    __nv_bfloat16 *pmap;
+};
+
+// mbarrier slots
+enum : int { kBarQK = 0, kBarSFull = 2, kBarSFree = 3, kBarV = 4, kBarUFull = 6, kBarUFree = 8, kBarP = 10,
+             kNumBars = 11 };
+
+template <int D, int MAXC>
+__global__ void __launch_bounds__(kThreads, 1)
+fwd_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__ CUtensorMap map_k,
+           const __grid_constant__ CUtensorMap map_v, const FwdArgs a) {
+    using L = FwdLayout<D>;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *sm = (uint8_t *)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
+    uint64_t *bars = (uint64_t *)(sm + L::kBars);
+    uint32_t *tmem_slot = (uint32_t *)(bars + 16);
+    volatile int *abort_flag = (volatile int *)(tmem_slot + 1);
+    float *red_max = (float *)(sm + L::kRed);     // [2][128]
+    float *red_sum = red_max + 256;               // [2][128]
+
+    const Shape &s = a.s;
+    const int H = s.H, W = s.W, BM = a.BM, span = a.span;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int64_t t0 = (int64_t)blockIdx.x * BM;
+    const int64_t kbase = t0 - (W - 1);
+
+    validate_seqlens(s);
+    if (threadIdx.x == 0) {
+        for (int i = 0; i < kNumBars; ++i) {
+            uint32_t cnt = 1;
+            if (i == kBarSFree || i == kBarUFree || i == kBarUFree + 1 || i == kBarP)
+                cnt = kComputeThreads;
+            ptx::mbar_init(&bars[i], cnt);
+        }
+        *abort_flag = 0;
+        ptx::fence_mbar_init();
+    }
+    if (warp == 0) {
+        ptx::tmem_alloc(tmem_slot, 512);
+        ptx::tmem_relinquish();
+    }
+    ptx::tc_fence_before();
+    __syncthreads();
+    ptx::tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+
+    if (warp == kProducerWarp) {
+        if (lane == 0) {
+            ptx::prefetch_tensormap(&map_q);
+            ptx::prefetch_tensormap(&map_k);
+            ptx::prefetch_tensormap(&map_v);
+            const uint32_t qk_bytes = L::kQBytes + (D / 64) * span * 128;
+            const uint32_t v_bytes = (D / 64) * span * 128;
+            auto issue_qk = [&](int h) {
+                const int b = h & 1;
+                uint8_t *q = sm + (b ? L::kQ1 : L::kQ0);
+                uint8_t *k = sm + (b ? L::kK1 : L::kK0);
+                ptx::mbar_arrive_expect_tx(&bars[kBarQK + b], qk_bytes);
+                for (int kb = 0; kb < D / 64; ++kb) {
+                    ptx::tma_load_2d(q + kb * 16384, &map_q, h * D + kb * 64, (int)t0, &bars[kBarQK + b]);
+                    ptx::tma_load_2d(k + kb * L::kKHalf, &map_k, h * D + kb * 64, (int)kbase, &bars[kBarQK + b]);
+                }
+            };
+            auto issue_v = [&](int h) {
+                const int b = h & 1;
+                uint8_t *v = sm + (b ? L::kK1 : L::kK0);
+                ptx::mbar_arrive_expect_tx(&bars[kBarV + b], v_bytes);
+                for (int kb = 0; kb < D / 64; ++kb)
+                    ptx::tma_load_2d(v + kb * L::kKHalf, &map_v, h * D + kb * 64, (int)kbase, &bars[kBarV + b]);
+            };
+            const uint32_t id_s = ptx::idesc_bf16_f32(128, span, 0, 0);
+            const uint32_t id_pv = ptx::idesc_bf16_f32(128, D, 0, 1);
+
+            // ---- phase 1: S_h = Q_h K_h^T into the single S buffer (TMEM columns 0..)
+            for (int h = 0; h < H && h < 2; ++h) issue_qk(h);
+            for (int h = 0; h < H; ++h) {
+                const int b = h & 1;
+                bool ok = wait_bar(&bars[kBarQK + b], (uint32_t)(h >> 1) & 1, abort_flag);
+                if (h >= 1) ok = wait_bar(&bars[kBarSFree], (uint32_t)(h - 1) & 1, abort_flag) && ok;
+                ptx::tc_fence_after();
+                if (ok) {
+                    const uint32_t qa = ptx::smem_u32(sm + (b ? L::kQ1 : L::kQ0));
+                    const uint32_t ka = ptx::smem_u32(sm + (b ? L::kK1 : L::kK0));
+#pragma unroll
+                    for (int k = 0; k < D / 16; ++k) {
+                        const uint64_t ad = ptx::smem_desc_sw128(qa + (k >> 2) * 16384 + (k & 3) * 32, 16, 1024);
+                        const uint64_t bd = ptx::smem_desc_sw128(ka + (k >> 2) * L::kKHalf + (k & 3) * 32, 16, 1024);
+                        ptx::mma_bf16(tmem, ad, bd, id_s, k > 0);
+                    }
+                }
+                ptx::mma_commit(&bars[kBarSFull]);
+                if (h + 2 < H) {
+                    if (wait_bar(&bars[kBarSFull], (uint32_t)h & 1, abort_flag)) issue_qk(h + 2);
+                }
+            }
+            // ---- phase 2: U_h = P V_h.  V_h reuses the K buffer of the same parity once
+            // the last S MMA that read it has completed.
+            if (wait_bar(&bars[kBarSFull], (uint32_t)(H - 1) & 1, abort_flag)) {   // every S MMA done
+                for (int b = 0; b < 2 && b < H; ++b) issue_v(b);
+            }
+            bool p_ok = wait_bar(&bars[kBarP], 0, abort_flag);
+            const uint32_t pa = ptx::smem_u32(sm + L::kP);
+            for (int h = 0; h < H; ++h) {
+                const int b = h & 1;
+                const uint32_t n = (uint32_t)(h >> 1);
+                bool ok = wait_bar(&bars[kBarV + b], n & 1, abort_flag) && p_ok;
+                if (h >= 2) ok = wait_bar(&bars[kBarUFree + b], (n - 1) & 1, abort_flag) && ok;
+                ptx::tc_fence_after();
+                if (ok) {
+                    const uint32_t va = ptx::smem_u32(sm + (b ? L::kK1 : L::kK0));
+                    for (int k = 0; k < span / 16; ++k) {
+                        const uint64_t ad = ptx::smem_desc_sw128(pa + (k >> 2) * 16384 + (k & 3) * 32, 16, 1024);
+                        const uint64_t bd = ptx::smem_desc_sw128(va + k * 2048, L::kKHalf, 1024);
+                        ptx::mma_bf16(tmem + b * 256, ad, bd, id_pv, k > 0);
+                    }
+                }
+                ptx::mma_commit(&bars[kBarUFull + b]);
+                if (h + 2 < H) {
+                    if (wait_bar(&bars[kBarUFull + b], n & 1, abort_flag)) issue_v(h + 2);
+                }
+            }
+        }
+        __syncwarp();
+    } else {
+        // ---------------------------------------------------------------- compute warps
+        const int q = warp & 3, split = warp >> 2;
+        const int i = 32 * q + lane;                   // tile row = TMEM lane
+        const int64_t t = t0 + i;
+        const bool valid = (i < BM) && (t < s.N);
+        int clo = 1, chi = 0;                           // valid columns of this row: [clo, chi]
+        if (valid) {
+            clo = (int)(window_lo(s, t) - kbase);
+            chi = (int)(t - kbase);
+        }
+        const Band bd = make_band(q, split, BM, W, span);
+        const uint32_t lane_base = (uint32_t)(32 * q) << 16;
+        const float sl2 = s.scale * kLog2e;
+
+        const uint32_t s_cols = tmem + lane_base;          // S_h, columns [0, span)
+        const uint32_t p_cols = tmem + lane_base + 256;    // P, columns [256, 256 + span)
+
+        for (int h = 0; h < H; ++h) {
+            wait_bar(&bars[kBarSFull], (uint32_t)h & 1, abort_flag);
+            ptx::tc_fence_after();
+            float x[MAXC][8];
+            float mloc = -INFINITY;
+#pragma unroll
+            for (int cc = 0; cc < MAXC; ++cc) {
+                if (cc < bd.mync) {
+                    const int col = bd.cb + (bd.c0 + cc) * 8;
+                    ptx::tmem_ld8(s_cols + col, x[cc]);
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) {
+                        const int cidx = col + e;
+                        float v = x[cc][e] * sl2;
+                        v = (cidx >= clo && cidx <= chi) ? v : -INFINITY;
+                        x[cc][e] = v;
+                        mloc = fmaxf(mloc, v);
+                    }
+                }
+            }
+            ptx::tc_fence_before();
+            ptx::mbar_arrive(&bars[kBarSFree]);
+            red_max[split * 128 + i] = mloc;
+            pair_sync(q);
+            float m = fmaxf(red_max[i], red_max[128 + i]);
+            if (!valid) m = 0.f;
+            float zl = 0.f;
+#pragma unroll
+            for (int cc = 0; cc < MAXC; ++cc) {
+                if (cc < bd.mync) {
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) {
+                        const float ev = ex2(x[cc][e] - m);
+                        x[cc][e] = ev;
+                        zl += ev;
+                    }
+                }
+            }
+            red_sum[split * 128 + i] = zl;
+            pair_sync(q);
+            const float Z = red_sum[i] + red_sum[128 + i];
+            const float coef = valid ? __ldg(a.c + t * H + h) / Z : 0.f;
+#pragma unroll
+            for (int cc = 0; cc < MAXC; ++cc) {
+                if (cc < bd.mync) {
+                    const int col = bd.cb + (bd.c0 + cc) * 8;
+                    float pc[8];
+                    if (h == 0) {
+#pragma unroll
+                        for (int e = 0; e < 8; ++e) pc[e] = coef * x[cc][e];
+                    } else {
+                        ptx::tmem_ld8(p_cols + col, pc);
+#pragma unroll
+                        for (int e = 0; e < 8; ++e) pc[e] = fmaf(coef, x[cc][e], pc[e]);
+                    }
+                    ptx::tmem_st8(p_cols + col, pc);
+                }
+            }
+            if (split == 0 && valid && a.lse) a.lse[t * H + h] = (m + __log2f(Z)) * kLn2;
+        }
+
+        // ---- P tile (bf16, K-major, swizzled) in smem; zero the columns outside the band
+        uint8_t *ptile = sm + L::kP;
+#pragma unroll
+        for (int cc = 0; cc < MAXC; ++cc) {
+            if (cc < bd.mync) {
+                const int col = bd.cb + (bd.c0 + cc) * 8;
+                float pc[8];
+                ptx::tmem_ld8(p_cols + col, pc);
+                uint4 w4;
+                w4.x = pack_bf16x2(pc[0], pc[1]);
+                w4.y = pack_bf16x2(pc[2], pc[3]);
+                w4.z = pack_bf16x2(pc[4], pc[5]);
+                w4.w = pack_bf16x2(pc[6], pc[7]);
+                *(uint4 *)(ptile + sw128_offset(i, col)) = w4;
+            }
+        }
+        ptx::tc_fence_before();
+        {
+            const uint4 z4 = make_uint4(0, 0, 0, 0);
+            const int ce = bd.cb + bd.nch * 8;
+            if (split == 0) {
+                for (int col = 0; col < bd.cb && col < span; col += 8) *(uint4 *)(ptile + sw128_offset(i, col)) = z4;
+            } else {
+                for (int col = (ce > bd.cb ? ce : bd.cb); col < span; col += 8)
+                    *(uint4 *)(ptile + sw128_offset(i, col)) = z4;
+            }
+        }
+        ptx::fence_proxy_async_smem();
+        ptx::mbar_arrive(&bars[kBarP]);
+
+        // ---- band copy of P to pmap[t][w] = P(t, t-W+1+w): tile column i + w of row i
+        if (a.pmap) {
+            compute_sync();
+            for (int r = warp; r < BM; r += kComputeWarps) {
+                const int64_t tr = t0 + r;
+                if (tr >= s.N) break;
+                __nv_bfloat16 *dst = a.pmap + tr * W;
+                for (int w = lane; w < W; w += 32) {
+                    const uint16_t bits = *(const uint16_t *)(ptile + sw128_offset(r, r + w));
+                    reinterpret_cast<uint16_t *>(dst)[w] = bits;
+                }
+            }
+        }
+
+        // ---- epilogue: o_h = g[t,h] * U_h
+        const int cbase = split * (D / 2);
+        for (int h = 0; h < H; ++h) {
+            const int b = h & 1;
+            const uint32_t n = (uint32_t)(h >> 1);
+            wait_bar(&bars[kBarUFull + b], n & 1, abort_flag);
+            ptx::tc_fence_after();
+            const float gh = valid ? __ldg(a.g + t * H + h) : 0.f;
+#pragma unroll
+            for (int c16 = 0; c16 < D / 32; ++c16) {
+                float u[16];
+                ptx::tmem_ld16(tmem + lane_base + b * 256 + cbase + c16 * 16, u);
+                if (valid) {
+                    uint4 w0, w1;
+                    w0.x = pack_bf16x2(gh * u[0], gh * u[1]);
+                    w0.y = pack_bf16x2(gh * u[2], gh * u[3]);
+                    w0.z = pack_bf16x2(gh * u[4], gh * u[5]);
+                    w0.w = pack_bf16x2(gh * u[6], gh * u[7]);
+                    w1.x = pack_bf16x2(gh * u[8], gh * u[9]);
+                    w1.y = pack_bf16x2(gh * u[10], gh * u[11]);
+                    w1.z = pack_bf16x2(gh * u[12], gh * u[13]);
+                    w1.w = pack_bf16x2(gh * u[14], gh * u[15]);
+                    uint4 *dst = (uint4 *)(a.o + (t * H + h) * D + cbase + c16 * 16);
+                    dst[0] = w0;
+                    dst[1] = w1;
+                }
+            }
+            ptx::tc_fence_before();
+            ptx::mbar_arrive(&bars[kBarUFree + b]);
+        }
+    }
+
+    ptx::tc_fence_before();
+    __syncthreads();
+    if (warp == 0) {
+        ptx::tc_fence_after();
+        ptx::tmem_dealloc(tmem, 512);
+    }
+}
+
+}  // namespace tc
+}  // namespace dc

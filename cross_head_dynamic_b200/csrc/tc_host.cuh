@@ -1,24 +1,153 @@
-// tc_host.cuh -- tcgen05/TMA path (host side).  Placeholder until the kernels land.
+// tc_host.cuh -- host side of the tcgen05/TMA path: shape support, block-size
+// choice, TMA descriptors (cuTensorMapEncodeTiled through the runtime's
+// driver entry point, so the library does not link libcuda), launches.
 #pragma once
+
+#include <cuda.h>
+#include <mutex>
+
 #include "common.cuh"
+#include "simt.cuh"
+#include "tc_fwd.cuh"
 
 namespace dc {
 namespace tc {
 
-inline bool supports(const Shape &) { return false; }
+constexpr int kMaxWindow = 129;   // BM = 128 keeps the key tile (BM + W - 1 rows) within 256
 
-inline cudaError_t fwd(const Shape &, const void *, const void *, const void *, const float *, const float *,
-                       void *, float *, void *, cudaStream_t, int32_t *) {
+inline bool supports(const Shape &s) {
+    return (s.d == 64 || s.d == 128) && s.W >= 1 && s.W <= kMaxWindow && s.H >= 1 && s.H <= 16 &&
+           s.N <= (int64_t)INT32_MAX - 512;
+}
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *, const cuuint64_t *,
+                                  const cuuint64_t *, const cuuint32_t *, const cuuint32_t *, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+inline EncodeTiledFn encode_fn() {
+    static EncodeTiledFn fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void *p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = (EncodeTiledFn)p;
+    });
+    return fn;
+}
+
+// 2-D view [N rows][H*d bf16] of a [N][H][d] tensor; boxes of 64 columns x box_rows
+// rows, 128-byte swizzle, zero fill outside the tensor.
+inline cudaError_t make_map(CUtensorMap *m, const void *ptr, int64_t N, int H, int d, int box_rows) {
+    EncodeTiledFn enc = encode_fn();
+    if (!enc) return cudaErrorNotSupported;
+    cuuint64_t dims[2] = {(cuuint64_t)H * d, (cuuint64_t)N};
+    cuuint64_t strides[1] = {(cuuint64_t)H * d * 2};
+    cuuint32_t box[2] = {64, (cuuint32_t)box_rows};
+    cuuint32_t es[2] = {1, 1};
+    CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(ptr), dims, strides, box, es,
+                     CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                     CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
+}
+
+inline int sm_count() {
+    int dev = 0, n = 148;
+    if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+    return n > 0 ? n : 148;
+}
+
+inline int round16(int x) { return (x + 15) & ~15; }
+
+// Query-block size: the candidate (multiple of 16, <= 128, tile span <= 256)
+// minimising waves x per-CTA cost, with the per-CTA cost modelled as the tile
+// span plus a fixed overhead; one CTA per SM.
+inline int choose_block(int64_t N, int W, int sms) {
+    int best = 128;
+    double best_cost = 1e300;
+    for (int bm = 128; bm >= 64; bm -= 16) {
+        if (bm + W - 1 > 256) continue;
+        const int64_t blocks = (N + bm - 1) / bm;
+        const int64_t waves = (blocks + sms - 1) / sms;
+        const double cost = (double)waves * (round16(bm + W - 1) + 96);
+        if (cost < best_cost - 1e-9) {
+            best_cost = cost;
+            best = bm;
+        }
+    }
+    return best;
+}
+
+// register-array width of the softmax warps: chunks of 8 columns per thread
+inline int maxc_for(int W) {
+    const int need = (((31 + W + 7) / 8) + 1) / 2;
+    if (need <= 4) return 4;
+    if (need <= 6) return 6;
+    if (need <= 9) return 9;
+    return 10;
+}
+
+template <typename K>
+inline cudaError_t set_smem(K kernel, uint32_t bytes) {
+    return cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
+}
+
+template <int D, int MAXC>
+inline cudaError_t launch_fwd(const CUtensorMap &mq, const CUtensorMap &mk, const CUtensorMap &mv, const FwdArgs &a,
+                              cudaStream_t st) {
+    auto kern = fwd_kernel<D, MAXC>;
+    cudaError_t e = set_smem(kern, FwdLayout<D>::kAlloc);
+    if (e != cudaSuccess) return e;
+    const unsigned grid = (unsigned)((a.s.N + a.BM - 1) / a.BM);
+    kern<<<grid, kThreads, FwdLayout<D>::kAlloc, st>>>(mq, mk, mv, a);
+    return cudaGetLastError();
+}
+
+template <int D>
+inline cudaError_t launch_fwd_d(int maxc, const CUtensorMap &mq, const CUtensorMap &mk, const CUtensorMap &mv,
+                                const FwdArgs &a, cudaStream_t st) {
+    switch (maxc) {
+        case 4: return launch_fwd<D, 4>(mq, mk, mv, a, st);
+        case 6: return launch_fwd<D, 6>(mq, mk, mv, a, st);
+        case 9: return launch_fwd<D, 9>(mq, mk, mv, a, st);
+        default: return launch_fwd<D, 10>(mq, mk, mv, a, st);
+    }
+}
+
+inline cudaError_t fwd(const Shape &s, const void *q, const void *k, const void *v, const float *c, const float *g,
+                       void *o, float *lse, void *pmap, cudaStream_t st, int32_t *launches) {
+    FwdArgs a;
+    a.s = s;
+    a.BM = choose_block(s.N, s.W, sm_count());
+    a.span = round16(a.BM + s.W - 1);
+    a.c = c;
+    a.g = g;
+    a.o = (__nv_bfloat16 *)o;
+    a.lse = lse;
+    a.pmap = (__nv_bfloat16 *)pmap;
+    CUtensorMap mq, mk, mv;
+    cudaError_t e = make_map(&mq, q, s.N, s.H, s.d, 128);
+    if (e == cudaSuccess) e = make_map(&mk, k, s.N, s.H, s.d, a.span);
+    if (e == cudaSuccess) e = make_map(&mv, v, s.N, s.H, s.d, a.span);
+    if (e != cudaSuccess) return e;
+    const int maxc = maxc_for(s.W);
+    e = (s.d == 64) ? launch_fwd_d<64>(maxc, mq, mk, mv, a, st) : launch_fwd_d<128>(maxc, mq, mk, mv, a, st);
+    if (e == cudaSuccess) ++*launches;
+    return e;
+}
+
+// The tcgen05 backward kernels are not in place yet: the backward entry points
+// serve this path with the SIMT kernels (the pmap/lse formats are shared).
+constexpr bool kHasBwd = false;
+inline cudaError_t bwd_query(const Shape &, const void *, const void *, const void *, const float *, const float *,
+                             const void *, const float *, const void *, void *, float *, float *, float *,
+                             cudaStream_t, int32_t *) {
     return cudaErrorNotSupported;
 }
-inline cudaError_t bwd_query(const Shape &, const void *, const void *, const void *, const float *,
-                             const float *, const void *, const float *, const void *, void *, float *,
-                             float *, float *, cudaStream_t, int32_t *) {
-    return cudaErrorNotSupported;
-}
-inline cudaError_t bwd_key(const Shape &, const void *, const void *, const float *, const float *,
-                           const void *, const float *, const void *, const float *, const float *, void *,
-                           void *, cudaStream_t, int32_t *) {
+inline cudaError_t bwd_key(const Shape &, const void *, const void *, const float *, const float *, const void *,
+                           const float *, const void *, const float *, const float *, void *, void *, cudaStream_t,
+                           int32_t *) {
     return cudaErrorNotSupported;
 }
 
