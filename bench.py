@@ -1,0 +1,396 @@
+#!/usr/bin/env python
+"""Benchmark of libdcattn: Lightweight DC attention forward + backward on B200.
+
+One step = dc_attn_fwd + dc_attn_bwd_query + dc_attn_bwd_key over one batch of
+the GPT-2-small attention shape (B8 x T2048, H6 x d128, W112, one document per
+row, bf16, seeded synthetic inputs).  Prints one JSON line (rank 0).
+
+  python bench.py [--gpus N --steps K --warmup W]      # libdcattn
+  python bench.py --impl reference ...                 # the fp64 CPU oracle
+
+Multi-GPU runs are replicas (the path has no cross-GPU exchange): every rank
+runs the same workload on its own GPU; value = all tokens / max-over-ranks time.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from cross_head_dynamic_b200.inputs import CONFIGS, generate  # noqa: E402
+
+METRIC = "DC-attn fwd+bwd tokens/sec and % of roofline on 1 B200 (B8×T2048×H6×d128, W112)"
+UNIT = "tokens/s"
+WORKLOAD = "gpt2_fwdbwd"
+N_SETS = 4                                   # rotating input/output sets, each larger than L2
+PEAKS_FILE = os.path.join(ROOT, "MEASURED_PEAKS.json")
+TRAFFIC_FILE = os.path.join(ROOT, "profiles", "dram_traffic.txt")
+KERNEL_SOURCES = {
+    "fwd": ["cross_head_dynamic_b200/csrc/tc_fwd.cuh", "cross_head_dynamic_b200/csrc/tc_common.cuh"],
+    "bwd_query": ["cross_head_dynamic_b200/csrc/tc_bwd.cuh", "cross_head_dynamic_b200/csrc/tc_common.cuh"],
+    "bwd_key": ["cross_head_dynamic_b200/csrc/tc_bwd.cuh", "cross_head_dynamic_b200/csrc/tc_common.cuh"],
+}
+
+
+def algorithmic_bytes_per_token(H: int, d: int, e: int = 2) -> dict:
+    """Minimal HBM bytes per token each kernel must move (no LSE, pmap or dP band):
+    fwd reads q,k,v,c,g and writes o; bwd_query reads q,k,v,dO,c,g and writes
+    dq,dc,dg; bwd_key reads q,k,dO,c,g,dc and writes dk,dv.  The whole step's
+    minimum counts every tensor once: 11*H*d*e + 24*H."""
+    return {
+        "fwd": 4 * H * d * e + 8 * H,
+        "bwd_query": 5 * H * d * e + 16 * H,
+        "bwd_key": 5 * H * d * e + 12 * H,
+        "step": 11 * H * d * e + 24 * H,
+    }
+
+
+def source_hash(paths) -> str:
+    h = hashlib.sha1()
+    for p in paths:
+        with open(os.path.join(ROOT, p), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:12]
+
+
+def measured_traffic(kernel: str, tokens: int):
+    """dram bytes per launch from the committed ncu summary, scaled to `tokens`,
+    or None when absent or taken on a different version of the kernel source."""
+    if not os.path.exists(TRAFFIC_FILE):
+        return None
+    want = source_hash(KERNEL_SOURCES[kernel])
+    for line in open(TRAFFIC_FILE):
+        parts = line.split()
+        if len(parts) >= 4 and not line.startswith("#") and parts[0] == kernel:
+            bytes_per_launch, src, cap_tokens = float(parts[1]), parts[2], int(parts[3])
+            if src != want:
+                return None
+            return bytes_per_launch * tokens / cap_tokens
+    return None
+
+
+class ClockSampler:
+    """nvidia-smi sampling of SM clocks and throttle reasons while the GPU works."""
+
+    QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_index: int):
+        self.samples = []
+        self.proc = None
+        self.dev = device_index
+        self._thread = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.dev}", f"--query-gpu={self.QUERY}", "--format=csv,noheader,nounits",
+                 "-lms", "100"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except (OSError, ValueError):
+            self.proc = None
+            return
+        self._thread = threading.Thread(target=self._read, daemon=True)
+        self._thread.start()
+
+    def _read(self):
+        for line in self.proc.stdout:
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) >= 9:
+                self.samples.append((time.time(), parts))
+
+    def stop(self):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+        if self._thread is not None:
+            self._thread.join(timeout=2)
+
+    def summary(self, t0: float, t1: float):
+        win = [p for (ts, p) in self.samples if t0 <= ts <= t1]
+        if not win:
+            return None
+        def num(x):
+            try:
+                return float(x)
+            except ValueError:
+                return None
+        sm = [num(p[1]) for p in win if num(p[1]) is not None]
+        mx = [num(p[2]) for p in win if num(p[2]) is not None]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[k] for p in win for k in range(4) if p[5 + k].lower().startswith("active")})
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(mx) if mx else None,
+                "reasons": reasons, "samples": len(win)}
+
+
+def dist_setup(n_gpus: int):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    return world, rank, local
+
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def allreduce_max(x: float, world: int) -> float:
+    if world == 1:
+        return x
+    import torch.distributed as dist
+    t = torch.tensor([x], device="cuda", dtype=torch.float64)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def oracle_sample_rate(cfg, rows: int, reps: int = 1):
+    """fp64 oracle fwd+bwd on the first `rows` batch rows; tokens/s on host cores."""
+    import oracle
+    oracle.build()
+    sub = cfg.replace(batch=rows)
+    x = generate(sub)
+    t = time.perf_counter()
+    for _ in range(reps):
+        oracle.forward(x["q"], x["k"], x["v"], x["c"], x["g"], x["cu_seqlens"], x["window"], x["scale"])
+        oracle.backward(x["q"], x["k"], x["v"], x["c"], x["g"], x["dO"], x["cu_seqlens"], x["window"], x["scale"])
+    dt = time.perf_counter() - t
+    return rows * cfg.seqlen * reps / dt, oracle.num_threads(), dt
+
+
+def config_block(cfg, n_gpus):
+    return {"workload": f"{WORKLOAD}: B{cfg.batch} x T{cfg.seqlen}, H{cfg.heads} x d{cfg.head_dim}, "
+                        f"W{cfg.window}, one document per row, bf16 q/k/v/dO, fp32 c/g",
+            "tokens_per_gpu": cfg.total_tokens, "global_batch": cfg.batch * n_gpus, "seq_len": cfg.seqlen,
+            "heads": cfg.heads, "head_dim": cfg.head_dim, "window": cfg.window,
+            "parallelism": f"replicas x{n_gpus}",
+            "l2": f"{N_SETS} rotating input/output sets of ~190 MB each (> 126 MB L2)"}
+
+
+def run_reference(args):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return 0
+    cfg = CONFIGS[WORKLOAD]
+    rows = 1
+    for _ in range(args.warmup):
+        oracle_sample_rate(cfg, rows)
+    rates, cores = [], 1
+    t_all = 0.0
+    for _ in range(args.steps):
+        r, cores, dt = oracle_sample_rate(cfg, rows)
+        rates.append(r)
+        t_all += dt
+    value = args.steps * rows * cfg.seqlen / t_all
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * t_all / args.steps,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic", "config": config_block(cfg, 1),
+            "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle",
+                             "sample": f"fwd+bwd of {rows} row x {cfg.seqlen} tokens of the workload per step"},
+            "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--impl", choices=["dcattn", "reference"], default="dcattn")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        args.warmup = 3
+    if args.impl == "reference":
+        return run_reference(args)
+
+    from cross_head_dynamic_b200 import build, dcattn
+    world, rank, local = dist_setup(args.gpus)
+    if world == 1:
+        torch.cuda.set_device(0)
+    build.build()
+    dcattn.load_library()
+    dev = torch.device("cuda", torch.cuda.current_device())
+    cfg = CONFIGS[WORKLOAD]
+    host = generate(cfg)
+    N, H, d, W, scale = cfg.total_tokens, cfg.heads, cfg.head_dim, cfg.window, cfg.softmax_scale
+    impl = dcattn.dc_attn_resolve_impl(host["q"].to(dev), host["cu_seqlens"].to(dev), W, scale)
+
+    # rotating sets of device-resident inputs and outputs
+    sets = []
+    for _ in range(N_SETS):
+        x = {k: (v.to(dev) if isinstance(v, torch.Tensor) else v) for k, v in host.items()}
+        x["o"] = torch.empty_like(x["q"])
+        x["lse"] = torch.empty(N, H, device=dev)
+        x["pmap"] = torch.empty(N, W, device=dev, dtype=torch.bfloat16)
+        x["dq"], x["dk"], x["dv"] = (torch.empty_like(x["q"]) for _ in range(3))
+        x["dc"], x["dg"] = torch.empty(N, H, device=dev), torch.empty(N, H, device=dev)
+        x["ws"] = torch.empty(dcattn.dc_attn_bwd_workspace_size(x["q"], x["cu_seqlens"], W, scale),
+                              device=dev, dtype=torch.uint8)
+        sets.append(x)
+    stream = torch.cuda.current_stream()
+    launches = [0]
+
+    def step(x, ev=None):
+        if ev is not None:
+            ev[0].record(stream)
+        dcattn.dc_attn_fwd(x["q"], x["k"], x["v"], x["c"], x["g"], x["cu_seqlens"], W, scale,
+                           o=x["o"], lse=x["lse"], pmap=x["pmap"])
+        launches[0] += dcattn.dc_attn_last_launch_count()
+        if ev is not None:
+            ev[1].record(stream)
+        dcattn.dc_attn_bwd_query(x["q"], x["k"], x["v"], x["c"], x["g"], x["dO"], x["lse"], x["pmap"],
+                                 x["cu_seqlens"], W, scale, dq=x["dq"], dc=x["dc"], dg=x["dg"], workspace=x["ws"])
+        launches[0] += dcattn.dc_attn_last_launch_count()
+        if ev is not None:
+            ev[2].record(stream)
+        dcattn.dc_attn_bwd_key(x["q"], x["k"], x["c"], x["g"], x["dO"], x["lse"], x["pmap"], x["dc"], x["ws"],
+                               x["cu_seqlens"], W, scale, dk=x["dk"], dv=x["dv"])
+        launches[0] += dcattn.dc_attn_last_launch_count()
+        if ev is not None:
+            ev[3].record(stream)
+
+    sampler = ClockSampler(local)
+    sampler.start()
+    time.sleep(0.3)
+    for it in range(args.warmup):
+        step(sets[it % N_SETS])
+    torch.cuda.synchronize()
+    if dcattn.dc_attn_device_status() != 0:
+        raise RuntimeError("device status word reports an error after warm-up")
+
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
+    barrier(world)
+    torch.cuda.synchronize()
+    launches[0] = 0
+    t_wall0 = time.time()
+    for it in range(args.steps):
+        step(sets[it % N_SETS], evs[it])
+    torch.cuda.synchronize()
+    t_wall1 = time.time()
+    barrier(world)
+    total_ms = evs[0][0].elapsed_time(evs[-1][3])
+    per_kernel = {"fwd": 0.0, "bwd_query": 0.0, "bwd_key": 0.0}
+    for ev in evs:
+        per_kernel["fwd"] += ev[0].elapsed_time(ev[1])
+        per_kernel["bwd_query"] += ev[1].elapsed_time(ev[2])
+        per_kernel["bwd_key"] += ev[2].elapsed_time(ev[3])
+    per_kernel = {k: v / args.steps for k, v in per_kernel.items()}   # ms per launch
+    gpu_launches = launches[0]
+    total_ms = allreduce_max(total_ms, world)
+    ms_step = total_ms / args.steps
+    value = world * N / (ms_step * 1e-3)
+
+    clocks = sampler.summary(t_wall0, t_wall1)
+    clock_note = "sampled during the timed region"
+    if clocks is None or clocks.get("samples", 0) < 3:
+        # the timed region was too short for the sampler: keep the same step running
+        # (untimed) for about a second and sample that
+        t2 = time.time()
+        it = 0
+        while time.time() - t2 < 1.2:
+            step(sets[it % N_SETS])
+            it += 1
+            if it % 50 == 0:
+                torch.cuda.synchronize()
+        torch.cuda.synchronize()
+        clocks = sampler.summary(t2, time.time())
+        clock_note = "sampled over ~1 s of the same step right after the timed region"
+    sampler.stop()
+
+    # end to end through the public API: pinned host inputs -> device -> fwd+bwd -> host results
+    e2e = None
+    pin = {k: host[k].pin_memory() for k in ("q", "k", "v", "c", "g", "dO", "cu_seqlens")}
+    outs_host = {k: torch.empty(sets[0][k].shape, dtype=sets[0][k].dtype).pin_memory()
+                 for k in ("o", "dq", "dk", "dv", "dc", "dg")}
+    h2d = sum(t.numel() * t.element_size() for t in pin.values())
+    d2h = sum(t.numel() * t.element_size() for t in outs_host.values())
+    e2e_steps = max(3, min(args.steps, 20))
+    for rep in range(2):
+        if rep == 1:
+            barrier(world)
+            torch.cuda.synchronize()
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+        for it in range(e2e_steps if rep == 1 else 3):
+            x = sets[it % N_SETS]
+            for k2 in pin:
+                x[k2].copy_(pin[k2], non_blocking=True)
+            step(x)
+            for k2 in outs_host:
+                outs_host[k2].copy_(x[k2], non_blocking=True)
+        if rep == 1:
+            e1.record(stream)
+        torch.cuda.synchronize()
+    e2e_ms = allreduce_max(e0.elapsed_time(e1) / e2e_steps, world)
+    e2e = {"value": world * N / (e2e_ms * 1e-3), "unit": UNIT, "h2d_bytes_per_step": h2d,
+           "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms}
+
+    # roofline of the dominant kernel (HBM-bound path) against the measured copy bandwidth
+    peaks = json.load(open(PEAKS_FILE)) if os.path.exists(PEAKS_FILE) else {}
+    hbm = peaks.get("hbm_gbs")
+    peak_note = "of measured" if hbm else "of fallback"
+    hbm = hbm or 6650.0
+    abytes = algorithmic_bytes_per_token(H, d)
+    dom = max(per_kernel, key=per_kernel.get)
+    achieved = abytes[dom] * N / (per_kernel[dom] * 1e-3) / 1e9
+    traffic = measured_traffic(dom, N)
+    step_gbs = abytes["step"] * N / (ms_step * 1e-3) / 1e9
+
+    cpu = None
+    if rank == 0 and not args.no_cpu_baseline:
+        rate, cores, dt = oracle_sample_rate(cfg, rows=cfg.batch)
+        cpu = {"value": rate, "unit": UNIT, "cores": cores, "kind": "oracle",
+               "sample": f"one fwd+bwd of all {cfg.total_tokens} tokens of the workload in fp64 ({dt:.1f} s)"}
+
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "bf16", "data": "synthetic", "impl": "dcattn", "kernels": impl,
+            "config": config_block(cfg, world),
+            "roofline": {"bound": "hbm", "kernel": dom, "achieved": achieved, "peak": hbm, "unit": "GB/s",
+                         "frac": achieved / hbm, "peak_source": peak_note, "traffic": traffic,
+                         "algorithmic_bytes_per_launch": abytes[dom] * N},
+            "step_roofline": {"achieved": step_gbs, "peak": hbm, "unit": "GB/s", "frac": step_gbs / hbm,
+                              "algorithmic_bytes_per_step": abytes["step"] * N,
+                              "roofline_tokens_per_s": hbm * 1e9 / abytes["step"]},
+            "kernel_ms": per_kernel,
+            "cpu_baseline": cpu,
+            "e2e": e2e,
+            "gpu_launches": gpu_launches,
+            "clocks": dict(clocks or {}, note=clock_note),
+        }
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

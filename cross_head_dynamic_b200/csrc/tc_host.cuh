@@ -9,6 +9,7 @@
 #include "common.cuh"
 #include "simt.cuh"
 #include "tc_fwd.cuh"
+#include "tc_bwd.cuh"
 
 namespace dc {
 namespace tc {
@@ -63,11 +64,11 @@ inline int round16(int x) { return (x + 15) & ~15; }
 // Query-block size: the candidate (multiple of 16, <= 128, tile span <= 256)
 // minimising waves x per-CTA cost, with the per-CTA cost modelled as the tile
 // span plus a fixed overhead; one CTA per SM.
-inline int choose_block(int64_t N, int W, int sms) {
-    int best = 128;
+inline int choose_block(int64_t N, int W, int sms, int max_span = 256) {
+    int best = 64;
     double best_cost = 1e300;
     for (int bm = 128; bm >= 64; bm -= 16) {
-        if (bm + W - 1 > 256) continue;
+        if (round16(bm + W - 1) > max_span) continue;
         const int64_t blocks = (N + bm - 1) / bm;
         const int64_t waves = (blocks + sms - 1) / sms;
         const double cost = (double)waves * (round16(bm + W - 1) + 96);
@@ -137,18 +138,101 @@ inline cudaError_t fwd(const Shape &s, const void *q, const void *k, const void 
     return e;
 }
 
-// The tcgen05 backward kernels are not in place yet: the backward entry points
-// serve this path with the SIMT kernels (the pmap/lse formats are shared).
-constexpr bool kHasBwd = false;
-inline cudaError_t bwd_query(const Shape &, const void *, const void *, const void *, const float *, const float *,
-                             const void *, const float *, const void *, void *, float *, float *, float *,
-                             cudaStream_t, int32_t *) {
-    return cudaErrorNotSupported;
+constexpr bool kHasBwd = true;
+
+template <int D, int MAXC>
+inline cudaError_t launch_bwd_query(const CUtensorMap &mq, const CUtensorMap &mk, const CUtensorMap &mv,
+                                    const CUtensorMap &mdo, const BwdArgs &a, cudaStream_t st) {
+    auto kern = bwd_query_kernel<D, MAXC>;
+    const uint32_t smem = QSideLayout<D>(a.span).bytes + 1024;
+    cudaError_t e = set_smem(kern, smem);
+    if (e != cudaSuccess) return e;
+    const unsigned grid = (unsigned)((a.s.N + a.BM - 1) / a.BM);
+    kern<<<grid, kThreads, smem, st>>>(mq, mk, mv, mdo, a);
+    return cudaGetLastError();
 }
-inline cudaError_t bwd_key(const Shape &, const void *, const void *, const float *, const float *, const void *,
-                           const float *, const void *, const float *, const float *, void *, void *, cudaStream_t,
-                           int32_t *) {
-    return cudaErrorNotSupported;
+
+template <int D, int MAXC>
+inline cudaError_t launch_bwd_key(const CUtensorMap &mq, const CUtensorMap &mk, const CUtensorMap &mdo,
+                                  const BwdArgs &a, cudaStream_t st) {
+    auto kern = bwd_key_kernel<D, MAXC>;
+    const uint32_t smem = KSideLayout<D>(a.span).bytes + 1024;
+    cudaError_t e = set_smem(kern, smem);
+    if (e != cudaSuccess) return e;
+    const unsigned grid = (unsigned)((a.s.N + a.BM - 1) / a.BM);
+    kern<<<grid, kThreads, smem, st>>>(mq, mk, mdo, a);
+    return cudaGetLastError();
+}
+
+#define DC_TC_MAXC_SWITCH(maxc, CALL)        \
+    switch (maxc) {                          \
+        case 4: { constexpr int MC = 4; return CALL; }   \
+        case 6: { constexpr int MC = 6; return CALL; }   \
+        case 9: { constexpr int MC = 9; return CALL; }   \
+        default: { constexpr int MC = 10; return CALL; } \
+    }
+
+inline BwdArgs bwd_args(const Shape &s) {
+    BwdArgs a = {};
+    a.s = s;
+    a.BM = choose_block(s.N, s.W, sm_count(), kBwdMaxSpan);
+    a.span = round16(a.BM + s.W - 1);
+    return a;
+}
+
+inline cudaError_t bwd_query(const Shape &s, const void *q, const void *k, const void *v, const float *c,
+                             const float *g, const void *dO, const float *lse, const void *pmap, void *dq, float *dc_,
+                             float *dg, float *band, cudaStream_t st, int32_t *launches) {
+    BwdArgs a = bwd_args(s);
+    a.c = c;
+    a.g = g;
+    a.lse = lse;
+    a.pmap = (const __nv_bfloat16 *)pmap;
+    a.dq = (__nv_bfloat16 *)dq;
+    a.dc = dc_;
+    a.dg = dg;
+    a.band = band;
+    CUtensorMap mq, mk, mv, mdo;
+    cudaError_t e = make_map(&mq, q, s.N, s.H, s.d, 128);
+    if (e == cudaSuccess) e = make_map(&mk, k, s.N, s.H, s.d, a.span);
+    if (e == cudaSuccess) e = make_map(&mv, v, s.N, s.H, s.d, a.span);
+    if (e == cudaSuccess) e = make_map(&mdo, dO, s.N, s.H, s.d, 128);
+    if (e != cudaSuccess) return e;
+    e = [&]() -> cudaError_t {
+        if (s.d == 64) {
+            DC_TC_MAXC_SWITCH(maxc_for(s.W), (launch_bwd_query<64, MC>(mq, mk, mv, mdo, a, st)));
+        }
+        DC_TC_MAXC_SWITCH(maxc_for(s.W), (launch_bwd_query<128, MC>(mq, mk, mv, mdo, a, st)));
+    }();
+    if (e == cudaSuccess) ++*launches;
+    return e;
+}
+
+inline cudaError_t bwd_key(const Shape &s, const void *q, const void *k, const float *c, const float *g,
+                           const void *dO, const float *lse, const void *pmap, const float *dc_, const float *band,
+                           void *dk, void *dv, cudaStream_t st, int32_t *launches) {
+    BwdArgs a = bwd_args(s);
+    a.c = c;
+    a.g = g;
+    a.lse = lse;
+    a.pmap = (const __nv_bfloat16 *)pmap;
+    a.dc_in = dc_;
+    a.band = const_cast<float *>(band);
+    a.dk = (__nv_bfloat16 *)dk;
+    a.dv = (__nv_bfloat16 *)dv;
+    CUtensorMap mq, mk, mdo;
+    cudaError_t e = make_map(&mq, q, s.N, s.H, s.d, a.span);
+    if (e == cudaSuccess) e = make_map(&mk, k, s.N, s.H, s.d, 128);
+    if (e == cudaSuccess) e = make_map(&mdo, dO, s.N, s.H, s.d, a.span);
+    if (e != cudaSuccess) return e;
+    e = [&]() -> cudaError_t {
+        if (s.d == 64) {
+            DC_TC_MAXC_SWITCH(maxc_for(s.W), (launch_bwd_key<64, MC>(mq, mk, mdo, a, st)));
+        }
+        DC_TC_MAXC_SWITCH(maxc_for(s.W), (launch_bwd_key<128, MC>(mq, mk, mdo, a, st)));
+    }();
+    if (e == cudaSuccess) ++*launches;
+    return e;
 }
 
 }  // namespace tc
