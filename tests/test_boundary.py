@@ -30,7 +30,7 @@ def declared_functions():
 def test_header_declares_expected_api():
     names = declared_functions()
     assert set(dcattn.EXPORTED) <= set(names), names
-    assert set(names) <= set(dcattn.EXPORTED) | {"dc_attn_fwd_noalloc"}, names
+    assert set(names) <= set(dcattn.EXPORTED), names
 
 
 def test_library_exports_every_declared_symbol(lib):
