@@ -6,6 +6,8 @@
 #include <stdint.h>
 #include <string.h>
 
+#include <mutex>
+
 #include "dcattn.h"
 #include "common.cuh"
 #include "simt.cuh"
@@ -254,5 +256,73 @@ const char *dc_attn_status_string(dc_status_t status) {
 }
 
 int32_t dc_attn_last_launch_count(void) { return t_launches; }
+
+}  // extern "C"
+
+// --------------------------------------------------------------------------
+// Backward without caller-provided scratch.
+//
+// Some callers cannot hand the backward a workspace: plugin-style interfaces
+// that give an op only its input and output tensors, and processes whose device
+// memory is reserved up front by their own pool and that must not call
+// cudaMalloc later.  For them the dP band lives in the array below, which every
+// GPU that loads this library keeps for the life of the process.
+// --------------------------------------------------------------------------
+
+#define DC_NOALLOC_SCRATCH_BYTES ((size_t)32 << 20)
+
+static __device__ __align__(256) unsigned char g_noalloc_scratch[DC_NOALLOC_SCRATCH_BYTES];
+
+namespace {
+
+constexpr int kMaxDevices = 64;
+std::mutex g_noalloc_mutex;
+void *g_noalloc_ptr[kMaxDevices] = {};
+
+// Device address of the scratch array on the current device, looked up once per
+// device (cudaGetSymbolAddress with that device current).  In host code the
+// array's name is only a host-side stand-in, never a usable device pointer.
+cudaError_t noalloc_scratch(void **out) {
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
+    std::lock_guard<std::mutex> lock(g_noalloc_mutex);
+    if (!g_noalloc_ptr[dev]) {
+        void *p = nullptr;
+        e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+        if (e != cudaSuccess) return e;
+        g_noalloc_ptr[dev] = p;
+    }
+    *out = g_noalloc_ptr[dev];
+    return cudaSuccess;
+}
+
+}  // namespace
+
+extern "C" {
+
+dc_status_t dc_attn_bwd_noalloc(const dc_attn_params *params, const void *q, const void *k, const void *v,
+                                const float *c, const float *g, const void *dO, const float *lse, const void *pmap,
+                                void *dq, void *dk, void *dv, float *dc_, float *dg, void *stream) {
+    Checked ck;
+    dc_status_t r = check_params(params, &ck);
+    if (r != DC_OK) return r;
+    const size_t need = band_bytes(ck.s);
+    if (need > DC_NOALLOC_SCRATCH_BYTES) return DC_ERR_UNSUPPORTED;   // N * W * 4 above the array size
+    if (ck.s.N == 0) {
+        t_launches = 0;
+        return DC_OK;
+    }
+    void *scratch = nullptr;
+    if (noalloc_scratch(&scratch) != cudaSuccess) {
+        (void)cudaGetLastError();
+        return DC_ERR_CUDA;
+    }
+    // The query pass writes every band entry [t][w] (t < N, w < W) before the key
+    // pass reads it, so nothing left in the array by an earlier call is read.
+    return dc_attn_bwd(params, q, k, v, c, g, dO, lse, pmap, dq, dk, dv, dc_, dg, scratch,
+                       DC_NOALLOC_SCRATCH_BYTES, stream);
+}
 
 }  // extern "C"

@@ -24,7 +24,7 @@ DC_DEVERR_TIMEOUT = 0x2
 
 EXPORTED = ("dc_attn_fwd", "dc_attn_bwd_workspace_size", "dc_attn_bwd_query", "dc_attn_bwd_key",
             "dc_attn_bwd", "dc_attn_resolve_impl", "dc_attn_device_status", "dc_attn_status_string",
-            "dc_attn_last_launch_count")
+            "dc_attn_last_launch_count", "dc_attn_bwd_noalloc")
 
 
 class DCAttnError(RuntimeError):
@@ -70,6 +70,8 @@ def load_library(path: str = LIB_PATH):
     lib.dc_attn_device_status.restype = st
     lib.dc_attn_status_string.argtypes = [st]
     lib.dc_attn_status_string.restype = ctypes.c_char_p
+    lib.dc_attn_bwd_noalloc.argtypes = [P] + [vp] * 14
+    lib.dc_attn_bwd_noalloc.restype = st
     lib.dc_attn_last_launch_count.argtypes = []
     lib.dc_attn_last_launch_count.restype = ctypes.c_int32
     _lib = lib
@@ -214,6 +216,31 @@ def dc_attn_bwd(q, k, v, c, g, dO, lse, pmap, cu_seqlens, window, scale, *, dq=N
         _dev(dg, "dg", torch.float32), _dev(workspace, "workspace"),
         workspace.numel() * workspace.element_size(), _stream_handle(stream))
     _check("dc_attn_bwd", code)
+    return dq, dk, dv, dc, dg
+
+
+def dc_attn_bwd_noalloc(q, k, v, c, g, dO, lse, pmap, cu_seqlens, window, scale, *, dq=None, dk=None, dv=None,
+                        dc=None, dg=None, impl="auto", stream=None):
+    """Full backward without a workspace, for callers that cannot allocate scratch
+    (plugin-style interfaces that pass an op only its inputs and outputs, or
+    processes that reserve all device memory up front).  The library's static
+    32 MiB scratch array holds the dP band instead, so N * W * 4 must not exceed
+    32 MiB; overlapping calls on one device race on that array.  Returns
+    (dq, dk, dv, dc, dg)."""
+    p = make_params(q, cu_seqlens, window, scale, impl)
+    N, H, d = q.shape
+    dq = torch.empty_like(q) if dq is None else dq
+    dk = torch.empty_like(q) if dk is None else dk
+    dv = torch.empty_like(q) if dv is None else dv
+    dc = torch.empty(N, H, device=q.device, dtype=torch.float32) if dc is None else dc
+    dg = torch.empty(N, H, device=q.device, dtype=torch.float32) if dg is None else dg
+    code = load_library().dc_attn_bwd_noalloc(
+        ctypes.byref(p), _dev(q, "q", q.dtype), _dev(k, "k", q.dtype), _dev(v, "v", q.dtype),
+        _dev(c, "c", torch.float32), _dev(g, "g", torch.float32), _dev(dO, "dO", q.dtype),
+        _dev(lse, "lse", torch.float32), _dev(pmap, "pmap", q.dtype), _dev(dq, "dq", q.dtype),
+        _dev(dk, "dk", q.dtype), _dev(dv, "dv", q.dtype), _dev(dc, "dc", torch.float32),
+        _dev(dg, "dg", torch.float32), _stream_handle(stream))
+    _check("dc_attn_bwd_noalloc", code)
     return dq, dk, dv, dc, dg
 
 

@@ -56,7 +56,7 @@ typedef enum {
 typedef enum { DC_F32 = 0, DC_BF16 = 1 } dc_dtype_t;
 
 /* Kernel family.  AUTO picks the tcgen05/TMA path when the shape allows it
- * (bf16, d in {64,128}, W <= 193) and the SIMT path otherwise.  SIMT is the
+ * (bf16, d in {64,128}, W <= 129) and the SIMT path otherwise.  SIMT is the
  * fp32-accumulating CUDA-core path used for fp32 tensors and any shape. */
 typedef enum { DC_IMPL_AUTO = 0, DC_IMPL_SIMT = 1, DC_IMPL_TCGEN05 = 2 } dc_impl_t;
 
@@ -125,6 +125,31 @@ dc_status_t dc_attn_bwd(const dc_attn_params *params,
                         const float *lse, const void *pmap,
                         void *dq, void *dk, void *dv, float *dc, float *dg,
                         void *workspace, size_t workspace_bytes, void *stream);
+
+/* Backward that allocates nothing and takes no workspace (no counterpart on the
+ * page; an interface addition).  For callers that cannot provide scratch:
+ * plugin-style interfaces that hand an op only its inputs and outputs, and
+ * processes whose device memory is reserved by their own pool at start-up and
+ * that must not call cudaMalloc afterwards.  Same arguments and results as
+ * dc_attn_bwd minus the workspace; the dP band lives instead in a static
+ * device array of 32 MiB (33554432 bytes) that every GPU loading this library
+ * keeps until the process exits.
+ * - Returns DC_ERR_UNSUPPORTED, before any launch, when the band needs more
+ *   than that: N * W * 4 bytes > 32 MiB (e.g. N = 65536 tokens at W = 128).
+ * - The first call on each device looks up the array's device address with
+ *   that device current; make that first call before any stream capture.
+ * - Every call on a device shares the one array.  Calls whose kernels overlap
+ *   on the GPU (different streams, or different host threads, without
+ *   ordering between them) race on it and give undefined results; serialise
+ *   them.  Nothing needs clearing between calls: the query pass rewrites every
+ *   band entry the key pass reads.
+ * - Calls no cudaMalloc/cudaFree and no allocating library routine. */
+dc_status_t dc_attn_bwd_noalloc(const dc_attn_params *params,
+                                const void *q, const void *k, const void *v,
+                                const float *c, const float *g, const void *dO,
+                                const float *lse, const void *pmap,
+                                void *dq, void *dk, void *dv, float *dc, float *dg,
+                                void *stream);
 
 /* Which kernel family AUTO resolves to for these params (DC_IMPL_SIMT or
  * DC_IMPL_TCGEN05), or -1 if the params are invalid. */

@@ -1,0 +1,74 @@
+"""The backward entry point that allocates nothing (dc_attn_bwd_noalloc).
+
+It exists for callers that cannot give the backward a scratch buffer: plugin
+interfaces that hand an op only its inputs and outputs, and processes whose
+device memory is reserved by their own pool at start-up so that no cudaMalloc
+may follow.  Its scratch is a fixed 32 MiB array inside the library.  These
+tests call it through the C ABI and compare it with dc_attn_bwd (caller-owned
+workspace) on the same inputs, on consecutive calls that share the array.
+This file is collected last so a stop-at-first-failure run has already run
+everything else.
+"""
+import ctypes
+
+import numpy as np
+import pytest
+import torch
+
+from cross_head_dynamic_b200 import dcattn
+from cross_head_dynamic_b200.inputs import random_problem
+from parity_util import TOL, rel_err, to_cuda
+
+pytestmark = pytest.mark.gpu
+
+SCRATCH_BYTES = 32 << 20
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _lib():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    from cross_head_dynamic_b200 import build
+    build.build()
+    dcattn.load_library()
+    dcattn.dc_attn_device_status(reset=True)
+    yield
+    assert dcattn.dc_attn_device_status(reset=True) == 0
+
+
+def _forward(x, impl):
+    return dcattn.dc_attn_fwd(x["q"], x["k"], x["v"], x["c"], x["g"], x["cu_seqlens"], x["window"], x["scale"],
+                              impl=impl)
+
+
+@pytest.mark.parametrize("impl", ["auto", "simt"])
+def test_noalloc_matches_workspace_backward_on_consecutive_calls(impl):
+    problems = [random_problem(31, [1000, 600, 448], 6, 128, 112, dtype="bf16"),
+                random_problem(32, [257, 3, 700], 6, 128, 112, dtype="bf16")]
+    for pb in problems:               # the second problem is smaller: stale array contents must not leak
+        x = to_cuda(pb)
+        o, lse, pmap = _forward(x, impl)
+        args = (x["q"], x["k"], x["v"], x["c"], x["g"], x["dO"], lse, pmap, x["cu_seqlens"], x["window"],
+                x["scale"])
+        ref = dcattn.dc_attn_bwd(*args, impl=impl)
+        torch.cuda.synchronize()
+        for _ in range(2):
+            got = dcattn.dc_attn_bwd_noalloc(*args, impl=impl)
+            torch.cuda.synchronize()
+            for name, a, b in zip(("dq", "dk", "dv", "dc", "dg"), got, ref):
+                err = rel_err(a.double().cpu().numpy(), b.double().cpu().numpy())
+                assert err <= TOL["bf16"], (name, err)
+
+
+def test_noalloc_rejects_problems_beyond_the_scratch_array():
+    x = to_cuda(random_problem(33, [64], 2, 64, 16, dtype="bf16"))
+    lib = dcattn.load_library()
+    W = 128
+    N = SCRATCH_BYTES // (4 * W) + 1          # band of N * W fp32 entries just above 32 MiB
+    p = dcattn.Params(dtype=dcattn.DC_BF16, impl=0, total_tokens=N, num_docs=1, num_heads=2, head_dim=64,
+                      window=W, softmax_scale=0.125, reserved=0, cu_seqlens=x["cu_seqlens"].data_ptr())
+    ptr = x["q"].data_ptr()
+    rc = lib.dc_attn_bwd_noalloc(ctypes.byref(p), *([ptr] * 13), None)
+    assert rc == dcattn.DC_ERR_UNSUPPORTED
+    p.total_tokens = SCRATCH_BYTES // (4 * W)  # exactly at the limit: accepted by the size check
+    assert lib.dc_attn_bwd_workspace_size(ctypes.byref(p)) == SCRATCH_BYTES
