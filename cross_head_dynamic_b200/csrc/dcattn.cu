@@ -179,7 +179,7 @@ dc_status_t dc_attn_bwd_query(const dc_attn_params *params, const void *q, const
     if (workspace_bytes < band_bytes(ck.s)) return DC_ERR_INVALID_ARG;
     cudaStream_t st = (cudaStream_t)stream;
     float *band = (float *)workspace;
-    if (ck.impl == DC_IMPL_TCGEN05 && dc::tc::kHasBwd)
+    if (ck.impl == DC_IMPL_TCGEN05)
         return cuda_status(dc::tc::bwd_query(ck.s, q, k, v, c, g, dO, lse, pmap, dq, dc_, dg, band, st,
                                              &t_launches));
     return cuda_status(DC_DISPATCH(simt_bwd_query, ck.dtype, ck.s.d, ck.s, q, k, v, c, g, dO, lse, pmap, dq,
@@ -200,7 +200,7 @@ dc_status_t dc_attn_bwd_key(const dc_attn_params *params, const void *q, const v
     if (workspace_bytes < band_bytes(ck.s)) return DC_ERR_INVALID_ARG;
     cudaStream_t st = (cudaStream_t)stream;
     const float *band = (const float *)workspace;
-    if (ck.impl == DC_IMPL_TCGEN05 && dc::tc::kHasBwd)
+    if (ck.impl == DC_IMPL_TCGEN05)
         return cuda_status(dc::tc::bwd_key(ck.s, q, k, c, g, dO, lse, pmap, dc_, band, dk, dv, st,
                                            &t_launches));
     return cuda_status(DC_DISPATCH(simt_bwd_key, ck.dtype, ck.s.d, ck.s, q, k, c, g, dO, lse, pmap, dc_, band,

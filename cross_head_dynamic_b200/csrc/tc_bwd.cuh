@@ -7,8 +7,10 @@
 //
 // Query side (one CTA per block of BM query tokens, all heads):
 //   phase 1, per head: MMA E_h = dO_h V_h^T -> TMEM; SIMT dP += g_h E_h
-//            (registers), dg_h = sum_j P E_h with P from the forward's pmap;
-//            dP is then stored as a band [N][W] in the workspace.
+//            (registers), dg_h = sum_j P E_h with P from the forward's pmap
+//            (the CTA's pmap rows are staged in shared memory once); dP is then
+//            stored as a band [N][W] in the workspace for the key side, which
+//            must see exactly the dP that dc was computed from.
 //   phase 2, per head: MMA S_h = Q_h K_h^T -> TMEM; SIMT p_h from lse,
 //            dc_h = sum_j dP p_h, ds_h -> bf16 tile in smem; MMA dQ_h = ds_h K_h.
 // Key side (one CTA per block of BK key tokens; the queries that see them span
@@ -16,9 +18,12 @@
 //   phase 1, per head: scale the dO_h rows by g_h in smem; MMA dV_h = P^T gdO_h
 //            with P^T built once from pmap.
 //   phase 2, per head: MMA S^T_h = K_h Q_h^T -> TMEM; SIMT ds^T from lse, c,
-//            dc and the stored dP; MMA dK_h = ds^T_h Q_h.
-// Same thread roles as the forward: warps 0-7 SIMT (two per TMEM lane
-// quarter), warp 8 lane 0 issues TMA and MMA; every wait is bounded.
+//            dc and the query side's dP; MMA dK_h = ds^T_h Q_h.
+// In both phase-2 loops the gradient MMA of head h runs while the SIMT warps
+// work on the scores of head h+1: the producer issues S_{h+1} before dQ_h/dK_h,
+// and the warps drain head h's accumulator one iteration later.
+// Same thread roles as the forward: warps 0-11 SIMT (three per TMEM lane
+// quarter), warp 12 lane 0 issues TMA and MMA; every wait is bounded.
 #pragma once
 
 #include "tc_common.cuh"
@@ -45,6 +50,33 @@ struct BwdArgs {
     __nv_bfloat16 *dv;
 };
 
+// Drain this split's 16-column chunks of one row of a [128 x D] fp32 accumulator
+// (row base address taddr, output row dst): scale, round to bf16, store when `store`.
+template <int D>
+__device__ __forceinline__ void drain_row(uint32_t taddr, __nv_bfloat16 *dst, float mult, bool store, int split) {
+    int cb16, ce16;
+    acc_split(split, D / 16, cb16, ce16);
+    constexpr int kMaxC16 = (D / 16 + kSplits - 1) / kSplits;
+#pragma unroll
+    for (int c = 0; c < kMaxC16; ++c) {
+        if (cb16 + c < ce16) {   // one 16-column chunk per TMEM round trip keeps register use low
+            uint32_t r[16];
+            ptx::tmem_ld16_issue(taddr + (cb16 + c) * 16, r);
+            ptx::tmem_wait_ld();
+            ptx::reg_fence16(r);
+            if (store) {
+                uint32_t w[8];
+#pragma unroll
+                for (int e = 0; e < 8; ++e)
+                    w[e] = pack_bf16x2(mult * __uint_as_float(r[2 * e]), mult * __uint_as_float(r[2 * e + 1]));
+                uint4 *p = (uint4 *)(dst + (cb16 + c) * 16);
+                p[0] = make_uint4(w[0], w[1], w[2], w[3]);
+                p[1] = make_uint4(w[4], w[5], w[6], w[7]);
+            }
+        }
+    }
+}
+
 // --------------------------------------------------------------------------- query side
 enum : int { kQBarLd = 0, kQBarQ = 2, kQBarK = 3, kQBarXFull = 5, kQBarXFree = 6, kQBarDs = 7, kQBarDqFull = 8,
              kQBarDqFree = 10, kQNumBars = 12 };
@@ -60,7 +92,7 @@ struct QSideLayout {
         rq = 2 * tile_k;                  // Q (phase 2) / dO buffer 0 (phase 1)
         rd = rq + 128u * D * 2;           // ds tile (phase 2) / dO buffer 1 (phase 1)
         red = rd + 4u * 16384;
-        bars = red + 2 * 2 * 128 * 4;
+        bars = red + 2 * kSplits * 128 * 4;
         bytes = bars + 512;
     }
 };
@@ -78,7 +110,7 @@ bwd_query_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
     uint64_t *bars = (uint64_t *)(sm + L.bars);
     uint32_t *tmem_slot = (uint32_t *)(bars + 32);
     volatile int *abort_flag = (volatile int *)(tmem_slot + 1);
-    float *red = (float *)(sm + L.red);   // [2 parity][2 split][128]
+    float *red = (float *)(sm + L.red);   // [2 parity][kSplits][128]
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int64_t t0 = (int64_t)blockIdx.x * BM;
@@ -102,8 +134,9 @@ bwd_query_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
     ptx::tc_fence_after();
     const uint32_t tmem = *tmem_slot;
 
-    if (warp == kProducerWarp) {
-        if (lane == 0) {
+    if (warp >= kProducerWarp) {
+        regs_producer();
+        if (warp == kProducerWarp && lane == 0) {
             const uint32_t q_bytes = 128u * D * 2;
             auto issue_e = [&](int h) {   // phase 1 operands of head h: dO_h and V_h
                 const int b = h & 1;
@@ -130,6 +163,23 @@ bwd_query_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
             };
             const uint32_t id_x = ptx::idesc_bf16_f32(128, span, 0, 0);   // E and S: [128 x span]
             const uint32_t id_dq = ptx::idesc_bf16_f32(128, D, 0, 1);     // dQ: [128 x D], B MN-major
+            // dQ_h = ds_h K_h into accumulator buffer h & 1 (K_h is MN-major for this product)
+            auto mma_dq = [&](int h) {
+                const int b = h & 1;
+                bool ok = wait_bar(&bars[kQBarDs], (uint32_t)h & 1, abort_flag);
+                if (h >= 2) ok = wait_bar(&bars[kQBarDqFree + b], (uint32_t)((h >> 1) - 1) & 1, abort_flag) && ok;
+                ptx::tc_fence_after();
+                if (ok) {
+                    const uint32_t dsa = ptx::smem_u32(sm + L.rd);
+                    const uint32_t ka = ptx::smem_u32(sm + (b ? L.r1 : L.r0));
+                    for (int k = 0; k < span / 16; ++k) {
+                        const uint64_t ad = ptx::smem_desc_sw128(dsa + (k >> 2) * 16384 + (k & 3) * 32, 16, 1024);
+                        const uint64_t bd = ptx::smem_desc_sw128(ka + k * 2048, span * 128, 1024);
+                        ptx::mma_bf16(tmem + 256 + 128 * b, ad, bd, id_dq, k > 0);
+                    }
+                }
+                ptx::mma_commit(&bars[kQBarDqFull + b]);
+            };
 
             // ---- phase 1: E_h = dO_h V_h^T
             for (int h = 0; h < H && h < 2; ++h) issue_e(h);
@@ -149,9 +199,14 @@ bwd_query_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
                     }
                 }
                 ptx::mma_commit(&bars[kQBarXFull]);
+                // phase 2 reads Q_h and K_h: pull them into L2 while phase 1 runs
+                for (int kb = 0; kb < D / 64; ++kb) {
+                    ptx::tma_prefetch_l2_2d(&map_q, h * D + kb * 64, (int)t0);
+                    ptx::tma_prefetch_l2_2d(&map_k, h * D + kb * 64, (int)kbase);
+                }
                 if (h + 2 < H && wait_bar(&bars[kQBarXFull], (uint32_t)h & 1, abort_flag)) issue_e(h + 2);
             }
-            // ---- phase 2: S_h = Q_h K_h^T, then dQ_h = ds_h K_h
+            // ---- phase 2: S_h = Q_h K_h^T; dQ_{h-1} = ds_{h-1} K_{h-1} right after it
             if (wait_bar(&bars[kQBarXFull], (uint32_t)(H - 1) & 1, abort_flag)) {   // all E MMAs done
                 issue_q(0);
                 for (int h = 0; h < H && h < 2; ++h) issue_k(h);
@@ -163,9 +218,9 @@ bwd_query_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
                 ok = wait_bar(&bars[kQBarK + b], (uint32_t)(h >> 1) & 1, abort_flag) && ok;
                 ok = wait_bar(&bars[kQBarXFree], (ph - 1) & 1, abort_flag) && ok;
                 ptx::tc_fence_after();
-                const uint32_t ka = ptx::smem_u32(sm + (b ? L.r1 : L.r0));
                 if (ok) {
                     const uint32_t qa = ptx::smem_u32(sm + L.rq);
+                    const uint32_t ka = ptx::smem_u32(sm + (b ? L.r1 : L.r0));
 #pragma unroll
                     for (int k = 0; k < D / 16; ++k) {
                         const uint64_t ad = ptx::smem_desc_sw128(qa + (k >> 2) * 16384 + (k & 3) * 32, 16, 1024);
@@ -174,24 +229,18 @@ bwd_query_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
                     }
                 }
                 ptx::mma_commit(&bars[kQBarXFull]);
+                if (h >= 1) mma_dq(h - 1);
+                // refill: Q_{h+1} once S_h has read Q; K_{h+1} once dQ_{h-1} has read K_{h-1}
                 if (wait_bar(&bars[kQBarXFull], ph & 1, abort_flag) && h + 1 < H) issue_q(h + 1);
-                ok = wait_bar(&bars[kQBarDs], (uint32_t)h & 1, abort_flag);
-                if (h >= 2) ok = wait_bar(&bars[kQBarDqFree + b], (uint32_t)((h >> 1) - 1) & 1, abort_flag) && ok;
-                ptx::tc_fence_after();
-                if (ok) {
-                    const uint32_t dsa = ptx::smem_u32(sm + L.rd);
-                    for (int k = 0; k < span / 16; ++k) {
-                        const uint64_t ad = ptx::smem_desc_sw128(dsa + (k >> 2) * 16384 + (k & 3) * 32, 16, 1024);
-                        const uint64_t bd = ptx::smem_desc_sw128(ka + k * 2048, span * 128, 1024);
-                        ptx::mma_bf16(tmem + 256 + 128 * b, ad, bd, id_dq, k > 0);
-                    }
-                }
-                ptx::mma_commit(&bars[kQBarDqFull + b]);
-                if (h + 2 < H && wait_bar(&bars[kQBarDqFull + b], (uint32_t)(h >> 1) & 1, abort_flag)) issue_k(h + 2);
+                if (h >= 1 && h + 1 < H &&
+                    wait_bar(&bars[kQBarDqFull + ((h - 1) & 1)], (uint32_t)((h - 1) >> 1) & 1, abort_flag))
+                    issue_k(h + 1);
             }
+            mma_dq(H - 1);
         }
         __syncwarp();
     } else {
+        regs_compute();
         // ---------------------------------------------------------------- compute warps
         const int q = warp & 3, split = warp >> 2;
         const int i = 32 * q + lane;
@@ -207,156 +256,191 @@ bwd_query_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
         const uint32_t x_cols = tmem + lane_base;
         const float sl2 = s.scale * kLog2e;
 
-        // P(t, c) = pmap[t][c - i] for columns c in this row's window (re-read per head;
-        // the CTA's pmap rows stay in L1)
-        const uint16_t *prow = reinterpret_cast<const uint16_t *>(a.pmap) + t * W - i;
+        // Stage the CTA's pmap rows (one contiguous [BM][W] block) in the upper half of the
+        // ds tile region, unused until phase 2; P(t, c) = pmap[t][c - i].
+        uint16_t *pstage = (uint16_t *)(sm + L.rd + 32768);
+        {
+            const int64_t rows = min((int64_t)BM, s.N - t0);
+            const int64_t nh = rows * W;   // t0 * W is even
+            const uint32_t *src = reinterpret_cast<const uint32_t *>(a.pmap + t0 * W);
+            uint32_t *dst = reinterpret_cast<uint32_t *>(pstage);
+            for (int64_t x = threadIdx.x; x < nh / 2; x += kComputeThreads) dst[x] = __ldg(src + x);
+            if ((nh & 1) && threadIdx.x == 0) pstage[nh - 1] = reinterpret_cast<const uint16_t *>(a.pmap)[t0 * W + nh - 1];
+        }
+        compute_sync();
+        const uint16_t *prow = pstage + i * W - i;
         float dP[MAXC][8];
 #pragma unroll
         for (int cc = 0; cc < MAXC; ++cc)
 #pragma unroll
             for (int e = 0; e < 8; ++e) dP[cc][e] = 0.f;
 
-        // ---- phase 1: dP and dg
+        // ---- phase 1: dP and dg, three chunks of E_h per TMEM round trip
         for (int h = 0; h < H; ++h) {
             wait_bar(&bars[kQBarXFull], (uint32_t)h & 1, abort_flag);
             ptx::tc_fence_after();
             const float gh = valid ? __ldg(a.g + t * H + h) : 0.f;
             float dgp = 0.f;
+            constexpr int G = 3;
 #pragma unroll
-            for (int cc = 0; cc < MAXC; ++cc) {
-                if (cc < bd.mync) {
-                    const int col = bd.cb + (bd.c0 + cc) * 8;
-                    float E[8];
-                    ptx::tmem_ld8(x_cols + col, E);
+            for (int g0 = 0; g0 < MAXC; g0 += G) {
+                uint32_t er[G][8];
+                float pv[G][8];
 #pragma unroll
-                    for (int e = 0; e < 8; ++e) {
-                        const int cidx = col + e;
-                        const bool in = cidx >= clo && cidx <= chi;
-                        const float ev = in ? E[e] : 0.f;
-                        const float pv = in ? __uint_as_float((uint32_t)__ldg(prow + cidx) << 16) : 0.f;
-                        dP[cc][e] = fmaf(gh, ev, dP[cc][e]);
-                        dgp = fmaf(pv, ev, dgp);
+                for (int gi = 0; gi < G; ++gi) {
+                    const int cc = g0 + gi;
+                    if (cc < MAXC && cc < bd.mync) {
+                        const int col = bd.cb + (bd.c0 + cc) * 8;
+#pragma unroll
+                        for (int e = 0; e < 8; ++e) {
+                            const int cidx = col + e;
+                            pv[gi][e] = (cidx >= clo && cidx <= chi) ? __uint_as_float((uint32_t)prow[cidx] << 16) : 0.f;
+                        }
+                        ptx::tmem_ld8_issue(x_cols + col, er[gi]);
+                    }
+                }
+                ptx::tmem_wait_ld();
+#pragma unroll
+                for (int gi = 0; gi < G; ++gi) {
+                    const int cc = g0 + gi;
+                    if (cc < MAXC && cc < bd.mync) {
+                        ptx::reg_fence8(er[gi]);
+                        const int col = bd.cb + (bd.c0 + cc) * 8;
+#pragma unroll
+                        for (int e = 0; e < 8; ++e) {
+                            const int cidx = col + e;
+                            const float ev = (cidx >= clo && cidx <= chi) ? __uint_as_float(er[gi][e]) : 0.f;
+                            dP[cc][e] = fmaf(gh, ev, dP[cc][e]);
+                            dgp = fmaf(pv[gi][e], ev, dgp);
+                        }
                     }
                 }
             }
             ptx::tc_fence_before();
             ptx::mbar_arrive(&bars[kQBarXFree]);
-            float *rd = red + (h & 1) * 256;
+            float *rd = red + (h & 1) * (kSplits * 128);
             rd[split * 128 + i] = dgp;
             pair_sync(q);
-            if (split == 0 && valid) a.dg[t * H + h] = rd[i] + rd[128 + i];
+            if (split == 0 && valid) {
+                float sum = rd[i];
+#pragma unroll
+                for (int sp = 1; sp < kSplits; ++sp) sum += rd[sp * 128 + i];
+                a.dg[t * H + h] = sum;
+            }
         }
-        // dP band: band[t][w] = dP(t, t - W + 1 + w), tile column i + w
-        if (valid) {
-            float *brow = a.band + t * W - i;
+        // every compute warp has finished phase 1 (and its reads of the staged pmap)
+        compute_sync();
+        // dP band: band[t][w] = dP(t, t - W + 1 + w) = tile column i + w.  The CTA's rows
+        // are one contiguous [BM][W] block of the band: stage it in the ds tile region
+        // (free: every E MMA has completed) and copy it out with 16-byte stores.  The
+        // row stride W - 1 between lanes is odd for the usual even W, so the staging
+        // stores do not conflict.
+        {
+            float *stage = (float *)(sm + L.rd);
+            if (i < BM) {
 #pragma unroll
-            for (int cc = 0; cc < MAXC; ++cc) {
-                if (cc < bd.mync) {
-                    const int col = bd.cb + (bd.c0 + cc) * 8;
+                for (int cc = 0; cc < MAXC; ++cc) {
+                    if (cc < bd.mync) {
+                        const int col = bd.cb + (bd.c0 + cc) * 8;
 #pragma unroll
-                    for (int e = 0; e < 8; ++e) {
-                        const int cidx = col + e;
-                        if (cidx >= i && cidx < i + W) brow[cidx] = dP[cc][e];
+                        for (int e = 0; e < 8; ++e) {
+                            const int w = col + e - i;
+                            if (w >= 0 && w < W) stage[i * W + w] = dP[cc][e];
+                        }
                     }
                 }
             }
+            compute_sync();
+            const int64_t rows = min((int64_t)BM, s.N - t0);
+            const int64_t n = rows * W;
+            float *dst = a.band + t0 * W;
+            if ((W & 3) == 0) {
+                for (int64_t x4 = threadIdx.x; x4 < n / 4; x4 += kComputeThreads)
+                    *(float4 *)(dst + 4 * x4) = *(const float4 *)(stage + 4 * x4);
+            } else {
+                for (int64_t x = threadIdx.x; x < n; x += kComputeThreads) dst[x] = stage[x];
+            }
+            compute_sync();
         }
 
-        // ---- phase 2: the ds tile region held dO in phase 1; every E MMA has
-        // completed (waited above), so zero its columns outside this quarter's band once.
+        // ---- phase 2.  The ds tile region held dO, the pmap rows and the dP band in
+        // phase 1; zero its columns outside this quarter's band once.
         uint8_t *dtile = sm + L.rd;
-        {
-            const uint4 z4 = make_uint4(0, 0, 0, 0);
-            const int ce = bd.cb + bd.nch * 8;
-            if (split == 0) {
-                for (int col = 0; col < bd.cb && col < span; col += 8) *(uint4 *)(dtile + sw128_offset(i, col)) = z4;
-            } else {
-                for (int col = (ce > bd.cb ? ce : bd.cb); col < span; col += 8)
-                    *(uint4 *)(dtile + sw128_offset(i, col)) = z4;
-            }
-        }
+        zero_outside_band(dtile, i, split, bd, span);
+        auto drain_dq = [&](int h) {
+            const int b = h & 1;
+            wait_bar(&bars[kQBarDqFull + b], (uint32_t)(h >> 1) & 1, abort_flag);
+            ptx::tc_fence_after();
+            drain_row<D>(tmem + lane_base + 256 + 128 * b, a.dq + (t * H + h) * D, s.scale, valid, split);
+            ptx::tc_fence_before();
+            ptx::mbar_arrive(&bars[kQBarDqFree + b]);
+        };
         for (int h = 0; h < H; ++h) {
             const uint32_t ph = (uint32_t)(H + h);
             wait_bar(&bars[kQBarXFull], ph & 1, abort_flag);
             ptx::tc_fence_after();
             const float lse2 = valid ? __ldg(a.lse + t * H + h) * kLog2e : 0.f;
-            // pass 1: p_h and dc_h; p is parked (bf16) in this thread's own slots of the
-            // ds tile, whose previous contents the dQ MMA of head h-1 has finished reading
+            // p_h and dc_h, the band of S_h in two TMEM round trips
             float dcp = 0.f;
+            uint32_t pp[MAXC][4];   // p_h as packed bf16 pairs
+            constexpr int G2 = (MAXC + 1) / 2;
 #pragma unroll
-            for (int cc = 0; cc < MAXC; ++cc) {
-                if (cc < bd.mync) {
-                    const int col = bd.cb + (bd.c0 + cc) * 8;
-                    float x[8];
-                    ptx::tmem_ld8(x_cols + col, x);
+            for (int g0 = 0; g0 < MAXC; g0 += G2) {
+                uint32_t xr[G2][8];
 #pragma unroll
-                    for (int e = 0; e < 8; ++e) {
-                        const int cidx = col + e;
-                        const float p = (cidx >= clo && cidx <= chi) ? ex2(x[e] * sl2 - lse2) : 0.f;
-                        x[e] = p;
-                        dcp = fmaf(dP[cc][e], p, dcp);
+                for (int gi = 0; gi < G2; ++gi) {
+                    const int cc = g0 + gi;
+                    if (cc < MAXC && cc < bd.mync) ptx::tmem_ld8_issue(x_cols + bd.cb + (bd.c0 + cc) * 8, xr[gi]);
+                }
+                ptx::tmem_wait_ld();
+#pragma unroll
+                for (int gi = 0; gi < G2; ++gi) {
+                    const int cc = g0 + gi;
+                    if (cc < MAXC && cc < bd.mync) {
+                        ptx::reg_fence8(xr[gi]);
+                        const int col = bd.cb + (bd.c0 + cc) * 8;
+                        float p[8];
+#pragma unroll
+                        for (int e = 0; e < 8; ++e) {
+                            const int cidx = col + e;
+                            p[e] = (cidx >= clo && cidx <= chi) ? ex2(__uint_as_float(xr[gi][e]) * sl2 - lse2) : 0.f;
+                            dcp = fmaf(dP[cc][e], p[e], dcp);
+                        }
+#pragma unroll
+                        for (int e = 0; e < 4; ++e) pp[cc][e] = pack_bf16x2(p[2 * e], p[2 * e + 1]);
                     }
-                    *(uint4 *)(dtile + sw128_offset(i, col)) =
-                        make_uint4(pack_bf16x2(x[0], x[1]), pack_bf16x2(x[2], x[3]), pack_bf16x2(x[4], x[5]),
-                                   pack_bf16x2(x[6], x[7]));
                 }
             }
             ptx::tc_fence_before();
             ptx::mbar_arrive(&bars[kQBarXFree]);
-            float *rd = red + (ph & 1) * 256;
+            float *rd = red + (ph & 1) * (kSplits * 128);
             rd[split * 128 + i] = dcp;
             pair_sync(q);
-            const float dch = rd[i] + rd[128 + i];
+            float dch = rd[i];
+#pragma unroll
+            for (int sp = 1; sp < kSplits; ++sp) dch += rd[sp * 128 + i];
             if (split == 0 && valid) a.dc[t * H + h] = dch;
             const float ch = valid ? __ldg(a.c + t * H + h) : 0.f;
-            // pass 2: ds_h = c_h p_h (dP - dc_h) over the parked p
+            // the previous head's dQ MMA has been running meanwhile; drain it, which also
+            // frees the ds tile for this head
+            if (h >= 1) drain_dq(h - 1);
 #pragma unroll
             for (int cc = 0; cc < MAXC; ++cc) {
                 if (cc < bd.mync) {
                     const int col = bd.cb + (bd.c0 + cc) * 8;
-                    uint4 *slot = (uint4 *)(dtile + sw128_offset(i, col));
-                    const uint4 pv = *slot;
-                    const uint32_t pw[4] = {pv.x, pv.y, pv.z, pv.w};
                     uint32_t w[4];
 #pragma unroll
                     for (int e = 0; e < 4; ++e) {
-                        const float p0 = __uint_as_float(pw[e] << 16), p1 = __uint_as_float(pw[e] & 0xFFFF0000u);
+                        const float p0 = __uint_as_float(pp[cc][e] << 16), p1 = __uint_as_float(pp[cc][e] & 0xFFFF0000u);
                         w[e] = pack_bf16x2(ch * p0 * (dP[cc][2 * e] - dch), ch * p1 * (dP[cc][2 * e + 1] - dch));
                     }
-                    *slot = make_uint4(w[0], w[1], w[2], w[3]);
+                    *(uint4 *)(dtile + sw128_offset(i, col)) = make_uint4(w[0], w[1], w[2], w[3]);
                 }
             }
             ptx::fence_proxy_async_smem();
             ptx::mbar_arrive(&bars[kQBarDs]);
-
-            // drain dQ_h (the next head rewrites the ds tile only after this MMA completed)
-            const int b = h & 1;
-            wait_bar(&bars[kQBarDqFull + b], (uint32_t)(h >> 1) & 1, abort_flag);
-            ptx::tc_fence_after();
-            const int cbase = split * (D / 2);
-#pragma unroll
-            for (int c16 = 0; c16 < D / 32; ++c16) {
-                float u[16];
-                ptx::tmem_ld16(tmem + lane_base + 256 + 128 * b + cbase + c16 * 16, u);
-                if (valid) {
-                    uint4 w0, w1;
-                    const float sc = s.scale;
-                    w0.x = pack_bf16x2(sc * u[0], sc * u[1]);
-                    w0.y = pack_bf16x2(sc * u[2], sc * u[3]);
-                    w0.z = pack_bf16x2(sc * u[4], sc * u[5]);
-                    w0.w = pack_bf16x2(sc * u[6], sc * u[7]);
-                    w1.x = pack_bf16x2(sc * u[8], sc * u[9]);
-                    w1.y = pack_bf16x2(sc * u[10], sc * u[11]);
-                    w1.z = pack_bf16x2(sc * u[12], sc * u[13]);
-                    w1.w = pack_bf16x2(sc * u[14], sc * u[15]);
-                    uint4 *dst = (uint4 *)(a.dq + (t * H + h) * D + cbase + c16 * 16);
-                    dst[0] = w0;
-                    dst[1] = w1;
-                }
-            }
-            ptx::tc_fence_before();
-            ptx::mbar_arrive(&bars[kQBarDqFree + b]);
         }
+        drain_dq(H - 1);
     }
 
     ptx::tc_fence_before();
@@ -374,16 +458,20 @@ enum : int { kKBarLd = 0, kKBarScaled = 2, kKBarPt = 4, kKBarAccFull = 5, kKBarA
 template <int D>
 struct KSideLayout {
     uint32_t tile_s;   // dO or Q tile over the query span: D/64 boxes of span rows x 128 B
-    uint32_t ra, rb0, rb1, rk, colv, bars, bytes;
-    __host__ __device__ KSideLayout(int span) {
+    uint32_t ra, rb0, rb1, rk, colv, bars, bytes, stage, stage_bytes;
+    bool stage_in_b1;  // the pmap staging rows fit in buffer 1 + the K/V buffer (dO_0 can load early)
+    __host__ __device__ KSideLayout(int span, int W) {
         tile_s = (uint32_t)(D / 64) * span * 128;
         ra = 0;                            // P^T tile (phase 1) / ds^T tile (phase 2): 64 KiB
         rb0 = 4u * 16384;                  // dO buffer 0 (phase 1) / Q buffer 0 (phase 2)
         rb1 = rb0 + tile_s;
-        rk = rb1 + tile_s;                 // K of the key block (phase 2)
+        rk = rb1 + tile_s;                 // V_h (phase 1) / K_h (phase 2) of the key block
         colv = rk + 128u * D * 2;          // per-query vectors [2][3][256] fp32
         bars = colv + 2 * 3 * 256 * 4;
         bytes = bars + 512;
+        stage_bytes = (uint32_t)span * W * 2;   // pmap rows of the query span, read once
+        stage_in_b1 = tile_s + 128u * D * 2 >= stage_bytes;
+        stage = stage_in_b1 ? rb1 : rb0;
     }
 };
 
@@ -395,7 +483,7 @@ bwd_key_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant_
     uint8_t *sm = (uint8_t *)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
     const Shape &s = a.s;
     const int H = s.H, W = s.W, BK = a.BM, span = a.span;
-    const KSideLayout<D> L(span);
+    const KSideLayout<D> L(span, W);
     uint64_t *bars = (uint64_t *)(sm + L.bars);
     uint32_t *tmem_slot = (uint32_t *)(bars + 32);
     volatile int *abort_flag = (volatile int *)(tmem_slot + 1);
@@ -422,9 +510,10 @@ bwd_key_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant_
     ptx::tc_fence_after();
     const uint32_t tmem = *tmem_slot;
 
-    if (warp == kProducerWarp) {
-        if (lane == 0) {
-            // load sequence a = 0 .. 2H-1 into buffers a & 1: dO_a for a < H, Q_{a-H} after
+    if (warp >= kProducerWarp) {
+        regs_producer();
+        if (warp == kProducerWarp && lane == 0) {
+            // load sequence idx = 0 .. 2H-1 into buffers idx & 1: dO_idx for idx < H, Q_{idx-H} after
             auto issue_ld = [&](int idx) {
                 const int b = idx & 1;
                 uint8_t *dst = sm + (b ? L.rb1 : L.rb0);
@@ -441,65 +530,73 @@ bwd_key_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant_
             };
             const uint32_t id_acc = ptx::idesc_bf16_f32(128, D, 0, 1);     // dV, dK: B MN-major
             const uint32_t id_st = ptx::idesc_bf16_f32(128, span, 0, 0);   // S^T: [128 keys x span]
-            issue_ld(0);
-            if (2 * H > 1) issue_ld(1);
-            issue_k(0);
-            // ---- phase 1: dV_h = P^T (g_h dO_h)
-            bool pt_ok = wait_bar(&bars[kKBarPt], 0, abort_flag);
             const uint32_t ra = ptx::smem_u32(sm + L.ra);
-            for (int h = 0; h < H; ++h) {
-                const int idx = h, b = idx & 1;
+            const uint32_t rk = ptx::smem_u32(sm + L.rk);
+            // accumulator product number idx (dV_idx for idx < H, dK_{idx-H} after) into
+            // buffer idx & 1: A = the tile in region A (P^T or ds^T), B = load buffer idx & 1
+            // (g-scaled dO or Q), MN-major
+            auto mma_acc = [&](int idx, bool ok) {
+                const int b = idx & 1;
                 const uint32_t n = (uint32_t)(idx >> 1);
-                bool ok = wait_bar(&bars[kKBarScaled + b], n & 1, abort_flag) && pt_ok;
                 if (idx >= 2) ok = wait_bar(&bars[kKBarAccFree + b], (n - 1) & 1, abort_flag) && ok;
                 ptx::tc_fence_after();
                 if (ok) {
-                    const uint32_t da = ptx::smem_u32(sm + (b ? L.rb1 : L.rb0));
+                    const uint32_t ba = ptx::smem_u32(sm + (b ? L.rb1 : L.rb0));
                     for (int k = 0; k < span / 16; ++k) {
                         const uint64_t ad = ptx::smem_desc_sw128(ra + (k >> 2) * 16384 + (k & 3) * 32, 16, 1024);
-                        const uint64_t bd2 = ptx::smem_desc_sw128(da + k * 2048, span * 128, 1024);
+                        const uint64_t bd2 = ptx::smem_desc_sw128(ba + k * 2048, span * 128, 1024);
                         ptx::mma_bf16(tmem + 256 + 128 * b, ad, bd2, id_acc, k > 0);
                     }
                 }
                 ptx::mma_commit(&bars[kKBarAccFull + b]);
+            };
+            if (L.stage_in_b1) issue_ld(0);   // buffer 0 does not overlap the pmap staging rows
+            // ---- phase 1: dV_h = P^T (g_h dO_h)
+            const bool pt_ok = wait_bar(&bars[kKBarPt], 0, abort_flag);   // staging area consumed
+            if (!L.stage_in_b1) issue_ld(0);
+            if (H > 1) issue_ld(1);
+            issue_k(0);
+            for (int h = 0; h < H; ++h) {
+                const int idx = h, b = idx & 1;
+                const uint32_t n = (uint32_t)(idx >> 1);
+                const bool ok = wait_bar(&bars[kKBarScaled + b], n & 1, abort_flag) && pt_ok;
+                mma_acc(idx, ok);
+                // phase 2 reads Q_h and K_h: pull them into L2 while phase 1 runs
+                for (int kb = 0; kb < D / 64; ++kb) {
+                    ptx::tma_prefetch_l2_2d(&map_q, h * D + kb * 64, (int)j0);
+                    ptx::tma_prefetch_l2_2d(&map_k, h * D + kb * 64, (int)j0);
+                }
                 if (idx + 2 < 2 * H && wait_bar(&bars[kKBarAccFull + b], n & 1, abort_flag)) issue_ld(idx + 2);
             }
-            // ---- phase 2: S^T_h = K_h Q_h^T, dK_h = ds^T_h Q_h
+            // ---- phase 2: S^T_h = K_h Q_h^T, then dK_{h-1} = ds^T_{h-1} Q_{h-1}
             for (int h = 0; h < H; ++h) {
                 const int idx = H + h, b = idx & 1;
-                const uint32_t n = (uint32_t)(idx >> 1);
                 bool ok = wait_bar(&bars[kKBarK], (uint32_t)h & 1, abort_flag);
-                ok = wait_bar(&bars[kKBarLd + b], n & 1, abort_flag) && ok;
+                ok = wait_bar(&bars[kKBarLd + b], (uint32_t)(idx >> 1) & 1, abort_flag) && ok;
                 if (h >= 1) ok = wait_bar(&bars[kKBarXFree], (uint32_t)(h - 1) & 1, abort_flag) && ok;
                 ptx::tc_fence_after();
-                const uint32_t qa = ptx::smem_u32(sm + (b ? L.rb1 : L.rb0));
                 if (ok) {
-                    const uint32_t ka = ptx::smem_u32(sm + L.rk);
+                    const uint32_t qa = ptx::smem_u32(sm + (b ? L.rb1 : L.rb0));
 #pragma unroll
                     for (int k = 0; k < D / 16; ++k) {
-                        const uint64_t ad = ptx::smem_desc_sw128(ka + (k >> 2) * 16384 + (k & 3) * 32, 16, 1024);
+                        const uint64_t ad = ptx::smem_desc_sw128(rk + (k >> 2) * 16384 + (k & 3) * 32, 16, 1024);
                         const uint64_t bd2 = ptx::smem_desc_sw128(qa + (k >> 2) * span * 128 + (k & 3) * 32, 16, 1024);
                         ptx::mma_bf16(tmem, ad, bd2, id_st, k > 0);
                     }
                 }
                 ptx::mma_commit(&bars[kKBarXFull]);
+                if (h >= 1) mma_acc(idx - 1, wait_bar(&bars[kKBarDs], (uint32_t)(h - 1) & 1, abort_flag));
+                // refill: K_{h+1} once S^T_h has read K; Q_{h+1} once dK_{h-1} has read Q_{h-1}
                 if (wait_bar(&bars[kKBarXFull], (uint32_t)h & 1, abort_flag) && h + 1 < H) issue_k(h + 1);
-                ok = wait_bar(&bars[kKBarDs], (uint32_t)h & 1, abort_flag);
-                if (idx >= 2) ok = wait_bar(&bars[kKBarAccFree + b], (n - 1) & 1, abort_flag) && ok;
-                ptx::tc_fence_after();
-                if (ok) {
-                    for (int k = 0; k < span / 16; ++k) {
-                        const uint64_t ad = ptx::smem_desc_sw128(ra + (k >> 2) * 16384 + (k & 3) * 32, 16, 1024);
-                        const uint64_t bd2 = ptx::smem_desc_sw128(qa + k * 2048, span * 128, 1024);
-                        ptx::mma_bf16(tmem + 256 + 128 * b, ad, bd2, id_acc, k > 0);
-                    }
-                }
-                ptx::mma_commit(&bars[kKBarAccFull + b]);
-                if (idx + 2 < 2 * H && wait_bar(&bars[kKBarAccFull + b], n & 1, abort_flag)) issue_ld(idx + 2);
+                if (h >= 1 && idx + 1 < 2 * H &&
+                    wait_bar(&bars[kKBarAccFull + ((idx - 1) & 1)], (uint32_t)((idx - 1) >> 1) & 1, abort_flag))
+                    issue_ld(idx + 1);
             }
+            mma_acc(2 * H - 1, wait_bar(&bars[kKBarDs], (uint32_t)(H - 1) & 1, abort_flag));
         }
         __syncwarp();
     } else {
+        regs_compute();
         // ---------------------------------------------------------------- compute warps
         const int tid = threadIdx.x;   // 0 .. 255
         const int q = warp & 3, split = warp >> 2;
@@ -514,14 +611,28 @@ bwd_key_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant_
             if (hi > dend - 1) hi = dend - 1;
             chi = (int)(hi - j0);
         }
+        // column c is in this row's window iff (unsigned)(c - span_lo) <= span_n; a row with an
+        // empty window (clo > chi: past the block or past N) gets span_lo = ~0u, so no c passes
+        const uint32_t span_lo = (chi >= clo) ? (uint32_t)clo : ~0u;
+        const uint32_t span_n = (chi >= clo) ? (uint32_t)(chi - clo) : 0u;
         const Band bd = make_band(q, split, BK, W, span);
         const uint32_t lane_base = (uint32_t)(32 * q) << 16;
         const float sl2 = s.scale * kLog2e;
 
+        // ---- stage pmap rows j0 .. j0+span-1 (one contiguous block) with coalesced loads
+        uint16_t *stage = (uint16_t *)(sm + L.stage);
+        {
+            const int64_t rows = min((int64_t)span, s.N - j0);
+            const int64_t nh = rows * W;                              // bf16 elements; j0 * W is even
+            const uint32_t *src = reinterpret_cast<const uint32_t *>(a.pmap + j0 * W);
+            uint32_t *dst = reinterpret_cast<uint32_t *>(stage);
+            for (int64_t x = tid; x < nh / 2; x += kComputeThreads) dst[x] = __ldg(src + x);
+            if ((nh & 1) && tid == 0) stage[nh - 1] = reinterpret_cast<const uint16_t *>(a.pmap)[j0 * W + nh - 1];
+        }
+        compute_sync();
         // ---- P^T tile: P^T(i, c) = P(j0 + c, j0 + i) = pmap[j0 + c][i - c + W - 1]
         uint8_t *atile = sm + L.ra;
         {
-            const uint16_t *pm = reinterpret_cast<const uint16_t *>(a.pmap);
 #pragma unroll
             for (int cc = 0; cc < MAXC; ++cc) {
                 if (cc < bd.mync) {
@@ -529,51 +640,42 @@ bwd_key_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant_
                     uint32_t w[4];
 #pragma unroll
                     for (int e = 0; e < 8; e += 2) {
-                        const int c0 = col + e, c1 = col + e + 1;
-                        const uint32_t v0 =
-                            (c0 >= clo && c0 <= chi) ? __ldg(pm + (j0 + c0) * W + (i - c0 + W - 1)) : 0u;
-                        const uint32_t v1 =
-                            (c1 >= clo && c1 <= chi) ? __ldg(pm + (j0 + c1) * W + (i - c1 + W - 1)) : 0u;
+                        const uint32_t c0 = (uint32_t)(col + e), c1 = c0 + 1;
+                        const uint32_t v0 = (c0 - span_lo <= span_n) ? stage[c0 * W + (i - (int)c0 + W - 1)] : 0u;
+                        const uint32_t v1 = (c1 - span_lo <= span_n) ? stage[c1 * W + (i - (int)c1 + W - 1)] : 0u;
                         w[e >> 1] = v0 | (v1 << 16);
                     }
                     *(uint4 *)(atile + sw128_offset(i, col)) = make_uint4(w[0], w[1], w[2], w[3]);
                 }
             }
-            const uint4 z4 = make_uint4(0, 0, 0, 0);
-            const int ce = bd.cb + bd.nch * 8;
-            if (split == 0) {
-                for (int col = 0; col < bd.cb && col < span; col += 8) *(uint4 *)(atile + sw128_offset(i, col)) = z4;
-            } else {
-                for (int col = (ce > bd.cb ? ce : bd.cb); col < span; col += 8)
-                    *(uint4 *)(atile + sw128_offset(i, col)) = z4;
-            }
+            zero_outside_band(atile, i, split, bd, span);
         }
         ptx::fence_proxy_async_smem();
         ptx::mbar_arrive(&bars[kKBarPt]);
 
-        // scale the rows of dO_h (buffer h & 1) by g[t, h] in place
+        // Scale the rows of dO_h (buffer h & 1) by g[t, h] in place.  Eight threads
+        // share one 128-byte row (one 16-byte chunk each), so every quarter warp
+        // touches one row: no bank conflicts.
         auto scale_do = [&](int h) {
             const int b = h & 1;
             wait_bar(&bars[kKBarLd + b], (uint32_t)(h >> 1) & 1, abort_flag);
             uint8_t *tile = sm + (b ? L.rb1 : L.rb0);
             const int rows = span * (D / 64);
-            for (int hr = tid; hr < rows; hr += kComputeThreads) {
+            const int chunk = tid & 7;
+            for (int hr = tid >> 3; hr < rows; hr += kComputeThreads / 8) {
                 const int r = hr % span;
                 const int64_t tr = j0 + r;
                 const float gv = (tr < s.N) ? __ldg(a.g + tr * H + h) : 0.f;
-                uint4 *row = (uint4 *)(tile + (hr / span) * span * 128 + r * 128);
+                uint4 *p = (uint4 *)(tile + (hr / span) * span * 128 + r * 128) + chunk;
+                uint4 v = *p;
+                uint32_t *u = &v.x;
 #pragma unroll
-                for (int k = 0; k < 8; ++k) {
-                    uint4 v = row[k];
-                    uint32_t *u = &v.x;
-#pragma unroll
-                    for (int e = 0; e < 4; ++e) {
-                        const float f0 = __uint_as_float(u[e] << 16) * gv;
-                        const float f1 = __uint_as_float(u[e] & 0xFFFF0000u) * gv;
-                        u[e] = pack_bf16x2(f0, f1);
-                    }
-                    row[k] = v;
+                for (int e = 0; e < 4; ++e) {
+                    const float f0 = __uint_as_float(u[e] << 16) * gv;
+                    const float f1 = __uint_as_float(u[e] & 0xFFFF0000u) * gv;
+                    u[e] = pack_bf16x2(f0, f1);
                 }
+                *p = v;
             }
             ptx::fence_proxy_async_smem();
             ptx::mbar_arrive(&bars[kKBarScaled + b]);
@@ -582,26 +684,7 @@ bwd_key_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant_
             const int b = idx & 1;
             wait_bar(&bars[kKBarAccFull + b], (uint32_t)(idx >> 1) & 1, abort_flag);
             ptx::tc_fence_after();
-            const int cbase = split * (D / 2);
-#pragma unroll
-            for (int c16 = 0; c16 < D / 32; ++c16) {
-                float u[16];
-                ptx::tmem_ld16(tmem + lane_base + 256 + 128 * b + cbase + c16 * 16, u);
-                if (validk) {
-                    uint4 w0, w1;
-                    w0.x = pack_bf16x2(mult * u[0], mult * u[1]);
-                    w0.y = pack_bf16x2(mult * u[2], mult * u[3]);
-                    w0.z = pack_bf16x2(mult * u[4], mult * u[5]);
-                    w0.w = pack_bf16x2(mult * u[6], mult * u[7]);
-                    w1.x = pack_bf16x2(mult * u[8], mult * u[9]);
-                    w1.y = pack_bf16x2(mult * u[10], mult * u[11]);
-                    w1.z = pack_bf16x2(mult * u[12], mult * u[13]);
-                    w1.w = pack_bf16x2(mult * u[14], mult * u[15]);
-                    uint4 *dst = (uint4 *)(out + (j * H + h) * D + cbase + c16 * 16);
-                    dst[0] = w0;
-                    dst[1] = w1;
-                }
-            }
+            drain_row<D>(tmem + lane_base + 256 + 128 * b, out + (j * H + h) * D, mult, validk, split);
             ptx::tc_fence_before();
             ptx::mbar_arrive(&bars[kKBarAccFree + b]);
         };
@@ -621,9 +704,9 @@ bwd_key_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant_
                 const int col = bd.cb + (bd.c0 + cc) * 8;
 #pragma unroll
                 for (int e = 0; e < 8; ++e) {
-                    const int cidx = col + e;
-                    dPT[cc][e] = (cidx >= clo && cidx <= chi) ? __ldg(a.band + (j0 + cidx) * W + (i - cidx + W - 1))
-                                                             : 0.f;
+                    const uint32_t cidx = (uint32_t)(col + e);
+                    dPT[cc][e] = (cidx - span_lo <= span_n)
+                                     ? __ldg(a.band + (j0 + (int)cidx) * W + (i - (int)cidx + W - 1)) : 0.f;
                 }
             }
         }
@@ -638,39 +721,57 @@ bwd_key_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant_
                 cv[512 + cidx] = ok ? __ldg(a.dc_in + tq * H + h) : 0.f;
             }
             compute_sync();
+            // drain the previous head's dK (its MMA ran while this head's S^T was computed),
+            // which also frees the ds^T tile for this head
+            if (h >= 1) drain(H + h - 1, a.dk, h - 1, s.scale);
             wait_bar(&bars[kKBarXFull], (uint32_t)h & 1, abort_flag);
             ptx::tc_fence_after();
+            uint32_t dsp[MAXC][4];   // ds^T as packed bf16 pairs
+            constexpr int G2 = (MAXC + 1) / 2;   // the band of S^T_h in two TMEM round trips
 #pragma unroll
-            for (int cc = 0; cc < MAXC; ++cc) {
-                if (cc < bd.mync) {
-                    const int col = bd.cb + (bd.c0 + cc) * 8;
-                    float x[8];
-                    ptx::tmem_ld8(tmem + lane_base + col, x);
-                    uint32_t w[4];
+            for (int g0 = 0; g0 < MAXC; g0 += G2) {
+                uint32_t xr[G2][8];
 #pragma unroll
-                    for (int e = 0; e < 8; e += 2) {
-                        float dsv[2];
+                for (int gi = 0; gi < G2; ++gi) {
+                    const int cc = g0 + gi;
+                    if (cc < MAXC && cc < bd.mync)
+                        ptx::tmem_ld8_issue(tmem + lane_base + bd.cb + (bd.c0 + cc) * 8, xr[gi]);
+                }
+                ptx::tmem_wait_ld();
 #pragma unroll
-                        for (int u = 0; u < 2; ++u) {
-                            const int cidx = col + e + u;
-                            float v = 0.f;
-                            if (cidx >= clo && cidx <= chi) {
-                                const float p = ex2(x[e + u] * sl2 - cv[cidx]);
-                                v = cv[256 + cidx] * p * (dPT[cc][e + u] - cv[512 + cidx]);
+                for (int gi = 0; gi < G2; ++gi) {
+                    const int cc = g0 + gi;
+                    if (cc < MAXC && cc < bd.mync) {
+                        ptx::reg_fence8(xr[gi]);
+                        const int col = bd.cb + (bd.c0 + cc) * 8;
+#pragma unroll
+                        for (int e = 0; e < 8; e += 2) {
+                            float dsv[2];
+#pragma unroll
+                            for (int u = 0; u < 2; ++u) {
+                                const uint32_t cidx = (uint32_t)(col + e + u);
+                                const float p = ex2(__uint_as_float(xr[gi][e + u]) * sl2 - cv[cidx]);
+                                const float v = cv[256 + cidx] * p * (dPT[cc][e + u] - cv[512 + cidx]);
+                                dsv[u] = (cidx - span_lo <= span_n) ? v : 0.f;
                             }
-                            dsv[u] = v;
+                            dsp[cc][e >> 1] = pack_bf16x2(dsv[0], dsv[1]);
                         }
-                        w[e >> 1] = pack_bf16x2(dsv[0], dsv[1]);
                     }
-                    *(uint4 *)(dtile + sw128_offset(i, col)) = make_uint4(w[0], w[1], w[2], w[3]);
                 }
             }
             ptx::tc_fence_before();
             ptx::mbar_arrive(&bars[kKBarXFree]);
+#pragma unroll
+            for (int cc = 0; cc < MAXC; ++cc) {
+                if (cc < bd.mync) {
+                    const int col = bd.cb + (bd.c0 + cc) * 8;
+                    *(uint4 *)(dtile + sw128_offset(i, col)) = make_uint4(dsp[cc][0], dsp[cc][1], dsp[cc][2], dsp[cc][3]);
+                }
+            }
             ptx::fence_proxy_async_smem();
             ptx::mbar_arrive(&bars[kKBarDs]);
-            drain(H + h, a.dk, h, s.scale);
         }
+        drain(2 * H - 1, a.dk, H - 1, s.scale);
     }
 
     ptx::tc_fence_before();

@@ -8,11 +8,34 @@
 namespace dc {
 namespace tc {
 
-// 8 compute warps (two per TMEM lane quarter) + 1 producer warp (TMA + MMA issue).
-constexpr int kComputeWarps = 8;
+// Four warpgroups: warpgroups 0-2 are the 12 compute warps, three per TMEM lane
+// quarter (warp w reads lanes 32*(w%4) .. +31 and takes part w/4 of the
+// quarter's columns); warp 12 (warpgroup 3) issues TMA and MMA, warps 13-15
+// only lend their registers.  The kernels launch with 128 registers per thread
+// (512 threads fill the 64K register file); warpgroup 3 then drops to
+// kRegsProducer and the compute warpgroups rise to kRegsCompute, which sums to
+// the launch budget (a larger sum would make setmaxnreg.inc wait forever).
+// The build checks that ptxas gives every tcgen05 kernel exactly kLaunchRegs.
+constexpr int kSplits = 3;
+constexpr int kComputeWarps = 4 * kSplits;
 constexpr int kComputeThreads = kComputeWarps * 32;
-constexpr int kThreads = kComputeThreads + 32;
+constexpr int kThreads = kComputeThreads + 128;
 constexpr int kProducerWarp = kComputeWarps;
+constexpr int kLaunchRegs = 128;
+constexpr int kRegsProducer = 80;
+constexpr int kRegsCompute = 144;
+static_assert(kThreads * kLaunchRegs <= 65536, "launch register budget exceeds the register file");
+static_assert(kComputeThreads * kRegsCompute + (kThreads - kComputeThreads) * kRegsProducer <= kThreads * kLaunchRegs,
+              "register split exceeds the launch budget");
+static_assert(kRegsCompute % 8 == 0 && kRegsProducer % 8 == 0 && kRegsProducer >= 24 && kRegsCompute <= 256,
+              "setmaxnreg counts must be multiples of 8 in [24, 256]");
+
+__device__ __forceinline__ void regs_producer() {
+    asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kRegsProducer));
+}
+__device__ __forceinline__ void regs_compute() {
+    asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kRegsCompute));
+}
 constexpr uint64_t kWaitNs = 2000000000ull;   // a legitimate wait lasts microseconds
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kLn2 = 0.6931471805599453f;
@@ -46,8 +69,8 @@ __device__ __forceinline__ bool wait_bar(uint64_t *bar, uint32_t parity, volatil
 __device__ __forceinline__ void named_sync(int id, int nthreads) {
     asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
 }
-// The two compute warps that share TMEM lane quarter q.
-__device__ __forceinline__ void pair_sync(int q) { named_sync(1 + q, 64); }
+// The compute warps that share TMEM lane quarter q.
+__device__ __forceinline__ void pair_sync(int q) { named_sync(1 + q, 32 * kSplits); }
 // All compute warps.
 __device__ __forceinline__ void compute_sync() { named_sync(5, kComputeThreads); }
 
@@ -65,12 +88,12 @@ __device__ __forceinline__ uint32_t sw128_offset(int row, int col) {
 // Column band of TMEM lane quarter q in a [128 x span] score tile whose column
 // c holds key kbase + c (kbase = block start - (W - 1)): rows 32q .. 32q+31
 // (those below `rows`) need columns [32q, 32q + rows_q - 1 + W - 1].  Split in
-// 8-column chunks between the two warps of the quarter.
+// 8-column chunks between the kSplits warps of the quarter.
 struct Band {
     int cb;      // first column of the quarter's band
     int nch;     // chunks of 8 columns in the band
-    int c0;      // first chunk of this thread's half
-    int mync;    // chunks in this thread's half
+    int c0;      // first chunk of this thread's part
+    int mync;    // chunks in this thread's part
 };
 
 __device__ __forceinline__ Band make_band(int q, int split, int rows, int W, int span) {
@@ -85,10 +108,29 @@ __device__ __forceinline__ Band make_band(int q, int split, int rows, int W, int
         if (ce > span) ce = span;
         b.nch = (ce - b.cb) >> 3;
     }
-    const int half = (b.nch + 1) >> 1;
-    b.c0 = split * half;
-    b.mync = max(0, min(b.nch - b.c0, half));
+    const int per = (b.nch + kSplits - 1) / kSplits;
+    b.c0 = split * per;
+    b.mync = max(0, min(b.nch - b.c0, per));
     return b;
+}
+
+// Zero the columns of tile row `row` outside its quarter's band (split 0 takes the
+// columns before the band, the last split those after it).
+__device__ __forceinline__ void zero_outside_band(uint8_t *tile, int row, int split, const Band &bd, int span) {
+    const uint4 z4 = make_uint4(0, 0, 0, 0);
+    const int ce = bd.cb + bd.nch * 8;
+    if (split == 0) {
+        for (int col = 0; col < bd.cb && col < span; col += 8) *(uint4 *)(tile + sw128_offset(row, col)) = z4;
+    } else if (split == kSplits - 1) {
+        for (int col = (ce > bd.cb ? ce : bd.cb); col < span; col += 8) *(uint4 *)(tile + sw128_offset(row, col)) = z4;
+    }
+}
+
+// 16-column chunks [begin, end) of a D-column accumulator row drained by this split.
+__device__ __forceinline__ void acc_split(int split, int nchunk16, int &begin, int &end) {
+    const int per = (nchunk16 + kSplits - 1) / kSplits;
+    begin = min(split * per, nchunk16);
+    end = min(begin + per, nchunk16);
 }
 
 }  // namespace tc

@@ -11,14 +11,15 @@
 //   SIMT    pull the row band of S_h into registers (which frees the S columns
 //           for the next head's MMA), mask to the causal window inside the
 //           document, softmax per row, P += c[t,h] * p_h with P accumulated in
-//           TMEM columns [256, 256 + span) (the H maps never leave the chip)
+//           registers (the H maps never leave the chip); V_h is prefetched
+//           into L2 meanwhile
 // Phase 2:
 //   SIMT    P -> bf16 tile in smem (K-major, swizzled), band copy -> pmap
 //   per head: TMA V_h [span x d]; MMA U_h = P V_h -> TMEM [128 x d];
 //           SIMT o_h = g[t,h] * U_h -> bf16 -> global
 //
-// Warps 0-7 do the SIMT work: warp w reads TMEM lanes 32*(w%4).. (rows of
-// the tile) and half (w/4) of its quarter's column band.  Warp 8 lane 0
+// Warps 0-11 do the SIMT work: warp w reads TMEM lanes 32*(w%4).. (rows of
+// the tile) and part w/4 of its quarter's column band.  Warp 12 lane 0
 // issues every TMA and MMA.  All waits are bounded (see wait_bar).
 #pragma once
 
@@ -40,7 +41,7 @@ struct FwdLayout {
     // the P tile reuses the Q buffers when they are large enough (free after the last S MMA)
     static constexpr uint32_t kP = (2 * kQBytes >= kPBytes) ? 0u : kK1 + kKBytes;
     static constexpr uint32_t kRed = (kP == 0 ? kK1 + kKBytes : kP + kPBytes);
-    static constexpr uint32_t kBars = kRed + 2 * 2 * 128 * 4;
+    static constexpr uint32_t kBars = kRed + 2 * kSplits * 128 * 4;
     static constexpr uint32_t kBytes = kBars + 256;
     static constexpr uint32_t kAlloc = kBytes + 1024;        // slack to align the base to 1 KiB
 };
@@ -70,8 +71,8 @@ fwd_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__ CU
     uint64_t *bars = (uint64_t *)(sm + L::kBars);
     uint32_t *tmem_slot = (uint32_t *)(bars + 16);
     volatile int *abort_flag = (volatile int *)(tmem_slot + 1);
-    float *red_max = (float *)(sm + L::kRed);     // [2][128]
-    float *red_sum = red_max + 256;               // [2][128]
+    float *red_max = (float *)(sm + L::kRed);     // [kSplits][128]
+    float *red_sum = red_max + kSplits * 128;     // [kSplits][128]
 
     const Shape &s = a.s;
     const int H = s.H, W = s.W, BM = a.BM, span = a.span;
@@ -99,8 +100,9 @@ fwd_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__ CU
     ptx::tc_fence_after();
     const uint32_t tmem = *tmem_slot;
 
-    if (warp == kProducerWarp) {
-        if (lane == 0) {
+    if (warp >= kProducerWarp) {
+        regs_producer();
+        if (warp == kProducerWarp && lane == 0) {
             ptx::prefetch_tensormap(&map_q);
             ptx::prefetch_tensormap(&map_k);
             ptx::prefetch_tensormap(&map_v);
@@ -144,6 +146,8 @@ fwd_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__ CU
                     }
                 }
                 ptx::mma_commit(&bars[kBarSFull]);
+                // V_h is not needed before phase 2; pull it into L2 now, while HBM has slack
+                for (int kb = 0; kb < D / 64; ++kb) ptx::tma_prefetch_l2_2d(&map_v, h * D + kb * 64, (int)kbase);
                 if (h + 2 < H) {
                     if (wait_bar(&bars[kBarSFull], (uint32_t)h & 1, abort_flag)) issue_qk(h + 2);
                 }
@@ -177,6 +181,7 @@ fwd_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__ CU
         }
         __syncwarp();
     } else {
+        regs_compute();
         // ---------------------------------------------------------------- compute warps
         const int q = warp & 3, split = warp >> 2;
         const int i = 32 * q + lane;                   // tile row = TMEM lane
@@ -192,33 +197,49 @@ fwd_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__ CU
         const float sl2 = s.scale * kLog2e;
 
         const uint32_t s_cols = tmem + lane_base;          // S_h, columns [0, span)
-        const uint32_t p_cols = tmem + lane_base + 256;    // P, columns [256, 256 + span)
+
+        // composed map of this thread's band, accumulated over heads in registers
+        float P[MAXC][8];
+#pragma unroll
+        for (int cc = 0; cc < MAXC; ++cc)
+#pragma unroll
+            for (int e = 0; e < 8; ++e) P[cc][e] = 0.f;
+        // column c is in this row's window iff (unsigned)(c - span_lo) <= span_n; a row with an
+        // empty window (clo > chi: past the block or past N) gets span_lo = ~0u, so no c passes
+        const uint32_t span_lo = (chi >= clo) ? (uint32_t)clo : ~0u;
+        const uint32_t span_n = (chi >= clo) ? (uint32_t)(chi - clo) : 0u;
 
         for (int h = 0; h < H; ++h) {
             wait_bar(&bars[kBarSFull], (uint32_t)h & 1, abort_flag);
             ptx::tc_fence_after();
-            float x[MAXC][8];
+            // pull this thread's band of S_h into registers with one wait
+            uint32_t xr[MAXC][8];
+#pragma unroll
+            for (int cc = 0; cc < MAXC; ++cc)
+                if (cc < bd.mync) ptx::tmem_ld8_issue(s_cols + bd.cb + (bd.c0 + cc) * 8, xr[cc]);
+            ptx::tmem_wait_ld();
             float mloc = -INFINITY;
 #pragma unroll
             for (int cc = 0; cc < MAXC; ++cc) {
                 if (cc < bd.mync) {
-                    const int col = bd.cb + (bd.c0 + cc) * 8;
-                    ptx::tmem_ld8(s_cols + col, x[cc]);
+                    ptx::reg_fence8(xr[cc]);
+                    const uint32_t col = (uint32_t)(bd.cb + (bd.c0 + cc) * 8);
 #pragma unroll
                     for (int e = 0; e < 8; ++e) {
-                        const int cidx = col + e;
-                        float v = x[cc][e] * sl2;
-                        v = (cidx >= clo && cidx <= chi) ? v : -INFINITY;
-                        x[cc][e] = v;
+                        float v = __uint_as_float(xr[cc][e]) * sl2;
+                        v = (col + e - span_lo <= span_n) ? v : -INFINITY;
+                        xr[cc][e] = __float_as_uint(v);
                         mloc = fmaxf(mloc, v);
                     }
                 }
             }
             ptx::tc_fence_before();
-            ptx::mbar_arrive(&bars[kBarSFree]);
+            ptx::mbar_arrive(&bars[kBarSFree]);   // S columns free for the next head's MMA
             red_max[split * 128 + i] = mloc;
             pair_sync(q);
-            float m = fmaxf(red_max[i], red_max[128 + i]);
+            float m = red_max[i];
+#pragma unroll
+            for (int sp = 1; sp < kSplits; ++sp) m = fmaxf(m, red_max[sp * 128 + i]);
             if (!valid) m = 0.f;
             float zl = 0.f;
 #pragma unroll
@@ -226,32 +247,23 @@ fwd_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__ CU
                 if (cc < bd.mync) {
 #pragma unroll
                     for (int e = 0; e < 8; ++e) {
-                        const float ev = ex2(x[cc][e] - m);
-                        x[cc][e] = ev;
+                        const float ev = ex2(__uint_as_float(xr[cc][e]) - m);
+                        xr[cc][e] = __float_as_uint(ev);
                         zl += ev;
                     }
                 }
             }
             red_sum[split * 128 + i] = zl;
             pair_sync(q);
-            const float Z = red_sum[i] + red_sum[128 + i];
+            float Z = red_sum[i];
+#pragma unroll
+            for (int sp = 1; sp < kSplits; ++sp) Z += red_sum[sp * 128 + i];
             const float coef = valid ? __ldg(a.c + t * H + h) / Z : 0.f;
 #pragma unroll
-            for (int cc = 0; cc < MAXC; ++cc) {
-                if (cc < bd.mync) {
-                    const int col = bd.cb + (bd.c0 + cc) * 8;
-                    float pc[8];
-                    if (h == 0) {
+            for (int cc = 0; cc < MAXC; ++cc)
+                if (cc < bd.mync)
 #pragma unroll
-                        for (int e = 0; e < 8; ++e) pc[e] = coef * x[cc][e];
-                    } else {
-                        ptx::tmem_ld8(p_cols + col, pc);
-#pragma unroll
-                        for (int e = 0; e < 8; ++e) pc[e] = fmaf(coef, x[cc][e], pc[e]);
-                    }
-                    ptx::tmem_st8(p_cols + col, pc);
-                }
-            }
+                    for (int e = 0; e < 8; ++e) P[cc][e] = fmaf(coef, __uint_as_float(xr[cc][e]), P[cc][e]);
             if (split == 0 && valid && a.lse) a.lse[t * H + h] = (m + __log2f(Z)) * kLn2;
         }
 
@@ -261,69 +273,80 @@ fwd_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__ CU
         for (int cc = 0; cc < MAXC; ++cc) {
             if (cc < bd.mync) {
                 const int col = bd.cb + (bd.c0 + cc) * 8;
-                float pc[8];
-                ptx::tmem_ld8(p_cols + col, pc);
                 uint4 w4;
-                w4.x = pack_bf16x2(pc[0], pc[1]);
-                w4.y = pack_bf16x2(pc[2], pc[3]);
-                w4.z = pack_bf16x2(pc[4], pc[5]);
-                w4.w = pack_bf16x2(pc[6], pc[7]);
+                w4.x = pack_bf16x2(P[cc][0], P[cc][1]);
+                w4.y = pack_bf16x2(P[cc][2], P[cc][3]);
+                w4.z = pack_bf16x2(P[cc][4], P[cc][5]);
+                w4.w = pack_bf16x2(P[cc][6], P[cc][7]);
                 *(uint4 *)(ptile + sw128_offset(i, col)) = w4;
             }
         }
-        ptx::tc_fence_before();
-        {
-            const uint4 z4 = make_uint4(0, 0, 0, 0);
-            const int ce = bd.cb + bd.nch * 8;
-            if (split == 0) {
-                for (int col = 0; col < bd.cb && col < span; col += 8) *(uint4 *)(ptile + sw128_offset(i, col)) = z4;
-            } else {
-                for (int col = (ce > bd.cb ? ce : bd.cb); col < span; col += 8)
-                    *(uint4 *)(ptile + sw128_offset(i, col)) = z4;
-            }
-        }
+        zero_outside_band(ptile, i, split, bd, span);
         ptx::fence_proxy_async_smem();
         ptx::mbar_arrive(&bars[kBarP]);
 
-        // ---- band copy of P to pmap[t][w] = P(t, t-W+1+w): tile column i + w of row i
+        // ---- band copy of P to pmap[t][w] = P(t, t-W+1+w) = tile(r, r + w)
         if (a.pmap) {
             compute_sync();
-            for (int r = warp; r < BM; r += kComputeWarps) {
-                const int64_t tr = t0 + r;
-                if (tr >= s.N) break;
-                __nv_bfloat16 *dst = a.pmap + tr * W;
-                for (int w = lane; w < W; w += 32) {
-                    const uint16_t bits = *(const uint16_t *)(ptile + sw128_offset(r, r + w));
-                    reinterpret_cast<uint16_t *>(dst)[w] = bits;
+            if ((W & 7) == 0) {
+                // 16-byte stores: lane l writes w in [8l, 8l + 8) of one row
+                const int nl = W >> 3;
+                for (int r0 = warp * (32 / nl > 0 ? 32 / nl : 1); r0 < BM; r0 += kComputeWarps * (32 / nl > 0 ? 32 / nl : 1)) {
+                    const int rows_per_iter = 32 / nl > 0 ? 32 / nl : 1;
+                    for (int l0 = lane; l0 < rows_per_iter * nl; l0 += 32) {
+                        const int r = r0 + l0 / nl, wl = (l0 % nl) * 8;
+                        if (r >= BM || t0 + r >= s.N) continue;
+                        uint32_t w[4];
+#pragma unroll
+                        for (int e = 0; e < 4; ++e) {
+                            const uint32_t lo = *(const uint16_t *)(ptile + sw128_offset(r, r + wl + 2 * e));
+                            const uint32_t hi = *(const uint16_t *)(ptile + sw128_offset(r, r + wl + 2 * e + 1));
+                            w[e] = lo | (hi << 16);
+                        }
+                        *(uint4 *)(a.pmap + (t0 + r) * W + wl) = make_uint4(w[0], w[1], w[2], w[3]);
+                    }
+                }
+            } else {
+                for (int r = warp; r < BM; r += kComputeWarps) {
+                    const int64_t tr = t0 + r;
+                    if (tr >= s.N) break;
+                    __nv_bfloat16 *dst = a.pmap + tr * W;
+                    for (int w = lane; w < W; w += 32) {
+                        const uint16_t bits = *(const uint16_t *)(ptile + sw128_offset(r, r + w));
+                        reinterpret_cast<uint16_t *>(dst)[w] = bits;
+                    }
                 }
             }
         }
 
-        // ---- epilogue: o_h = g[t,h] * U_h
-        const int cbase = split * (D / 2);
+        // ---- epilogue: o_h = g[t,h] * U_h; this split drains 16-column chunks [cb16, ce16)
+        int cb16, ce16;
+        acc_split(split, D / 16, cb16, ce16);
+        constexpr int kMaxC16 = (D / 16 + kSplits - 1) / kSplits;
         for (int h = 0; h < H; ++h) {
             const int b = h & 1;
             const uint32_t n = (uint32_t)(h >> 1);
             wait_bar(&bars[kBarUFull + b], n & 1, abort_flag);
             ptx::tc_fence_after();
             const float gh = valid ? __ldg(a.g + t * H + h) : 0.f;
+            uint32_t ur[kMaxC16][16];
 #pragma unroll
-            for (int c16 = 0; c16 < D / 32; ++c16) {
-                float u[16];
-                ptx::tmem_ld16(tmem + lane_base + b * 256 + cbase + c16 * 16, u);
-                if (valid) {
-                    uint4 w0, w1;
-                    w0.x = pack_bf16x2(gh * u[0], gh * u[1]);
-                    w0.y = pack_bf16x2(gh * u[2], gh * u[3]);
-                    w0.z = pack_bf16x2(gh * u[4], gh * u[5]);
-                    w0.w = pack_bf16x2(gh * u[6], gh * u[7]);
-                    w1.x = pack_bf16x2(gh * u[8], gh * u[9]);
-                    w1.y = pack_bf16x2(gh * u[10], gh * u[11]);
-                    w1.z = pack_bf16x2(gh * u[12], gh * u[13]);
-                    w1.w = pack_bf16x2(gh * u[14], gh * u[15]);
-                    uint4 *dst = (uint4 *)(a.o + (t * H + h) * D + cbase + c16 * 16);
-                    dst[0] = w0;
-                    dst[1] = w1;
+            for (int c = 0; c < kMaxC16; ++c)
+                if (cb16 + c < ce16) ptx::tmem_ld16_issue(tmem + lane_base + b * 256 + (cb16 + c) * 16, ur[c]);
+            ptx::tmem_wait_ld();
+#pragma unroll
+            for (int c = 0; c < kMaxC16; ++c) {
+                if (cb16 + c < ce16) {
+                    ptx::reg_fence16(ur[c]);
+                    if (valid) {
+                        uint32_t w[8];
+#pragma unroll
+                        for (int e = 0; e < 8; ++e)
+                            w[e] = pack_bf16x2(gh * __uint_as_float(ur[c][2 * e]), gh * __uint_as_float(ur[c][2 * e + 1]));
+                        uint4 *dst = (uint4 *)(a.o + (t * H + h) * D + (cb16 + c) * 16);
+                        dst[0] = make_uint4(w[0], w[1], w[2], w[3]);
+                        dst[1] = make_uint4(w[4], w[5], w[6], w[7]);
+                    }
                 }
             }
             ptx::tc_fence_before();

@@ -81,12 +81,13 @@ inline int choose_block(int64_t N, int W, int sms, int max_span = 256) {
 }
 
 // register-array width of the softmax warps: chunks of 8 columns per thread
+// (a quarter's band of 31 + W columns split between kSplits warps)
 inline int maxc_for(int W) {
-    const int need = (((31 + W + 7) / 8) + 1) / 2;
+    const int need = (((31 + W + 7) / 8) + kSplits - 1) / kSplits;
+    if (need <= 3) return 3;
     if (need <= 4) return 4;
     if (need <= 6) return 6;
-    if (need <= 9) return 9;
-    return 10;
+    return 7;
 }
 
 template <typename K>
@@ -109,10 +110,10 @@ template <int D>
 inline cudaError_t launch_fwd_d(int maxc, const CUtensorMap &mq, const CUtensorMap &mk, const CUtensorMap &mv,
                                 const FwdArgs &a, cudaStream_t st) {
     switch (maxc) {
+        case 3: return launch_fwd<D, 3>(mq, mk, mv, a, st);
         case 4: return launch_fwd<D, 4>(mq, mk, mv, a, st);
         case 6: return launch_fwd<D, 6>(mq, mk, mv, a, st);
-        case 9: return launch_fwd<D, 9>(mq, mk, mv, a, st);
-        default: return launch_fwd<D, 10>(mq, mk, mv, a, st);
+        default: return launch_fwd<D, 7>(mq, mk, mv, a, st);
     }
 }
 
@@ -138,8 +139,6 @@ inline cudaError_t fwd(const Shape &s, const void *q, const void *k, const void 
     return e;
 }
 
-constexpr bool kHasBwd = true;
-
 template <int D, int MAXC>
 inline cudaError_t launch_bwd_query(const CUtensorMap &mq, const CUtensorMap &mk, const CUtensorMap &mv,
                                     const CUtensorMap &mdo, const BwdArgs &a, cudaStream_t st) {
@@ -156,7 +155,9 @@ template <int D, int MAXC>
 inline cudaError_t launch_bwd_key(const CUtensorMap &mq, const CUtensorMap &mk, const CUtensorMap &mdo,
                                   const BwdArgs &a, cudaStream_t st) {
     auto kern = bwd_key_kernel<D, MAXC>;
-    const uint32_t smem = KSideLayout<D>(a.span).bytes + 1024;
+    const KSideLayout<D> L(a.span, a.s.W);
+    if (L.stage + L.stage_bytes > L.colv) return cudaErrorInvalidValue;   // staging must fit before colv
+    const uint32_t smem = L.bytes + 1024;
     cudaError_t e = set_smem(kern, smem);
     if (e != cudaSuccess) return e;
     const unsigned grid = (unsigned)((a.s.N + a.BM - 1) / a.BM);
@@ -166,10 +167,10 @@ inline cudaError_t launch_bwd_key(const CUtensorMap &mq, const CUtensorMap &mk, 
 
 #define DC_TC_MAXC_SWITCH(maxc, CALL)        \
     switch (maxc) {                          \
+        case 3: { constexpr int MC = 3; return CALL; }   \
         case 4: { constexpr int MC = 4; return CALL; }   \
         case 6: { constexpr int MC = 6; return CALL; }   \
-        case 9: { constexpr int MC = 9; return CALL; }   \
-        default: { constexpr int MC = 10; return CALL; } \
+        default: { constexpr int MC = 7; return CALL; }  \
     }
 
 inline BwdArgs bwd_args(const Shape &s) {
