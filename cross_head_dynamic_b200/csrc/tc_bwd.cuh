@@ -51,9 +51,11 @@ struct BwdArgs {
 };
 
 // Drain this split's 16-column chunks of one row of a [128 x D] fp32 accumulator
-// (row base address taddr, output row dst): scale, round to bf16, store when `store`.
+// (row base address taddr, output row dst): scale, round to bf16, store when `store`
+// (full 32-byte sectors; aligned32 says whether the output buffer allows 256-bit stores).
 template <int D>
-__device__ __forceinline__ void drain_row(uint32_t taddr, __nv_bfloat16 *dst, float mult, bool store, int split) {
+__device__ __forceinline__ void drain_row(uint32_t taddr, __nv_bfloat16 *dst, float mult, bool store, int split,
+                                          bool aligned32) {
     int cb16, ce16;
     acc_split(split, D / 16, cb16, ce16);
     constexpr int kMaxC16 = (D / 16 + kSplits - 1) / kSplits;
@@ -69,9 +71,7 @@ __device__ __forceinline__ void drain_row(uint32_t taddr, __nv_bfloat16 *dst, fl
 #pragma unroll
                 for (int e = 0; e < 8; ++e)
                     w[e] = pack_bf16x2(mult * __uint_as_float(r[2 * e]), mult * __uint_as_float(r[2 * e + 1]));
-                uint4 *p = (uint4 *)(dst + (cb16 + c) * 16);
-                p[0] = make_uint4(w[0], w[1], w[2], w[3]);
-                p[1] = make_uint4(w[4], w[5], w[6], w[7]);
+                ptx::st_global_32b(dst + (cb16 + c) * 16, w, aligned32);
             }
         }
     }
@@ -79,7 +79,28 @@ __device__ __forceinline__ void drain_row(uint32_t taddr, __nv_bfloat16 *dst, fl
 
 // --------------------------------------------------------------------------- query side
 enum : int { kQBarLd = 0, kQBarQ = 2, kQBarK = 3, kQBarXFull = 5, kQBarXFree = 6, kQBarDs = 7, kQBarDqFull = 8,
-             kQBarDqFree = 10, kQNumBars = 12 };
+             kQBarDqFree = 10, kQBarPmap = 12, kQNumBars = 13 };
+
+// Copy `bytes` bytes of global memory to shared memory: a bulk copy of the 16-byte
+// multiple (completing on `bar`) and plain copies of the rest.  The caller's arrive on
+// `bar` (expect_tx) publishes both.
+__device__ __forceinline__ void stage_in(void *sdst, const void *gsrc, uint32_t bytes, uint64_t *bar) {
+    const uint32_t main = bytes & ~15u;
+    for (uint32_t x = main; x < bytes; x += 2)
+        *(uint16_t *)((uint8_t *)sdst + x) = *(const uint16_t *)((const uint8_t *)gsrc + x);
+    ptx::mbar_arrive_expect_tx(bar, main);
+    if (main) ptx::bulk_load(sdst, gsrc, main, bar);
+}
+
+// Copy `bytes` bytes of shared memory to global memory: a bulk copy of the 16-byte
+// multiple (committed to this thread's bulk group) and plain copies of the rest.
+__device__ __forceinline__ void stage_out(void *gdst, const void *ssrc, uint32_t bytes) {
+    const uint32_t main = bytes & ~15u;
+    for (uint32_t x = main; x < bytes; x += 2)
+        *(uint16_t *)((uint8_t *)gdst + x) = *(const uint16_t *)((const uint8_t *)ssrc + x);
+    if (main) ptx::bulk_store(gdst, ssrc, main);
+    ptx::bulk_commit();
+}
 
 template <int D>
 struct QSideLayout {
@@ -181,6 +202,10 @@ bwd_query_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
                 ptx::mma_commit(&bars[kQBarDqFull + b]);
             };
 
+            // the CTA's pmap rows (one contiguous [BM][W] run) into the upper half of the ds
+            // tile region, which phase 1 does not use
+            stage_in(sm + L.rd + 32768, a.pmap + t0 * W, (uint32_t)(min((int64_t)BM, s.N - t0) * W * 2),
+                     &bars[kQBarPmap]);
             // ---- phase 1: E_h = dO_h V_h^T
             for (int h = 0; h < H && h < 2; ++h) issue_e(h);
             for (int h = 0; h < H; ++h) {
@@ -256,18 +281,9 @@ bwd_query_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
         const uint32_t x_cols = tmem + lane_base;
         const float sl2 = s.scale * kLog2e;
 
-        // Stage the CTA's pmap rows (one contiguous [BM][W] block) in the upper half of the
-        // ds tile region, unused until phase 2; P(t, c) = pmap[t][c - i].
-        uint16_t *pstage = (uint16_t *)(sm + L.rd + 32768);
-        {
-            const int64_t rows = min((int64_t)BM, s.N - t0);
-            const int64_t nh = rows * W;   // t0 * W is even
-            const uint32_t *src = reinterpret_cast<const uint32_t *>(a.pmap + t0 * W);
-            uint32_t *dst = reinterpret_cast<uint32_t *>(pstage);
-            for (int64_t x = threadIdx.x; x < nh / 2; x += kComputeThreads) dst[x] = __ldg(src + x);
-            if ((nh & 1) && threadIdx.x == 0) pstage[nh - 1] = reinterpret_cast<const uint16_t *>(a.pmap)[t0 * W + nh - 1];
-        }
-        compute_sync();
+        // the CTA's pmap rows, staged by the producer; P(t, c) = pmap[t][c - i]
+        const uint16_t *pstage = (const uint16_t *)(sm + L.rd + 32768);
+        wait_bar(&bars[kQBarPmap], 0, abort_flag);
         const uint16_t *prow = pstage + i * W - i;
         float dP[MAXC][8];
 #pragma unroll
@@ -350,15 +366,11 @@ bwd_query_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
                     }
                 }
             }
+            ptx::fence_proxy_async_smem();
             compute_sync();
-            const int64_t rows = min((int64_t)BM, s.N - t0);
-            const int64_t n = rows * W;
-            float *dst = a.band + t0 * W;
-            if ((W & 3) == 0) {
-                for (int64_t x4 = threadIdx.x; x4 < n / 4; x4 += kComputeThreads)
-                    *(float4 *)(dst + 4 * x4) = *(const float4 *)(stage + 4 * x4);
-            } else {
-                for (int64_t x = threadIdx.x; x < n; x += kComputeThreads) dst[x] = stage[x];
+            if (threadIdx.x == 0) {
+                stage_out(a.band + t0 * W, stage, (uint32_t)(min((int64_t)BM, s.N - t0) * W * 4));
+                ptx::bulk_wait_read();
             }
             compute_sync();
         }
@@ -371,7 +383,8 @@ bwd_query_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
             const int b = h & 1;
             wait_bar(&bars[kQBarDqFull + b], (uint32_t)(h >> 1) & 1, abort_flag);
             ptx::tc_fence_after();
-            drain_row<D>(tmem + lane_base + 256 + 128 * b, a.dq + (t * H + h) * D, s.scale, valid, split);
+            drain_row<D>(tmem + lane_base + 256 + 128 * b, a.dq + (t * H + h) * D, s.scale, valid, split,
+                         ((uintptr_t)a.dq & 31) == 0);
             ptx::tc_fence_before();
             ptx::mbar_arrive(&bars[kQBarDqFree + b]);
         };
@@ -443,6 +456,7 @@ bwd_query_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
         drain_dq(H - 1);
     }
 
+    if (threadIdx.x == 0) ptx::bulk_wait_all();   // the dP band copy has completed
     ptx::tc_fence_before();
     __syncthreads();
     if (warp == 0) {
@@ -453,7 +467,7 @@ bwd_query_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
 
 // --------------------------------------------------------------------------- key side
 enum : int { kKBarLd = 0, kKBarScaled = 2, kKBarPt = 4, kKBarAccFull = 5, kKBarAccFree = 7, kKBarK = 9,
-             kKBarXFull = 10, kKBarXFree = 11, kKBarDs = 12, kKNumBars = 13 };
+             kKBarXFull = 10, kKBarXFree = 11, kKBarDs = 12, kKBarPmap = 13, kKNumBars = 14 };
 
 template <int D>
 struct KSideLayout {
@@ -550,6 +564,9 @@ bwd_key_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant_
                 }
                 ptx::mma_commit(&bars[kKBarAccFull + b]);
             };
+            // pmap rows j0 .. j0+span-1 (one contiguous run) into the staging area
+            stage_in(sm + L.stage, a.pmap + j0 * W, (uint32_t)(min((int64_t)span, s.N - j0) * W * 2),
+                     &bars[kKBarPmap]);
             if (L.stage_in_b1) issue_ld(0);   // buffer 0 does not overlap the pmap staging rows
             // ---- phase 1: dV_h = P^T (g_h dO_h)
             const bool pt_ok = wait_bar(&bars[kKBarPt], 0, abort_flag);   // staging area consumed
@@ -619,17 +636,9 @@ bwd_key_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant_
         const uint32_t lane_base = (uint32_t)(32 * q) << 16;
         const float sl2 = s.scale * kLog2e;
 
-        // ---- stage pmap rows j0 .. j0+span-1 (one contiguous block) with coalesced loads
-        uint16_t *stage = (uint16_t *)(sm + L.stage);
-        {
-            const int64_t rows = min((int64_t)span, s.N - j0);
-            const int64_t nh = rows * W;                              // bf16 elements; j0 * W is even
-            const uint32_t *src = reinterpret_cast<const uint32_t *>(a.pmap + j0 * W);
-            uint32_t *dst = reinterpret_cast<uint32_t *>(stage);
-            for (int64_t x = tid; x < nh / 2; x += kComputeThreads) dst[x] = __ldg(src + x);
-            if ((nh & 1) && tid == 0) stage[nh - 1] = reinterpret_cast<const uint16_t *>(a.pmap)[j0 * W + nh - 1];
-        }
-        compute_sync();
+        // ---- pmap rows j0 .. j0+span-1, staged by the producer
+        const uint16_t *stage = (const uint16_t *)(sm + L.stage);
+        wait_bar(&bars[kKBarPmap], 0, abort_flag);
         // ---- P^T tile: P^T(i, c) = P(j0 + c, j0 + i) = pmap[j0 + c][i - c + W - 1]
         uint8_t *atile = sm + L.ra;
         {
@@ -684,7 +693,8 @@ bwd_key_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant_
             const int b = idx & 1;
             wait_bar(&bars[kKBarAccFull + b], (uint32_t)(idx >> 1) & 1, abort_flag);
             ptx::tc_fence_after();
-            drain_row<D>(tmem + lane_base + 256 + 128 * b, out + (j * H + h) * D, mult, validk, split);
+            drain_row<D>(tmem + lane_base + 256 + 128 * b, out + (j * H + h) * D, mult, validk, split,
+                         ((uintptr_t)out & 31) == 0);
             ptx::tc_fence_before();
             ptx::mbar_arrive(&bars[kKBarAccFree + b]);
         };

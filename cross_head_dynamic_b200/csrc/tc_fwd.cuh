@@ -42,8 +42,12 @@ struct FwdLayout {
     static constexpr uint32_t kP = (2 * kQBytes >= kPBytes) ? 0u : kK1 + kKBytes;
     static constexpr uint32_t kRed = (kP == 0 ? kK1 + kKBytes : kP + kPBytes);
     static constexpr uint32_t kBars = kRed + 2 * kSplits * 128 * 4;
-    static constexpr uint32_t kBytes = kBars + 256;
+    // pmap rows of the block, contiguous as in global memory, written out by one bulk copy
+    static constexpr uint32_t kStage = kBars + 256;
+    static constexpr uint32_t kStageBytes = 30u * 1024;
+    static constexpr uint32_t kBytes = kStage + kStageBytes;
     static constexpr uint32_t kAlloc = kBytes + 1024;        // slack to align the base to 1 KiB
+    static_assert(kAlloc <= 227u * 1024, "forward tile layout exceeds shared memory");
 };
 
 struct FwdArgs {
@@ -285,37 +289,42 @@ fwd_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__ CU
         ptx::fence_proxy_async_smem();
         ptx::mbar_arrive(&bars[kBarP]);
 
-        // ---- band copy of P to pmap[t][w] = P(t, t-W+1+w) = tile(r, r + w)
+        // ---- pmap[t][w] = P(t, t-W+1+w) = P at tile column i + w.  The block's rows are one
+        // contiguous run of pmap: build it in shared memory from the registers (passes of
+        // `rpp` rows when it does not fit) and write it with one bulk copy per pass.
         if (a.pmap) {
-            compute_sync();
-            if ((W & 7) == 0) {
-                // 16-byte stores: lane l writes w in [8l, 8l + 8) of one row
-                const int nl = W >> 3;
-                for (int r0 = warp * (32 / nl > 0 ? 32 / nl : 1); r0 < BM; r0 += kComputeWarps * (32 / nl > 0 ? 32 / nl : 1)) {
-                    const int rows_per_iter = 32 / nl > 0 ? 32 / nl : 1;
-                    for (int l0 = lane; l0 < rows_per_iter * nl; l0 += 32) {
-                        const int r = r0 + l0 / nl, wl = (l0 % nl) * 8;
-                        if (r >= BM || t0 + r >= s.N) continue;
-                        uint32_t w[4];
+            const int rows_blk = (int)min((int64_t)BM, s.N - t0);
+            const int rpp = min(BM, (int)(L::kStageBytes / (uint32_t)(2 * W)) & ~7);   // rows per pass
+            uint16_t *stage = (uint16_t *)(sm + L::kStage);
+            for (int r0 = 0; r0 < rows_blk; r0 += rpp) {
+                const int nr = min(rpp, rows_blk - r0);
+                if (i >= r0 && i < r0 + nr) {
+                    uint16_t *srow = stage + (i - r0) * W - i;   // srow[col] = pmap[t][col - i]
 #pragma unroll
-                        for (int e = 0; e < 4; ++e) {
-                            const uint32_t lo = *(const uint16_t *)(ptile + sw128_offset(r, r + wl + 2 * e));
-                            const uint32_t hi = *(const uint16_t *)(ptile + sw128_offset(r, r + wl + 2 * e + 1));
-                            w[e] = lo | (hi << 16);
+                    for (int cc = 0; cc < MAXC; ++cc) {
+                        if (cc < bd.mync) {
+                            const int col = bd.cb + (bd.c0 + cc) * 8;
+#pragma unroll
+                            for (int e = 0; e < 8; ++e) {
+                                const uint32_t w = (uint32_t)(col + e - i);
+                                if (w < (uint32_t)W) srow[col + e] = __bfloat16_as_ushort(__float2bfloat16_rn(P[cc][e]));
+                            }
                         }
-                        *(uint4 *)(a.pmap + (t0 + r) * W + wl) = make_uint4(w[0], w[1], w[2], w[3]);
                     }
                 }
-            } else {
-                for (int r = warp; r < BM; r += kComputeWarps) {
-                    const int64_t tr = t0 + r;
-                    if (tr >= s.N) break;
-                    __nv_bfloat16 *dst = a.pmap + tr * W;
-                    for (int w = lane; w < W; w += 32) {
-                        const uint16_t bits = *(const uint16_t *)(ptile + sw128_offset(r, r + w));
-                        reinterpret_cast<uint16_t *>(dst)[w] = bits;
-                    }
+                ptx::fence_proxy_async_smem();
+                compute_sync();
+                if (threadIdx.x == 0) {
+                    const uint32_t bytes = (uint32_t)nr * W * 2;
+                    uint8_t *dst = (uint8_t *)(a.pmap + (t0 + r0) * W);
+                    const uint32_t main = bytes & ~15u;
+                    for (uint32_t x = main; x < bytes; x += 2)   // ragged end of the tensor
+                        *(uint16_t *)(dst + x) = *(const uint16_t *)((const uint8_t *)stage + x);
+                    if (main) ptx::bulk_store(dst, stage, main);
+                    ptx::bulk_commit();
+                    if (r0 + rpp < rows_blk) ptx::bulk_wait_read();
                 }
+                if (r0 + rpp < rows_blk) compute_sync();
             }
         }
 
@@ -323,6 +332,7 @@ fwd_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__ CU
         int cb16, ce16;
         acc_split(split, D / 16, cb16, ce16);
         constexpr int kMaxC16 = (D / 16 + kSplits - 1) / kSplits;
+        const bool o_aligned32 = ((uintptr_t)a.o & 31) == 0;
         for (int h = 0; h < H; ++h) {
             const int b = h & 1;
             const uint32_t n = (uint32_t)(h >> 1);
@@ -343,9 +353,7 @@ fwd_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__ CU
 #pragma unroll
                         for (int e = 0; e < 8; ++e)
                             w[e] = pack_bf16x2(gh * __uint_as_float(ur[c][2 * e]), gh * __uint_as_float(ur[c][2 * e + 1]));
-                        uint4 *dst = (uint4 *)(a.o + (t * H + h) * D + (cb16 + c) * 16);
-                        dst[0] = make_uint4(w[0], w[1], w[2], w[3]);
-                        dst[1] = make_uint4(w[4], w[5], w[6], w[7]);
+                        ptx::st_global_32b(a.o + (t * H + h) * D + (cb16 + c) * 16, w, o_aligned32);
                     }
                 }
             }
@@ -354,6 +362,7 @@ fwd_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__ CU
         }
     }
 
+    if (threadIdx.x == 0) ptx::bulk_wait_all();   // the pmap copy has left shared memory
     ptx::tc_fence_before();
     __syncthreads();
     if (warp == 0) {
