@@ -229,13 +229,18 @@ bwd_query_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
                     ptx::tma_prefetch_l2_2d(&map_q, h * D + kb * 64, (int)t0);
                     ptx::tma_prefetch_l2_2d(&map_k, h * D + kb * 64, (int)kbase);
                 }
-                if (h + 2 < H && wait_bar(&bars[kQBarXFull], (uint32_t)h & 1, abort_flag)) issue_e(h + 2);
+                // once E_h has completed its buffers are reused: by dO_{h+2} / V_{h+2}, or, for
+                // the last use of buffer b, by the phase-2 tiles K_b (and Q_0 for buffer 0)
+                if (wait_bar(&bars[kQBarXFull], (uint32_t)h & 1, abort_flag)) {
+                    if (h + 2 < H) {
+                        issue_e(h + 2);
+                    } else {
+                        if (b == 0) issue_q(0);
+                        issue_k(b);
+                    }
+                }
             }
             // ---- phase 2: S_h = Q_h K_h^T; dQ_{h-1} = ds_{h-1} K_{h-1} right after it
-            if (wait_bar(&bars[kQBarXFull], (uint32_t)(H - 1) & 1, abort_flag)) {   // all E MMAs done
-                issue_q(0);
-                for (int h = 0; h < H && h < 2; ++h) issue_k(h);
-            }
             for (int h = 0; h < H; ++h) {
                 const int b = h & 1;
                 const uint32_t ph = (uint32_t)(H + h);
@@ -281,39 +286,48 @@ bwd_query_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
         const uint32_t x_cols = tmem + lane_base;
         const float sl2 = s.scale * kLog2e;
 
-        // the CTA's pmap rows, staged by the producer; P(t, c) = pmap[t][c - i]
-        const uint16_t *pstage = (const uint16_t *)(sm + L.rd + 32768);
-        wait_bar(&bars[kQBarPmap], 0, abort_flag);
-        const uint16_t *prow = pstage + i * W - i;
+        // P(t, c) = pmap[t][c - i] on this thread's band, from the CTA's pmap rows staged by
+        // the producer; zero outside the window.  Kept in registers (bf16 pairs) for all heads.
+        uint32_t pvp[MAXC][4];
+        {
+            const uint16_t *prow = (const uint16_t *)(sm + L.rd + 32768) + i * W - i;
+            wait_bar(&bars[kQBarPmap], 0, abort_flag);
+#pragma unroll
+            for (int cc = 0; cc < MAXC; ++cc) {
+                if (cc < bd.mync) {
+                    const int col = bd.cb + (bd.c0 + cc) * 8;
+#pragma unroll
+                    for (int e = 0; e < 8; e += 2) {
+                        const int c0 = col + e, c1 = c0 + 1;
+                        const uint32_t lo = (c0 >= clo && c0 <= chi) ? prow[c0] : 0u;
+                        const uint32_t hi = (c1 >= clo && c1 <= chi) ? prow[c1] : 0u;
+                        pvp[cc][e >> 1] = lo | (hi << 16);
+                    }
+                }
+            }
+        }
         float dP[MAXC][8];
 #pragma unroll
         for (int cc = 0; cc < MAXC; ++cc)
 #pragma unroll
             for (int e = 0; e < 8; ++e) dP[cc][e] = 0.f;
 
-        // ---- phase 1: dP and dg, three chunks of E_h per TMEM round trip
+        // ---- phase 1: dP and dg, three chunks of E_h per TMEM round trip.  dP is left
+        // unmasked: outside the window it only ever meets p = 0 (and the key side reads
+        // the band inside the window only); P is zero there, so dg needs no mask either.
         for (int h = 0; h < H; ++h) {
             wait_bar(&bars[kQBarXFull], (uint32_t)h & 1, abort_flag);
             ptx::tc_fence_after();
             const float gh = valid ? __ldg(a.g + t * H + h) : 0.f;
-            float dgp = 0.f;
+            float dga = 0.f, dgb = 0.f;
             constexpr int G = 3;
 #pragma unroll
             for (int g0 = 0; g0 < MAXC; g0 += G) {
                 uint32_t er[G][8];
-                float pv[G][8];
 #pragma unroll
                 for (int gi = 0; gi < G; ++gi) {
                     const int cc = g0 + gi;
-                    if (cc < MAXC && cc < bd.mync) {
-                        const int col = bd.cb + (bd.c0 + cc) * 8;
-#pragma unroll
-                        for (int e = 0; e < 8; ++e) {
-                            const int cidx = col + e;
-                            pv[gi][e] = (cidx >= clo && cidx <= chi) ? __uint_as_float((uint32_t)prow[cidx] << 16) : 0.f;
-                        }
-                        ptx::tmem_ld8_issue(x_cols + col, er[gi]);
-                    }
+                    if (cc < MAXC && cc < bd.mync) ptx::tmem_ld8_issue(x_cols + bd.cb + (bd.c0 + cc) * 8, er[gi]);
                 }
                 ptx::tmem_wait_ld();
 #pragma unroll
@@ -321,17 +335,18 @@ bwd_query_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
                     const int cc = g0 + gi;
                     if (cc < MAXC && cc < bd.mync) {
                         ptx::reg_fence8(er[gi]);
-                        const int col = bd.cb + (bd.c0 + cc) * 8;
 #pragma unroll
-                        for (int e = 0; e < 8; ++e) {
-                            const int cidx = col + e;
-                            const float ev = (cidx >= clo && cidx <= chi) ? __uint_as_float(er[gi][e]) : 0.f;
-                            dP[cc][e] = fmaf(gh, ev, dP[cc][e]);
-                            dgp = fmaf(pv[gi][e], ev, dgp);
+                        for (int e = 0; e < 8; e += 2) {
+                            const float e0 = __uint_as_float(er[gi][e]), e1 = __uint_as_float(er[gi][e + 1]);
+                            dP[cc][e] = fmaf(gh, e0, dP[cc][e]);
+                            dP[cc][e + 1] = fmaf(gh, e1, dP[cc][e + 1]);
+                            dga = fmaf(__uint_as_float(pvp[cc][e >> 1] << 16), e0, dga);
+                            dgb = fmaf(__uint_as_float(pvp[cc][e >> 1] & 0xFFFF0000u), e1, dgb);
                         }
                     }
                 }
             }
+            const float dgp = dga + dgb;
             ptx::tc_fence_before();
             ptx::mbar_arrive(&bars[kQBarXFree]);
             float *rd = red + (h & 1) * (kSplits * 128);
@@ -394,7 +409,7 @@ bwd_query_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
             ptx::tc_fence_after();
             const float lse2 = valid ? __ldg(a.lse + t * H + h) * kLog2e : 0.f;
             // p_h and dc_h, the band of S_h in two TMEM round trips
-            float dcp = 0.f;
+            float dca = 0.f, dcb = 0.f;   // two independent chains
             uint32_t pp[MAXC][4];   // p_h as packed bf16 pairs
             constexpr int G2 = (MAXC + 1) / 2;
 #pragma unroll
@@ -417,7 +432,8 @@ bwd_query_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
                         for (int e = 0; e < 8; ++e) {
                             const int cidx = col + e;
                             p[e] = (cidx >= clo && cidx <= chi) ? ex2(__uint_as_float(xr[gi][e]) * sl2 - lse2) : 0.f;
-                            dcp = fmaf(dP[cc][e], p[e], dcp);
+                            if (e & 1) dcb = fmaf(dP[cc][e], p[e], dcb);
+                            else dca = fmaf(dP[cc][e], p[e], dca);
                         }
 #pragma unroll
                         for (int e = 0; e < 4; ++e) pp[cc][e] = pack_bf16x2(p[2 * e], p[2 * e + 1]);
@@ -427,7 +443,7 @@ bwd_query_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
             ptx::tc_fence_before();
             ptx::mbar_arrive(&bars[kQBarXFree]);
             float *rd = red + (ph & 1) * (kSplits * 128);
-            rd[split * 128 + i] = dcp;
+            rd[split * 128 + i] = dca + dcb;
             pair_sync(q);
             float dch = rd[i];
 #pragma unroll
@@ -664,27 +680,38 @@ bwd_key_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant_
 
         // Scale the rows of dO_h (buffer h & 1) by g[t, h] in place.  Eight threads
         // share one 128-byte row (one 16-byte chunk each), so every quarter warp
-        // touches one row: no bank conflicts.
+        // touches one row: no bank conflicts.  The g values of a thread's rows are
+        // fetched together, before the wait for the tile.
+        constexpr int kRowsPerPass = kComputeThreads / 8;
+        constexpr int kPasses = (kBwdMaxSpan + kRowsPerPass - 1) / kRowsPerPass;
         auto scale_do = [&](int h) {
             const int b = h & 1;
+            float gv[kPasses];
+#pragma unroll
+            for (int it = 0; it < kPasses; ++it) {
+                const int r = (tid >> 3) + it * kRowsPerPass;
+                gv[it] = (r < span && j0 + r < s.N) ? __ldg(a.g + (j0 + r) * H + h) : 0.f;
+            }
             wait_bar(&bars[kKBarLd + b], (uint32_t)(h >> 1) & 1, abort_flag);
             uint8_t *tile = sm + (b ? L.rb1 : L.rb0);
-            const int rows = span * (D / 64);
-            const int chunk = tid & 7;
-            for (int hr = tid >> 3; hr < rows; hr += kComputeThreads / 8) {
-                const int r = hr % span;
-                const int64_t tr = j0 + r;
-                const float gv = (tr < s.N) ? __ldg(a.g + tr * H + h) : 0.f;
-                uint4 *p = (uint4 *)(tile + (hr / span) * span * 128 + r * 128) + chunk;
-                uint4 v = *p;
-                uint32_t *u = &v.x;
 #pragma unroll
-                for (int e = 0; e < 4; ++e) {
-                    const float f0 = __uint_as_float(u[e] << 16) * gv;
-                    const float f1 = __uint_as_float(u[e] & 0xFFFF0000u) * gv;
-                    u[e] = pack_bf16x2(f0, f1);
+            for (int kb = 0; kb < D / 64; ++kb) {
+#pragma unroll
+                for (int it = 0; it < kPasses; ++it) {
+                    const int r = (tid >> 3) + it * kRowsPerPass;
+                    if (r < span) {
+                        uint4 *p = (uint4 *)(tile + kb * span * 128 + r * 128) + (tid & 7);
+                        uint4 v = *p;
+                        uint32_t *u = &v.x;
+#pragma unroll
+                        for (int e = 0; e < 4; ++e) {
+                            const float f0 = __uint_as_float(u[e] << 16) * gv[it];
+                            const float f1 = __uint_as_float(u[e] & 0xFFFF0000u) * gv[it];
+                            u[e] = pack_bf16x2(f0, f1);
+                        }
+                        *p = v;
+                    }
                 }
-                *p = v;
             }
             ptx::fence_proxy_async_smem();
             ptx::mbar_arrive(&bars[kKBarScaled + b]);
@@ -721,16 +748,31 @@ bwd_key_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant_
             }
         }
         uint8_t *dtile = sm + L.ra;   // ds^T tile reuses the P^T region (every dV MMA has completed)
-        for (int h = 0; h < H; ++h) {
-            float *cv = colv + (h & 1) * 768;   // [lse * log2e | c | dc] for query columns
-            for (int cidx = tid; cidx < span; cidx += kComputeThreads) {
-                const int64_t tq = j0 + cidx;
-                const bool ok = tq < s.N;
-                cv[cidx] = ok ? __ldg(a.lse + tq * H + h) * kLog2e : 0.f;
-                cv[256 + cidx] = ok ? __ldg(a.c + tq * H + h) : 0.f;
-                cv[512 + cidx] = ok ? __ldg(a.dc_in + tq * H + h) : 0.f;
+        // per-query vectors of head h in colv[h & 1]: [lse * log2e | c | dc], one query column
+        // per thread (span <= 256 < kComputeThreads); head h+1's values are fetched while
+        // head h is processed
+        float nv0 = 0.f, nv1 = 0.f, nv2 = 0.f;
+        auto fetch_colv = [&](int h) {
+            const int64_t tq = j0 + tid;
+            const bool ok = tid < span && tq < s.N;
+            nv0 = ok ? __ldg(a.lse + tq * H + h) * kLog2e : 0.f;
+            nv1 = ok ? __ldg(a.c + tq * H + h) : 0.f;
+            nv2 = ok ? __ldg(a.dc_in + tq * H + h) : 0.f;
+        };
+        auto store_colv = [&](int h) {
+            float *cv = colv + (h & 1) * 768;
+            if (tid < 256) {
+                cv[tid] = nv0;
+                cv[256 + tid] = nv1;
+                cv[512 + tid] = nv2;
             }
-            compute_sync();
+        };
+        fetch_colv(0);
+        store_colv(0);
+        for (int h = 0; h < H; ++h) {
+            const float *cv = colv + (h & 1) * 768;
+            compute_sync();   // colv[h & 1] written; every warp is done with head h - 1
+            if (h + 1 < H) fetch_colv(h + 1);
             // drain the previous head's dK (its MMA ran while this head's S^T was computed),
             // which also frees the ds^T tile for this head
             if (h >= 1) drain(H + h - 1, a.dk, h - 1, s.scale);
@@ -753,15 +795,22 @@ bwd_key_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant_
                     const int cc = g0 + gi;
                     if (cc < MAXC && cc < bd.mync) {
                         ptx::reg_fence8(xr[gi]);
-                        const int col = bd.cb + (bd.c0 + cc) * 8;
+                        const int col = bd.cb + (bd.c0 + cc) * 8;   // the same for every lane
+                        float lv[8], cvv[8], dcv[8];
+                        *(float4 *)&lv[0] = *(const float4 *)(cv + col);
+                        *(float4 *)&lv[4] = *(const float4 *)(cv + col + 4);
+                        *(float4 *)&cvv[0] = *(const float4 *)(cv + 256 + col);
+                        *(float4 *)&cvv[4] = *(const float4 *)(cv + 256 + col + 4);
+                        *(float4 *)&dcv[0] = *(const float4 *)(cv + 512 + col);
+                        *(float4 *)&dcv[4] = *(const float4 *)(cv + 512 + col + 4);
 #pragma unroll
                         for (int e = 0; e < 8; e += 2) {
                             float dsv[2];
 #pragma unroll
                             for (int u = 0; u < 2; ++u) {
                                 const uint32_t cidx = (uint32_t)(col + e + u);
-                                const float p = ex2(__uint_as_float(xr[gi][e + u]) * sl2 - cv[cidx]);
-                                const float v = cv[256 + cidx] * p * (dPT[cc][e + u] - cv[512 + cidx]);
+                                const float p = ex2(__uint_as_float(xr[gi][e + u]) * sl2 - lv[e + u]);
+                                const float v = cvv[e + u] * p * (dPT[cc][e + u] - dcv[e + u]);
                                 dsv[u] = (cidx - span_lo <= span_n) ? v : 0.f;
                             }
                             dsp[cc][e >> 1] = pack_bf16x2(dsv[0], dsv[1]);
@@ -780,6 +829,7 @@ bwd_key_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant_
             }
             ptx::fence_proxy_async_smem();
             ptx::mbar_arrive(&bars[kKBarDs]);
+            if (h + 1 < H) store_colv(h + 1);
         }
         drain(2 * H - 1, a.dk, H - 1, s.scale);
     }

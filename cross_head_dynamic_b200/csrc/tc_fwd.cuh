@@ -222,7 +222,7 @@ fwd_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__ CU
             for (int cc = 0; cc < MAXC; ++cc)
                 if (cc < bd.mync) ptx::tmem_ld8_issue(s_cols + bd.cb + (bd.c0 + cc) * 8, xr[cc]);
             ptx::tmem_wait_ld();
-            float mloc = -INFINITY;
+            float mx[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};   // independent chains
 #pragma unroll
             for (int cc = 0; cc < MAXC; ++cc) {
                 if (cc < bd.mync) {
@@ -233,10 +233,11 @@ fwd_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__ CU
                         float v = __uint_as_float(xr[cc][e]) * sl2;
                         v = (col + e - span_lo <= span_n) ? v : -INFINITY;
                         xr[cc][e] = __float_as_uint(v);
-                        mloc = fmaxf(mloc, v);
+                        mx[e & 3] = fmaxf(mx[e & 3], v);
                     }
                 }
             }
+            const float mloc = fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3]));
             ptx::tc_fence_before();
             ptx::mbar_arrive(&bars[kBarSFree]);   // S columns free for the next head's MMA
             red_max[split * 128 + i] = mloc;
@@ -245,7 +246,7 @@ fwd_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__ CU
 #pragma unroll
             for (int sp = 1; sp < kSplits; ++sp) m = fmaxf(m, red_max[sp * 128 + i]);
             if (!valid) m = 0.f;
-            float zl = 0.f;
+            float zs[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
             for (int cc = 0; cc < MAXC; ++cc) {
                 if (cc < bd.mync) {
@@ -253,10 +254,11 @@ fwd_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__ CU
                     for (int e = 0; e < 8; ++e) {
                         const float ev = ex2(__uint_as_float(xr[cc][e]) - m);
                         xr[cc][e] = __float_as_uint(ev);
-                        zl += ev;
+                        zs[e & 3] += ev;
                     }
                 }
             }
+            const float zl = (zs[0] + zs[1]) + (zs[2] + zs[3]);
             red_sum[split * 128 + i] = zl;
             pair_sync(q);
             float Z = red_sum[i];
