@@ -224,11 +224,6 @@ bwd_query_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
                     }
                 }
                 ptx::mma_commit(&bars[kQBarXFull]);
-                // phase 2 reads Q_h and K_h: pull them into L2 while phase 1 runs
-                for (int kb = 0; kb < D / 64; ++kb) {
-                    ptx::tma_prefetch_l2_2d(&map_q, h * D + kb * 64, (int)t0);
-                    ptx::tma_prefetch_l2_2d(&map_k, h * D + kb * 64, (int)kbase);
-                }
                 // once E_h has completed its buffers are reused: by dO_{h+2} / V_{h+2}, or, for
                 // the last use of buffer b, by the phase-2 tiles K_b (and Q_0 for buffer 0)
                 if (wait_bar(&bars[kQBarXFull], (uint32_t)h & 1, abort_flag)) {
@@ -450,9 +445,9 @@ bwd_query_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
             for (int sp = 1; sp < kSplits; ++sp) dch += rd[sp * 128 + i];
             if (split == 0 && valid) a.dc[t * H + h] = dch;
             const float ch = valid ? __ldg(a.c + t * H + h) : 0.f;
-            // the previous head's dQ MMA has been running meanwhile; drain it, which also
-            // frees the ds tile for this head
-            if (h >= 1) drain_dq(h - 1);
+            // the previous head's dQ MMA has been running meanwhile; once it has completed the
+            // ds tile is free for this head (its accumulator is drained after the tile is handed on)
+            if (h >= 1) wait_bar(&bars[kQBarDqFull + ((h - 1) & 1)], (uint32_t)((h - 1) >> 1) & 1, abort_flag);
 #pragma unroll
             for (int cc = 0; cc < MAXC; ++cc) {
                 if (cc < bd.mync) {
@@ -468,6 +463,7 @@ bwd_query_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
             }
             ptx::fence_proxy_async_smem();
             ptx::mbar_arrive(&bars[kQBarDs]);
+            if (h >= 1) drain_dq(h - 1);   // overlaps the dQ_h MMA (other accumulator buffer)
         }
         drain_dq(H - 1);
     }
@@ -594,11 +590,6 @@ bwd_key_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant_
                 const uint32_t n = (uint32_t)(idx >> 1);
                 const bool ok = wait_bar(&bars[kKBarScaled + b], n & 1, abort_flag) && pt_ok;
                 mma_acc(idx, ok);
-                // phase 2 reads Q_h and K_h: pull them into L2 while phase 1 runs
-                for (int kb = 0; kb < D / 64; ++kb) {
-                    ptx::tma_prefetch_l2_2d(&map_q, h * D + kb * 64, (int)j0);
-                    ptx::tma_prefetch_l2_2d(&map_k, h * D + kb * 64, (int)j0);
-                }
                 if (idx + 2 < 2 * H && wait_bar(&bars[kKBarAccFull + b], n & 1, abort_flag)) issue_ld(idx + 2);
             }
             // ---- phase 2: S^T_h = K_h Q_h^T, then dK_{h-1} = ds^T_{h-1} Q_{h-1}
@@ -773,9 +764,6 @@ bwd_key_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant_
             const float *cv = colv + (h & 1) * 768;
             compute_sync();   // colv[h & 1] written; every warp is done with head h - 1
             if (h + 1 < H) fetch_colv(h + 1);
-            // drain the previous head's dK (its MMA ran while this head's S^T was computed),
-            // which also frees the ds^T tile for this head
-            if (h >= 1) drain(H + h - 1, a.dk, h - 1, s.scale);
             wait_bar(&bars[kKBarXFull], (uint32_t)h & 1, abort_flag);
             ptx::tc_fence_after();
             uint32_t dsp[MAXC][4];   // ds^T as packed bf16 pairs
@@ -820,6 +808,10 @@ bwd_key_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant_
             }
             ptx::tc_fence_before();
             ptx::mbar_arrive(&bars[kKBarXFree]);
+            // the previous head's dK MMA (running while this head's S^T was computed) must have
+            // read the ds^T tile before it is overwritten; its accumulator is drained afterwards
+            if (h >= 1)
+                wait_bar(&bars[kKBarAccFull + ((H + h - 1) & 1)], (uint32_t)((H + h - 1) >> 1) & 1, abort_flag);
 #pragma unroll
             for (int cc = 0; cc < MAXC; ++cc) {
                 if (cc < bd.mync) {
@@ -829,6 +821,7 @@ bwd_key_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant_
             }
             ptx::fence_proxy_async_smem();
             ptx::mbar_arrive(&bars[kKBarDs]);
+            if (h >= 1) drain(H + h - 1, a.dk, h - 1, s.scale);   // overlaps the dK_h MMA
             if (h + 1 < H) store_colv(h + 1);
         }
         drain(2 * H - 1, a.dk, H - 1, s.scale);

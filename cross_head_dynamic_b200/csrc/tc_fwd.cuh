@@ -11,8 +11,7 @@
 //   SIMT    pull the row band of S_h into registers (which frees the S columns
 //           for the next head's MMA), mask to the causal window inside the
 //           document, softmax per row, P += c[t,h] * p_h with P accumulated in
-//           registers (the H maps never leave the chip); V_h is prefetched
-//           into L2 meanwhile
+//           registers (the H maps never leave the chip)
 // Phase 2:
 //   SIMT    P -> bf16 tile in smem (K-major, swizzled), band copy -> pmap
 //   per head: TMA V_h [span x d]; MMA U_h = P V_h -> TMEM [128 x d];
@@ -150,8 +149,6 @@ fwd_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__ CU
                     }
                 }
                 ptx::mma_commit(&bars[kBarSFull]);
-                // V_h is not needed before phase 2; pull it into L2 now, while HBM has slack
-                for (int kb = 0; kb < D / 64; ++kb) ptx::tma_prefetch_l2_2d(&map_v, h * D + kb * 64, (int)kbase);
                 if (h + 2 < H) {
                     if (wait_bar(&bars[kBarSFull], (uint32_t)h & 1, abort_flag)) issue_qk(h + 2);
                 }

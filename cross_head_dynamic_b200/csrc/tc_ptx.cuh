@@ -119,11 +119,6 @@ __device__ __forceinline__ void st_global_32b(void *p, const uint32_t (&w)[8], b
     }
 }
 
-// Bring the box at (x, y) into L2 without a shared-memory destination.
-__device__ __forceinline__ void tma_prefetch_l2_2d(const CUtensorMap *map, int x, int y) {
-    asm volatile("cp.async.bulk.prefetch.tensor.2d.L2.global.tile [%0, {%1, %2}];" ::"l"((uint64_t)map), "r"(x), "r"(y)
-                 : "memory");
-}
 __device__ __forceinline__ void prefetch_tensormap(const CUtensorMap *map) {
     asm volatile("prefetch.tensormap [%0];" ::"l"((uint64_t)map) : "memory");
 }
