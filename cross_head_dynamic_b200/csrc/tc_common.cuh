@@ -37,7 +37,6 @@ __device__ __forceinline__ void regs_compute() {
     asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kRegsCompute));
 }
 constexpr uint64_t kWaitNs = 2000000000ull;   // a legitimate wait lasts microseconds
-
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kLn2 = 0.6931471805599453f;
 

@@ -40,10 +40,11 @@ struct FwdLayout {
     // the P tile reuses the Q buffers when they are large enough (free after the last S MMA)
     static constexpr uint32_t kP = (2 * kQBytes >= kPBytes) ? 0u : kK1 + kKBytes;
     static constexpr uint32_t kRed = (kP == 0 ? kK1 + kKBytes : kP + kPBytes);
-    static constexpr uint32_t kBars = kRed + 2 * kSplits * 128 * 4;
+    // per-row (max, sum) of each split, double-buffered by head parity: [2][kSplits][128] float2
+    static constexpr uint32_t kBars = kRed + 2 * kSplits * 128 * 8;
     // pmap rows of the block, contiguous as in global memory, written out by one bulk copy
     static constexpr uint32_t kStage = kBars + 256;
-    static constexpr uint32_t kStageBytes = 30u * 1024;
+    static constexpr uint32_t kStageBytes = 27u * 1024 + 512;
     static constexpr uint32_t kBytes = kStage + kStageBytes;
     static constexpr uint32_t kAlloc = kBytes + 1024;        // slack to align the base to 1 KiB
     static_assert(kAlloc <= 227u * 1024, "forward tile layout exceeds shared memory");
@@ -74,8 +75,7 @@ fwd_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__ CU
     uint64_t *bars = (uint64_t *)(sm + L::kBars);
     uint32_t *tmem_slot = (uint32_t *)(bars + 16);
     volatile int *abort_flag = (volatile int *)(tmem_slot + 1);
-    float *red_max = (float *)(sm + L::kRed);     // [kSplits][128]
-    float *red_sum = red_max + kSplits * 128;     // [kSplits][128]
+    float2 *red = (float2 *)(sm + L::kRed);       // [2][kSplits][128] (max, sum)
 
     const Shape &s = a.s;
     const int H = s.H, W = s.W, BM = a.BM, span = a.span;
@@ -225,43 +225,58 @@ fwd_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__ CU
                 if (cc < bd.mync) {
                     ptx::reg_fence8(xr[cc]);
                     const uint32_t col = (uint32_t)(bd.cb + (bd.c0 + cc) * 8);
+                    // chunks inside every lane's window (most of the band) skip the mask
+                    if (__all_sync(0xffffffffu, col - span_lo <= span_n && col + 7 - span_lo <= span_n)) {
 #pragma unroll
-                    for (int e = 0; e < 8; ++e) {
-                        float v = __uint_as_float(xr[cc][e]) * sl2;
-                        v = (col + e - span_lo <= span_n) ? v : -INFINITY;
-                        xr[cc][e] = __float_as_uint(v);
-                        mx[e & 3] = fmaxf(mx[e & 3], v);
+                        for (int e = 0; e < 8; ++e) {
+                            const float v = __uint_as_float(xr[cc][e]) * sl2;
+                            xr[cc][e] = __float_as_uint(v);
+                            mx[e & 3] = fmaxf(mx[e & 3], v);
+                        }
+                    } else {
+#pragma unroll
+                        for (int e = 0; e < 8; ++e) {
+                            float v = __uint_as_float(xr[cc][e]) * sl2;
+                            v = (col + e - span_lo <= span_n) ? v : -INFINITY;
+                            xr[cc][e] = __float_as_uint(v);
+                            mx[e & 3] = fmaxf(mx[e & 3], v);
+                        }
                     }
                 }
             }
-            const float mloc = fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3]));
             ptx::tc_fence_before();
             ptx::mbar_arrive(&bars[kBarSFree]);   // S columns free for the next head's MMA
-            red_max[split * 128 + i] = mloc;
-            pair_sync(q);
-            float m = red_max[i];
-#pragma unroll
-            for (int sp = 1; sp < kSplits; ++sp) m = fmaxf(m, red_max[sp * 128 + i]);
-            if (!valid) m = 0.f;
+            // Softmax with this split's own maximum; the splits' (max, sum) pairs are then
+            // combined in one exchange: Z = sum_s Z_s 2^(m_s - m), p = e_s 2^(m_s - m) / Z.
+            const float mloc = fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3]));
+            const bool any = mloc != -INFINITY;   // this split has a column in the row's window
+            const float mref = any ? mloc : 0.f;
             float zs[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
             for (int cc = 0; cc < MAXC; ++cc) {
                 if (cc < bd.mync) {
 #pragma unroll
                     for (int e = 0; e < 8; ++e) {
-                        const float ev = ex2(__uint_as_float(xr[cc][e]) - m);
+                        const float ev = ex2(__uint_as_float(xr[cc][e]) - mref);
                         xr[cc][e] = __float_as_uint(ev);
                         zs[e & 3] += ev;
                     }
                 }
             }
-            const float zl = (zs[0] + zs[1]) + (zs[2] + zs[3]);
-            red_sum[split * 128 + i] = zl;
+            float2 *rd = red + (h & 1) * (kSplits * 128);
+            rd[split * 128 + i] = make_float2(mloc, (zs[0] + zs[1]) + (zs[2] + zs[3]));
             pair_sync(q);
-            float Z = red_sum[i];
+            float2 ms[kSplits];
 #pragma unroll
-            for (int sp = 1; sp < kSplits; ++sp) Z += red_sum[sp * 128 + i];
-            const float coef = valid ? __ldg(a.c + t * H + h) / Z : 0.f;
+            for (int sp = 0; sp < kSplits; ++sp) ms[sp] = rd[sp * 128 + i];
+            float m = ms[0].x;
+#pragma unroll
+            for (int sp = 1; sp < kSplits; ++sp) m = fmaxf(m, ms[sp].x);
+            if (!valid) m = 0.f;
+            float Z = 0.f;
+#pragma unroll
+            for (int sp = 0; sp < kSplits; ++sp) Z += ms[sp].y > 0.f ? ms[sp].y * ex2(ms[sp].x - m) : 0.f;
+            const float coef = (valid && any) ? __ldg(a.c + t * H + h) * ex2(mref - m) / Z : 0.f;
 #pragma unroll
             for (int cc = 0; cc < MAXC; ++cc)
                 if (cc < bd.mync)
@@ -272,16 +287,14 @@ fwd_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__ CU
 
         // ---- P tile (bf16, K-major, swizzled) in smem; zero the columns outside the band
         uint8_t *ptile = sm + L::kP;
+        uint32_t Pb[MAXC][4];   // P rounded to bf16 pairs, also the pmap values
 #pragma unroll
         for (int cc = 0; cc < MAXC; ++cc) {
             if (cc < bd.mync) {
                 const int col = bd.cb + (bd.c0 + cc) * 8;
-                uint4 w4;
-                w4.x = pack_bf16x2(P[cc][0], P[cc][1]);
-                w4.y = pack_bf16x2(P[cc][2], P[cc][3]);
-                w4.z = pack_bf16x2(P[cc][4], P[cc][5]);
-                w4.w = pack_bf16x2(P[cc][6], P[cc][7]);
-                *(uint4 *)(ptile + sw128_offset(i, col)) = w4;
+#pragma unroll
+                for (int e = 0; e < 4; ++e) Pb[cc][e] = pack_bf16x2(P[cc][2 * e], P[cc][2 * e + 1]);
+                *(uint4 *)(ptile + sw128_offset(i, col)) = make_uint4(Pb[cc][0], Pb[cc][1], Pb[cc][2], Pb[cc][3]);
             }
         }
         zero_outside_band(ptile, i, split, bd, span);
@@ -306,7 +319,7 @@ fwd_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__ CU
 #pragma unroll
                             for (int e = 0; e < 8; ++e) {
                                 const uint32_t w = (uint32_t)(col + e - i);
-                                if (w < (uint32_t)W) srow[col + e] = __bfloat16_as_ushort(__float2bfloat16_rn(P[cc][e]));
+                                if (w < (uint32_t)W) srow[col + e] = (uint16_t)(Pb[cc][e >> 1] >> (16 * (e & 1)));
                             }
                         }
                     }
