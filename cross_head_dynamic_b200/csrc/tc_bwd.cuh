@@ -236,32 +236,35 @@ bwd_query_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
                 }
             }
             // ---- phase 2: S_h = Q_h K_h^T; dQ_{h-1} = ds_{h-1} K_{h-1} right after it
-            for (int h = 0; h < H; ++h) {
-                const int b = h & 1;
+            for (int h = 0; h <= H; ++h) {   // h == H only issues dQ_{H-1}
                 const uint32_t ph = (uint32_t)(H + h);
-                bool ok = wait_bar(&bars[kQBarQ], (uint32_t)h & 1, abort_flag);
-                ok = wait_bar(&bars[kQBarK + b], (uint32_t)(h >> 1) & 1, abort_flag) && ok;
-                ok = wait_bar(&bars[kQBarXFree], (ph - 1) & 1, abort_flag) && ok;
-                ptx::tc_fence_after();
-                if (ok) {
-                    const uint32_t qa = ptx::smem_u32(sm + L.rq);
-                    const uint32_t ka = ptx::smem_u32(sm + (b ? L.r1 : L.r0));
+                if (h < H) {
+                    const int b = h & 1;
+                    bool ok = wait_bar(&bars[kQBarQ], (uint32_t)h & 1, abort_flag);
+                    ok = wait_bar(&bars[kQBarK + b], (uint32_t)(h >> 1) & 1, abort_flag) && ok;
+                    ok = wait_bar(&bars[kQBarXFree], (ph - 1) & 1, abort_flag) && ok;
+                    ptx::tc_fence_after();
+                    if (ok) {
+                        const uint32_t qa = ptx::smem_u32(sm + L.rq);
+                        const uint32_t ka = ptx::smem_u32(sm + (b ? L.r1 : L.r0));
 #pragma unroll
-                    for (int k = 0; k < D / 16; ++k) {
-                        const uint64_t ad = ptx::smem_desc_sw128(qa + (k >> 2) * 16384 + (k & 3) * 32, 16, 1024);
-                        const uint64_t bd = ptx::smem_desc_sw128(ka + (k >> 2) * span * 128 + (k & 3) * 32, 16, 1024);
-                        ptx::mma_bf16(tmem, ad, bd, id_x, k > 0);
+                        for (int k = 0; k < D / 16; ++k) {
+                            const uint64_t ad = ptx::smem_desc_sw128(qa + (k >> 2) * 16384 + (k & 3) * 32, 16, 1024);
+                            const uint64_t bd = ptx::smem_desc_sw128(ka + (k >> 2) * span * 128 + (k & 3) * 32, 16, 1024);
+                            ptx::mma_bf16(tmem, ad, bd, id_x, k > 0);
+                        }
                     }
+                    ptx::mma_commit(&bars[kQBarXFull]);
                 }
-                ptx::mma_commit(&bars[kQBarXFull]);
                 if (h >= 1) mma_dq(h - 1);
-                // refill: Q_{h+1} once S_h has read Q; K_{h+1} once dQ_{h-1} has read K_{h-1}
-                if (wait_bar(&bars[kQBarXFull], ph & 1, abort_flag) && h + 1 < H) issue_q(h + 1);
-                if (h >= 1 && h + 1 < H &&
-                    wait_bar(&bars[kQBarDqFull + ((h - 1) & 1)], (uint32_t)((h - 1) >> 1) & 1, abort_flag))
-                    issue_k(h + 1);
+                if (h < H) {
+                    // refill: Q_{h+1} once S_h has read Q; K_{h+1} once dQ_{h-1} has read K_{h-1}
+                    if (wait_bar(&bars[kQBarXFull], ph & 1, abort_flag) && h + 1 < H) issue_q(h + 1);
+                    if (h >= 1 && h + 1 < H &&
+                        wait_bar(&bars[kQBarDqFull + ((h - 1) & 1)], (uint32_t)((h - 1) >> 1) & 1, abort_flag))
+                        issue_k(h + 1);
+                }
             }
-            mma_dq(H - 1);
         }
         __syncwarp();
     } else {
@@ -398,74 +401,75 @@ bwd_query_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
             ptx::tc_fence_before();
             ptx::mbar_arrive(&bars[kQBarDqFree + b]);
         };
-        for (int h = 0; h < H; ++h) {
-            const uint32_t ph = (uint32_t)(H + h);
-            wait_bar(&bars[kQBarXFull], ph & 1, abort_flag);
-            ptx::tc_fence_after();
-            const float lse2 = valid ? __ldg(a.lse + t * H + h) * kLog2e : 0.f;
-            // p_h and dc_h, the band of S_h in two TMEM round trips
-            float dca = 0.f, dcb = 0.f;   // two independent chains
-            uint32_t pp[MAXC][4];   // p_h as packed bf16 pairs
-            constexpr int G2 = (MAXC + 1) / 2;
+        for (int h = 0; h <= H; ++h) {   // h == H only drains dQ_{H-1}
+            if (h < H) {
+                const uint32_t ph = (uint32_t)(H + h);
+                wait_bar(&bars[kQBarXFull], ph & 1, abort_flag);
+                ptx::tc_fence_after();
+                const float lse2 = valid ? __ldg(a.lse + t * H + h) * kLog2e : 0.f;
+                // p_h and dc_h, the band of S_h in two TMEM round trips
+                float dca = 0.f, dcb = 0.f;   // two independent chains
+                uint32_t pp[MAXC][4];   // p_h as packed bf16 pairs
+                constexpr int G2 = (MAXC + 1) / 2;
 #pragma unroll
-            for (int g0 = 0; g0 < MAXC; g0 += G2) {
-                uint32_t xr[G2][8];
+                for (int g0 = 0; g0 < MAXC; g0 += G2) {
+                    uint32_t xr[G2][8];
 #pragma unroll
-                for (int gi = 0; gi < G2; ++gi) {
-                    const int cc = g0 + gi;
-                    if (cc < MAXC && cc < bd.mync) ptx::tmem_ld8_issue(x_cols + bd.cb + (bd.c0 + cc) * 8, xr[gi]);
-                }
-                ptx::tmem_wait_ld();
+                    for (int gi = 0; gi < G2; ++gi) {
+                        const int cc = g0 + gi;
+                        if (cc < MAXC && cc < bd.mync) ptx::tmem_ld8_issue(x_cols + bd.cb + (bd.c0 + cc) * 8, xr[gi]);
+                    }
+                    ptx::tmem_wait_ld();
 #pragma unroll
-                for (int gi = 0; gi < G2; ++gi) {
-                    const int cc = g0 + gi;
-                    if (cc < MAXC && cc < bd.mync) {
-                        ptx::reg_fence8(xr[gi]);
-                        const int col = bd.cb + (bd.c0 + cc) * 8;
-                        float p[8];
+                    for (int gi = 0; gi < G2; ++gi) {
+                        const int cc = g0 + gi;
+                        if (cc < MAXC && cc < bd.mync) {
+                            ptx::reg_fence8(xr[gi]);
+                            const int col = bd.cb + (bd.c0 + cc) * 8;
+                            float p[8];
 #pragma unroll
-                        for (int e = 0; e < 8; ++e) {
-                            const int cidx = col + e;
-                            p[e] = (cidx >= clo && cidx <= chi) ? ex2(__uint_as_float(xr[gi][e]) * sl2 - lse2) : 0.f;
-                            if (e & 1) dcb = fmaf(dP[cc][e], p[e], dcb);
-                            else dca = fmaf(dP[cc][e], p[e], dca);
+                            for (int e = 0; e < 8; ++e) {
+                                const int cidx = col + e;
+                                p[e] = (cidx >= clo && cidx <= chi) ? ex2(__uint_as_float(xr[gi][e]) * sl2 - lse2) : 0.f;
+                                if (e & 1) dcb = fmaf(dP[cc][e], p[e], dcb);
+                                else dca = fmaf(dP[cc][e], p[e], dca);
+                            }
+#pragma unroll
+                            for (int e = 0; e < 4; ++e) pp[cc][e] = pack_bf16x2(p[2 * e], p[2 * e + 1]);
                         }
-#pragma unroll
-                        for (int e = 0; e < 4; ++e) pp[cc][e] = pack_bf16x2(p[2 * e], p[2 * e + 1]);
                     }
                 }
-            }
-            ptx::tc_fence_before();
-            ptx::mbar_arrive(&bars[kQBarXFree]);
-            float *rd = red + (ph & 1) * (kSplits * 128);
-            rd[split * 128 + i] = dca + dcb;
-            pair_sync(q);
-            float dch = rd[i];
+                ptx::tc_fence_before();
+                ptx::mbar_arrive(&bars[kQBarXFree]);
+                float *rd = red + (ph & 1) * (kSplits * 128);
+                rd[split * 128 + i] = dca + dcb;
+                pair_sync(q);
+                float dch = rd[i];
 #pragma unroll
-            for (int sp = 1; sp < kSplits; ++sp) dch += rd[sp * 128 + i];
-            if (split == 0 && valid) a.dc[t * H + h] = dch;
-            const float ch = valid ? __ldg(a.c + t * H + h) : 0.f;
-            // the previous head's dQ MMA has been running meanwhile; once it has completed the
-            // ds tile is free for this head (its accumulator is drained after the tile is handed on)
-            if (h >= 1) wait_bar(&bars[kQBarDqFull + ((h - 1) & 1)], (uint32_t)((h - 1) >> 1) & 1, abort_flag);
+                for (int sp = 1; sp < kSplits; ++sp) dch += rd[sp * 128 + i];
+                if (split == 0 && valid) a.dc[t * H + h] = dch;
+                const float ch = valid ? __ldg(a.c + t * H + h) : 0.f;
+                // the previous head's dQ MMA has been running meanwhile; once it has completed the
+                // ds tile is free for this head (its accumulator is drained after the tile is handed on)
+                if (h >= 1) wait_bar(&bars[kQBarDqFull + ((h - 1) & 1)], (uint32_t)((h - 1) >> 1) & 1, abort_flag);
 #pragma unroll
-            for (int cc = 0; cc < MAXC; ++cc) {
-                if (cc < bd.mync) {
-                    const int col = bd.cb + (bd.c0 + cc) * 8;
-                    uint32_t w[4];
+                for (int cc = 0; cc < MAXC; ++cc) {
+                    if (cc < bd.mync) {
+                        const int col = bd.cb + (bd.c0 + cc) * 8;
+                        uint32_t w[4];
 #pragma unroll
-                    for (int e = 0; e < 4; ++e) {
-                        const float p0 = __uint_as_float(pp[cc][e] << 16), p1 = __uint_as_float(pp[cc][e] & 0xFFFF0000u);
-                        w[e] = pack_bf16x2(ch * p0 * (dP[cc][2 * e] - dch), ch * p1 * (dP[cc][2 * e + 1] - dch));
+                        for (int e = 0; e < 4; ++e) {
+                            const float p0 = __uint_as_float(pp[cc][e] << 16), p1 = __uint_as_float(pp[cc][e] & 0xFFFF0000u);
+                            w[e] = pack_bf16x2(ch * p0 * (dP[cc][2 * e] - dch), ch * p1 * (dP[cc][2 * e + 1] - dch));
+                        }
+                        *(uint4 *)(dtile + sw128_offset(i, col)) = make_uint4(w[0], w[1], w[2], w[3]);
                     }
-                    *(uint4 *)(dtile + sw128_offset(i, col)) = make_uint4(w[0], w[1], w[2], w[3]);
                 }
+                ptx::fence_proxy_async_smem();
+                ptx::mbar_arrive(&bars[kQBarDs]);
             }
-            ptx::fence_proxy_async_smem();
-            ptx::mbar_arrive(&bars[kQBarDs]);
             if (h >= 1) drain_dq(h - 1);   // overlaps the dQ_h MMA (other accumulator buffer)
         }
-        drain_dq(H - 1);
     }
 
     if (threadIdx.x == 0) ptx::bulk_wait_all();   // the dP band copy has completed
@@ -593,30 +597,33 @@ bwd_key_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant_
                 if (idx + 2 < 2 * H && wait_bar(&bars[kKBarAccFull + b], n & 1, abort_flag)) issue_ld(idx + 2);
             }
             // ---- phase 2: S^T_h = K_h Q_h^T, then dK_{h-1} = ds^T_{h-1} Q_{h-1}
-            for (int h = 0; h < H; ++h) {
+            for (int h = 0; h <= H; ++h) {   // h == H only issues dK_{H-1}
                 const int idx = H + h, b = idx & 1;
-                bool ok = wait_bar(&bars[kKBarK], (uint32_t)h & 1, abort_flag);
-                ok = wait_bar(&bars[kKBarLd + b], (uint32_t)(idx >> 1) & 1, abort_flag) && ok;
-                if (h >= 1) ok = wait_bar(&bars[kKBarXFree], (uint32_t)(h - 1) & 1, abort_flag) && ok;
-                ptx::tc_fence_after();
-                if (ok) {
-                    const uint32_t qa = ptx::smem_u32(sm + (b ? L.rb1 : L.rb0));
+                if (h < H) {
+                    bool ok = wait_bar(&bars[kKBarK], (uint32_t)h & 1, abort_flag);
+                    ok = wait_bar(&bars[kKBarLd + b], (uint32_t)(idx >> 1) & 1, abort_flag) && ok;
+                    if (h >= 1) ok = wait_bar(&bars[kKBarXFree], (uint32_t)(h - 1) & 1, abort_flag) && ok;
+                    ptx::tc_fence_after();
+                    if (ok) {
+                        const uint32_t qa = ptx::smem_u32(sm + (b ? L.rb1 : L.rb0));
 #pragma unroll
-                    for (int k = 0; k < D / 16; ++k) {
-                        const uint64_t ad = ptx::smem_desc_sw128(rk + (k >> 2) * 16384 + (k & 3) * 32, 16, 1024);
-                        const uint64_t bd2 = ptx::smem_desc_sw128(qa + (k >> 2) * span * 128 + (k & 3) * 32, 16, 1024);
-                        ptx::mma_bf16(tmem, ad, bd2, id_st, k > 0);
+                        for (int k = 0; k < D / 16; ++k) {
+                            const uint64_t ad = ptx::smem_desc_sw128(rk + (k >> 2) * 16384 + (k & 3) * 32, 16, 1024);
+                            const uint64_t bd2 = ptx::smem_desc_sw128(qa + (k >> 2) * span * 128 + (k & 3) * 32, 16, 1024);
+                            ptx::mma_bf16(tmem, ad, bd2, id_st, k > 0);
+                        }
                     }
+                    ptx::mma_commit(&bars[kKBarXFull]);
                 }
-                ptx::mma_commit(&bars[kKBarXFull]);
                 if (h >= 1) mma_acc(idx - 1, wait_bar(&bars[kKBarDs], (uint32_t)(h - 1) & 1, abort_flag));
-                // refill: K_{h+1} once S^T_h has read K; Q_{h+1} once dK_{h-1} has read Q_{h-1}
-                if (wait_bar(&bars[kKBarXFull], (uint32_t)h & 1, abort_flag) && h + 1 < H) issue_k(h + 1);
-                if (h >= 1 && idx + 1 < 2 * H &&
-                    wait_bar(&bars[kKBarAccFull + ((idx - 1) & 1)], (uint32_t)((idx - 1) >> 1) & 1, abort_flag))
-                    issue_ld(idx + 1);
+                if (h < H) {
+                    // refill: K_{h+1} once S^T_h has read K; Q_{h+1} once dK_{h-1} has read Q_{h-1}
+                    if (wait_bar(&bars[kKBarXFull], (uint32_t)h & 1, abort_flag) && h + 1 < H) issue_k(h + 1);
+                    if (h >= 1 && idx + 1 < 2 * H &&
+                        wait_bar(&bars[kKBarAccFull + ((idx - 1) & 1)], (uint32_t)((idx - 1) >> 1) & 1, abort_flag))
+                        issue_ld(idx + 1);
+                }
             }
-            mma_acc(2 * H - 1, wait_bar(&bars[kKBarDs], (uint32_t)(H - 1) & 1, abort_flag));
         }
         __syncwarp();
     } else {
@@ -717,11 +724,10 @@ bwd_key_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant_
             ptx::mbar_arrive(&bars[kKBarAccFree + b]);
         };
 
-        // ---- phase 1: dV
-        scale_do(0);
-        for (int h = 0; h < H; ++h) {
-            if (h + 1 < H) scale_do(h + 1);
-            drain(h, a.dv, h, 1.f);
+        // ---- phase 1: dV (scaling dO_h runs ahead of draining dV_{h-1}; one copy of each)
+        for (int h = 0; h <= H; ++h) {
+            if (h < H) scale_do(h);
+            if (h >= 1) drain(h - 1, a.dv, h - 1, 1.f);
         }
 
         // ---- phase 2: dK.  dP(t, j) for this row's band from the query side's workspace
@@ -760,71 +766,72 @@ bwd_key_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant_
         };
         fetch_colv(0);
         store_colv(0);
-        for (int h = 0; h < H; ++h) {
-            const float *cv = colv + (h & 1) * 768;
-            compute_sync();   // colv[h & 1] written; every warp is done with head h - 1
-            if (h + 1 < H) fetch_colv(h + 1);
-            wait_bar(&bars[kKBarXFull], (uint32_t)h & 1, abort_flag);
-            ptx::tc_fence_after();
-            uint32_t dsp[MAXC][4];   // ds^T as packed bf16 pairs
-            constexpr int G2 = (MAXC + 1) / 2;   // the band of S^T_h in two TMEM round trips
+        for (int h = 0; h <= H; ++h) {   // h == H only drains dK_{H-1}
+            if (h < H) {
+                const float *cv = colv + (h & 1) * 768;
+                compute_sync();   // colv[h & 1] written; every warp is done with head h - 1
+                if (h + 1 < H) fetch_colv(h + 1);
+                wait_bar(&bars[kKBarXFull], (uint32_t)h & 1, abort_flag);
+                ptx::tc_fence_after();
+                uint32_t dsp[MAXC][4];   // ds^T as packed bf16 pairs
+                constexpr int G2 = (MAXC + 1) / 2;   // the band of S^T_h in two TMEM round trips
 #pragma unroll
-            for (int g0 = 0; g0 < MAXC; g0 += G2) {
-                uint32_t xr[G2][8];
+                for (int g0 = 0; g0 < MAXC; g0 += G2) {
+                    uint32_t xr[G2][8];
 #pragma unroll
-                for (int gi = 0; gi < G2; ++gi) {
-                    const int cc = g0 + gi;
-                    if (cc < MAXC && cc < bd.mync)
-                        ptx::tmem_ld8_issue(tmem + lane_base + bd.cb + (bd.c0 + cc) * 8, xr[gi]);
-                }
-                ptx::tmem_wait_ld();
+                    for (int gi = 0; gi < G2; ++gi) {
+                        const int cc = g0 + gi;
+                        if (cc < MAXC && cc < bd.mync)
+                            ptx::tmem_ld8_issue(tmem + lane_base + bd.cb + (bd.c0 + cc) * 8, xr[gi]);
+                    }
+                    ptx::tmem_wait_ld();
 #pragma unroll
-                for (int gi = 0; gi < G2; ++gi) {
-                    const int cc = g0 + gi;
-                    if (cc < MAXC && cc < bd.mync) {
-                        ptx::reg_fence8(xr[gi]);
-                        const int col = bd.cb + (bd.c0 + cc) * 8;   // the same for every lane
-                        float lv[8], cvv[8], dcv[8];
-                        *(float4 *)&lv[0] = *(const float4 *)(cv + col);
-                        *(float4 *)&lv[4] = *(const float4 *)(cv + col + 4);
-                        *(float4 *)&cvv[0] = *(const float4 *)(cv + 256 + col);
-                        *(float4 *)&cvv[4] = *(const float4 *)(cv + 256 + col + 4);
-                        *(float4 *)&dcv[0] = *(const float4 *)(cv + 512 + col);
-                        *(float4 *)&dcv[4] = *(const float4 *)(cv + 512 + col + 4);
+                    for (int gi = 0; gi < G2; ++gi) {
+                        const int cc = g0 + gi;
+                        if (cc < MAXC && cc < bd.mync) {
+                            ptx::reg_fence8(xr[gi]);
+                            const int col = bd.cb + (bd.c0 + cc) * 8;   // the same for every lane
+                            float lv[8], cvv[8], dcv[8];
+                            *(float4 *)&lv[0] = *(const float4 *)(cv + col);
+                            *(float4 *)&lv[4] = *(const float4 *)(cv + col + 4);
+                            *(float4 *)&cvv[0] = *(const float4 *)(cv + 256 + col);
+                            *(float4 *)&cvv[4] = *(const float4 *)(cv + 256 + col + 4);
+                            *(float4 *)&dcv[0] = *(const float4 *)(cv + 512 + col);
+                            *(float4 *)&dcv[4] = *(const float4 *)(cv + 512 + col + 4);
 #pragma unroll
-                        for (int e = 0; e < 8; e += 2) {
-                            float dsv[2];
+                            for (int e = 0; e < 8; e += 2) {
+                                float dsv[2];
 #pragma unroll
-                            for (int u = 0; u < 2; ++u) {
-                                const uint32_t cidx = (uint32_t)(col + e + u);
-                                const float p = ex2(__uint_as_float(xr[gi][e + u]) * sl2 - lv[e + u]);
-                                const float v = cvv[e + u] * p * (dPT[cc][e + u] - dcv[e + u]);
-                                dsv[u] = (cidx - span_lo <= span_n) ? v : 0.f;
+                                for (int u = 0; u < 2; ++u) {
+                                    const uint32_t cidx = (uint32_t)(col + e + u);
+                                    const float p = ex2(__uint_as_float(xr[gi][e + u]) * sl2 - lv[e + u]);
+                                    const float v = cvv[e + u] * p * (dPT[cc][e + u] - dcv[e + u]);
+                                    dsv[u] = (cidx - span_lo <= span_n) ? v : 0.f;
+                                }
+                                dsp[cc][e >> 1] = pack_bf16x2(dsv[0], dsv[1]);
                             }
-                            dsp[cc][e >> 1] = pack_bf16x2(dsv[0], dsv[1]);
                         }
                     }
                 }
-            }
-            ptx::tc_fence_before();
-            ptx::mbar_arrive(&bars[kKBarXFree]);
-            // the previous head's dK MMA (running while this head's S^T was computed) must have
-            // read the ds^T tile before it is overwritten; its accumulator is drained afterwards
-            if (h >= 1)
-                wait_bar(&bars[kKBarAccFull + ((H + h - 1) & 1)], (uint32_t)((H + h - 1) >> 1) & 1, abort_flag);
+                ptx::tc_fence_before();
+                ptx::mbar_arrive(&bars[kKBarXFree]);
+                // the previous head's dK MMA (running while this head's S^T was computed) must have
+                // read the ds^T tile before it is overwritten; its accumulator is drained afterwards
+                if (h >= 1)
+                    wait_bar(&bars[kKBarAccFull + ((H + h - 1) & 1)], (uint32_t)((H + h - 1) >> 1) & 1, abort_flag);
 #pragma unroll
-            for (int cc = 0; cc < MAXC; ++cc) {
-                if (cc < bd.mync) {
-                    const int col = bd.cb + (bd.c0 + cc) * 8;
-                    *(uint4 *)(dtile + sw128_offset(i, col)) = make_uint4(dsp[cc][0], dsp[cc][1], dsp[cc][2], dsp[cc][3]);
+                for (int cc = 0; cc < MAXC; ++cc) {
+                    if (cc < bd.mync) {
+                        const int col = bd.cb + (bd.c0 + cc) * 8;
+                        *(uint4 *)(dtile + sw128_offset(i, col)) = make_uint4(dsp[cc][0], dsp[cc][1], dsp[cc][2], dsp[cc][3]);
+                    }
                 }
+                ptx::fence_proxy_async_smem();
+                ptx::mbar_arrive(&bars[kKBarDs]);
             }
-            ptx::fence_proxy_async_smem();
-            ptx::mbar_arrive(&bars[kKBarDs]);
             if (h >= 1) drain(H + h - 1, a.dk, h - 1, s.scale);   // overlaps the dK_h MMA
             if (h + 1 < H) store_colv(h + 1);
         }
-        drain(2 * H - 1, a.dk, H - 1, s.scale);
     }
 
     ptx::tc_fence_before();

@@ -36,7 +36,7 @@ __device__ __forceinline__ void regs_producer() {
 __device__ __forceinline__ void regs_compute() {
     asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kRegsCompute));
 }
-constexpr uint64_t kWaitNs = 2000000000ull;   // a legitimate wait lasts microseconds
+constexpr uint32_t kWaitNs = 2000000000u;   // a legitimate wait lasts microseconds
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kLn2 = 0.6931471805599453f;
 
@@ -49,20 +49,23 @@ __device__ __forceinline__ float ex2(float x) {
 // Bounded wait on an mbarrier phase.  After the first timeout anywhere in the
 // CTA every later wait returns immediately (false) so the CTA drains to its
 // teardown instead of hanging; the status word records the event.
+// The loop is compact and not unrolled: it is inlined at every wait of every
+// kernel, and small code keeps instruction-cache misses down.  The abort flag and
+// the clock are looked at every 64 polls.
 __device__ __forceinline__ bool wait_bar(uint64_t *bar, uint32_t parity, volatile int *abort_flag) {
     if (*abort_flag) return false;
-    if (ptx::mbar_try_wait(bar, parity)) return true;
-    const uint64_t t0 = ptx::globaltimer();
-    while (true) {
-        for (int i = 0; i < 32; ++i)
-            if (ptx::mbar_try_wait(bar, parity)) return true;
-        if (*abort_flag) return false;
-        if (ptx::globaltimer() - t0 > kWaitNs) {
-            *abort_flag = 1;
-            raise_status(DC_DEVERR_TIMEOUT);
-            return false;
+    uint32_t t0 = 0;
+#pragma unroll 1
+    for (uint32_t n = 1;; ++n) {
+        if (ptx::mbar_try_wait(bar, parity)) return true;
+        if ((n & 63) == 0) {
+            if (n == 64) t0 = ptx::globaltimer_lo();
+            if (*abort_flag || ptx::globaltimer_lo() - t0 > kWaitNs) break;
         }
     }
+    *abort_flag = 1;   // after a timeout anywhere in the CTA every later wait returns at once
+    raise_status(DC_DEVERR_TIMEOUT);
+    return false;
 }
 
 // Named barrier among `nthreads` threads (barrier 0 is __syncthreads).
