@@ -361,9 +361,9 @@ bwd_query_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
         compute_sync();
         // dP band: band[t][w] = dP(t, t - W + 1 + w) = tile column i + w.  The CTA's rows
         // are one contiguous [BM][W] block of the band: stage it in the ds tile region
-        // (free: every E MMA has completed) and copy it out with 16-byte stores.  The
-        // row stride W - 1 between lanes is odd for the usual even W, so the staging
-        // stores do not conflict.
+        // (free: every E MMA has completed) and write it with one bulk copy.  The row
+        // stride W - 1 between lanes is odd for the usual even W, so the staging stores
+        // do not conflict.
         {
             float *stage = (float *)(sm + L.rd);
             if (i < BM) {
@@ -381,17 +381,13 @@ bwd_query_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
             }
             ptx::fence_proxy_async_smem();
             compute_sync();
-            if (threadIdx.x == 0) {
-                stage_out(a.band + t0 * W, stage, (uint32_t)(min((int64_t)BM, s.N - t0) * W * 4));
-                ptx::bulk_wait_read();
-            }
-            compute_sync();
+            if (threadIdx.x == 0) stage_out(a.band + t0 * W, stage, (uint32_t)(min((int64_t)BM, s.N - t0) * W * 4));
         }
 
-        // ---- phase 2.  The ds tile region held dO, the pmap rows and the dP band in
-        // phase 1; zero its columns outside this quarter's band once.
+        // ---- phase 2.  The ds tile region held dO, the pmap rows and the dP band; the band
+        // copy reads it while head 0's scores are processed, and it is reused from head 0's
+        // ds tile on (columns outside this quarter's band zeroed once).
         uint8_t *dtile = sm + L.rd;
-        zero_outside_band(dtile, i, split, bd, span);
         auto drain_dq = [&](int h) {
             const int b = h & 1;
             wait_bar(&bars[kQBarDqFull + b], (uint32_t)(h >> 1) & 1, abort_flag);
@@ -451,7 +447,13 @@ bwd_query_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
                 const float ch = valid ? __ldg(a.c + t * H + h) : 0.f;
                 // the previous head's dQ MMA has been running meanwhile; once it has completed the
                 // ds tile is free for this head (its accumulator is drained after the tile is handed on)
-                if (h >= 1) wait_bar(&bars[kQBarDqFull + ((h - 1) & 1)], (uint32_t)((h - 1) >> 1) & 1, abort_flag);
+                if (h >= 1) {
+                    wait_bar(&bars[kQBarDqFull + ((h - 1) & 1)], (uint32_t)((h - 1) >> 1) & 1, abort_flag);
+                } else {
+                    if (threadIdx.x == 0) ptx::bulk_wait_read();   // the band copy has left the region
+                    compute_sync();
+                    zero_outside_band(dtile, i, split, bd, span);
+                }
 #pragma unroll
                 for (int cc = 0; cc < MAXC; ++cc) {
                     if (cc < bd.mync) {
