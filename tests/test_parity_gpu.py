@@ -81,6 +81,11 @@ EDGE_CASES = [
     ("bf16_d64_h12", [400, 129], 12, 64, 64, "bf16"),
     ("bf16_w1", [260], 6, 128, 1, "bf16"),
     ("bf16_short_docs", [5, 17, 3, 200, 9], 6, 128, 112, "bf16"),
+    # the widest window the tcgen05 kernels take (7 chunks of 8 columns per thread), the
+    # most heads, and the first window past it (served by the SIMT kernels)
+    ("bf16_w129", [700, 45], 4, 128, 129, "bf16"),
+    ("bf16_w120_h16_d64", [520], 16, 64, 120, "bf16"),
+    ("bf16_w130", [300], 2, 64, 130, "bf16"),
 ]
 
 
