@@ -256,23 +256,24 @@ def main():
     launches = [0]
 
     def step(x, ev=None):
+        # everything on the current stream (the capture stream while a graph is recorded)
         if ev is not None:
-            ev[0].record(stream)
+            ev[0].record()
         dcattn.dc_attn_fwd(x["q"], x["k"], x["v"], x["c"], x["g"], x["cu_seqlens"], W, scale,
                            o=x["o"], lse=x["lse"], pmap=x["pmap"])
         launches[0] += dcattn.dc_attn_last_launch_count()
         if ev is not None:
-            ev[1].record(stream)
+            ev[1].record()
         dcattn.dc_attn_bwd_query(x["q"], x["k"], x["v"], x["c"], x["g"], x["dO"], x["lse"], x["pmap"],
                                  x["cu_seqlens"], W, scale, dq=x["dq"], dc=x["dc"], dg=x["dg"], workspace=x["ws"])
         launches[0] += dcattn.dc_attn_last_launch_count()
         if ev is not None:
-            ev[2].record(stream)
+            ev[2].record()
         dcattn.dc_attn_bwd_key(x["q"], x["k"], x["c"], x["g"], x["dO"], x["lse"], x["pmap"], x["dc"], x["ws"],
                                x["cu_seqlens"], W, scale, dk=x["dk"], dv=x["dv"])
         launches[0] += dcattn.dc_attn_last_launch_count()
         if ev is not None:
-            ev[3].record(stream)
+            ev[3].record()
 
     sampler = ClockSampler(local)
     sampler.start()
@@ -283,24 +284,48 @@ def main():
     if dcattn.dc_attn_device_status() != 0:
         raise RuntimeError("device status word reports an error after warm-up")
 
-    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
+    # Timed region: one CUDA graph per input set holds one whole step (the three kernels);
+    # the graphs are replayed back to back with nothing between the kernels.
+    graphs = []
+    launches[0] = 0
+    for x in sets:
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            step(x)
+        graphs.append(g)
+    launches_per_step = launches[0] // N_SETS
+    torch.cuda.synchronize()
+    for it in range(args.warmup):
+        graphs[it % N_SETS].replay()
+    torch.cuda.synchronize()
+    if dcattn.dc_attn_device_status() != 0:
+        raise RuntimeError("device status word reports an error after the graph warm-up")
+    t_start, t_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     barrier(world)
     torch.cuda.synchronize()
-    launches[0] = 0
     t_wall0 = time.time()
+    t_start.record(stream)
     for it in range(args.steps):
-        step(sets[it % N_SETS], evs[it])
+        graphs[it % N_SETS].replay()
+    t_end.record(stream)
     torch.cuda.synchronize()
     t_wall1 = time.time()
     barrier(world)
-    total_ms = evs[0][0].elapsed_time(evs[-1][3])
-    per_kernel = {"fwd": 0.0, "bwd_query": 0.0, "bwd_key": 0.0}
-    for ev in evs:
-        per_kernel["fwd"] += ev[0].elapsed_time(ev[1])
-        per_kernel["bwd_query"] += ev[1].elapsed_time(ev[2])
-        per_kernel["bwd_key"] += ev[2].elapsed_time(ev[3])
-    per_kernel = {k: v / args.steps for k, v in per_kernel.items()}   # ms per launch
-    gpu_launches = launches[0]
+    total_ms = t_start.elapsed_time(t_end)
+    gpu_launches = launches_per_step * args.steps
+
+    # Per-kernel split: a second timed pass of the same steps, launched directly on the
+    # stream with CUDA events between the kernels (events inside the timed graphs would
+    # themselves slow the step down).
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
+    torch.cuda.synchronize()
+    for it in range(args.steps):
+        step(sets[it % N_SETS], evs[it])
+    torch.cuda.synchronize()
+    names = ("fwd", "bwd_query", "bwd_key")
+    per_kernel = {n: sum(ev[j].elapsed_time(ev[j + 1]) for ev in evs) / args.steps
+                  for j, n in enumerate(names)}   # ms per launch
+    split_ms_step = evs[0][0].elapsed_time(evs[-1][3]) / args.steps
     total_ms = allreduce_max(total_ms, world)
     ms_step = total_ms / args.steps
     value = world * N / (ms_step * 1e-3)
@@ -313,7 +338,7 @@ def main():
         t2 = time.time()
         it = 0
         while time.time() - t2 < 1.2:
-            step(sets[it % N_SETS])
+            graphs[it % N_SETS].replay()
             it += 1
             if it % 50 == 0:
                 torch.cuda.synchronize()
@@ -322,33 +347,63 @@ def main():
         clock_note = "sampled over ~1 s of the same step right after the timed region"
     sampler.stop()
 
-    # end to end through the public API: pinned host inputs -> device -> fwd+bwd -> host results
+    # end to end through the public API: pinned host inputs -> device -> fwd+bwd -> host
+    # results, every step.  The copies run on their own streams, so step i's upload and
+    # step i-1's read-back overlap step i's kernels (as a training loop would pipeline them);
+    # each set's buffers are reused only after their previous read-back has finished.
     e2e = None
     pin = {k: host[k].pin_memory() for k in ("q", "k", "v", "c", "g", "dO", "cu_seqlens")}
-    outs_host = {k: torch.empty(sets[0][k].shape, dtype=sets[0][k].dtype).pin_memory()
-                 for k in ("o", "dq", "dk", "dv", "dc", "dg")}
+    out_keys = ("o", "dq", "dk", "dv", "dc", "dg")
+    outs_host = [{k: torch.empty(sets[0][k].shape, dtype=sets[0][k].dtype).pin_memory() for k in out_keys}
+                 for _ in range(N_SETS)]
     h2d = sum(t.numel() * t.element_size() for t in pin.values())
-    d2h = sum(t.numel() * t.element_size() for t in outs_host.values())
+    d2h = sum(t.numel() * t.element_size() for t in outs_host[0].values())
+    up, down = torch.cuda.Stream(), torch.cuda.Stream()
     e2e_steps = max(3, min(args.steps, 20))
-    for rep in range(2):
-        if rep == 1:
-            barrier(world)
-            torch.cuda.synchronize()
-            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-            e0.record(stream)
-        for it in range(e2e_steps if rep == 1 else 3):
-            x = sets[it % N_SETS]
-            for k2 in pin:
-                x[k2].copy_(pin[k2], non_blocking=True)
+
+    def e2e_run(n):
+        freed = [None] * N_SETS            # read-back of the set's previous outputs done
+        for it in range(n):
+            si = it % N_SETS
+            x = sets[si]
+            ev_in = torch.cuda.Event()
+            with torch.cuda.stream(up):
+                if freed[si] is not None:
+                    up.wait_event(freed[si])
+                for k2 in pin:
+                    x[k2].copy_(pin[k2], non_blocking=True)
+                ev_in.record(up)
+            stream.wait_event(ev_in)
+            if freed[si] is not None:
+                stream.wait_event(freed[si])
             step(x)
-            for k2 in outs_host:
-                outs_host[k2].copy_(x[k2], non_blocking=True)
-        if rep == 1:
-            e1.record(stream)
-        torch.cuda.synchronize()
+            ev_out = torch.cuda.Event()
+            ev_out.record(stream)
+            with torch.cuda.stream(down):
+                down.wait_event(ev_out)
+                for k2 in out_keys:
+                    outs_host[si][k2].copy_(x[k2], non_blocking=True)
+                done = torch.cuda.Event()
+                done.record(down)
+            freed[si] = done
+        for f in freed:
+            if f is not None:
+                stream.wait_event(f)
+
+    e2e_run(3)
+    torch.cuda.synchronize()
+    barrier(world)
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    e2e_run(e2e_steps)
+    e1.record(stream)
+    torch.cuda.synchronize()
     e2e_ms = allreduce_max(e0.elapsed_time(e1) / e2e_steps, world)
     e2e = {"value": world * N / (e2e_ms * 1e-3), "unit": UNIT, "h2d_bytes_per_step": h2d,
-           "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms}
+           "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms,
+           "note": "dc_attn_* calls; inputs uploaded and outputs read back every step on copy streams "
+                   "that overlap neighbouring steps"}
 
     # roofline of the dominant kernel (HBM-bound path) against the measured copy bandwidth
     peaks = json.load(open(PEAKS_FILE)) if os.path.exists(PEAKS_FILE) else {}
@@ -373,6 +428,10 @@ def main():
             "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "bf16", "data": "synthetic", "impl": "dcattn", "kernels": impl,
             "config": config_block(cfg, world),
+            "timing": (f"value: {args.steps} back-to-back replays of one CUDA graph per input set (one graph = "
+                       f"one fwd+bwd step, {launches_per_step} kernels); kernel_ms: a second pass of the same "
+                       f"{args.steps} steps launched directly with CUDA events between the kernels "
+                       f"({split_ms_step * 1e3:.1f} us per step there)"),
             "roofline": {"bound": "hbm", "kernel": dom, "achieved": achieved, "peak": hbm, "unit": "GB/s",
                          "frac": achieved / hbm, "peak_source": peak_note, "traffic": traffic,
                          "algorithmic_bytes_per_launch": abytes[dom] * N},
