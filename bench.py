@@ -7,6 +7,7 @@ row, bf16, seeded synthetic inputs).  Prints one JSON line (rank 0).
 
   python bench.py [--gpus N --steps K --warmup W]      # libdcattn
   python bench.py --impl reference ...                 # the fp64 CPU oracle
+  python bench.py --sweep [--steps K --warmup W]       # every workload, one line each
 
 Multi-GPU runs are replicas (the path has no cross-GPU exchange): every rank
 runs the same workload on its own GPU; value = all tokens / max-over-ranks time.
@@ -215,6 +216,86 @@ def run_reference(args):
     return 0
 
 
+def run_sweep(args):
+    """One JSON line per workload of the inputs module (rank 0 only): the same graph-timed
+    step (forward, plus both backward kernels where the workload has a backward) on two
+    rotating input sets, with the step's fraction of the HBM roofline.  Shows which kernels
+    serve each shape (tcgen05 or SIMT)."""
+    from cross_head_dynamic_b200 import build, dcattn
+    if int(os.environ.get("RANK", "0")) != 0:
+        return 0
+    torch.cuda.set_device(0)
+    build.build()
+    dcattn.load_library()
+    dev = torch.device("cuda", 0)
+    peaks = json.load(open(PEAKS_FILE)) if os.path.exists(PEAKS_FILE) else {}
+    hbm = peaks.get("hbm_gbs") or 6650.0
+    for name, cfg in CONFIGS.items():
+        host = generate(cfg)
+        N, H, d, W, scale = cfg.total_tokens, cfg.heads, cfg.head_dim, cfg.window, cfg.softmax_scale
+        dt = host["q"].dtype
+        impl = dcattn.dc_attn_resolve_impl(host["q"].to(dev), host["cu_seqlens"].to(dev), W, scale)
+        sets = []
+        for r in range(2):
+            x = {k: (v.to(dev) if isinstance(v, torch.Tensor) else v) for k, v in host.items()}
+            if r:
+                for k in ("q", "k", "v", "dO"):
+                    if isinstance(x.get(k), torch.Tensor):
+                        x[k] = x[k].roll(1, dims=0).contiguous()
+            x["o"] = torch.empty_like(x["q"])
+            x["lse"] = torch.empty(N, H, device=dev)
+            x["pmap"] = torch.empty(N, W, device=dev, dtype=dt)
+            if cfg.backward:
+                x["dq"], x["dk"], x["dv"] = (torch.empty_like(x["q"]) for _ in range(3))
+                x["dc"], x["dg"] = torch.empty(N, H, device=dev), torch.empty(N, H, device=dev)
+                x["ws"] = torch.empty(max(16, dcattn.dc_attn_bwd_workspace_size(x["q"], x["cu_seqlens"], W, scale)),
+                                      device=dev, dtype=torch.uint8)
+            sets.append(x)
+
+        def step(x):
+            dcattn.dc_attn_fwd(x["q"], x["k"], x["v"], x["c"], x["g"], x["cu_seqlens"], W, scale,
+                               o=x["o"], lse=x["lse"], pmap=x["pmap"])
+            if cfg.backward:
+                dcattn.dc_attn_bwd_query(x["q"], x["k"], x["v"], x["c"], x["g"], x["dO"], x["lse"], x["pmap"],
+                                         x["cu_seqlens"], W, scale, dq=x["dq"], dc=x["dc"], dg=x["dg"],
+                                         workspace=x["ws"])
+                dcattn.dc_attn_bwd_key(x["q"], x["k"], x["c"], x["g"], x["dO"], x["lse"], x["pmap"], x["dc"],
+                                       x["ws"], x["cu_seqlens"], W, scale, dk=x["dk"], dv=x["dv"])
+
+        for x in sets:
+            step(x)
+        torch.cuda.synchronize()
+        graphs = []
+        for x in sets:
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g):
+                step(x)
+            graphs.append(g)
+        for it in range(args.warmup):
+            graphs[it % 2].replay()
+        torch.cuda.synchronize()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record()
+        for it in range(args.steps):
+            graphs[it % 2].replay()
+        b.record()
+        torch.cuda.synchronize()
+        if dcattn.dc_attn_device_status() != 0:
+            raise RuntimeError(f"device status word reports an error on {name}")
+        ms = a.elapsed_time(b) / args.steps
+        e = 4 if cfg.dtype == "f32" else 2
+        per_tok = (11 * H * d * e + 24 * H) if cfg.backward else (4 * H * d * e + 8 * H)
+        gbs = per_tok * N / (ms * 1e-3) / 1e9
+        print(json.dumps({"workload": name, "pass": "fwd+bwd" if cfg.backward else "fwd", "kernels": impl,
+                          "tokens": N, "heads": H, "head_dim": d, "window": W, "dtype": cfg.dtype,
+                          "docs": cfg.docs, "ms_per_step": ms, "tokens_per_s": N / (ms * 1e-3),
+                          "roofline": {"bound": "hbm", "achieved": gbs, "peak": hbm, "unit": "GB/s",
+                                       "frac": gbs / hbm, "algorithmic_bytes_per_token": per_tok}}), flush=True)
+        del graphs, sets
+        torch.cuda.empty_cache()
+    return 0
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -222,11 +303,15 @@ def main():
     ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--impl", choices=["dcattn", "reference"], default="dcattn")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--sweep", action="store_true",
+                    help="one JSON line per workload of the inputs module instead of the headline line")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
     if args.impl == "reference":
         return run_reference(args)
+    if args.sweep:
+        return run_sweep(args)
 
     from cross_head_dynamic_b200 import build, dcattn
     world, rank, local = dist_setup(args.gpus)
