@@ -14,17 +14,39 @@ namespace simt {
 
 constexpr int kMaxHeads = 16;
 
+// Floats of the per-warp row tile used by dot_rows32 (32 rows of d + 1).
+__host__ __device__ inline size_t tile_floats(int d) { return 32 * ((size_t)d + 1); }
 // Bytes of shared memory one warp needs in each kernel.
-inline size_t fwd_smem_per_warp(int H, int d, int W) { return sizeof(float) * ((size_t)H * d + kMaxHeads + W); }
-inline size_t bwdq_smem_per_warp(int H, int d, int W) { return sizeof(float) * (2 * (size_t)H * d + 3 * (size_t)W); }
-inline size_t bwdk_smem_per_warp(int H, int d, int W) { return sizeof(float) * ((size_t)H * d); }
+inline size_t fwd_smem_per_warp(int H, int d, int W) {
+    return sizeof(float) * ((size_t)H * d + kMaxHeads + W + tile_floats(d));
+}
+inline size_t bwdq_smem_per_warp(int H, int d, int W) {
+    return sizeof(float) * (2 * (size_t)H * d + 3 * (size_t)W + tile_floats(d));
+}
+inline size_t bwdk_smem_per_warp(int H, int d, int W) { return sizeof(float) * ((size_t)H * d + tile_floats(d)); }
 
+// <xs, row(lane)> for up to 32 consecutive rows, row r at rows + r * stride (d = 32 * DPL
+// elements, xs in shared memory).  The rows pass through this warp's tile with coalesced
+// loads (the warp reads one row at a time), then every lane takes its own row from the
+// tile; rows are d + 1 floats apart, so those reads hit 32 distinct banks.  All lanes
+// call it; lanes >= cnt get 0.
 template <typename T, int DPL>
-__device__ __forceinline__ float dot_row(const float *xs, const T *row) {
-    // <xs, row> over d = 32*DPL elements; xs is in shared memory (broadcast read).
+__device__ __forceinline__ float dot_rows32(const float *xs, const T *rows, int64_t stride, int cnt, float *tile) {
+    constexpr int d = 32 * DPL;
+    const int lane = threadIdx.x & 31;
+    __syncwarp();
+    for (int r = 0; r < cnt; ++r) {
+        const T *src = rows + r * stride;
+#pragma unroll
+        for (int i = 0; i < DPL; ++i) tile[r * (d + 1) + lane + 32 * i] = ldf<T>(src + lane + 32 * i);
+    }
+    __syncwarp();
     float acc = 0.f;
+    if (lane < cnt) {
+        const float *tr = tile + lane * (d + 1);
 #pragma unroll 8
-    for (int e = 0; e < 32 * DPL; ++e) acc = fmaf(xs[e], ldf<T>(row + e), acc);
+        for (int e = 0; e < d; ++e) acc = fmaf(xs[e], tr[e], acc);
+    }
     return acc;
 }
 
@@ -42,9 +64,10 @@ __global__ void fwd_kernel(Shape s, const T *__restrict__ q, const T *__restrict
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int64_t t = (int64_t)blockIdx.x * (blockDim.x >> 5) + warp;
     if (t >= s.N) return;
-    float *qs = smem + (size_t)warp * (H * d + kMaxHeads + W);
+    float *qs = smem + (size_t)warp * (H * d + kMaxHeads + W + tile_floats(d));
     float *ls = qs + H * d;
     float *Pw = ls + kMaxHeads;
+    float *tile = Pw + W;
 
     for (int i = lane; i < H * d; i += 32) qs[i] = ldf<T>(q + t * H * d + i);
     __syncwarp();
@@ -53,13 +76,17 @@ __global__ void fwd_kernel(Shape s, const T *__restrict__ q, const T *__restrict
 
     for (int h = 0; h < H; ++h) {
         float m = -INFINITY, z = 0.f;
-        for (int jj = lane; jj < n; jj += 32) {
-            float x = s.scale * dot_row<T, DPL>(qs + h * d, k + ((lo + jj) * H + h) * d);
-            if (x > m) {
-                z = z * expf(m - x) + 1.f;
-                m = x;
-            } else {
-                z += expf(x - m);
+        for (int base = 0; base < n; base += 32) {
+            const int cnt = min(32, n - base);
+            const float x = s.scale * dot_rows32<T, DPL>(qs + h * d, k + ((lo + base) * H + h) * d, (int64_t)H * d,
+                                                         cnt, tile);
+            if (lane < cnt) {
+                if (x > m) {
+                    z = z * expf(m - x) + 1.f;
+                    m = x;
+                } else {
+                    z += expf(x - m);
+                }
             }
         }
         const float M = warp_max(m);
@@ -72,13 +99,15 @@ __global__ void fwd_kernel(Shape s, const T *__restrict__ q, const T *__restrict
         }
     }
     __syncwarp();
-    for (int jj = lane; jj < n; jj += 32) {
+    for (int base = 0; base < n; base += 32) {
+        const int cnt = min(32, n - base);
         float P = 0.f;
         for (int h = 0; h < H; ++h) {
-            float x = s.scale * dot_row<T, DPL>(qs + h * d, k + ((lo + jj) * H + h) * d);
+            const float x = s.scale * dot_rows32<T, DPL>(qs + h * d, k + ((lo + base) * H + h) * d, (int64_t)H * d,
+                                                         cnt, tile);
             P = fmaf(__ldg(c + t * H + h), expf(x - ls[h]), P);
         }
-        Pw[jj] = P;
+        if (lane < cnt) Pw[base + lane] = P;
     }
     __syncwarp();
     if (pmap) {
@@ -119,11 +148,12 @@ __global__ void bwd_query_kernel(Shape s, const T *__restrict__ q, const T *__re
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int64_t t = (int64_t)blockIdx.x * (blockDim.x >> 5) + warp;
     if (t >= s.N) return;
-    float *qs = smem + (size_t)warp * (2 * H * d + 3 * W);
+    float *qs = smem + (size_t)warp * (2 * H * d + 3 * W + tile_floats(d));
     float *dos = qs + H * d;
     float *Pw = dos + H * d;
     float *dPw = Pw + W;
     float *sw = dPw + W;
+    float *tile = sw + W;
 
     for (int i = lane; i < H * d; i += 32) {
         qs[i] = ldf<T>(q + t * H * d + i);
@@ -139,18 +169,23 @@ __global__ void bwd_query_kernel(Shape s, const T *__restrict__ q, const T *__re
     float dgp[kMaxHeads];
 #pragma unroll
     for (int h = 0; h < kMaxHeads; ++h) dgp[h] = 0.f;
-    for (int jj = lane; jj < n; jj += 32) {
+    for (int base = 0; base < n; base += 32) {
+        const int cnt = min(32, n - base);
+        const int jj = base + lane;
+        const float pj = lane < cnt ? Pw[jj] : 0.f;
         float dP = 0.f;
 #pragma unroll
         for (int h = 0; h < kMaxHeads; ++h) {
             if (h < H) {
-                const float E = dot_row<T, DPL>(dos + h * d, v + ((lo + jj) * H + h) * d);
+                const float E = dot_rows32<T, DPL>(dos + h * d, v + ((lo + base) * H + h) * d, (int64_t)H * d, cnt, tile);
                 dP = fmaf(__ldg(g + t * H + h), E, dP);
-                dgp[h] = fmaf(Pw[jj], E, dgp[h]);
+                dgp[h] = fmaf(pj, E, dgp[h]);
             }
         }
-        dPw[jj] = dP;
-        dPband[t * W + w0 + jj] = dP;
+        if (lane < cnt) {
+            dPw[jj] = dP;
+            dPband[t * W + w0 + jj] = dP;
+        }
     }
 #pragma unroll
     for (int h = 0; h < kMaxHeads; ++h) {
@@ -164,11 +199,15 @@ __global__ void bwd_query_kernel(Shape s, const T *__restrict__ q, const T *__re
     for (int h = 0; h < H; ++h) {
         const float l = __ldg(lse + t * H + h);
         float dcp = 0.f;
-        for (int jj = lane; jj < n; jj += 32) {
-            const float x = s.scale * dot_row<T, DPL>(qs + h * d, k + ((lo + jj) * H + h) * d);
-            const float p = expf(x - l);
-            sw[jj] = p;
-            dcp = fmaf(dPw[jj], p, dcp);
+        for (int base = 0; base < n; base += 32) {
+            const int cnt = min(32, n - base);
+            const float x = s.scale * dot_rows32<T, DPL>(qs + h * d, k + ((lo + base) * H + h) * d, (int64_t)H * d,
+                                                         cnt, tile);
+            if (lane < cnt) {
+                const float p = expf(x - l);
+                sw[base + lane] = p;
+                dcp = fmaf(dPw[base + lane], p, dcp);
+            }
         }
         const float dch = warp_sum(dcp);
         if (lane == 0) dc[t * H + h] = dch;
@@ -206,7 +245,8 @@ __global__ void bwd_key_kernel(Shape s, const T *__restrict__ q, const T *__rest
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int64_t j = (int64_t)blockIdx.x * (blockDim.x >> 5) + warp;
     if (j >= s.N) return;
-    float *ks = smem + (size_t)warp * (H * d);
+    float *ks = smem + (size_t)warp * (H * d + tile_floats(d));
+    float *tile = ks + H * d;
     for (int i = lane; i < H * d; i += 32) ks[i] = ldf<T>(k + j * H * d + i);
     __syncwarp();
     int64_t hi = j + W - 1;
@@ -220,10 +260,12 @@ __global__ void bwd_key_kernel(Shape s, const T *__restrict__ q, const T *__rest
         for (int i = 0; i < DPL; ++i) ak[i] = av[i] = 0.f;
         for (int base = 0; base < n; base += 32) {
             float ds = 0.f, pg = 0.f;
+            const int cnt0 = min(32, n - base);
+            const float x = s.scale * dot_rows32<T, DPL>(ks + h * d, q + ((j + base) * H + h) * d, (int64_t)H * d,
+                                                         cnt0, tile);
             if (base + lane < n) {
                 const int64_t t = j + base + lane;
                 const int64_t w = j - (t - W + 1);
-                const float x = s.scale * dot_row<T, DPL>(ks + h * d, q + (t * H + h) * d);
                 const float p = expf(x - __ldg(lse + t * H + h));
                 ds = __ldg(c + t * H + h) * p * (__ldg(dPband + t * W + w) - __ldg(dc + t * H + h));
                 pg = ldf<T>(pmap + t * W + w) * __ldg(g + t * H + h);
