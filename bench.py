@@ -161,9 +161,19 @@ def allreduce_max(x: float, world: int) -> float:
     if world == 1:
         return x
     import torch.distributed as dist
-    t = torch.tensor([x], device="cuda", dtype=torch.float64)
+    dev = "cuda" if dist.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([x], device=dev, dtype=torch.float64)
     dist.all_reduce(t, op=dist.ReduceOp.MAX)
     return float(t.item())
+
+
+def replica_throughput(tokens_per_rank: int, local_ms: float, steps: int, world: int):
+    """Whole-job throughput of `world` replicas that each ran `steps` steps of
+    `tokens_per_rank` tokens in `local_ms` (device time): every rank's work over the
+    slowest rank's time.  Returns (tokens/s, ms per step)."""
+    total_ms = allreduce_max(local_ms, world)
+    ms_step = total_ms / steps
+    return world * tokens_per_rank / (ms_step * 1e-3), ms_step
 
 
 def oracle_sample_rate(cfg, rows: int, reps: int = 1):
@@ -411,9 +421,7 @@ def main():
     per_kernel = {n: sum(ev[j].elapsed_time(ev[j + 1]) for ev in evs) / args.steps
                   for j, n in enumerate(names)}   # ms per launch
     split_ms_step = evs[0][0].elapsed_time(evs[-1][3]) / args.steps
-    total_ms = allreduce_max(total_ms, world)
-    ms_step = total_ms / args.steps
-    value = world * N / (ms_step * 1e-3)
+    value, ms_step = replica_throughput(N, total_ms, args.steps, world)
 
     clocks = sampler.summary(t_wall0, t_wall1)
     clock_note = "sampled during the timed region"
