@@ -8,9 +8,10 @@
 // Query side (one CTA per block of BM query tokens, all heads):
 //   phase 1, per head: MMA E_h = dO_h V_h^T -> TMEM; SIMT dP += g_h E_h
 //            (registers), dg_h = sum_j P E_h with P from the forward's pmap
-//            (the CTA's pmap rows are staged in shared memory once); dP is then
-//            stored as a band [N][W] in the workspace for the key side, which
-//            must see exactly the dP that dc was computed from.
+//            (the CTA's pmap rows arrive by one bulk load and are kept in
+//            registers); dP is then written, by one bulk store, as a band [N][W]
+//            in the workspace for the key side, which must see exactly the dP
+//            that dc was computed from.
 //   phase 2, per head: MMA S_h = Q_h K_h^T -> TMEM; SIMT p_h from lse,
 //            dc_h = sum_j dP p_h, ds_h -> bf16 tile in smem; MMA dQ_h = ds_h K_h.
 // Key side (one CTA per block of BK key tokens; the queries that see them span
@@ -20,8 +21,9 @@
 //   phase 2, per head: MMA S^T_h = K_h Q_h^T -> TMEM; SIMT ds^T from lse, c,
 //            dc and the query side's dP; MMA dK_h = ds^T_h Q_h.
 // In both phase-2 loops the gradient MMA of head h runs while the SIMT warps
-// work on the scores of head h+1: the producer issues S_{h+1} before dQ_h/dK_h,
-// and the warps drain head h's accumulator one iteration later.
+// work on the scores of head h+1: the producer issues S_{h+1} before dQ_h/dK_h;
+// the warps write the next ds tile once that MMA has read the current one and
+// then drain its accumulator (two accumulator buffers in TMEM).
 // Same thread roles as the forward: warps 0-11 SIMT (three per TMEM lane
 // quarter), warp 12 lane 0 issues TMA and MMA; every wait is bounded.
 #pragma once

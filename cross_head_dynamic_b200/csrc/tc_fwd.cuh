@@ -13,9 +13,10 @@
 //           document, softmax per row, P += c[t,h] * p_h with P accumulated in
 //           registers (the H maps never leave the chip)
 // Phase 2:
-//   SIMT    P -> bf16 tile in smem (K-major, swizzled), band copy -> pmap
-//   per head: TMA V_h [span x d]; MMA U_h = P V_h -> TMEM [128 x d];
-//           SIMT o_h = g[t,h] * U_h -> bf16 -> global
+//   SIMT    P -> bf16 tile in smem (K-major, swizzled); the block's pmap rows
+//           -> smem -> one bulk copy to global
+//   per head: TMA V_h [span x d]; MMA U_h = P V_h -> TMEM [128 x d] (two
+//           buffers); SIMT o_h = g[t,h] * U_h -> bf16 -> global (32-byte stores)
 //
 // Warps 0-11 do the SIMT work: warp w reads TMEM lanes 32*(w%4).. (rows of
 // the tile) and part w/4 of its quarter's column band.  Warp 12 lane 0
