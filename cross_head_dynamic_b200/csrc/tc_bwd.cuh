@@ -728,13 +728,9 @@ bwd_key_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant_
             ptx::mbar_arrive(&bars[kKBarAccFree + b]);
         };
 
-        // ---- phase 1: dV (scaling dO_h runs ahead of draining dV_{h-1}; one copy of each)
-        for (int h = 0; h <= H; ++h) {
-            if (h < H) scale_do(h);
-            if (h >= 1) drain(h - 1, a.dv, h - 1, 1.f);
-        }
-
-        // ---- phase 2: dK.  dP(t, j) for this row's band from the query side's workspace
+        // Phase-2 inputs that phase 1 does not touch are fetched now, so that their loads run
+        // during phase 1: dP(t, j) for this row's band from the query side's workspace, and
+        // head 0's per-query vectors.
         float dPT[MAXC][8];
 #pragma unroll
         for (int cc = 0; cc < MAXC; ++cc) {
@@ -748,7 +744,6 @@ bwd_key_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant_
                 }
             }
         }
-        uint8_t *dtile = sm + L.ra;   // ds^T tile reuses the P^T region (every dV MMA has completed)
         // per-query vectors of head h in colv[h & 1]: [lse * log2e | c | dc], one query column
         // per thread (span <= 256 < kComputeThreads); head h+1's values are fetched while
         // head h is processed
@@ -769,7 +764,16 @@ bwd_key_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant_
             }
         };
         fetch_colv(0);
-        store_colv(0);
+        store_colv(0);   // published by the first phase-2 compute_sync
+
+        // ---- phase 1: dV (scaling dO_h runs ahead of draining dV_{h-1}; one copy of each)
+        for (int h = 0; h <= H; ++h) {
+            if (h < H) scale_do(h);
+            if (h >= 1) drain(h - 1, a.dv, h - 1, 1.f);
+        }
+
+        // ---- phase 2: dK
+        uint8_t *dtile = sm + L.ra;   // ds^T tile reuses the P^T region (every dV MMA has completed)
         for (int h = 0; h <= H; ++h) {   // h == H only drains dK_{H-1}
             if (h < H) {
                 const float *cv = colv + (h & 1) * 768;
