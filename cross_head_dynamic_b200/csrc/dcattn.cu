@@ -154,6 +154,11 @@ dc_status_t dc_attn_fwd(const dc_attn_params *params, const void *q, const void 
     r = ptrs_ok({q, k, v, c, g, o}, {lse, pmap});
     if (r != DC_OK) return r;
     cudaStream_t st = (cudaStream_t)stream;
+    // a window cut into segments keeps the per-segment LSE in lse: without it, SIMT
+    if (ck.impl == DC_IMPL_TCGEN05 && dc::tc::segmented(ck.s) && !lse) {
+        if (params->impl == DC_IMPL_TCGEN05) return DC_ERR_UNSUPPORTED;
+        ck.impl = DC_IMPL_SIMT;
+    }
     if (ck.impl == DC_IMPL_TCGEN05)
         return cuda_status(dc::tc::fwd(ck.s, q, k, v, c, g, o, lse, pmap, st, &t_launches));
     return cuda_status(DC_DISPATCH(simt_fwd, ck.dtype, ck.s.d, ck.s, q, k, v, c, g, o, lse, pmap, st));

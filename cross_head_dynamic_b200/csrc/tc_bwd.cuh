@@ -50,12 +50,20 @@ struct BwdArgs {
     float *band;           // dP band [N][W]: written by the query side, read by the key side
     __nv_bfloat16 *dk;     // key side out
     __nv_bfloat16 *dv;
+    Seg seg;               // window segment (segmented instantiations only)
 };
+
+// Segmented query side, launched in this order: the far segment's dP band, dg and dc
+// (partial sums); the near segment, which completes dg and dc and writes its share of
+// dq; the far segment again, which adds its share of dq (it needs the complete dc).
+enum : int { kQSegFarPart1 = 1, kQSegNear = 2, kQSegFarPart2 = 3 };
+// Segmented key side: the first segment writes dk and dv, the next one adds to them.
+enum : int { kKSegWrite = 1, kKSegAdd = 2 };
 
 // Drain this split's 16-column chunks of one row of a [128 x D] fp32 accumulator
 // (row base address taddr, output row dst): scale, round to bf16, store when `store`
 // (full 32-byte sectors; aligned32 says whether the output buffer allows 256-bit stores).
-template <int D>
+template <int D, bool ADD = false>
 __device__ __forceinline__ void drain_row(uint32_t taddr, __nv_bfloat16 *dst, float mult, bool store, int split,
                                           bool aligned32) {
     int cb16, ce16;
@@ -73,6 +81,7 @@ __device__ __forceinline__ void drain_row(uint32_t taddr, __nv_bfloat16 *dst, fl
 #pragma unroll
                 for (int e = 0; e < 8; ++e)
                     w[e] = pack_bf16x2(mult * __uint_as_float(r[2 * e]), mult * __uint_as_float(r[2 * e + 1]));
+                if constexpr (ADD) add_bf16x16(w, dst + (cb16 + c) * 16, mult, r);   // dst += mult * acc
                 ptx::st_global_32b(dst + (cb16 + c) * 16, w, aligned32);
             }
         }
@@ -120,7 +129,7 @@ struct QSideLayout {
     }
 };
 
-template <int D, int MAXC>
+template <int D, int MAXC, bool SEG = false>
 __global__ void __launch_bounds__(kThreads, 1)
 bwd_query_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__ CUtensorMap map_k,
                  const __grid_constant__ CUtensorMap map_v, const __grid_constant__ CUtensorMap map_do,
@@ -137,7 +146,10 @@ bwd_query_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int64_t t0 = (int64_t)blockIdx.x * BM;
-    const int64_t kbase = t0 - (W - 1);
+    const int64_t kbase = SEG ? t0 - a.seg.shift - (W - 1) : t0 - (W - 1);
+    const bool do_p1 = !SEG || a.seg.mode != kQSegFarPart2;   // phase 1 (E, dP band, dg)
+    const bool do_dq = !SEG || a.seg.mode != kQSegFarPart1;   // ds and dQ
+    const int ph0 = do_p1 ? H : 0;                            // X-buffer phases before phase 2
 
     validate_seqlens(s);
     if (threadIdx.x == 0) {
@@ -205,12 +217,17 @@ bwd_query_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
             };
 
             // the CTA's pmap rows (one contiguous [BM][W] run) into the upper half of the ds
-            // tile region, which phase 1 does not use
-            stage_in(sm + L.rd + 32768, a.pmap + t0 * W, (uint32_t)(min((int64_t)BM, s.N - t0) * W * 2),
-                     &bars[kQBarPmap]);
+            // tile region, which phase 1 does not use (a segment reads its columns directly)
+            if (!SEG)
+                stage_in(sm + L.rd + 32768, a.pmap + t0 * W, (uint32_t)(min((int64_t)BM, s.N - t0) * W * 2),
+                         &bars[kQBarPmap]);
+            if (!do_p1) {   // no phase 1: the phase-2 tiles load at once
+                issue_q(0);
+                for (int b = 0; b < 2 && b < H; ++b) issue_k(b);
+            }
             // ---- phase 1: E_h = dO_h V_h^T
-            for (int h = 0; h < H && h < 2; ++h) issue_e(h);
-            for (int h = 0; h < H; ++h) {
+            for (int h = 0; h < (do_p1 ? H : 0) && h < 2; ++h) issue_e(h);
+            for (int h = 0; h < (do_p1 ? H : 0); ++h) {
                 const int b = h & 1;
                 bool ok = wait_bar(&bars[kQBarLd + b], (uint32_t)(h >> 1) & 1, abort_flag);
                 if (h >= 1) ok = wait_bar(&bars[kQBarXFree], (uint32_t)(h - 1) & 1, abort_flag) && ok;
@@ -239,12 +256,12 @@ bwd_query_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
             }
             // ---- phase 2: S_h = Q_h K_h^T; dQ_{h-1} = ds_{h-1} K_{h-1} right after it
             for (int h = 0; h <= H; ++h) {   // h == H only issues dQ_{H-1}
-                const uint32_t ph = (uint32_t)(H + h);
+                const uint32_t ph = (uint32_t)(ph0 + h);
                 if (h < H) {
                     const int b = h & 1;
                     bool ok = wait_bar(&bars[kQBarQ], (uint32_t)h & 1, abort_flag);
                     ok = wait_bar(&bars[kQBarK + b], (uint32_t)(h >> 1) & 1, abort_flag) && ok;
-                    ok = wait_bar(&bars[kQBarXFree], (ph - 1) & 1, abort_flag) && ok;
+                    if (ph >= 1) ok = wait_bar(&bars[kQBarXFree], (ph - 1) & 1, abort_flag) && ok;
                     ptx::tc_fence_after();
                     if (ok) {
                         const uint32_t qa = ptx::smem_u32(sm + L.rq);
@@ -258,12 +275,15 @@ bwd_query_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
                     }
                     ptx::mma_commit(&bars[kQBarXFull]);
                 }
-                if (h >= 1) mma_dq(h - 1);
+                if (h >= 1 && do_dq) mma_dq(h - 1);
                 if (h < H) {
-                    // refill: Q_{h+1} once S_h has read Q; K_{h+1} once dQ_{h-1} has read K_{h-1}
-                    if (wait_bar(&bars[kQBarXFull], ph & 1, abort_flag) && h + 1 < H) issue_q(h + 1);
+                    // refill: Q_{h+1} once S_h has read Q; K_{h+1} once dQ_{h-1} (or, with no dQ,
+                    // S_{h-1}, which completed before S_h) has read K_{h-1}
+                    const bool s_done = wait_bar(&bars[kQBarXFull], ph & 1, abort_flag);
+                    if (s_done && h + 1 < H) issue_q(h + 1);
                     if (h >= 1 && h + 1 < H &&
-                        wait_bar(&bars[kQBarDqFull + ((h - 1) & 1)], (uint32_t)((h - 1) >> 1) & 1, abort_flag))
+                        (do_dq ? wait_bar(&bars[kQBarDqFull + ((h - 1) & 1)], (uint32_t)((h - 1) >> 1) & 1, abort_flag)
+                               : s_done))
                         issue_k(h + 1);
                 }
             }
@@ -278,8 +298,16 @@ bwd_query_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
         const bool valid = (i < BM) && (t < s.N);
         int clo = 1, chi = 0;
         if (valid) {
-            clo = (int)(window_lo(s, t) - kbase);
-            chi = (int)(t - kbase);
+            if constexpr (SEG) {
+                int64_t lo, hi;
+                if (seg_window(s, t, a.seg.shift, lo, hi)) {
+                    clo = (int)(lo - kbase);
+                    chi = (int)(hi - kbase);
+                }
+            } else {
+                clo = (int)(window_lo(s, t) - kbase);
+                chi = (int)(t - kbase);
+            }
         }
         const Band bd = make_band(q, split, BM, W, span);
         const uint32_t lane_base = (uint32_t)(32 * q) << 16;
@@ -288,8 +316,24 @@ bwd_query_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
 
         // P(t, c) = pmap[t][c - i] on this thread's band, from the CTA's pmap rows staged by
         // the producer; zero outside the window.  Kept in registers (bf16 pairs) for all heads.
+        // A segment reads its columns of the row from global memory.
         uint32_t pvp[MAXC][4];
-        {
+        if constexpr (SEG) {
+            const uint16_t *prow = (const uint16_t *)a.pmap + t * a.seg.wrow + a.seg.wofs - i;   // prow[c], c in window
+#pragma unroll
+            for (int cc = 0; cc < MAXC; ++cc) {
+                if (cc < bd.mync) {
+                    const int col = bd.cb + (bd.c0 + cc) * 8;
+#pragma unroll
+                    for (int e = 0; e < 8; e += 2) {
+                        const int c0 = col + e, c1 = c0 + 1;
+                        const uint32_t lo = (do_p1 && c0 >= clo && c0 <= chi) ? __ldg(prow + c0) : 0u;
+                        const uint32_t hi = (do_p1 && c1 >= clo && c1 <= chi) ? __ldg(prow + c1) : 0u;
+                        pvp[cc][e >> 1] = lo | (hi << 16);
+                    }
+                }
+            }
+        } else {
             const uint16_t *prow = (const uint16_t *)(sm + L.rd + 32768) + i * W - i;
             wait_bar(&bars[kQBarPmap], 0, abort_flag);
 #pragma unroll
@@ -311,11 +355,25 @@ bwd_query_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
         for (int cc = 0; cc < MAXC; ++cc)
 #pragma unroll
             for (int e = 0; e < 8; ++e) dP[cc][e] = 0.f;
+        if (SEG && !do_p1) {   // dP from the band the first far-segment launch wrote
+            const float *brow = a.band + t * a.seg.wrow + a.seg.wofs - i;   // brow[c], c in window
+#pragma unroll
+            for (int cc = 0; cc < MAXC; ++cc) {
+                if (cc < bd.mync) {
+                    const int col = bd.cb + (bd.c0 + cc) * 8;
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) {
+                        const int cidx = col + e;
+                        if (cidx >= clo && cidx <= chi) dP[cc][e] = __ldg(brow + cidx);
+                    }
+                }
+            }
+        }
 
         // ---- phase 1: dP and dg, three chunks of E_h per TMEM round trip.  dP is left
         // unmasked: outside the window it only ever meets p = 0 (and the key side reads
         // the band inside the window only); P is zero there, so dg needs no mask either.
-        for (int h = 0; h < H; ++h) {
+        for (int h = 0; h < (do_p1 ? H : 0); ++h) {
             wait_bar(&bars[kQBarXFull], (uint32_t)h & 1, abort_flag);
             ptx::tc_fence_after();
             const float gh = valid ? __ldg(a.g + t * H + h) : 0.f;
@@ -356,6 +414,9 @@ bwd_query_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
                 float sum = rd[i];
 #pragma unroll
                 for (int sp = 1; sp < kSplits; ++sp) sum += rd[sp * 128 + i];
+                if constexpr (SEG) {   // the near segment completes the far segment's partial sum
+                    if (a.seg.mode == kQSegNear) sum += a.dg[t * H + h];
+                }
                 a.dg[t * H + h] = sum;
             }
         }
@@ -365,8 +426,24 @@ bwd_query_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
         // are one contiguous [BM][W] block of the band: stage it in the ds tile region
         // (free: every E MMA has completed) and write it with one bulk copy.  The row
         // stride W - 1 between lanes is odd for the usual even W, so the staging stores
-        // do not conflict.
-        {
+        // do not conflict.  A segment owns only columns wofs .. wofs + W - 1 of each row: plain
+        // stores.
+        if constexpr (SEG) {
+            if (do_p1 && valid) {
+                float *brow = a.band + t * a.seg.wrow + a.seg.wofs;   // brow[w], w < W
+#pragma unroll
+                for (int cc = 0; cc < MAXC; ++cc) {
+                    if (cc < bd.mync) {
+                        const int col = bd.cb + (bd.c0 + cc) * 8;
+#pragma unroll
+                        for (int e = 0; e < 8; ++e) {
+                            const uint32_t w = (uint32_t)(col + e - i);
+                            if (w < (uint32_t)W) brow[w] = dP[cc][e];
+                        }
+                    }
+                }
+            }
+        } else {
             float *stage = (float *)(sm + L.rd);
             if (i < BM) {
 #pragma unroll
@@ -394,14 +471,18 @@ bwd_query_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
             const int b = h & 1;
             wait_bar(&bars[kQBarDqFull + b], (uint32_t)(h >> 1) & 1, abort_flag);
             ptx::tc_fence_after();
-            drain_row<D>(tmem + lane_base + 256 + 128 * b, a.dq + (t * H + h) * D, s.scale, valid, split,
-                         ((uintptr_t)a.dq & 31) == 0);
+            if (SEG && a.seg.mode == kQSegFarPart2)   // adds the far segment's share to dq
+                drain_row<D, true>(tmem + lane_base + 256 + 128 * b, a.dq + (t * H + h) * D, s.scale, valid, split,
+                                   ((uintptr_t)a.dq & 31) == 0);
+            else
+                drain_row<D>(tmem + lane_base + 256 + 128 * b, a.dq + (t * H + h) * D, s.scale, valid, split,
+                             ((uintptr_t)a.dq & 31) == 0);
             ptx::tc_fence_before();
             ptx::mbar_arrive(&bars[kQBarDqFree + b]);
         };
-        for (int h = 0; h <= H; ++h) {   // h == H only drains dQ_{H-1}
+        for (int h = 0; h <= (do_dq ? H : H - 1); ++h) {   // h == H only drains dQ_{H-1}
             if (h < H) {
-                const uint32_t ph = (uint32_t)(H + h);
+                const uint32_t ph = (uint32_t)(ph0 + h);
                 wait_bar(&bars[kQBarXFull], ph & 1, abort_flag);
                 ptx::tc_fence_after();
                 const float lse2 = valid ? __ldg(a.lse + t * H + h) * kLog2e : 0.f;
@@ -439,20 +520,30 @@ bwd_query_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
                 }
                 ptx::tc_fence_before();
                 ptx::mbar_arrive(&bars[kQBarXFree]);
-                float *rd = red + (ph & 1) * (kSplits * 128);
-                rd[split * 128 + i] = dca + dcb;
-                pair_sync(q);
-                float dch = rd[i];
+                float dch;
+                if (SEG && a.seg.mode == kQSegFarPart2) {   // dc is complete: the near launch wrote it
+                    dch = valid ? a.dc[t * H + h] : 0.f;
+                } else {
+                    // the near segment adds the far segment's partial dc (read before any split
+                    // of this row writes the sum)
+                    const float dc_far = (SEG && a.seg.mode == kQSegNear && valid) ? a.dc[t * H + h] : 0.f;
+                    float *rd = red + (ph & 1) * (kSplits * 128);
+                    rd[split * 128 + i] = dca + dcb;
+                    pair_sync(q);
+                    dch = rd[i];
 #pragma unroll
-                for (int sp = 1; sp < kSplits; ++sp) dch += rd[sp * 128 + i];
-                if (split == 0 && valid) a.dc[t * H + h] = dch;
+                    for (int sp = 1; sp < kSplits; ++sp) dch += rd[sp * 128 + i];
+                    if constexpr (SEG) dch += dc_far;
+                    if (split == 0 && valid) a.dc[t * H + h] = dch;
+                }
+                if (!do_dq) continue;   // the first far-segment launch stops at dc
                 const float ch = valid ? __ldg(a.c + t * H + h) : 0.f;
                 // the previous head's dQ MMA has been running meanwhile; once it has completed the
                 // ds tile is free for this head (its accumulator is drained after the tile is handed on)
                 if (h >= 1) {
                     wait_bar(&bars[kQBarDqFull + ((h - 1) & 1)], (uint32_t)((h - 1) >> 1) & 1, abort_flag);
                 } else {
-                    if (threadIdx.x == 0) ptx::bulk_wait_read();   // the band copy has left the region
+                    if (!SEG && threadIdx.x == 0) ptx::bulk_wait_read();   // the band copy has left the region
                     compute_sync();
                     zero_outside_band(dtile, i, split, bd, span);
                 }
@@ -509,7 +600,7 @@ struct KSideLayout {
     }
 };
 
-template <int D, int MAXC>
+template <int D, int MAXC, bool SEG = false>
 __global__ void __launch_bounds__(kThreads, 1)
 bwd_key_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__ CUtensorMap map_k,
                const __grid_constant__ CUtensorMap map_do, const BwdArgs a) {
@@ -525,6 +616,8 @@ bwd_key_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant_
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int64_t j0 = (int64_t)blockIdx.x * BK;
+    // first query of the span: a segment's queries start `shift` tokens after the key block
+    const int64_t qbase = SEG ? j0 + a.seg.shift : j0;
 
     if (threadIdx.x == 0) {
         for (int i = 0; i < kKNumBars; ++i) {
@@ -555,7 +648,7 @@ bwd_key_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant_
                 const int h = idx < H ? idx : idx - H;
                 ptx::mbar_arrive_expect_tx(&bars[kKBarLd + b], L.tile_s);
                 for (int kb = 0; kb < D / 64; ++kb)
-                    ptx::tma_load_2d(dst + kb * span * 128, map, h * D + kb * 64, (int)j0, &bars[kKBarLd + b]);
+                    ptx::tma_load_2d(dst + kb * span * 128, map, h * D + kb * 64, (int)qbase, &bars[kKBarLd + b]);
             };
             auto issue_k = [&](int h) {
                 ptx::mbar_arrive_expect_tx(&bars[kKBarK], 128u * D * 2);
@@ -584,14 +677,16 @@ bwd_key_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant_
                 }
                 ptx::mma_commit(&bars[kKBarAccFull + b]);
             };
-            // pmap rows j0 .. j0+span-1 (one contiguous run) into the staging area
-            stage_in(sm + L.stage, a.pmap + j0 * W, (uint32_t)(min((int64_t)span, s.N - j0) * W * 2),
-                     &bars[kKBarPmap]);
-            if (L.stage_in_b1) issue_ld(0);   // buffer 0 does not overlap the pmap staging rows
+            // pmap rows j0 .. j0+span-1 (one contiguous run) into the staging area (a segment
+            // reads its columns of the rows directly)
+            if (!SEG)
+                stage_in(sm + L.stage, a.pmap + j0 * W, (uint32_t)(min((int64_t)span, s.N - j0) * W * 2),
+                         &bars[kKBarPmap]);
+            if (SEG || L.stage_in_b1) issue_ld(0);   // buffer 0 does not overlap the pmap staging rows
             // ---- phase 1: dV_h = P^T (g_h dO_h)
             const bool pt_ok = wait_bar(&bars[kKBarPt], 0, abort_flag);   // staging area consumed
-            if (!L.stage_in_b1) issue_ld(0);
-            if (H > 1) issue_ld(1);
+            if (!SEG && !L.stage_in_b1) issue_ld(0);
+            issue_ld(1);   // dO_1, or Q_0 when H == 1 (there are 2H >= 2 loads)
             issue_k(0);
             for (int h = 0; h < H; ++h) {
                 const int idx = h, b = idx & 1;
@@ -638,13 +733,22 @@ bwd_key_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant_
         const int i = 32 * q + lane;                 // key row
         const int64_t j = j0 + i;
         const bool validk = (i < BK) && (j < s.N);
-        int clo = 1, chi = 0;                         // query columns c (t = j0 + c) that see key j
+        int clo = 1, chi = 0;                         // query columns c (t = qbase + c) that see key j
         if (validk) {
-            clo = i;
             const int64_t dend = doc_end(s, j);
-            int64_t hi = j + W - 1;
-            if (hi > dend - 1) hi = dend - 1;
-            chi = (int)(hi - j0);
+            if constexpr (SEG) {   // queries j + shift .. j + shift + W - 1 of j's document
+                if (j + a.seg.shift <= dend - 1) {
+                    clo = i;
+                    int64_t hi = j + a.seg.shift + W - 1;
+                    if (hi > dend - 1) hi = dend - 1;
+                    chi = (int)(hi - qbase);
+                }
+            } else {
+                clo = i;
+                int64_t hi = j + W - 1;
+                if (hi > dend - 1) hi = dend - 1;
+                chi = (int)(hi - j0);
+            }
         }
         // column c is in this row's window iff (unsigned)(c - span_lo) <= span_n; a row with an
         // empty window (clo > chi: past the block or past N) gets span_lo = ~0u, so no c passes
@@ -656,10 +760,29 @@ bwd_key_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant_
 
         // ---- pmap rows j0 .. j0+span-1, staged by the producer
         const uint16_t *stage = (const uint16_t *)(sm + L.stage);
-        wait_bar(&bars[kKBarPmap], 0, abort_flag);
+        if (!SEG) wait_bar(&bars[kKBarPmap], 0, abort_flag);
         // ---- P^T tile: P^T(i, c) = P(j0 + c, j0 + i) = pmap[j0 + c][i - c + W - 1]
+        // (segment: P(qbase + c, j0 + i) = pmap[qbase + c][wofs + i - c + W - 1], from global memory)
         uint8_t *atile = sm + L.ra;
-        {
+        if constexpr (SEG) {
+            const uint16_t *pm = (const uint16_t *)a.pmap + qbase * a.seg.wrow + a.seg.wofs + i + W - 1;
+#pragma unroll
+            for (int cc = 0; cc < MAXC; ++cc) {
+                if (cc < bd.mync) {
+                    const int col = bd.cb + (bd.c0 + cc) * 8;
+                    uint32_t w[4];
+#pragma unroll
+                    for (int e = 0; e < 8; e += 2) {
+                        const uint32_t c0 = (uint32_t)(col + e), c1 = c0 + 1;
+                        const uint32_t v0 = (c0 - span_lo <= span_n) ? __ldg(pm + (int64_t)c0 * a.seg.wrow - (int)c0) : 0u;
+                        const uint32_t v1 = (c1 - span_lo <= span_n) ? __ldg(pm + (int64_t)c1 * a.seg.wrow - (int)c1) : 0u;
+                        w[e >> 1] = v0 | (v1 << 16);
+                    }
+                    *(uint4 *)(atile + sw128_offset(i, col)) = make_uint4(w[0], w[1], w[2], w[3]);
+                }
+            }
+            zero_outside_band(atile, i, split, bd, span);
+        } else {
 #pragma unroll
             for (int cc = 0; cc < MAXC; ++cc) {
                 if (cc < bd.mync) {
@@ -692,7 +815,7 @@ bwd_key_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant_
 #pragma unroll
             for (int it = 0; it < kPasses; ++it) {
                 const int r = (tid >> 3) + it * kRowsPerPass;
-                gv[it] = (r < span && j0 + r < s.N) ? __ldg(a.g + (j0 + r) * H + h) : 0.f;
+                gv[it] = (r < span && qbase + r < s.N) ? __ldg(a.g + (qbase + r) * H + h) : 0.f;
             }
             wait_bar(&bars[kKBarLd + b], (uint32_t)(h >> 1) & 1, abort_flag);
             uint8_t *tile = sm + (b ? L.rb1 : L.rb0);
@@ -722,8 +845,12 @@ bwd_key_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant_
             const int b = idx & 1;
             wait_bar(&bars[kKBarAccFull + b], (uint32_t)(idx >> 1) & 1, abort_flag);
             ptx::tc_fence_after();
-            drain_row<D>(tmem + lane_base + 256 + 128 * b, out + (j * H + h) * D, mult, validk, split,
-                         ((uintptr_t)out & 31) == 0);
+            if (SEG && a.seg.mode == kKSegAdd)   // a later segment adds its share
+                drain_row<D, true>(tmem + lane_base + 256 + 128 * b, out + (j * H + h) * D, mult, validk, split,
+                                   ((uintptr_t)out & 31) == 0);
+            else
+                drain_row<D>(tmem + lane_base + 256 + 128 * b, out + (j * H + h) * D, mult, validk, split,
+                             ((uintptr_t)out & 31) == 0);
             ptx::tc_fence_before();
             ptx::mbar_arrive(&bars[kKBarAccFree + b]);
         };
@@ -739,8 +866,13 @@ bwd_key_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant_
 #pragma unroll
                 for (int e = 0; e < 8; ++e) {
                     const uint32_t cidx = (uint32_t)(col + e);
-                    dPT[cc][e] = (cidx - span_lo <= span_n)
-                                     ? __ldg(a.band + (j0 + (int)cidx) * W + (i - (int)cidx + W - 1)) : 0.f;
+                    if constexpr (SEG)
+                        dPT[cc][e] = (cidx - span_lo <= span_n)
+                                         ? __ldg(a.band + (qbase + (int)cidx) * a.seg.wrow + a.seg.wofs + (i - (int)cidx + W - 1))
+                                         : 0.f;
+                    else
+                        dPT[cc][e] = (cidx - span_lo <= span_n)
+                                         ? __ldg(a.band + (j0 + (int)cidx) * W + (i - (int)cidx + W - 1)) : 0.f;
                 }
             }
         }
@@ -749,7 +881,7 @@ bwd_key_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant_
         // head h is processed
         float nv0 = 0.f, nv1 = 0.f, nv2 = 0.f;
         auto fetch_colv = [&](int h) {
-            const int64_t tq = j0 + tid;
+            const int64_t tq = qbase + tid;
             const bool ok = tid < span && tq < s.N;
             nv0 = ok ? __ldg(a.lse + tq * H + h) * kLog2e : 0.f;
             nv1 = ok ? __ldg(a.c + tq * H + h) : 0.f;

@@ -82,6 +82,18 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float a, float b) {
     return *reinterpret_cast<uint32_t *>(&v);
 }
 
+// w = bf16(old + mult * acc) for 16 consecutive values: old read from `src` (16-byte
+// aligned), acc the fp32 accumulator words.  Used where a window segment adds its share
+// to an output that an earlier segment wrote.
+__device__ __forceinline__ void add_bf16x16(uint32_t w[8], const __nv_bfloat16 *src, float mult, const uint32_t acc[16]) {
+    const uint4 o0 = *(const uint4 *)src, o1 = *(const uint4 *)(src + 8);
+    const uint32_t old[8] = {o0.x, o0.y, o0.z, o0.w, o1.x, o1.y, o1.z, o1.w};
+#pragma unroll
+    for (int e = 0; e < 8; ++e)
+        w[e] = pack_bf16x2(__uint_as_float(old[e] << 16) + mult * __uint_as_float(acc[2 * e]),
+                           __uint_as_float(old[e] & 0xFFFF0000u) + mult * __uint_as_float(acc[2 * e + 1]));
+}
+
 // Byte offset of element (row, col) of a K-major, 128-byte-swizzled bf16 tile
 // made of 64-column blocks of 128 rows (16 KiB each).
 __device__ __forceinline__ uint32_t sw128_offset(int row, int col) {
@@ -127,6 +139,28 @@ __device__ __forceinline__ void zero_outside_band(uint8_t *tile, int row, int sp
     } else if (split == kSplits - 1) {
         for (int col = (ce > bd.cb ? ce : bd.cb); col < span; col += 8) *(uint4 *)(tile + sw128_offset(row, col)) = z4;
     }
+}
+
+// Window segments.  A window wider than the tile geometry allows (W > 129) is cut into
+// segments of at most 128 keys counted back from the query: segment k of query t holds
+// keys t - shift - Wseg + 1 .. t - shift (shift = 128 k), inside t's document.  Each
+// segment runs the kernels with W = Wseg; pmap and the dP band keep rows of the full
+// width `wrow`, where the segment's keys start at column wofs = wrow - shift - Wseg.
+struct Seg {
+    int shift;   // keys of the segment end `shift` tokens before the query
+    int wrow;    // row length of pmap and the dP band (the full window W)
+    int wofs;    // first column of the segment in those rows
+    int mode;    // what this launch of the kernel does (per-kernel enum)
+};
+
+// Keys [lo, hi] of query t in the segment (Wseg = s.W); false when it holds none.
+__device__ __forceinline__ bool seg_window(const Shape &s, int64_t t, int shift, int64_t &lo, int64_t &hi) {
+    int64_t a = __ldg(s.cu + doc_index(s.cu, s.num_docs, t));
+    if (a < 0) a = 0;
+    hi = t - shift;
+    lo = hi - s.W + 1;
+    if (lo < a) lo = a;
+    return hi >= lo;
 }
 
 // 16-column chunks [begin, end) of a D-column accumulator row drained by this split.

@@ -60,13 +60,19 @@ struct FwdArgs {
     __nv_bfloat16 *o;
     float *lse;
     __nv_bfloat16 *pmap;
+    Seg seg;      // window segment (segmented instantiation only)
 };
+
+// Launches of the segmented forward, in order: the LSE of every segment merged into lse
+// (phase 1 only), then every segment composes its part of P with that LSE and adds its
+// share of o (the first one writes o, the others add to it).
+enum : int { kFwdSegStatsFirst = 1, kFwdSegStatsMerge = 2, kFwdSegApplyWrite = 3, kFwdSegApplyAdd = 4 };
 
 // mbarrier slots
 enum : int { kBarQK = 0, kBarSFull = 2, kBarSFree = 3, kBarV = 4, kBarUFull = 6, kBarUFree = 8, kBarP = 10,
              kNumBars = 11 };
 
-template <int D, int MAXC>
+template <int D, int MAXC, bool SEG = false>
 __global__ void __launch_bounds__(kThreads, 1)
 fwd_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__ CUtensorMap map_k,
            const __grid_constant__ CUtensorMap map_v, const FwdArgs a) {
@@ -82,7 +88,9 @@ fwd_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__ CU
     const int H = s.H, W = s.W, BM = a.BM, span = a.span;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int64_t t0 = (int64_t)blockIdx.x * BM;
-    const int64_t kbase = t0 - (W - 1);
+    const int64_t kbase = SEG ? t0 - a.seg.shift - (W - 1) : t0 - (W - 1);
+    // segmented LSE launches stop after phase 1
+    const bool stats_only = SEG && a.seg.mode <= kFwdSegStatsMerge;
 
     validate_seqlens(s);
     if (threadIdx.x == 0) {
@@ -156,12 +164,12 @@ fwd_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__ CU
             }
             // ---- phase 2: U_h = P V_h.  V_h reuses the K buffer of the same parity once
             // the last S MMA that read it has completed.
-            if (wait_bar(&bars[kBarSFull], (uint32_t)(H - 1) & 1, abort_flag)) {   // every S MMA done
+            if (!stats_only && wait_bar(&bars[kBarSFull], (uint32_t)(H - 1) & 1, abort_flag)) {   // every S MMA done
                 for (int b = 0; b < 2 && b < H; ++b) issue_v(b);
             }
-            bool p_ok = wait_bar(&bars[kBarP], 0, abort_flag);
+            bool p_ok = !stats_only && wait_bar(&bars[kBarP], 0, abort_flag);
             const uint32_t pa = ptx::smem_u32(sm + L::kP);
-            for (int h = 0; h < H; ++h) {
+            for (int h = 0; h < (stats_only ? 0 : H); ++h) {
                 const int b = h & 1;
                 const uint32_t n = (uint32_t)(h >> 1);
                 bool ok = wait_bar(&bars[kBarV + b], n & 1, abort_flag) && p_ok;
@@ -191,8 +199,16 @@ fwd_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__ CU
         const bool valid = (i < BM) && (t < s.N);
         int clo = 1, chi = 0;                           // valid columns of this row: [clo, chi]
         if (valid) {
-            clo = (int)(window_lo(s, t) - kbase);
-            chi = (int)(t - kbase);
+            if constexpr (SEG) {
+                int64_t lo, hi;
+                if (seg_window(s, t, a.seg.shift, lo, hi)) {
+                    clo = (int)(lo - kbase);
+                    chi = (int)(hi - kbase);
+                }
+            } else {
+                clo = (int)(window_lo(s, t) - kbase);
+                chi = (int)(t - kbase);
+            }
         }
         const Band bd = make_band(q, split, BM, W, span);
         const uint32_t lane_base = (uint32_t)(32 * q) << 16;
@@ -247,6 +263,19 @@ fwd_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__ CU
             }
             ptx::tc_fence_before();
             ptx::mbar_arrive(&bars[kBarSFree]);   // S columns free for the next head's MMA
+            if constexpr (SEG) {
+                if (!stats_only) {   // p_h = 2^(s log2e - lse log2e) with the whole window's LSE
+                    const float lref = valid ? __ldg(a.lse + t * H + h) * kLog2e : 0.f;
+                    const float coef = valid ? __ldg(a.c + t * H + h) : 0.f;
+#pragma unroll
+                    for (int cc = 0; cc < MAXC; ++cc)
+                        if (cc < bd.mync)
+#pragma unroll
+                            for (int e = 0; e < 8; ++e)
+                                P[cc][e] = fmaf(coef, ex2(__uint_as_float(xr[cc][e]) - lref), P[cc][e]);
+                    continue;
+                }
+            }
             // Softmax with this split's own maximum; the splits' (max, sum) pairs are then
             // combined in one exchange: Z = sum_s Z_s 2^(m_s - m), p = e_s 2^(m_s - m) / Z.
             const float mloc = fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3]));
@@ -277,6 +306,19 @@ fwd_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__ CU
             float Z = 0.f;
 #pragma unroll
             for (int sp = 0; sp < kSplits; ++sp) Z += ms[sp].y > 0.f ? ms[sp].y * ex2(ms[sp].x - m) : 0.f;
+            if constexpr (SEG) {   // LSE launch: this segment's log-sum-exp, merged into lse
+                if (split == 0 && valid) {
+                    const float ls = Z > 0.f ? (m + __log2f(Z)) * kLn2 : -INFINITY;   // -inf: no key here
+                    float out = ls;
+                    if (a.seg.mode == kFwdSegStatsMerge) {
+                        const float l0 = a.lse[t * H + h];
+                        const float hi = fmaxf(l0, ls), lo = fminf(l0, ls);
+                        out = (lo == -INFINITY) ? hi : hi + log1pf(expf(lo - hi));
+                    }
+                    a.lse[t * H + h] = out;
+                }
+                continue;
+            }
             const float coef = (valid && any) ? __ldg(a.c + t * H + h) * ex2(mref - m) / Z : 0.f;
 #pragma unroll
             for (int cc = 0; cc < MAXC; ++cc)
@@ -286,33 +328,30 @@ fwd_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__ CU
             if (split == 0 && valid && a.lse) a.lse[t * H + h] = (m + __log2f(Z)) * kLn2;
         }
 
-        // ---- P tile (bf16, K-major, swizzled) in smem; zero the columns outside the band
-        uint8_t *ptile = sm + L::kP;
-        uint32_t Pb[MAXC][4];   // P rounded to bf16 pairs, also the pmap values
+        if (!stats_only) {   // phase 2 (the segmented LSE launches stop here)
+            // ---- P tile (bf16, K-major, swizzled) in smem; zero the columns outside the band
+            uint8_t *ptile = sm + L::kP;
+            uint32_t Pb[MAXC][4];   // P rounded to bf16 pairs, also the pmap values
 #pragma unroll
-        for (int cc = 0; cc < MAXC; ++cc) {
-            if (cc < bd.mync) {
-                const int col = bd.cb + (bd.c0 + cc) * 8;
+            for (int cc = 0; cc < MAXC; ++cc) {
+                if (cc < bd.mync) {
+                    const int col = bd.cb + (bd.c0 + cc) * 8;
 #pragma unroll
-                for (int e = 0; e < 4; ++e) Pb[cc][e] = pack_bf16x2(P[cc][2 * e], P[cc][2 * e + 1]);
-                *(uint4 *)(ptile + sw128_offset(i, col)) = make_uint4(Pb[cc][0], Pb[cc][1], Pb[cc][2], Pb[cc][3]);
+                    for (int e = 0; e < 4; ++e) Pb[cc][e] = pack_bf16x2(P[cc][2 * e], P[cc][2 * e + 1]);
+                    *(uint4 *)(ptile + sw128_offset(i, col)) = make_uint4(Pb[cc][0], Pb[cc][1], Pb[cc][2], Pb[cc][3]);
+                }
             }
-        }
-        zero_outside_band(ptile, i, split, bd, span);
-        ptx::fence_proxy_async_smem();
-        ptx::mbar_arrive(&bars[kBarP]);
+            zero_outside_band(ptile, i, split, bd, span);
+            ptx::fence_proxy_async_smem();
+            ptx::mbar_arrive(&bars[kBarP]);
 
-        // ---- pmap[t][w] = P(t, t-W+1+w) = P at tile column i + w.  The block's rows are one
-        // contiguous run of pmap: build it in shared memory from the registers (passes of
-        // `rpp` rows when it does not fit) and write it with one bulk copy per pass.
-        if (a.pmap) {
-            const int rows_blk = (int)min((int64_t)BM, s.N - t0);
-            const int rpp = min(BM, (int)(L::kStageBytes / (uint32_t)(2 * W)) & ~7);   // rows per pass
-            uint16_t *stage = (uint16_t *)(sm + L::kStage);
-            for (int r0 = 0; r0 < rows_blk; r0 += rpp) {
-                const int nr = min(rpp, rows_blk - r0);
-                if (i >= r0 && i < r0 + nr) {
-                    uint16_t *srow = stage + (i - r0) * W - i;   // srow[col] = pmap[t][col - i]
+            // ---- pmap[t][w] = P(t, t-W+1+w) = P at tile column i + w.  The block's rows are one
+            // contiguous run of pmap: build it in shared memory from the registers (passes of
+            // `rpp` rows when it does not fit) and write it with one bulk copy per pass.
+            // A segment owns only columns wofs .. wofs + W - 1 of each row: plain stores.
+            if (SEG && a.pmap) {
+                if (valid) {
+                    uint16_t *prow = (uint16_t *)a.pmap + t * a.seg.wrow + a.seg.wofs;   // prow[w], w < W
 #pragma unroll
                     for (int cc = 0; cc < MAXC; ++cc) {
                         if (cc < bd.mync) {
@@ -320,58 +359,83 @@ fwd_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__ CU
 #pragma unroll
                             for (int e = 0; e < 8; ++e) {
                                 const uint32_t w = (uint32_t)(col + e - i);
-                                if (w < (uint32_t)W) srow[col + e] = (uint16_t)(Pb[cc][e >> 1] >> (16 * (e & 1)));
+                                if (w < (uint32_t)W) prow[w] = (uint16_t)(Pb[cc][e >> 1] >> (16 * (e & 1)));
                             }
                         }
                     }
                 }
-                ptx::fence_proxy_async_smem();
-                compute_sync();
-                if (threadIdx.x == 0) {
-                    const uint32_t bytes = (uint32_t)nr * W * 2;
-                    uint8_t *dst = (uint8_t *)(a.pmap + (t0 + r0) * W);
-                    const uint32_t main = bytes & ~15u;
-                    for (uint32_t x = main; x < bytes; x += 2)   // ragged end of the tensor
-                        *(uint16_t *)(dst + x) = *(const uint16_t *)((const uint8_t *)stage + x);
-                    if (main) ptx::bulk_store(dst, stage, main);
-                    ptx::bulk_commit();
-                    if (r0 + rpp < rows_blk) ptx::bulk_wait_read();
+            } else if (a.pmap) {
+                const int rows_blk = (int)min((int64_t)BM, s.N - t0);
+                const int rpp = min(BM, (int)(L::kStageBytes / (uint32_t)(2 * W)) & ~7);   // rows per pass
+                uint16_t *stage = (uint16_t *)(sm + L::kStage);
+                for (int r0 = 0; r0 < rows_blk; r0 += rpp) {
+                    const int nr = min(rpp, rows_blk - r0);
+                    if (i >= r0 && i < r0 + nr) {
+                        uint16_t *srow = stage + (i - r0) * W - i;   // srow[col] = pmap[t][col - i]
+#pragma unroll
+                        for (int cc = 0; cc < MAXC; ++cc) {
+                            if (cc < bd.mync) {
+                                const int col = bd.cb + (bd.c0 + cc) * 8;
+#pragma unroll
+                                for (int e = 0; e < 8; ++e) {
+                                    const uint32_t w = (uint32_t)(col + e - i);
+                                    if (w < (uint32_t)W) srow[col + e] = (uint16_t)(Pb[cc][e >> 1] >> (16 * (e & 1)));
+                                }
+                            }
+                        }
+                    }
+                    ptx::fence_proxy_async_smem();
+                    compute_sync();
+                    if (threadIdx.x == 0) {
+                        const uint32_t bytes = (uint32_t)nr * W * 2;
+                        uint8_t *dst = (uint8_t *)(a.pmap + (t0 + r0) * W);
+                        const uint32_t main = bytes & ~15u;
+                        for (uint32_t x = main; x < bytes; x += 2)   // ragged end of the tensor
+                            *(uint16_t *)(dst + x) = *(const uint16_t *)((const uint8_t *)stage + x);
+                        if (main) ptx::bulk_store(dst, stage, main);
+                        ptx::bulk_commit();
+                        if (r0 + rpp < rows_blk) ptx::bulk_wait_read();
+                    }
+                    if (r0 + rpp < rows_blk) compute_sync();
                 }
-                if (r0 + rpp < rows_blk) compute_sync();
             }
-        }
 
-        // ---- epilogue: o_h = g[t,h] * U_h; this split drains 16-column chunks [cb16, ce16)
-        int cb16, ce16;
-        acc_split(split, D / 16, cb16, ce16);
-        constexpr int kMaxC16 = (D / 16 + kSplits - 1) / kSplits;
-        const bool o_aligned32 = ((uintptr_t)a.o & 31) == 0;
-        for (int h = 0; h < H; ++h) {
-            const int b = h & 1;
-            const uint32_t n = (uint32_t)(h >> 1);
-            wait_bar(&bars[kBarUFull + b], n & 1, abort_flag);
-            ptx::tc_fence_after();
-            const float gh = valid ? __ldg(a.g + t * H + h) : 0.f;
-            uint32_t ur[kMaxC16][16];
+            // ---- epilogue: o_h = g[t,h] * U_h; this split drains 16-column chunks [cb16, ce16)
+            int cb16, ce16;
+            acc_split(split, D / 16, cb16, ce16);
+            constexpr int kMaxC16 = (D / 16 + kSplits - 1) / kSplits;
+            const bool o_aligned32 = ((uintptr_t)a.o & 31) == 0;
+            for (int h = 0; h < H; ++h) {
+                const int b = h & 1;
+                const uint32_t n = (uint32_t)(h >> 1);
+                wait_bar(&bars[kBarUFull + b], n & 1, abort_flag);
+                ptx::tc_fence_after();
+                const float gh = valid ? __ldg(a.g + t * H + h) : 0.f;
+                uint32_t ur[kMaxC16][16];
 #pragma unroll
-            for (int c = 0; c < kMaxC16; ++c)
-                if (cb16 + c < ce16) ptx::tmem_ld16_issue(tmem + lane_base + b * 256 + (cb16 + c) * 16, ur[c]);
-            ptx::tmem_wait_ld();
+                for (int c = 0; c < kMaxC16; ++c)
+                    if (cb16 + c < ce16) ptx::tmem_ld16_issue(tmem + lane_base + b * 256 + (cb16 + c) * 16, ur[c]);
+                ptx::tmem_wait_ld();
 #pragma unroll
-            for (int c = 0; c < kMaxC16; ++c) {
-                if (cb16 + c < ce16) {
-                    ptx::reg_fence16(ur[c]);
-                    if (valid) {
-                        uint32_t w[8];
+                for (int c = 0; c < kMaxC16; ++c) {
+                    if (cb16 + c < ce16) {
+                        ptx::reg_fence16(ur[c]);
+                        if (valid) {
+                            uint32_t w[8];
 #pragma unroll
-                        for (int e = 0; e < 8; ++e)
-                            w[e] = pack_bf16x2(gh * __uint_as_float(ur[c][2 * e]), gh * __uint_as_float(ur[c][2 * e + 1]));
-                        ptx::st_global_32b(a.o + (t * H + h) * D + (cb16 + c) * 16, w, o_aligned32);
+                            for (int e = 0; e < 8; ++e)
+                                w[e] = pack_bf16x2(gh * __uint_as_float(ur[c][2 * e]), gh * __uint_as_float(ur[c][2 * e + 1]));
+                            if constexpr (SEG) {   // later segments add their share to o
+                                if (a.seg.mode == kFwdSegApplyAdd)
+                                    add_bf16x16(w, a.o + (t * H + h) * D + (cb16 + c) * 16, gh, ur[c]);
+                            }
+                            ptx::st_global_32b(a.o + (t * H + h) * D + (cb16 + c) * 16, w, o_aligned32);
+                        }
                     }
                 }
+                ptx::tc_fence_before();
+                ptx::mbar_arrive(&bars[kBarUFree + b]);
             }
-            ptx::tc_fence_before();
-            ptx::mbar_arrive(&bars[kBarUFree + b]);
         }
     }
 

@@ -14,11 +14,27 @@
 namespace dc {
 namespace tc {
 
-constexpr int kMaxWindow = 129;   // BM = 128 keeps the key tile (BM + W - 1 rows) within 256
+constexpr int kMaxWindow = 129;      // BM = 128 keeps the key tile (BM + W - 1 rows) within 256
+constexpr int kSegWidth = 128;       // wider windows run as segments of this many keys
+constexpr int kMaxSegWindow = 2 * kSegWidth;
 
 inline bool supports(const Shape &s) {
-    return (s.d == 64 || s.d == 128) && s.W >= 1 && s.W <= kMaxWindow && s.H >= 1 && s.H <= 16 &&
+    return (s.d == 64 || s.d == 128) && s.W >= 1 && s.W <= kMaxSegWindow && s.H >= 1 && s.H <= 16 &&
            s.N <= (int64_t)INT32_MAX - 512;
+}
+
+inline bool segmented(const Shape &s) { return s.W > kMaxWindow; }
+
+// Segment k of a segmented window (k = 0: the kSegWidth keys ending at the query; k = 1:
+// the rest): the shape the kernels run with (W = the segment's width) and its Seg.
+inline Shape seg_shape(const Shape &s, int k, int mode, Seg *seg) {
+    Shape r = s;
+    r.W = k == 0 ? kSegWidth : s.W - kSegWidth;
+    seg->shift = k * kSegWidth;
+    seg->wrow = s.W;
+    seg->wofs = s.W - seg->shift - r.W;
+    seg->mode = mode;
+    return r;
 }
 
 typedef CUresult (*EncodeTiledFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *, const cuuint64_t *,
@@ -95,10 +111,10 @@ inline cudaError_t set_smem(K kernel, uint32_t bytes) {
     return cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
 }
 
-template <int D, int MAXC>
+template <int D, int MAXC, bool SEG = false>
 inline cudaError_t launch_fwd(const CUtensorMap &mq, const CUtensorMap &mk, const CUtensorMap &mv, const FwdArgs &a,
                               cudaStream_t st) {
-    auto kern = fwd_kernel<D, MAXC>;
+    auto kern = fwd_kernel<D, MAXC, SEG>;
     cudaError_t e = set_smem(kern, FwdLayout<D>::kAlloc);
     if (e != cudaSuccess) return e;
     const unsigned grid = (unsigned)((a.s.N + a.BM - 1) / a.BM);
@@ -117,8 +133,45 @@ inline cudaError_t launch_fwd_d(int maxc, const CUtensorMap &mq, const CUtensorM
     }
 }
 
+// Window of more than kMaxWindow keys: the LSE of the near and the far segment merged
+// into lse, then the far segment writes its part of pmap and its share of o and the near
+// segment adds its share (four launches; lse is required).
+inline cudaError_t fwd_segmented(const Shape &s, const void *q, const void *k, const void *v, const float *c,
+                                 const float *g, void *o, float *lse, void *pmap, cudaStream_t st, int32_t *launches) {
+    if (!lse) return cudaErrorInvalidValue;
+    const int BM = choose_block(s.N, kSegWidth, sm_count());
+    CUtensorMap mq, mk[2], mv[2];
+    cudaError_t e = make_map(&mq, q, s.N, s.H, s.d, 128);
+    for (int sk = 0; sk < 2 && e == cudaSuccess; ++sk) {
+        Seg sg;
+        const int span = round16(BM + seg_shape(s, sk, 0, &sg).W - 1);
+        e = make_map(&mk[sk], k, s.N, s.H, s.d, span);
+        if (e == cudaSuccess) e = make_map(&mv[sk], v, s.N, s.H, s.d, span);
+    }
+    if (e != cudaSuccess) return e;
+    const int order[4][2] = {{0, kFwdSegStatsFirst}, {1, kFwdSegStatsMerge}, {1, kFwdSegApplyWrite},
+                             {0, kFwdSegApplyAdd}};
+    for (const auto &step : order) {
+        FwdArgs a;
+        a.s = seg_shape(s, step[0], step[1], &a.seg);
+        a.BM = BM;
+        a.span = round16(BM + a.s.W - 1);
+        a.c = c;
+        a.g = g;
+        a.o = (__nv_bfloat16 *)o;
+        a.lse = lse;
+        a.pmap = (__nv_bfloat16 *)pmap;
+        const CUtensorMap &kk = mk[step[0]], &vv = mv[step[0]];
+        e = (s.d == 64) ? launch_fwd<64, 7, true>(mq, kk, vv, a, st) : launch_fwd<128, 7, true>(mq, kk, vv, a, st);
+        if (e != cudaSuccess) return e;
+        ++*launches;
+    }
+    return cudaSuccess;
+}
+
 inline cudaError_t fwd(const Shape &s, const void *q, const void *k, const void *v, const float *c, const float *g,
                        void *o, float *lse, void *pmap, cudaStream_t st, int32_t *launches) {
+    if (segmented(s)) return fwd_segmented(s, q, k, v, c, g, o, lse, pmap, st, launches);
     FwdArgs a;
     a.s = s;
     a.BM = choose_block(s.N, s.W, sm_count());
@@ -139,10 +192,10 @@ inline cudaError_t fwd(const Shape &s, const void *q, const void *k, const void 
     return e;
 }
 
-template <int D, int MAXC>
+template <int D, int MAXC, bool SEG = false>
 inline cudaError_t launch_bwd_query(const CUtensorMap &mq, const CUtensorMap &mk, const CUtensorMap &mv,
                                     const CUtensorMap &mdo, const BwdArgs &a, cudaStream_t st) {
-    auto kern = bwd_query_kernel<D, MAXC>;
+    auto kern = bwd_query_kernel<D, MAXC, SEG>;
     const uint32_t smem = QSideLayout<D>(a.span).bytes + 1024;
     cudaError_t e = set_smem(kern, smem);
     if (e != cudaSuccess) return e;
@@ -151,12 +204,12 @@ inline cudaError_t launch_bwd_query(const CUtensorMap &mq, const CUtensorMap &mk
     return cudaGetLastError();
 }
 
-template <int D, int MAXC>
+template <int D, int MAXC, bool SEG = false>
 inline cudaError_t launch_bwd_key(const CUtensorMap &mq, const CUtensorMap &mk, const CUtensorMap &mdo,
                                   const BwdArgs &a, cudaStream_t st) {
-    auto kern = bwd_key_kernel<D, MAXC>;
+    auto kern = bwd_key_kernel<D, MAXC, SEG>;
     const KSideLayout<D> L(a.span, a.s.W);
-    if (L.stage + L.stage_bytes > L.colv) return cudaErrorInvalidValue;   // staging must fit before colv
+    if (!SEG && L.stage + L.stage_bytes > L.colv) return cudaErrorInvalidValue;   // staging must fit before colv
     const uint32_t smem = L.bytes + 1024;
     cudaError_t e = set_smem(kern, smem);
     if (e != cudaSuccess) return e;
@@ -181,9 +234,49 @@ inline BwdArgs bwd_args(const Shape &s) {
     return a;
 }
 
+// Segmented query side: far segment (dP band, partial dg and dc), near segment (complete
+// dg and dc, its share of dq), far segment again (adds its share of dq).
+inline cudaError_t bwd_query_segmented(const Shape &s, const void *q, const void *k, const void *v, const float *c,
+                                       const float *g, const void *dO, const float *lse, const void *pmap, void *dq,
+                                       float *dc_, float *dg, float *band, cudaStream_t st, int32_t *launches) {
+    const int BM = choose_block(s.N, kSegWidth, sm_count(), kBwdMaxSpan);
+    CUtensorMap mq, mdo, mk[2], mv[2];
+    cudaError_t e = make_map(&mq, q, s.N, s.H, s.d, 128);
+    if (e == cudaSuccess) e = make_map(&mdo, dO, s.N, s.H, s.d, 128);
+    for (int sk = 0; sk < 2 && e == cudaSuccess; ++sk) {
+        Seg sg;
+        const int span = round16(BM + seg_shape(s, sk, 0, &sg).W - 1);
+        e = make_map(&mk[sk], k, s.N, s.H, s.d, span);
+        if (e == cudaSuccess) e = make_map(&mv[sk], v, s.N, s.H, s.d, span);
+    }
+    if (e != cudaSuccess) return e;
+    const int order[3][2] = {{1, kQSegFarPart1}, {0, kQSegNear}, {1, kQSegFarPart2}};
+    for (const auto &step : order) {
+        BwdArgs a = {};
+        a.s = seg_shape(s, step[0], step[1], &a.seg);
+        a.BM = BM;
+        a.span = round16(BM + a.s.W - 1);
+        a.c = c;
+        a.g = g;
+        a.lse = lse;
+        a.pmap = (const __nv_bfloat16 *)pmap;
+        a.dq = (__nv_bfloat16 *)dq;
+        a.dc = dc_;
+        a.dg = dg;
+        a.band = band;
+        const CUtensorMap &kk = mk[step[0]], &vv = mv[step[0]];
+        e = (s.d == 64) ? launch_bwd_query<64, 7, true>(mq, kk, vv, mdo, a, st)
+                        : launch_bwd_query<128, 7, true>(mq, kk, vv, mdo, a, st);
+        if (e != cudaSuccess) return e;
+        ++*launches;
+    }
+    return cudaSuccess;
+}
+
 inline cudaError_t bwd_query(const Shape &s, const void *q, const void *k, const void *v, const float *c,
                              const float *g, const void *dO, const float *lse, const void *pmap, void *dq, float *dc_,
                              float *dg, float *band, cudaStream_t st, int32_t *launches) {
+    if (segmented(s)) return bwd_query_segmented(s, q, k, v, c, g, dO, lse, pmap, dq, dc_, dg, band, st, launches);
     BwdArgs a = bwd_args(s);
     a.c = c;
     a.g = g;
@@ -209,9 +302,46 @@ inline cudaError_t bwd_query(const Shape &s, const void *q, const void *k, const
     return e;
 }
 
+// Segmented key side: the near segment's queries write dk and dv, the far segment's add.
+inline cudaError_t bwd_key_segmented(const Shape &s, const void *q, const void *k, const float *c, const float *g,
+                                     const void *dO, const float *lse, const void *pmap, const float *dc_,
+                                     const float *band, void *dk, void *dv, cudaStream_t st, int32_t *launches) {
+    const int BK = choose_block(s.N, kSegWidth, sm_count(), kBwdMaxSpan);
+    CUtensorMap mk, mq[2], mdo[2];
+    cudaError_t e = make_map(&mk, k, s.N, s.H, s.d, 128);
+    for (int sk = 0; sk < 2 && e == cudaSuccess; ++sk) {
+        Seg sg;
+        const int span = round16(BK + seg_shape(s, sk, 0, &sg).W - 1);
+        e = make_map(&mq[sk], q, s.N, s.H, s.d, span);
+        if (e == cudaSuccess) e = make_map(&mdo[sk], dO, s.N, s.H, s.d, span);
+    }
+    if (e != cudaSuccess) return e;
+    const int order[2][2] = {{0, kKSegWrite}, {1, kKSegAdd}};
+    for (const auto &step : order) {
+        BwdArgs a = {};
+        a.s = seg_shape(s, step[0], step[1], &a.seg);
+        a.BM = BK;
+        a.span = round16(BK + a.s.W - 1);
+        a.c = c;
+        a.g = g;
+        a.lse = lse;
+        a.pmap = (const __nv_bfloat16 *)pmap;
+        a.dc_in = dc_;
+        a.band = const_cast<float *>(band);
+        a.dk = (__nv_bfloat16 *)dk;
+        a.dv = (__nv_bfloat16 *)dv;
+        const CUtensorMap &qq = mq[step[0]], &dd = mdo[step[0]];
+        e = (s.d == 64) ? launch_bwd_key<64, 7, true>(qq, mk, dd, a, st) : launch_bwd_key<128, 7, true>(qq, mk, dd, a, st);
+        if (e != cudaSuccess) return e;
+        ++*launches;
+    }
+    return cudaSuccess;
+}
+
 inline cudaError_t bwd_key(const Shape &s, const void *q, const void *k, const float *c, const float *g,
                            const void *dO, const float *lse, const void *pmap, const float *dc_, const float *band,
                            void *dk, void *dv, cudaStream_t st, int32_t *launches) {
+    if (segmented(s)) return bwd_key_segmented(s, q, k, c, g, dO, lse, pmap, dc_, band, dk, dv, st, launches);
     BwdArgs a = bwd_args(s);
     a.c = c;
     a.g = g;

@@ -56,8 +56,15 @@ typedef enum {
 typedef enum { DC_F32 = 0, DC_BF16 = 1 } dc_dtype_t;
 
 /* Kernel family.  AUTO picks the tcgen05/TMA path when the shape allows it
- * (bf16, d in {64,128}, W <= 129) and the SIMT path otherwise.  SIMT is the
- * fp32-accumulating CUDA-core path used for fp32 tensors and any shape. */
+ * (bf16, d in {64,128}, W <= 256) and the SIMT path otherwise.  SIMT is the
+ * fp32-accumulating CUDA-core path used for fp32 tensors and any shape.
+ * On tcgen05 a window of W > 129 keys runs as two segments (the 128 keys
+ * ending at the query, then the rest): the forward first merges the two
+ * segments' log-sum-exp values in `lse` and so needs that buffer (AUTO
+ * without lse runs such a forward on SIMT; TCGEN05 without lse returns
+ * DC_ERR_UNSUPPORTED), and the second segment adds its share to o, dq, dk
+ * and dv after the first one has written them, which rounds that partial
+ * sum to bf16 once. */
 typedef enum { DC_IMPL_AUTO = 0, DC_IMPL_SIMT = 1, DC_IMPL_TCGEN05 = 2 } dc_impl_t;
 
 /* Bits of the device status word. */

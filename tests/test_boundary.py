@@ -115,11 +115,12 @@ def test_resolve_impl(lib):
 
 
 def test_resolve_impl_tcgen05_range(lib):
-    # bf16 with d in {64, 128} and 1 <= W <= 129 runs on tcgen05, other bf16 shapes on SIMT;
-    # more than 16 heads is refused on every path
+    # bf16 with d in {64, 128} and 1 <= W <= 256 runs on tcgen05 (W > 129 as two window
+    # segments), other bf16 shapes on SIMT; more than 16 heads is refused on every path
     tc, simt = dcattn.IMPLS["tcgen05"], dcattn.IMPLS["simt"]
-    for W, d, H, want in ((1, 128, 6, tc), (112, 128, 6, tc), (129, 128, 4, tc), (130, 64, 2, simt),
-                          (256, 128, 6, simt), (64, 64, 16, tc), (64, 96, 6, simt), (64, 64, 17, -1)):
+    for W, d, H, want in ((1, 128, 6, tc), (112, 128, 6, tc), (129, 128, 4, tc), (130, 64, 2, tc),
+                          (256, 128, 6, tc), (257, 128, 6, simt), (64, 64, 16, tc), (64, 96, 6, simt),
+                          (64, 64, 17, -1)):
         p = _params(dtype=dcattn.DC_BF16, window=W, head_dim=d, num_heads=H)
         assert lib.dc_attn_resolve_impl(ctypes.byref(p)) == want, (W, d, H)
 

@@ -81,11 +81,20 @@ EDGE_CASES = [
     ("bf16_d64_h12", [400, 129], 12, 64, 64, "bf16"),
     ("bf16_w1", [260], 6, 128, 1, "bf16"),
     ("bf16_short_docs", [5, 17, 3, 200, 9], 6, 128, 112, "bf16"),
-    # the widest window the tcgen05 kernels take (7 chunks of 8 columns per thread), the
-    # most heads, and the first window past it (served by the SIMT kernels)
+    ("bf16_h1", [300, 50], 1, 128, 112, "bf16"),
+    # the widest window the tcgen05 kernels take in one piece (7 chunks of 8 columns per
+    # thread), the most heads, and the first window past it
     ("bf16_w129", [700, 45], 4, 128, 129, "bf16"),
     ("bf16_w120_h16_d64", [520], 16, 64, 120, "bf16"),
+    # W > 129: a near segment of 128 keys and a far one of W - 128 (2 keys at W = 130); documents
+    # shorter than the near segment (far segment empty), windows past the document start,
+    # segment offsets that are not multiples of 8 (W = 200, 250), one head, sixteen heads
     ("bf16_w130", [300], 2, 64, 130, "bf16"),
+    ("bf16_w256_docs", [700, 45, 200, 3, 130], 6, 128, 256, "bf16"),
+    ("bf16_w200_h12_d64", [600, 90], 12, 64, 200, "bf16"),
+    ("bf16_w250_h16_d64", [520], 16, 64, 250, "bf16"),
+    ("bf16_w256_h1", [1100], 1, 128, 256, "bf16"),
+    ("bf16_w256_short", [100, 60], 4, 128, 256, "bf16"),
 ]
 
 
@@ -137,9 +146,11 @@ def test_deterministic():
         assert np.array_equal(a[n], b[n]), n
 
 
-def test_guard_bands_untouched():
-    """Outputs written into the middle of larger buffers: sentinels around them survive."""
-    inp = to_cuda(random_problem(7, [257, 130], 6, 128, 112, dtype="bf16"))
+@pytest.mark.parametrize("W", [112, 256])
+def test_guard_bands_untouched(W):
+    """Outputs written into the middle of larger buffers: sentinels around them survive
+    (W = 256: the window-segment kernels, which add into o, dq, dk and dv)."""
+    inp = to_cuda(random_problem(7, [257, 130], 6, 128, W, dtype="bf16"))
     N, H, d = inp["q"].shape
     W = inp["window"]
     G = 4096
@@ -167,6 +178,19 @@ def test_guard_bands_untouched():
     torch.cuda.synchronize()
     for buf in [bo, bl, bp, bws] + [b for b, _ in bufs.values()]:
         assert bool((buf[:G] == 7).all()) and bool((buf[-G:] == 7).all())
+
+
+def test_segmented_forward_without_lse():
+    """W > 129 without an lse buffer: AUTO serves it on the SIMT kernels, an explicit
+    tcgen05 request is refused before any launch."""
+    inp = to_cuda(random_problem(9, [300], 2, 64, 200, dtype="bf16"))
+    args = (inp["q"], inp["k"], inp["v"], inp["c"], inp["g"], inp["cu_seqlens"], 200, inp["scale"])
+    o, lse, pmap = dcattn.dc_attn_fwd(*args, need_backward=False)
+    assert lse is None and pmap is None
+    o_ref, _, _ = dcattn.dc_attn_fwd(*args, impl="simt")
+    assert torch.equal(o, o_ref)
+    with pytest.raises(dcattn.DCAttnError):
+        dcattn.dc_attn_fwd(*args, need_backward=False, impl="tcgen05")
 
 
 def test_malformed_seqlens_flagged_not_faulting():
