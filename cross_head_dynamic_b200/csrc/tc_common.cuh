@@ -170,5 +170,14 @@ __device__ __forceinline__ void acc_split(int split, int nchunk16, int &begin, i
     end = min(begin + per, nchunk16);
 }
 
+// Prefetch into L2 the 16-column chunks of a D-column bf16 output row that this split
+// drains: a segment that adds into an output reads them just before its stores.
+template <int D>
+__device__ __forceinline__ void prefetch_drain_row(const __nv_bfloat16 *row, int split) {
+    int cb16, ce16;
+    acc_split(split, D / 16, cb16, ce16);
+    for (int c = cb16; c < ce16; ++c) ptx::prefetch_l2(row + c * 16);
+}
+
 }  // namespace tc
 }  // namespace dc

@@ -63,10 +63,11 @@ struct FwdArgs {
     Seg seg;      // window segment (segmented instantiation only)
 };
 
-// Launches of the segmented forward, in order: the LSE of every segment merged into lse
-// (phase 1 only), then every segment composes its part of P with that LSE and adds its
-// share of o (the first one writes o, the others add to it).
-enum : int { kFwdSegStatsFirst = 1, kFwdSegStatsMerge = 2, kFwdSegApplyWrite = 3, kFwdSegApplyAdd = 4 };
+// Launches of the segmented forward, in order: the far segment's LSE into lse (phase 1
+// only); the near segment, which merges its own LSE with it (the whole window's LSE, kept
+// in lse), composes its part of P with that and writes o; the far segment again, which
+// composes its part with the whole window's LSE and adds its share to o.
+enum : int { kFwdSegStats = 1, kFwdSegNear = 2, kFwdSegFarApply = 3 };
 
 // mbarrier slots
 enum : int { kBarQK = 0, kBarSFull = 2, kBarSFree = 3, kBarV = 4, kBarUFull = 6, kBarUFree = 8, kBarP = 10,
@@ -89,8 +90,8 @@ fwd_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__ CU
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int64_t t0 = (int64_t)blockIdx.x * BM;
     const int64_t kbase = SEG ? t0 - a.seg.shift - (W - 1) : t0 - (W - 1);
-    // segmented LSE launches stop after phase 1
-    const bool stats_only = SEG && a.seg.mode <= kFwdSegStatsMerge;
+    // the segmented LSE launch stops after phase 1
+    const bool stats_only = SEG && a.seg.mode == kFwdSegStats;
 
     validate_seqlens(s);
     if (threadIdx.x == 0) {
@@ -264,7 +265,7 @@ fwd_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__ CU
             ptx::tc_fence_before();
             ptx::mbar_arrive(&bars[kBarSFree]);   // S columns free for the next head's MMA
             if constexpr (SEG) {
-                if (!stats_only) {   // p_h = 2^(s log2e - lse log2e) with the whole window's LSE
+                if (a.seg.mode == kFwdSegFarApply) {   // p_h = 2^(s log2e - lse log2e), whole window's LSE
                     const float lref = valid ? __ldg(a.lse + t * H + h) * kLog2e : 0.f;
                     const float coef = valid ? __ldg(a.c + t * H + h) : 0.f;
 #pragma unroll
@@ -293,6 +294,10 @@ fwd_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__ CU
                     }
                 }
             }
+            // near segment: the far segment's LSE (log2 units), read before any split of this
+            // row writes the merged value
+            float lfar2 = 0.f;
+            if constexpr (SEG) lfar2 = (valid && !stats_only) ? a.lse[t * H + h] * kLog2e : 0.f;
             float2 *rd = red + (h & 1) * (kSplits * 128);
             rd[split * 128 + i] = make_float2(mloc, (zs[0] + zs[1]) + (zs[2] + zs[3]));
             pair_sync(q);
@@ -306,17 +311,23 @@ fwd_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__ CU
             float Z = 0.f;
 #pragma unroll
             for (int sp = 0; sp < kSplits; ++sp) Z += ms[sp].y > 0.f ? ms[sp].y * ex2(ms[sp].x - m) : 0.f;
-            if constexpr (SEG) {   // LSE launch: this segment's log-sum-exp, merged into lse
-                if (split == 0 && valid) {
-                    const float ls = Z > 0.f ? (m + __log2f(Z)) * kLn2 : -INFINITY;   // -inf: no key here
-                    float out = ls;
-                    if (a.seg.mode == kFwdSegStatsMerge) {
-                        const float l0 = a.lse[t * H + h];
-                        const float hi = fmaxf(l0, ls), lo = fminf(l0, ls);
-                        out = (lo == -INFINITY) ? hi : hi + log1pf(expf(lo - hi));
-                    }
-                    a.lse[t * H + h] = out;
+            if constexpr (SEG) {
+                // log2 of this segment's normalizer (-inf: no key of the row in it)
+                const float l2 = Z > 0.f ? m + __log2f(Z) : -INFINITY;
+                if (stats_only) {   // far segment's LSE
+                    if (split == 0 && valid) a.lse[t * H + h] = l2 * kLn2;
+                    continue;
                 }
+                // near segment: the whole window's normalizer, log2(2^l2 + 2^lfar2)
+                const float hi = fmaxf(l2, lfar2), lo = fminf(l2, lfar2);
+                const float lw2 = (lo == -INFINITY) ? hi : hi + __log2f(1.f + ex2(lo - hi));
+                const float coef = (valid && any) ? __ldg(a.c + t * H + h) * ex2(mref - lw2) : 0.f;
+#pragma unroll
+                for (int cc = 0; cc < MAXC; ++cc)
+                    if (cc < bd.mync)
+#pragma unroll
+                        for (int e = 0; e < 8; ++e) P[cc][e] = fmaf(coef, __uint_as_float(xr[cc][e]), P[cc][e]);
+                if (split == 0 && valid) a.lse[t * H + h] = lw2 * kLn2;
                 continue;
             }
             const float coef = (valid && any) ? __ldg(a.c + t * H + h) * ex2(mref - m) / Z : 0.f;
@@ -328,7 +339,11 @@ fwd_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__ CU
             if (split == 0 && valid && a.lse) a.lse[t * H + h] = (m + __log2f(Z)) * kLn2;
         }
 
-        if (!stats_only) {   // phase 2 (the segmented LSE launches stop here)
+        if (!stats_only) {   // phase 2 (the segmented LSE launch stops here)
+            // the far segment adds to o: bring the rows it reads into L2 two heads ahead
+            const bool o_add = SEG && a.seg.mode == kFwdSegFarApply && valid;
+            if (o_add)
+                for (int h = 0; h < H && h < 2; ++h) prefetch_drain_row<D>(a.o + (t * H + h) * D, split);
             // ---- P tile (bf16, K-major, swizzled) in smem; zero the columns outside the band
             uint8_t *ptile = sm + L::kP;
             uint32_t Pb[MAXC][4];   // P rounded to bf16 pairs, also the pmap values
@@ -408,6 +423,7 @@ fwd_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__ CU
             for (int h = 0; h < H; ++h) {
                 const int b = h & 1;
                 const uint32_t n = (uint32_t)(h >> 1);
+                if (o_add && h + 2 < H) prefetch_drain_row<D>(a.o + (t * H + h + 2) * D, split);
                 wait_bar(&bars[kBarUFull + b], n & 1, abort_flag);
                 ptx::tc_fence_after();
                 const float gh = valid ? __ldg(a.g + t * H + h) : 0.f;
@@ -426,7 +442,7 @@ fwd_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__ CU
                             for (int e = 0; e < 8; ++e)
                                 w[e] = pack_bf16x2(gh * __uint_as_float(ur[c][2 * e]), gh * __uint_as_float(ur[c][2 * e + 1]));
                             if constexpr (SEG) {   // later segments add their share to o
-                                if (a.seg.mode == kFwdSegApplyAdd)
+                                if (a.seg.mode == kFwdSegFarApply)
                                     add_bf16x16(w, a.o + (t * H + h) * D + (cb16 + c) * 16, gh, ur[c]);
                             }
                             ptx::st_global_32b(a.o + (t * H + h) * D + (cb16 + c) * 16, w, o_aligned32);

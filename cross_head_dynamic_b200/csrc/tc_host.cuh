@@ -133,9 +133,9 @@ inline cudaError_t launch_fwd_d(int maxc, const CUtensorMap &mq, const CUtensorM
     }
 }
 
-// Window of more than kMaxWindow keys: the LSE of the near and the far segment merged
-// into lse, then the far segment writes its part of pmap and its share of o and the near
-// segment adds its share (four launches; lse is required).
+// Window of more than kMaxWindow keys: the far segment's LSE into lse; the near segment
+// merges its own LSE into it, writes its part of pmap and its share of o; the far segment
+// writes its part of pmap and adds its share of o (three launches; lse is required).
 inline cudaError_t fwd_segmented(const Shape &s, const void *q, const void *k, const void *v, const float *c,
                                  const float *g, void *o, float *lse, void *pmap, cudaStream_t st, int32_t *launches) {
     if (!lse) return cudaErrorInvalidValue;
@@ -149,8 +149,7 @@ inline cudaError_t fwd_segmented(const Shape &s, const void *q, const void *k, c
         if (e == cudaSuccess) e = make_map(&mv[sk], v, s.N, s.H, s.d, span);
     }
     if (e != cudaSuccess) return e;
-    const int order[4][2] = {{0, kFwdSegStatsFirst}, {1, kFwdSegStatsMerge}, {1, kFwdSegApplyWrite},
-                             {0, kFwdSegApplyAdd}};
+    const int order[3][2] = {{1, kFwdSegStats}, {0, kFwdSegNear}, {1, kFwdSegFarApply}};
     for (const auto &step : order) {
         FwdArgs a;
         a.s = seg_shape(s, step[0], step[1], &a.seg);

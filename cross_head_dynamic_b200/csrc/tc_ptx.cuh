@@ -126,6 +126,11 @@ __device__ __forceinline__ void st_global_32b(void *p, const uint32_t (&w)[8], b
     }
 }
 
+// Bring the line holding p into L2 (no register result, nothing to wait for).
+__device__ __forceinline__ void prefetch_l2(const void *p) {
+    asm volatile("prefetch.global.L2 [%0];" ::"l"(p));
+}
+
 __device__ __forceinline__ void prefetch_tensormap(const CUtensorMap *map) {
     asm volatile("prefetch.tensormap [%0];" ::"l"((uint64_t)map) : "memory");
 }
