@@ -138,7 +138,19 @@ cudaError_t simt_bwd_key(const dc::Shape &s, const void *q, const void *k, const
         }                                                                           \
     }()
 
+// The smallest workspace the backward takes: the dP band [N][W] fp32.
 size_t band_bytes(const dc::Shape &s) { return sizeof(float) * (size_t)s.N * (size_t)s.W; }
+
+// The workspace the backward asks for: on the tcgen05 path with a one-piece window also
+// room for the ds band (used when given; with only band_bytes the key side recomputes ds).
+size_t ws_need(const Checked &ck) {
+    size_t b = band_bytes(ck.s);
+    if (ck.impl == DC_IMPL_TCGEN05 && !dc::tc::segmented(ck.s)) {
+        const size_t d = dc::tc::dsb_bytes(ck.s);
+        if (d > b) b = d;
+    }
+    return b;
+}
 
 }  // namespace
 
@@ -167,7 +179,7 @@ dc_status_t dc_attn_fwd(const dc_attn_params *params, const void *q, const void 
 size_t dc_attn_bwd_workspace_size(const dc_attn_params *params) {
     Checked ck;
     if (check_params(params, &ck) != DC_OK) return 0;
-    return band_bytes(ck.s);
+    return ws_need(ck);
 }
 
 dc_status_t dc_attn_bwd_query(const dc_attn_params *params, const void *q, const void *k, const void *v,
@@ -185,8 +197,8 @@ dc_status_t dc_attn_bwd_query(const dc_attn_params *params, const void *q, const
     cudaStream_t st = (cudaStream_t)stream;
     float *band = (float *)workspace;
     if (ck.impl == DC_IMPL_TCGEN05)
-        return cuda_status(dc::tc::bwd_query(ck.s, q, k, v, c, g, dO, lse, pmap, dq, dc_, dg, band, st,
-                                             &t_launches));
+        return cuda_status(dc::tc::bwd_query(ck.s, q, k, v, c, g, dO, lse, pmap, dq, dc_, dg, workspace,
+                                             workspace_bytes, st, &t_launches));
     return cuda_status(DC_DISPATCH(simt_bwd_query, ck.dtype, ck.s.d, ck.s, q, k, v, c, g, dO, lse, pmap, dq,
                                    dc_, dg, band, st));
 }
@@ -206,8 +218,8 @@ dc_status_t dc_attn_bwd_key(const dc_attn_params *params, const void *q, const v
     cudaStream_t st = (cudaStream_t)stream;
     const float *band = (const float *)workspace;
     if (ck.impl == DC_IMPL_TCGEN05)
-        return cuda_status(dc::tc::bwd_key(ck.s, q, k, c, g, dO, lse, pmap, dc_, band, dk, dv, st,
-                                           &t_launches));
+        return cuda_status(dc::tc::bwd_key(ck.s, q, k, c, g, dO, lse, pmap, dc_, workspace, workspace_bytes, dk, dv,
+                                           st, &t_launches));
     return cuda_status(DC_DISPATCH(simt_bwd_key, ck.dtype, ck.s.d, ck.s, q, k, c, g, dO, lse, pmap, dc_, band,
                                    dk, dv, st));
 }

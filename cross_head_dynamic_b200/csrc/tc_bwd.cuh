@@ -34,6 +34,9 @@ namespace dc {
 namespace tc {
 
 constexpr int kBwdMaxSpan = 240;   // key/query tile rows, keeps both kernels within 227 KiB of smem
+// Row length of the ds band for every W <= 129 (129 rounded up to 8): a constant, so that the
+// query side's band stores of one head all address from one base register.
+constexpr int kDsbRow = 136;
 
 struct BwdArgs {
     Shape s;
@@ -51,6 +54,7 @@ struct BwdArgs {
     __nv_bfloat16 *dk;     // key side out
     __nv_bfloat16 *dv;
     Seg seg;               // window segment (segmented instantiations only)
+    __nv_bfloat16 *dsb;    // ds band [H][N][kDsbRow], key-major (see bwd_key_kernel)
 };
 
 // Segmented query side, launched in this order: the far segment's dP band, dg and dc
@@ -129,7 +133,7 @@ struct QSideLayout {
     }
 };
 
-template <int D, int MAXC, bool SEG = false>
+template <int D, int MAXC, bool SEG = false, bool DSB = false>
 __global__ void __launch_bounds__(kThreads, 1)
 bwd_query_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__ CUtensorMap map_k,
                  const __grid_constant__ CUtensorMap map_v, const __grid_constant__ CUtensorMap map_do,
@@ -313,6 +317,18 @@ bwd_query_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
         const uint32_t lane_base = (uint32_t)(32 * q) << 16;
         const uint32_t x_cols = tmem + lane_base;
         const float sl2 = s.scale * kLog2e;
+        // column c is in this row's window iff (unsigned)(c - win_lo) <= win_n (never for a row
+        // with an empty window)
+        const uint32_t win_lo = (chi >= clo) ? (uint32_t)clo : ~0u;
+        const uint32_t win_n = (chi >= clo) ? (uint32_t)(chi - clo) : 0u;
+        // ds band row of this query for head h, from the first column of this thread's part of
+        // the band: tile column c = c_first + k is element dsrow + k (kDsbRow - 1) (key
+        // j = kbase + c, offset t - j = i + W - 1 - c)
+        uint16_t *dsrow = nullptr;
+        if constexpr (DSB) {
+            const int c_first = bd.cb + bd.c0 * 8;
+            dsrow = (uint16_t *)a.dsb + (kbase + c_first) * kDsbRow + (i + W - 1 - c_first);
+        }
 
         // P(t, c) = pmap[t][c - i] on this thread's band, from the CTA's pmap rows staged by
         // the producer; zero outside the window.  Kept in registers (bf16 pairs) for all heads.
@@ -443,7 +459,7 @@ bwd_query_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
                     }
                 }
             }
-        } else {
+        } else if constexpr (!DSB) {   // (with the ds band the key side needs no dP)
             float *stage = (float *)(sm + L.rd);
             if (i < BM) {
 #pragma unroll
@@ -543,7 +559,7 @@ bwd_query_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
                 if (h >= 1) {
                     wait_bar(&bars[kQBarDqFull + ((h - 1) & 1)], (uint32_t)((h - 1) >> 1) & 1, abort_flag);
                 } else {
-                    if (!SEG && threadIdx.x == 0) ptx::bulk_wait_read();   // the band copy has left the region
+                    if (!SEG && !DSB && threadIdx.x == 0) ptx::bulk_wait_read();   // the band copy has left the region
                     compute_sync();
                     zero_outside_band(dtile, i, split, bd, span);
                 }
@@ -558,10 +574,26 @@ bwd_query_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
                             w[e] = pack_bf16x2(ch * p0 * (dP[cc][2 * e] - dch), ch * p1 * (dP[cc][2 * e + 1] - dch));
                         }
                         *(uint4 *)(dtile + sw128_offset(i, col)) = make_uint4(w[0], w[1], w[2], w[3]);
+                        if constexpr (DSB) {
+                            // ds_h(t, j) into the key-major band, dsb[h][j][t - j], for the columns in the
+                            // row's window: for one column all lanes (consecutive t) write consecutive
+                            // elements.  Column c of this row is element dsrow + c (kDsbRow - 1).
+                            uint16_t *pc = dsrow + cc * 8 * (kDsbRow - 1);
+                            const uint32_t c0 = (uint32_t)col - win_lo;
+                            if (__all_sync(0xffffffffu, c0 <= win_n && c0 + 7 <= win_n)) {
+#pragma unroll
+                                for (int e = 0; e < 8; ++e) pc[e * (kDsbRow - 1)] = (uint16_t)(w[e >> 1] >> (16 * (e & 1)));
+                            } else {
+#pragma unroll
+                                for (int e = 0; e < 8; ++e)
+                                    if (c0 + e <= win_n) pc[e * (kDsbRow - 1)] = (uint16_t)(w[e >> 1] >> (16 * (e & 1)));
+                            }
+                        }
                     }
                 }
                 ptx::fence_proxy_async_smem();
                 ptx::mbar_arrive(&bars[kQBarDs]);
+                if constexpr (DSB) dsrow += s.N * kDsbRow;   // next head's band
             }
             if (h >= 1) drain_dq(h - 1);   // overlaps the dQ_h MMA (other accumulator buffer)
         }
@@ -600,9 +632,11 @@ struct KSideLayout {
     }
 };
 
+// Key side that recomputes ds^T from S^T (and reads dP from the band): used for window
+// segments, and when the workspace cannot hold the ds band.
 template <int D, int MAXC, bool SEG = false>
 __global__ void __launch_bounds__(kThreads, 1)
-bwd_key_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__ CUtensorMap map_k,
+bwd_key_seg_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__ CUtensorMap map_k,
                const __grid_constant__ CUtensorMap map_do, const BwdArgs a) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t *sm = (uint8_t *)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
@@ -971,6 +1005,283 @@ bwd_key_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant_
             }
             if (h >= 1) drain(H + h - 1, a.dk, h - 1, s.scale);   // overlaps the dK_h MMA
             if (h + 1 < H) store_colv(h + 1);
+        }
+    }
+
+    ptx::tc_fence_before();
+    __syncthreads();
+    if (warp == 0) {
+        ptx::tc_fence_after();
+        ptx::tmem_dealloc(tmem, 512);
+    }
+}
+
+// --------------------------------------------------------------------------- key side, ds from the band
+// The query side wrote every ds_h(t, j) it used for dQ into the key-major band
+// dsb[h][j][t - j] (bf16).  A key block's rows of it are one contiguous [BK][wp] run per
+// head: one bulk copy brings them to shared memory, and each key row's band of ds^T is
+// read from there.  No S^T product, no K tile, no dP band and no per-query vectors.
+//   phase 1, per head: scale the dO_h rows by g_h in smem; MMA dV_h = P^T gdO_h.
+//   phase 2, per head: ds^T_h tile from the staged rows; MMA dK_h = ds^T_h Q_h, drained
+//            while the next head's tile is built.
+enum : int { kDBarLd = 0, kDBarScaled = 2, kDBarPt = 4, kDBarAccFull = 5, kDBarAccFree = 7, kDBarDsIn = 9,
+             kDBarDs = 10, kDBarPmap = 11, kDNumBars = 12 };
+
+template <int D>
+struct DSideLayout {
+    uint32_t tile_s;   // dO or Q tile over the query span: D/64 boxes of span rows x 128 B
+    uint32_t ra, rb0, rb1, rs, bars, bytes, stage, stage_bytes;
+    bool stage_in_b1;  // the pmap staging rows fit in buffer 1 (dO_0 can load early)
+    __host__ __device__ DSideLayout(int span, int W, int BK, int wp) {
+        tile_s = (uint32_t)(D / 64) * span * 128;
+        ra = 0;                                  // P^T tile (phase 1) / ds^T tile (phase 2): 64 KiB
+        rb0 = 4u * 16384;                        // dO buffer 0 (phase 1) / Q buffer 0 (phase 2)
+        rb1 = rb0 + tile_s;
+        rs = rb1 + tile_s;                       // ds rows of the key block [BK][wp] bf16
+        bars = rs + (((uint32_t)BK * wp * 2 + 127) & ~127u);
+        bytes = bars + 512;
+        stage_bytes = (uint32_t)span * W * 2;    // pmap rows of the query span, read once
+        stage_in_b1 = tile_s >= stage_bytes;
+        stage = stage_in_b1 ? rb1 : rb0;         // else it spans buffers 0 and 1
+    }
+};
+
+template <int D, int MAXC>
+__global__ void __launch_bounds__(kThreads, 1)
+bwd_key_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__ CUtensorMap map_do,
+               const BwdArgs a) {
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *sm = (uint8_t *)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
+    const Shape &s = a.s;
+    const int H = s.H, W = s.W, BK = a.BM, span = a.span;
+    constexpr int wp = kDsbRow;
+    const DSideLayout<D> L(span, W, BK, wp);
+    uint64_t *bars = (uint64_t *)(sm + L.bars);
+    uint32_t *tmem_slot = (uint32_t *)(bars + 32);
+    volatile int *abort_flag = (volatile int *)(tmem_slot + 1);
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int64_t j0 = (int64_t)blockIdx.x * BK;
+    const int rows_blk = (int)min((int64_t)BK, s.N - j0);   // key rows of this block
+
+    if (threadIdx.x == 0) {
+        for (int i = 0; i < kDNumBars; ++i) {
+            const bool many = (i == kDBarScaled || i == kDBarScaled + 1 || i == kDBarPt || i == kDBarAccFree ||
+                               i == kDBarAccFree + 1 || i == kDBarDs);
+            ptx::mbar_init(&bars[i], many ? kComputeThreads : 1);
+        }
+        *abort_flag = 0;
+        ptx::fence_mbar_init();
+    }
+    if (warp == 0) {
+        ptx::tmem_alloc(tmem_slot, 512);
+        ptx::tmem_relinquish();
+    }
+    ptx::tc_fence_before();
+    __syncthreads();
+    ptx::tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+
+    if (warp >= kProducerWarp) {
+        regs_producer();
+        if (warp == kProducerWarp && lane == 0) {
+            // load sequence idx = 0 .. 2H-1 into buffers idx & 1: dO_idx for idx < H, Q_{idx-H} after
+            auto issue_ld = [&](int idx) {
+                const int b = idx & 1;
+                uint8_t *dst = sm + (b ? L.rb1 : L.rb0);
+                const CUtensorMap *map = idx < H ? &map_do : &map_q;
+                const int h = idx < H ? idx : idx - H;
+                ptx::mbar_arrive_expect_tx(&bars[kDBarLd + b], L.tile_s);
+                for (int kb = 0; kb < D / 64; ++kb)
+                    ptx::tma_load_2d(dst + kb * span * 128, map, h * D + kb * 64, (int)j0, &bars[kDBarLd + b]);
+            };
+            // the block's ds rows of head h (contiguous; wp * 2 is a multiple of 16 bytes)
+            auto issue_ds = [&](int h) {
+                stage_in(sm + L.rs, a.dsb + ((int64_t)h * s.N + j0) * wp, (uint32_t)rows_blk * wp * 2,
+                         &bars[kDBarDsIn]);
+            };
+            const uint32_t id_acc = ptx::idesc_bf16_f32(128, D, 0, 1);     // dV, dK: B MN-major
+            const uint32_t ra = ptx::smem_u32(sm + L.ra);
+            // accumulator product number idx (dV_idx for idx < H, dK_{idx-H} after) into
+            // buffer idx & 1: A = the tile in region A (P^T or ds^T), B = load buffer idx & 1
+            // (g-scaled dO or Q), MN-major
+            auto mma_acc = [&](int idx, bool ok) {
+                const int b = idx & 1;
+                const uint32_t n = (uint32_t)(idx >> 1);
+                if (idx >= 2) ok = wait_bar(&bars[kDBarAccFree + b], (n - 1) & 1, abort_flag) && ok;
+                ptx::tc_fence_after();
+                if (ok) {
+                    const uint32_t ba = ptx::smem_u32(sm + (b ? L.rb1 : L.rb0));
+                    for (int k = 0; k < span / 16; ++k) {
+                        const uint64_t ad = ptx::smem_desc_sw128(ra + (k >> 2) * 16384 + (k & 3) * 32, 16, 1024);
+                        const uint64_t bd2 = ptx::smem_desc_sw128(ba + k * 2048, span * 128, 1024);
+                        ptx::mma_bf16(tmem + 256 + 128 * b, ad, bd2, id_acc, k > 0);
+                    }
+                }
+                ptx::mma_commit(&bars[kDBarAccFull + b]);
+            };
+            // pmap rows j0 .. j0+span-1 (one contiguous run) into the staging area; head 0's ds rows
+            stage_in(sm + L.stage, a.pmap + j0 * W, (uint32_t)(min((int64_t)span, s.N - j0) * W * 2),
+                     &bars[kDBarPmap]);
+            issue_ds(0);
+            if (L.stage_in_b1) issue_ld(0);   // buffer 0 does not overlap the pmap staging rows
+            // ---- phase 1: dV_h = P^T (g_h dO_h)
+            const bool pt_ok = wait_bar(&bars[kDBarPt], 0, abort_flag);   // staging area consumed
+            if (!L.stage_in_b1) issue_ld(0);
+            issue_ld(1);   // dO_1, or Q_0 when H == 1 (there are 2H >= 2 loads)
+            for (int h = 0; h < H; ++h) {
+                const int idx = h, b = idx & 1;
+                const uint32_t n = (uint32_t)(idx >> 1);
+                const bool ok = wait_bar(&bars[kDBarScaled + b], n & 1, abort_flag) && pt_ok;
+                mma_acc(idx, ok);
+                if (idx + 2 < 2 * H && wait_bar(&bars[kDBarAccFull + b], n & 1, abort_flag)) issue_ld(idx + 2);
+            }
+            // ---- phase 2: dK_h = ds^T_h Q_h
+            for (int h = 0; h < H; ++h) {
+                const int idx = H + h, b = idx & 1;
+                const uint32_t n = (uint32_t)(idx >> 1);
+                bool ok = wait_bar(&bars[kDBarDs], (uint32_t)h & 1, abort_flag);   // tile h written, rows read
+                if (ok && h + 1 < H) issue_ds(h + 1);
+                ok = wait_bar(&bars[kDBarLd + b], n & 1, abort_flag) && ok;        // Q_h
+                mma_acc(idx, ok);
+                if (idx + 2 < 2 * H && wait_bar(&bars[kDBarAccFull + b], n & 1, abort_flag)) issue_ld(idx + 2);
+            }
+        }
+        __syncwarp();
+    } else {
+        regs_compute();
+        // ---------------------------------------------------------------- compute warps
+        const int tid = threadIdx.x;   // 0 .. 383
+        const int q = warp & 3, split = warp >> 2;
+        const int i = 32 * q + lane;                 // key row
+        const int64_t j = j0 + i;
+        const bool validk = (i < BK) && (j < s.N);
+        int clo = 1, chi = 0;                         // query columns c (t = j0 + c) that see key j
+        if (validk) {
+            clo = i;
+            const int64_t dend = doc_end(s, j);
+            int64_t hi = j + W - 1;
+            if (hi > dend - 1) hi = dend - 1;
+            chi = (int)(hi - j0);
+        }
+        // column c is in this row's window iff (unsigned)(c - span_lo) <= span_n; a row with an
+        // empty window (clo > chi: past the block or past N) gets span_lo = ~0u, so no c passes
+        const uint32_t span_lo = (chi >= clo) ? (uint32_t)clo : ~0u;
+        const uint32_t span_n = (chi >= clo) ? (uint32_t)(chi - clo) : 0u;
+        const Band bd = make_band(q, split, BK, W, span);
+        const uint32_t lane_base = (uint32_t)(32 * q) << 16;
+
+        // ---- P^T tile: P^T(i, c) = P(j0 + c, j0 + i) = pmap[j0 + c][i - c + W - 1]
+        const uint16_t *stage = (const uint16_t *)(sm + L.stage);
+        wait_bar(&bars[kDBarPmap], 0, abort_flag);
+        uint8_t *atile = sm + L.ra;
+#pragma unroll
+        for (int cc = 0; cc < MAXC; ++cc) {
+            if (cc < bd.mync) {
+                const int col = bd.cb + (bd.c0 + cc) * 8;
+                uint32_t w[4];
+#pragma unroll
+                for (int e = 0; e < 8; e += 2) {
+                    const uint32_t c0 = (uint32_t)(col + e), c1 = c0 + 1;
+                    const uint32_t v0 = (c0 - span_lo <= span_n) ? stage[c0 * W + (i - (int)c0 + W - 1)] : 0u;
+                    const uint32_t v1 = (c1 - span_lo <= span_n) ? stage[c1 * W + (i - (int)c1 + W - 1)] : 0u;
+                    w[e >> 1] = v0 | (v1 << 16);
+                }
+                *(uint4 *)(atile + sw128_offset(i, col)) = make_uint4(w[0], w[1], w[2], w[3]);
+            }
+        }
+        zero_outside_band(atile, i, split, bd, span);
+        ptx::fence_proxy_async_smem();
+        ptx::mbar_arrive(&bars[kDBarPt]);
+
+        // Scale the rows of dO_h (buffer h & 1) by g[t, h] in place.  Eight threads
+        // share one 128-byte row (one 16-byte chunk each), so every quarter warp
+        // touches one row: no bank conflicts.  The g values of a thread's rows are
+        // fetched together, before the wait for the tile.
+        constexpr int kRowsPerPass = kComputeThreads / 8;
+        constexpr int kPasses = (kBwdMaxSpan + kRowsPerPass - 1) / kRowsPerPass;
+        auto scale_do = [&](int h) {
+            const int b = h & 1;
+            float gv[kPasses];
+#pragma unroll
+            for (int it = 0; it < kPasses; ++it) {
+                const int r = (tid >> 3) + it * kRowsPerPass;
+                gv[it] = (r < span && j0 + r < s.N) ? __ldg(a.g + (j0 + r) * H + h) : 0.f;
+            }
+            wait_bar(&bars[kDBarLd + b], (uint32_t)(h >> 1) & 1, abort_flag);
+            uint8_t *tile = sm + (b ? L.rb1 : L.rb0);
+#pragma unroll
+            for (int kb = 0; kb < D / 64; ++kb) {
+#pragma unroll
+                for (int it = 0; it < kPasses; ++it) {
+                    const int r = (tid >> 3) + it * kRowsPerPass;
+                    if (r < span) {
+                        uint4 *p = (uint4 *)(tile + kb * span * 128 + r * 128) + (tid & 7);
+                        uint4 v = *p;
+                        uint32_t *u = &v.x;
+#pragma unroll
+                        for (int e = 0; e < 4; ++e) {
+                            const float f0 = __uint_as_float(u[e] << 16) * gv[it];
+                            const float f1 = __uint_as_float(u[e] & 0xFFFF0000u) * gv[it];
+                            u[e] = pack_bf16x2(f0, f1);
+                        }
+                        *p = v;
+                    }
+                }
+            }
+            ptx::fence_proxy_async_smem();
+            ptx::mbar_arrive(&bars[kDBarScaled + b]);
+        };
+        auto drain = [&](int idx, __nv_bfloat16 *out, int h, float mult) {
+            const int b = idx & 1;
+            wait_bar(&bars[kDBarAccFull + b], (uint32_t)(idx >> 1) & 1, abort_flag);
+            ptx::tc_fence_after();
+            drain_row<D>(tmem + lane_base + 256 + 128 * b, out + (j * H + h) * D, mult, validk, split,
+                         ((uintptr_t)out & 31) == 0);
+            ptx::tc_fence_before();
+            ptx::mbar_arrive(&bars[kDBarAccFree + b]);
+        };
+
+        // ---- phase 1: dV (scaling dO_h runs ahead of draining dV_{h-1}; one copy of each)
+        for (int h = 0; h <= H; ++h) {
+            if (h < H) scale_do(h);
+            if (h >= 1) drain(h - 1, a.dv, h - 1, 1.f);
+        }
+
+        // ---- phase 2: dK.  ds^T(i, c) = ds(j0 + c, j0 + i) = dsb[h][j0 + i][c - i], row i of the
+        // staged rows (stride wp); the tile reuses the P^T region (every dV MMA has completed).
+        const uint16_t *dsr = (const uint16_t *)(sm + L.rs) + i * wp - i;   // dsr[c], c in window
+        for (int h = 0; h <= H; ++h) {   // h == H only drains dK_{H-1}
+            if (h < H) {
+                wait_bar(&bars[kDBarDsIn], (uint32_t)h & 1, abort_flag);
+                uint32_t dsp[MAXC][4];
+#pragma unroll
+                for (int cc = 0; cc < MAXC; ++cc) {
+                    if (cc < bd.mync) {
+                        const int col = bd.cb + (bd.c0 + cc) * 8;
+#pragma unroll
+                        for (int e = 0; e < 8; e += 2) {
+                            const uint32_t c0 = (uint32_t)(col + e), c1 = c0 + 1;
+                            const uint32_t v0 = (c0 - span_lo <= span_n) ? dsr[c0] : 0u;
+                            const uint32_t v1 = (c1 - span_lo <= span_n) ? dsr[c1] : 0u;
+                            dsp[cc][e >> 1] = v0 | (v1 << 16);
+                        }
+                    }
+                }
+                // the previous head's dK MMA must have read the tile before it is overwritten
+                if (h >= 1)
+                    wait_bar(&bars[kDBarAccFull + ((H + h - 1) & 1)], (uint32_t)((H + h - 1) >> 1) & 1, abort_flag);
+#pragma unroll
+                for (int cc = 0; cc < MAXC; ++cc) {
+                    if (cc < bd.mync) {
+                        const int col = bd.cb + (bd.c0 + cc) * 8;
+                        *(uint4 *)(atile + sw128_offset(i, col)) = make_uint4(dsp[cc][0], dsp[cc][1], dsp[cc][2], dsp[cc][3]);
+                    }
+                }
+                ptx::fence_proxy_async_smem();
+                ptx::mbar_arrive(&bars[kDBarDs]);
+            }
+            if (h >= 1) drain(H + h - 1, a.dk, h - 1, s.scale);   // overlaps the dK_h MMA
         }
     }
 

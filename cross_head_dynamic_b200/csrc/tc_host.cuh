@@ -191,10 +191,10 @@ inline cudaError_t fwd(const Shape &s, const void *q, const void *k, const void 
     return e;
 }
 
-template <int D, int MAXC, bool SEG = false>
+template <int D, int MAXC, bool SEG = false, bool DSB = false>
 inline cudaError_t launch_bwd_query(const CUtensorMap &mq, const CUtensorMap &mk, const CUtensorMap &mv,
                                     const CUtensorMap &mdo, const BwdArgs &a, cudaStream_t st) {
-    auto kern = bwd_query_kernel<D, MAXC, SEG>;
+    auto kern = bwd_query_kernel<D, MAXC, SEG, DSB>;
     const uint32_t smem = QSideLayout<D>(a.span).bytes + 1024;
     cudaError_t e = set_smem(kern, smem);
     if (e != cudaSuccess) return e;
@@ -206,7 +206,7 @@ inline cudaError_t launch_bwd_query(const CUtensorMap &mq, const CUtensorMap &mk
 template <int D, int MAXC, bool SEG = false>
 inline cudaError_t launch_bwd_key(const CUtensorMap &mq, const CUtensorMap &mk, const CUtensorMap &mdo,
                                   const BwdArgs &a, cudaStream_t st) {
-    auto kern = bwd_key_kernel<D, MAXC, SEG>;
+    auto kern = bwd_key_seg_kernel<D, MAXC, SEG>;
     const KSideLayout<D> L(a.span, a.s.W);
     if (!SEG && L.stage + L.stage_bytes > L.colv) return cudaErrorInvalidValue;   // staging must fit before colv
     const uint32_t smem = L.bytes + 1024;
@@ -214,6 +214,18 @@ inline cudaError_t launch_bwd_key(const CUtensorMap &mq, const CUtensorMap &mk, 
     if (e != cudaSuccess) return e;
     const unsigned grid = (unsigned)((a.s.N + a.BM - 1) / a.BM);
     kern<<<grid, kThreads, smem, st>>>(mq, mk, mdo, a);
+    return cudaGetLastError();
+}
+
+template <int D, int MAXC>
+inline cudaError_t launch_bwd_key_dsb(const CUtensorMap &mq, const CUtensorMap &mdo, const BwdArgs &a,
+                                      cudaStream_t st) {
+    auto kern = bwd_key_kernel<D, MAXC>;
+    const uint32_t smem = DSideLayout<D>(a.span, a.s.W, a.BM, kDsbRow).bytes + 1024;
+    cudaError_t e = set_smem(kern, smem);
+    if (e != cudaSuccess) return e;
+    const unsigned grid = (unsigned)((a.s.N + a.BM - 1) / a.BM);
+    kern<<<grid, kThreads, smem, st>>>(mq, mdo, a);
     return cudaGetLastError();
 }
 
@@ -231,6 +243,26 @@ inline BwdArgs bwd_args(const Shape &s) {
     a.BM = choose_block(s.N, s.W, sm_count(), kBwdMaxSpan);
     a.span = round16(a.BM + s.W - 1);
     return a;
+}
+
+// Bytes of the key-major ds band [H][N][kDsbRow] bf16 the query side hands to the key side.
+inline size_t dsb_bytes(const Shape &s) { return (size_t)s.H * (size_t)s.N * (size_t)kDsbRow * 2; }
+
+// The backward pair that passes ds through the band (instead of the key side recomputing
+// it from S^T and the dP band) runs when the window is one piece, the workspace holds the
+// band and the key side's shared-memory layout fits (pmap staging rows before the ds rows).
+inline bool use_dsb(const Shape &s, size_t workspace_bytes) {
+    if (segmented(s) || workspace_bytes < dsb_bytes(s)) return false;
+    const BwdArgs a = bwd_args(s);
+    const bool fits128 = [&] {
+        const DSideLayout<128> L(a.span, s.W, a.BM, kDsbRow);
+        return L.stage + L.stage_bytes <= L.rs && L.bytes + 1024 <= 227u * 1024;
+    }();
+    const bool fits64 = [&] {
+        const DSideLayout<64> L(a.span, s.W, a.BM, kDsbRow);
+        return L.stage + L.stage_bytes <= L.rs && L.bytes + 1024 <= 227u * 1024;
+    }();
+    return s.d == 128 ? fits128 : fits64;
 }
 
 // Segmented query side: far segment (dP band, partial dg and dc), near segment (complete
@@ -274,9 +306,12 @@ inline cudaError_t bwd_query_segmented(const Shape &s, const void *q, const void
 
 inline cudaError_t bwd_query(const Shape &s, const void *q, const void *k, const void *v, const float *c,
                              const float *g, const void *dO, const float *lse, const void *pmap, void *dq, float *dc_,
-                             float *dg, float *band, cudaStream_t st, int32_t *launches) {
+                             float *dg, void *workspace, size_t workspace_bytes, cudaStream_t st, int32_t *launches) {
+    float *band = (float *)workspace;
     if (segmented(s)) return bwd_query_segmented(s, q, k, v, c, g, dO, lse, pmap, dq, dc_, dg, band, st, launches);
+    const bool dsb = use_dsb(s, workspace_bytes);
     BwdArgs a = bwd_args(s);
+    if (dsb) a.dsb = (__nv_bfloat16 *)workspace;
     a.c = c;
     a.g = g;
     a.lse = lse;
@@ -292,6 +327,12 @@ inline cudaError_t bwd_query(const Shape &s, const void *q, const void *k, const
     if (e == cudaSuccess) e = make_map(&mdo, dO, s.N, s.H, s.d, 128);
     if (e != cudaSuccess) return e;
     e = [&]() -> cudaError_t {
+        if (dsb) {
+            if (s.d == 64) {
+                DC_TC_MAXC_SWITCH(maxc_for(s.W), (launch_bwd_query<64, MC, false, true>(mq, mk, mv, mdo, a, st)));
+            }
+            DC_TC_MAXC_SWITCH(maxc_for(s.W), (launch_bwd_query<128, MC, false, true>(mq, mk, mv, mdo, a, st)));
+        }
         if (s.d == 64) {
             DC_TC_MAXC_SWITCH(maxc_for(s.W), (launch_bwd_query<64, MC>(mq, mk, mv, mdo, a, st)));
         }
@@ -338,10 +379,30 @@ inline cudaError_t bwd_key_segmented(const Shape &s, const void *q, const void *
 }
 
 inline cudaError_t bwd_key(const Shape &s, const void *q, const void *k, const float *c, const float *g,
-                           const void *dO, const float *lse, const void *pmap, const float *dc_, const float *band,
-                           void *dk, void *dv, cudaStream_t st, int32_t *launches) {
+                           const void *dO, const float *lse, const void *pmap, const float *dc_, const void *workspace,
+                           size_t workspace_bytes, void *dk, void *dv, cudaStream_t st, int32_t *launches) {
+    const float *band = (const float *)workspace;
     if (segmented(s)) return bwd_key_segmented(s, q, k, c, g, dO, lse, pmap, dc_, band, dk, dv, st, launches);
     BwdArgs a = bwd_args(s);
+    if (use_dsb(s, workspace_bytes)) {   // ds from the query side's band
+        a.pmap = (const __nv_bfloat16 *)pmap;
+        a.g = g;
+        a.dsb = (__nv_bfloat16 *)const_cast<void *>(workspace);
+        a.dk = (__nv_bfloat16 *)dk;
+        a.dv = (__nv_bfloat16 *)dv;
+        CUtensorMap mq, mdo;
+        cudaError_t e = make_map(&mq, q, s.N, s.H, s.d, a.span);
+        if (e == cudaSuccess) e = make_map(&mdo, dO, s.N, s.H, s.d, a.span);
+        if (e != cudaSuccess) return e;
+        e = [&]() -> cudaError_t {
+            if (s.d == 64) {
+                DC_TC_MAXC_SWITCH(maxc_for(s.W), (launch_bwd_key_dsb<64, MC>(mq, mdo, a, st)));
+            }
+            DC_TC_MAXC_SWITCH(maxc_for(s.W), (launch_bwd_key_dsb<128, MC>(mq, mdo, a, st)));
+        }();
+        if (e == cudaSuccess) ++*launches;
+        return e;
+    }
     a.c = c;
     a.g = g;
     a.lse = lse;

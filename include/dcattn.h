@@ -94,9 +94,14 @@ dc_status_t dc_attn_fwd(const dc_attn_params *params,
                         const float *c, const float *g,
                         void *o, float *lse, void *pmap, void *stream);
 
-/* Bytes of device scratch the backward entry points need (the composed-map
- * gradient dP(t, .) handed from the query pass to the key pass, fp32 [N][W]).
- * 0 when N == 0. */
+/* Bytes of device scratch the backward entry points ask for; 0 when N == 0.
+ * The least they accept is N * W * 4 (the composed-map gradient dP(t, .) handed
+ * from the query pass to the key pass, fp32 [N][W]).  On the tcgen05 path with
+ * W <= 129 the size returned also holds the ds band, H * N * round8(W) * 2
+ * bytes (bf16 ds_h(t, j) of the query pass, which the key pass then reads
+ * instead of recomputing it); a workspace smaller than that but at least
+ * N * W * 4 runs the recomputing key pass.  Give dc_attn_bwd_query and
+ * dc_attn_bwd_key the same workspace and the same size. */
 size_t dc_attn_bwd_workspace_size(const dc_attn_params *params);
 
 /* Backward, query side: dq [N][H][d], dc [N][H], dg [N][H] fp32, and dP into
@@ -115,7 +120,8 @@ dc_status_t dc_attn_bwd_query(const dc_attn_params *params,
                               void *workspace, size_t workspace_bytes, void *stream);
 
 /* Backward, key side: dk, dv [N][H][d].  Must follow dc_attn_bwd_query on the
- * same stream with the same workspace (it reads dc and the stored dP).
+ * same stream with the same workspace and size (it reads dc and the stored dP,
+ * or the stored ds).
  *   dk_h(j) = sigma sum_{t: j in window(t)} ds_h(t,j) q_h(t)
  *   dv_h(j) = sum_{t: j in window(t)} P(t,j) g[t,h] dO_h(t) */
 dc_status_t dc_attn_bwd_key(const dc_attn_params *params,

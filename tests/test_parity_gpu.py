@@ -180,6 +180,24 @@ def test_guard_bands_untouched(W):
         assert bool((buf[:G] == 7).all()) and bool((buf[-G:] == 7).all())
 
 
+@pytest.mark.parametrize("W", [112, 129])
+def test_backward_with_band_sized_workspace(W):
+    """A workspace of only N * W * 4 bytes (the dP band) is too small for the ds band, so
+    the key side recomputes ds from S^T; both backward pairs must match the oracle."""
+    inp = random_problem(10, [700, 45, 300], 6, 128, W, dtype="bf16")
+    x = to_cuda(inp)
+    N = x["q"].shape[0]
+    o, lse, pmap = dcattn.dc_attn_fwd(x["q"], x["k"], x["v"], x["c"], x["g"], x["cu_seqlens"], W, x["scale"])
+    ws = torch.empty(N * W * 4, device="cuda", dtype=torch.uint8)
+    assert ws.numel() < dcattn.dc_attn_bwd_workspace_size(x["q"], x["cu_seqlens"], W, x["scale"])
+    dq, dk, dv, dc, dg = dcattn.dc_attn_bwd(x["q"], x["k"], x["v"], x["c"], x["g"], x["dO"], lse, pmap,
+                                            x["cu_seqlens"], W, x["scale"], workspace=ws)
+    torch.cuda.synchronize()
+    gpu = {n: t.double().cpu().numpy() for n, t in dict(dq=dq, dk=dk, dv=dv, dc=dc, dg=dg).items()}
+    rows, ref = run_oracle(inp)
+    compare(gpu, rows, ref, TOL["bf16"], names=list(gpu))
+
+
 def test_segmented_forward_without_lse():
     """W > 129 without an lse buffer: AUTO serves it on the SIMT kernels, an explicit
     tcgen05 request is refused before any launch."""
