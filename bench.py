@@ -45,14 +45,14 @@ KERNEL_SOURCES = {
 
 
 def algorithmic_bytes_per_token(H: int, d: int, e: int = 2) -> dict:
-    """Minimal HBM bytes per token each kernel must move (no LSE, pmap or dP band):
+    """Minimal HBM bytes per token each kernel must move (no LSE, pmap or ds band):
     fwd reads q,k,v,c,g and writes o; bwd_query reads q,k,v,dO,c,g and writes
-    dq,dc,dg; bwd_key reads q,k,dO,c,g,dc and writes dk,dv.  The whole step's
-    minimum counts every tensor once: 11*H*d*e + 24*H."""
+    dq,dc,dg; bwd_key (given ds from the query side) reads q,dO,g and writes dk,dv.
+    The whole step's minimum counts every tensor once: 11*H*d*e + 24*H."""
     return {
         "fwd": 4 * H * d * e + 8 * H,
         "bwd_query": 5 * H * d * e + 16 * H,
-        "bwd_key": 5 * H * d * e + 12 * H,
+        "bwd_key": 4 * H * d * e + 4 * H,
         "step": 11 * H * d * e + 24 * H,
     }
 

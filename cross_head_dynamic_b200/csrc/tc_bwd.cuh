@@ -1025,7 +1025,7 @@ bwd_key_seg_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_const
 //   phase 2, per head: ds^T_h tile from the staged rows; MMA dK_h = ds^T_h Q_h, drained
 //            while the next head's tile is built.
 enum : int { kDBarLd = 0, kDBarScaled = 2, kDBarPt = 4, kDBarAccFull = 5, kDBarAccFree = 7, kDBarDsIn = 9,
-             kDBarDs = 10, kDBarPmap = 11, kDNumBars = 12 };
+             kDBarDs = 10, kDBarPmap = 11, kDBarRowsRead = 12, kDNumBars = 13 };
 
 template <int D>
 struct DSideLayout {
@@ -1067,7 +1067,7 @@ bwd_key_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant_
     if (threadIdx.x == 0) {
         for (int i = 0; i < kDNumBars; ++i) {
             const bool many = (i == kDBarScaled || i == kDBarScaled + 1 || i == kDBarPt || i == kDBarAccFree ||
-                               i == kDBarAccFree + 1 || i == kDBarDs);
+                               i == kDBarAccFree + 1 || i == kDBarDs || i == kDBarRowsRead);
             ptx::mbar_init(&bars[i], many ? kComputeThreads : 1);
         }
         *abort_flag = 0;
@@ -1140,8 +1140,9 @@ bwd_key_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant_
             for (int h = 0; h < H; ++h) {
                 const int idx = H + h, b = idx & 1;
                 const uint32_t n = (uint32_t)(idx >> 1);
-                bool ok = wait_bar(&bars[kDBarDs], (uint32_t)h & 1, abort_flag);   // tile h written, rows read
-                if (ok && h + 1 < H) issue_ds(h + 1);
+                // the next head's rows load as soon as this head's have been read into registers
+                if (h + 1 < H && wait_bar(&bars[kDBarRowsRead], (uint32_t)h & 1, abort_flag)) issue_ds(h + 1);
+                bool ok = wait_bar(&bars[kDBarDs], (uint32_t)h & 1, abort_flag);   // tile h written
                 ok = wait_bar(&bars[kDBarLd + b], n & 1, abort_flag) && ok;        // Q_h
                 mma_acc(idx, ok);
                 if (idx + 2 < 2 * H && wait_bar(&bars[kDBarAccFull + b], n & 1, abort_flag)) issue_ld(idx + 2);
@@ -1268,6 +1269,7 @@ bwd_key_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant_
                         }
                     }
                 }
+                ptx::mbar_arrive(&bars[kDBarRowsRead]);   // the staged rows may be replaced
                 // the previous head's dK MMA must have read the tile before it is overwritten
                 if (h >= 1)
                     wait_bar(&bars[kDBarAccFull + ((H + h - 1) & 1)], (uint32_t)((H + h - 1) >> 1) & 1, abort_flag);
