@@ -14,12 +14,17 @@
 //            that dc was computed from.
 //   phase 2, per head: MMA S_h = Q_h K_h^T -> TMEM; SIMT p_h from lse,
 //            dc_h = sum_j dP p_h, ds_h -> bf16 tile in smem; MMA dQ_h = ds_h K_h.
+//            With the ds band (DSB), every ds_h(t, j) also goes to the key-major
+//            band dsb[h][j][t - j] in the workspace, and no dP band is written.
 // Key side (one CTA per block of BK key tokens; the queries that see them span
 // round16(BK + W - 1) rows starting at the block):
 //   phase 1, per head: scale the dO_h rows by g_h in smem; MMA dV_h = P^T gdO_h
 //            with P^T built once from pmap.
-//   phase 2, per head: MMA S^T_h = K_h Q_h^T -> TMEM; SIMT ds^T from lse, c,
-//            dc and the query side's dP; MMA dK_h = ds^T_h Q_h.
+//   phase 2, per head, bwd_key_kernel: the block's rows of the ds band -> ds^T
+//            tile; MMA dK_h = ds^T_h Q_h.
+//   phase 2, per head, bwd_key_seg_kernel (window segments, or a workspace that
+//            holds only the dP band): MMA S^T_h = K_h Q_h^T -> TMEM; SIMT ds^T
+//            from lse, c, dc and the query side's dP; MMA dK_h = ds^T_h Q_h.
 // In both phase-2 loops the gradient MMA of head h runs while the SIMT warps
 // work on the scores of head h+1: the producer issues S_{h+1} before dQ_h/dK_h;
 // the warps write the next ds tile once that MMA has read the current one and
