@@ -224,7 +224,7 @@ def dc_attn_bwd_noalloc(q, k, v, c, g, dO, lse, pmap, cu_seqlens, window, scale,
     """Full backward without a workspace, for callers that cannot allocate scratch
     (plugin-style interfaces that pass an op only its inputs and outputs, or
     processes that reserve all device memory up front).  The library's static
-    32 MiB scratch array holds the dP band instead, so N * W * 4 must not exceed
+    32 MiB scratch array serves as the workspace, so N * W * 4 must not exceed
     32 MiB; overlapping calls on one device race on that array.  Returns
     (dq, dk, dv, dc, dg)."""
     p = make_params(q, cu_seqlens, window, scale, impl)

@@ -144,10 +144,11 @@ dc_status_t dc_attn_bwd(const dc_attn_params *params,
  * plugin-style interfaces that hand an op only its inputs and outputs, and
  * processes whose device memory is reserved by their own pool at start-up and
  * that must not call cudaMalloc afterwards.  Same arguments and results as
- * dc_attn_bwd minus the workspace; the dP band lives instead in a static
+ * dc_attn_bwd minus the workspace; the scratch lives instead in a static
  * device array of 32 MiB (33554432 bytes) that every GPU loading this library
- * keeps until the process exits.
- * - Returns DC_ERR_UNSUPPORTED, before any launch, when the band needs more
+ * keeps until the process exits (it is passed on as a workspace of that size,
+ * so the ds band is used when it fits).
+ * - Returns DC_ERR_UNSUPPORTED, before any launch, when the dP band needs more
  *   than that: N * W * 4 bytes > 32 MiB (e.g. N = 65536 tokens at W = 128).
  * - The first call on each device looks up the array's device address with
  *   that device current; make that first call before any stream capture.
