@@ -139,6 +139,14 @@ cudaError_t simt_bwd_key(const dc::Shape &s, const void *q, const void *k, const
     }()
 
 // The smallest workspace the backward takes: the dP band [N][W] fp32.
+// dst[i] += src[i] (fp32 sum, rounded once to T): the dk, dv partials a token-range
+// shard returns to the shard that owns the halo keys.
+template <typename T>
+__global__ void halo_add_kernel(T *dst, const T *src, int64_t n) {
+    for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n; i += (int64_t)gridDim.x * blockDim.x)
+        dc::stf<T>(dst + i, dc::ldf<T>(dst + i) + dc::ldf<T>(src + i));
+}
+
 size_t band_bytes(const dc::Shape &s) { return sizeof(float) * (size_t)s.N * (size_t)s.W; }
 
 // The workspace the backward asks for: on the tcgen05 path with a one-piece window also
@@ -235,6 +243,24 @@ dc_status_t dc_attn_bwd(const dc_attn_params *params, const void *q, const void 
     r = dc_attn_bwd_key(params, q, k, c, g, dO, lse, pmap, dc_, dk, dv, workspace, workspace_bytes, stream);
     t_launches += n1;
     return r;
+}
+
+dc_status_t dc_attn_halo_add(void *dst, const void *src, int64_t n, int32_t dtype, void *stream) {
+    if (n < 0 || (dtype != DC_F32 && dtype != DC_BF16)) return DC_ERR_INVALID_ARG;
+    t_launches = 0;
+    if (n == 0) return DC_OK;
+    dc_status_t r = ptrs_ok({dst, src}, {});
+    if (r != DC_OK) return r;
+    const int threads = 256;
+    const int64_t want = (n + threads - 1) / threads;
+    const unsigned blocks = (unsigned)(want < 148 * 16 ? want : 148 * 16);
+    cudaStream_t st = (cudaStream_t)stream;
+    if (dtype == DC_F32)
+        halo_add_kernel<float><<<blocks, threads, 0, st>>>((float *)dst, (const float *)src, n);
+    else
+        halo_add_kernel<__nv_bfloat16><<<blocks, threads, 0, st>>>((__nv_bfloat16 *)dst, (const __nv_bfloat16 *)src, n);
+    ++t_launches;
+    return cuda_status(cudaGetLastError());
 }
 
 int32_t dc_attn_resolve_impl(const dc_attn_params *params) {

@@ -24,7 +24,7 @@ DC_DEVERR_TIMEOUT = 0x2
 
 EXPORTED = ("dc_attn_fwd", "dc_attn_bwd_workspace_size", "dc_attn_bwd_query", "dc_attn_bwd_key",
             "dc_attn_bwd", "dc_attn_resolve_impl", "dc_attn_device_status", "dc_attn_status_string",
-            "dc_attn_last_launch_count", "dc_attn_bwd_noalloc")
+            "dc_attn_last_launch_count", "dc_attn_bwd_noalloc", "dc_attn_halo_add")
 
 
 class DCAttnError(RuntimeError):
@@ -74,6 +74,8 @@ def load_library(path: str = LIB_PATH):
     lib.dc_attn_bwd_noalloc.restype = st
     lib.dc_attn_last_launch_count.argtypes = []
     lib.dc_attn_last_launch_count.restype = ctypes.c_int32
+    lib.dc_attn_halo_add.argtypes = [vp, vp, ctypes.c_int64, ctypes.c_int32, vp]
+    lib.dc_attn_halo_add.restype = st
     _lib = lib
     return lib
 
@@ -254,3 +256,16 @@ def dc_attn_device_status(reset: bool = True, stream=None) -> int:
 
 def dc_attn_last_launch_count() -> int:
     return int(load_library().dc_attn_last_launch_count())
+
+
+def dc_attn_halo_add(dst, src, stream=None):
+    """dst += src in place (same shape, bf16 or fp32; fp32 sum rounded once), on the GPU."""
+    if dst.shape != src.shape or dst.dtype != src.dtype:
+        raise ValueError("dc_attn_halo_add: dst and src differ in shape or dtype")
+    dt = {torch.float32: DC_F32, torch.bfloat16: DC_BF16}.get(dst.dtype)
+    if dt is None:
+        raise ValueError(f"dc_attn_halo_add: unsupported dtype {dst.dtype}")
+    code = load_library().dc_attn_halo_add(_dev(dst, "dst", dst.dtype), _dev(src, "src", dst.dtype), dst.numel(),
+                                           dt, _stream_handle(stream))
+    _check("dc_attn_halo_add", code)
+    return dst

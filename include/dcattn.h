@@ -165,6 +165,14 @@ dc_status_t dc_attn_bwd_noalloc(const dc_attn_params *params,
                                 void *dq, void *dk, void *dv, float *dc, float *dg,
                                 void *stream);
 
+/* dst[i] += src[i] for i < n, in `dtype` (dc_dtype_t) with an fp32 sum rounded
+ * once (no counterpart on the page; an interface addition for token-range
+ * sharding of one long sequence over several GPUs: the dk and dv partials that
+ * a shard computes for the W - 1 keys before its range, which belong to its left
+ * neighbour, are added there).  dst and src: device, 16-byte aligned, not
+ * overlapping.  Asynchronous on `stream`. */
+dc_status_t dc_attn_halo_add(void *dst, const void *src, int64_t n, int32_t dtype, void *stream);
+
 /* Which kernel family AUTO resolves to for these params (DC_IMPL_SIMT or
  * DC_IMPL_TCGEN05), or -1 if the params are invalid. */
 int32_t dc_attn_resolve_impl(const dc_attn_params *params);
