@@ -92,6 +92,15 @@ def test_null_and_misaligned_pointers_rejected(lib):
     assert _fwd(lib, p, ptr=0x2008) == dcattn.DC_ERR_INVALID_ARG
 
 
+def test_halo_add_rejects_bad_arguments_on_host(lib):
+    ok = 0x4000
+    assert lib.dc_attn_halo_add(ok, ok, 16, 7, None) == dcattn.DC_ERR_INVALID_ARG          # dtype
+    assert lib.dc_attn_halo_add(ok, ok, -1, dcattn.DC_BF16, None) == dcattn.DC_ERR_INVALID_ARG
+    assert lib.dc_attn_halo_add(0, ok, 16, dcattn.DC_BF16, None) == dcattn.DC_ERR_INVALID_ARG   # null
+    assert lib.dc_attn_halo_add(ok, 0x4008, 16, dcattn.DC_F32, None) == dcattn.DC_ERR_INVALID_ARG  # misaligned
+    assert lib.dc_attn_halo_add(0, 0, 0, dcattn.DC_F32, None) == dcattn.DC_OK                # n = 0: no-op
+
+
 def test_empty_problem_is_a_noop(lib):
     p = _params(total_tokens=0, num_docs=0, cu_seqlens=0)
     assert _fwd(lib, p, ptr=0) == dcattn.DC_OK
