@@ -247,6 +247,8 @@ def run_sweep(args):
     peaks = json.load(open(PEAKS_FILE)) if os.path.exists(PEAKS_FILE) else {}
     hbm = peaks.get("hbm_gbs") or 6650.0
     for name, cfg in CONFIGS.items():
+        if args.workload and name not in args.workload:
+            continue
         host = generate(cfg)
         N, H, d, W, scale = cfg.total_tokens, cfg.heads, cfg.head_dim, cfg.window, cfg.softmax_scale
         dt = host["q"].dtype
@@ -321,6 +323,8 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--sweep", action="store_true",
                     help="one JSON line per workload of the inputs module instead of the headline line")
+    ap.add_argument("--workload", action="append", choices=list(CONFIGS),
+                    help="with --sweep: only these workloads (repeatable)")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
