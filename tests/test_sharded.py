@@ -50,6 +50,9 @@ CASES = {
     "even_w9": ([30, 5, 50, 1, 34], 9, None),
     "uneven_w16": ([70, 3, 47], 16, [(0, 20), (20, 90), (90, 120)]),
     "one_doc_w16": ([96], 16, None),
+    "w1_no_halo": ([40, 1, 39], 1, None),
+    # four ranges, the middle ones exactly as long as the halo their right neighbour needs
+    "min_ranges_w16": ([20, 45, 2, 33], 16, [(0, 40), (40, 55), (55, 70), (70, 100)]),
 }
 
 
@@ -84,9 +87,11 @@ def _rank_main(rank, world, port, case, out):
         dist.destroy_process_group()
 
 
-@pytest.mark.parametrize("world", [2, 3])
+@pytest.mark.parametrize("world", [2, 3, 4])
 @pytest.mark.parametrize("case", list(CASES))
 def test_sharded_matches_unsharded_oracle(case, world):
+    if world == 4 and case != "min_ranges_w16":
+        pytest.skip("four ranks run on the case built for them")
     port = _free_port()
     out = mp.get_context("spawn").Manager().dict()
     mp.spawn(_rank_main, args=(world, port, case, out), nprocs=world, join=True)
