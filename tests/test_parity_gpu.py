@@ -2,8 +2,9 @@
 
 Metric per output tensor: max|gpu - oracle| / max|oracle|; bound 1e-5 for fp32
 storage and 1.5e-2 for bf16 storage (fp32 accumulation on the GPU in both).
-Large workloads are checked on whole documents sampled from the full-size GPU
-run (documents are independent, so the oracle's values for them are exact).
+Every workload, the full-size ones included, is compared on every token of
+every output tensor: each document boundary of the packed varlen batch falls
+at its own offset inside a query block, and all of them are checked.
 """
 import json
 import math
@@ -85,6 +86,12 @@ EDGE_CASES = [
     # the widest window the tcgen05 kernels take in one piece (7 chunks of 8 columns per
     # thread), the most heads, and the first window past it
     ("bf16_w129", [700, 45], 4, 128, 129, "bf16"),
+    # windows of 97-113 keys hand ds from the query side to the key side as whole tiles
+    # (key tile starting 112 keys before the block): the smallest and largest such window,
+    # one in between with d = 64 and twelve heads, documents starting inside blocks
+    ("bf16_w97_tiles", [333, 90, 1], 6, 128, 97, "bf16"),
+    ("bf16_w113_tiles", [400, 2, 300], 3, 128, 113, "bf16"),
+    ("bf16_w100_d64_tiles", [500, 37, 260], 12, 64, 100, "bf16"),
     ("bf16_w120_h16_d64", [520], 16, 64, 120, "bf16"),
     # W > 129: a near segment of 128 keys and a far one of W - 128 (2 keys at W = 130); documents
     # shorter than the near segment (far segment empty), windows past the document start,
@@ -108,25 +115,17 @@ def test_edge_cases(case, impl):
     compare(gpu, rows, ref, TOL[dtype])
 
 
-def _sample_docs(cfg, cu):
-    n = len(cu) - 1
-    if cfg.docs == "rows":
-        # both end rows of short-row batches; the last row of long-row batches
-        return sorted({0, n - 1}) if cfg.seqlen <= 4096 else [n - 1]
-    # varlen: the first three documents, one in the middle, and the last one
-    return sorted({0, 1, 2, n // 2, n - 1})
-
-
 CONFIG_NAMES = [n for n in CONFIGS if n != "tiny_fp32"]
 
 
 @pytest.mark.parametrize("name", CONFIG_NAMES)
 def test_config_parity(name):
+    """Full-size workload in the launch configuration the benchmark times, every row."""
     cfg = CONFIGS[name]
     inp = generate(cfg)
     gpu = run_gpu(inp, backward=cfg.backward)
-    docs = _sample_docs(cfg, inp["cu_seqlens"])
-    rows, ref = run_oracle(inp, docs=docs, backward=cfg.backward)
+    rows, ref = run_oracle(inp, backward=cfg.backward)
+    assert len(rows) == cfg.total_tokens
     compare(gpu, rows, ref, TOL[cfg.dtype])
 
 
