@@ -23,6 +23,8 @@ struct Shape {
     int W;
     float scale;
     const int32_t *cu;
+    uint32_t wait_ns;   // limit of every bounded wait in the tcgen05 kernels (nanoseconds)
+    int inject;         // test hook: the tcgen05 forward's first CTA leaves out its first Q/K load
 };
 
 template <typename T> __device__ __forceinline__ float ldf(const T *p);

@@ -6,6 +6,7 @@
 #include <stdint.h>
 #include <string.h>
 
+#include <atomic>
 #include <mutex>
 
 #include "dcattn.h"
@@ -16,6 +17,11 @@
 namespace {
 
 thread_local int32_t t_launches = 0;
+
+// Test hooks: the limit of every bounded wait in the tcgen05 kernels launched from now
+// on, and a one-shot request that the next one-piece tcgen05 forward leaves out a load.
+std::atomic<uint32_t> g_wait_ns{dc::tc::kWaitNs};
+std::atomic<int> g_inject{0};
 
 struct Checked {
     dc::Shape s;
@@ -47,6 +53,8 @@ dc_status_t check_params(const dc_attn_params *p, Checked *out) {
     out->s.W = p->window;
     out->s.scale = p->softmax_scale;
     out->s.cu = p->cu_seqlens;
+    out->s.wait_ns = g_wait_ns.load(std::memory_order_relaxed);
+    out->s.inject = 0;
     out->dtype = p->dtype;
     const bool tc_ok = p->dtype == DC_BF16 && dc::tc::supports(out->s);
     if (p->impl == DC_IMPL_TCGEN05) {
@@ -154,7 +162,7 @@ size_t band_bytes(const dc::Shape &s) { return sizeof(float) * (size_t)s.N * (si
 size_t ws_need(const Checked &ck) {
     size_t b = band_bytes(ck.s);
     if (ck.impl == DC_IMPL_TCGEN05 && !dc::tc::segmented(ck.s)) {
-        const size_t d = dc::tc::dsb_bytes(ck.s);
+        const size_t d = dc::tc::dst_shape(ck.s) ? dc::tc::dst_bytes(ck.s) : dc::tc::dsb_bytes(ck.s);
         if (d > b) b = d;
     }
     return b;
@@ -179,8 +187,10 @@ dc_status_t dc_attn_fwd(const dc_attn_params *params, const void *q, const void 
         if (params->impl == DC_IMPL_TCGEN05) return DC_ERR_UNSUPPORTED;
         ck.impl = DC_IMPL_SIMT;
     }
-    if (ck.impl == DC_IMPL_TCGEN05)
+    if (ck.impl == DC_IMPL_TCGEN05) {
+        if (!dc::tc::segmented(ck.s)) ck.s.inject = g_inject.exchange(0);
         return cuda_status(dc::tc::fwd(ck.s, q, k, v, c, g, o, lse, pmap, st, &t_launches));
+    }
     return cuda_status(DC_DISPATCH(simt_fwd, ck.dtype, ck.s.d, ck.s, q, k, v, c, g, o, lse, pmap, st));
 }
 
@@ -300,6 +310,18 @@ const char *dc_attn_status_string(dc_status_t status) {
 
 int32_t dc_attn_last_launch_count(void) { return t_launches; }
 
+dc_status_t dc_attn_set_wait_limit(uint32_t ns) {
+    if (ns == 0) ns = dc::tc::kWaitNs;
+    if (ns < 100000u) return DC_ERR_INVALID_ARG;
+    g_wait_ns.store(ns, std::memory_order_relaxed);
+    return DC_OK;
+}
+
+dc_status_t dc_attn_inject_missing_load(void) {
+    g_inject.store(1);
+    return DC_OK;
+}
+
 }  // extern "C"
 
 // --------------------------------------------------------------------------
@@ -322,16 +344,23 @@ constexpr int kMaxDevices = 64;
 std::mutex g_noalloc_mutex;
 void *g_noalloc_ptr[kMaxDevices] = {};
 
-// Device address of the scratch array on the current device, looked up once per
-// device (cudaGetSymbolAddress with that device current).  In host code the
-// array's name is only a host-side stand-in, never a usable device pointer.
-cudaError_t noalloc_scratch(void **out) {
+// Device address of the scratch array on the current device.  In host code the
+// array's name is only a host-side stand-in, never a usable device pointer, so
+// the address comes from cudaGetSymbolAddress with that device current.  It is
+// looked up again on every call made outside stream capture (a cudaDeviceReset
+// in between would leave an older address dangling); a call made while `stream`
+// is being captured uses the address an earlier call found on the device, since
+// the lookup may load the module, which capture does not allow.
+cudaError_t noalloc_scratch(cudaStream_t stream, void **out) {
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess) return e;
     if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
+    cudaStreamCaptureStatus cap = cudaStreamCaptureStatusNone;
+    e = cudaStreamIsCapturing(stream, &cap);
+    if (e != cudaSuccess) return e;
     std::lock_guard<std::mutex> lock(g_noalloc_mutex);
-    if (!g_noalloc_ptr[dev]) {
+    if (cap == cudaStreamCaptureStatusNone || !g_noalloc_ptr[dev]) {
         void *p = nullptr;
         e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
         if (e != cudaSuccess) return e;
@@ -358,7 +387,7 @@ dc_status_t dc_attn_bwd_noalloc(const dc_attn_params *params, const void *q, con
         return DC_OK;
     }
     void *scratch = nullptr;
-    if (noalloc_scratch(&scratch) != cudaSuccess) {
+    if (noalloc_scratch((cudaStream_t)stream, &scratch) != cudaSuccess) {
         (void)cudaGetLastError();
         return DC_ERR_CUDA;
     }

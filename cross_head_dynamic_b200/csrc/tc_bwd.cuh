@@ -16,6 +16,9 @@
 //            dc_h = sum_j dP p_h, ds_h -> bf16 tile in smem; MMA dQ_h = ds_h K_h.
 //            With the ds band (DSB), every ds_h(t, j) also goes to the key-major
 //            band dsb[h][j][t - j] in the workspace, and no dP band is written.
+//            With the ds tile hand-off (DST) the key tile starts BM keys before the
+//            block (span = 2 BM), and the ds tile itself, [BM queries x 2 BM keys],
+//            goes to the workspace by TMA tensor stores; no dP band either.
 // Key side (one CTA per block of BK key tokens; the queries that see them span
 // round16(BK + W - 1) rows starting at the block):
 //   phase 1, per head: scale the dO_h rows by g_h in smem; MMA dV_h = P^T gdO_h
@@ -25,6 +28,10 @@
 //   phase 2, per head, bwd_key_seg_kernel (window segments, or a workspace that
 //            holds only the dP band): MMA S^T_h = K_h Q_h^T -> TMEM; SIMT ds^T
 //            from lse, c, dc and the query side's dP; MMA dK_h = ds^T_h Q_h.
+//   bwd_key_dst_kernel (ds tiles): the key block's ds^T_h arrives by four TMA boxes
+//            of the query side's tiles (its own block's and the next block's) and is
+//            used as it lands, as an MN-major A operand; the compute warps only build
+//            the P tile once, scale dO and drain.
 // In both phase-2 loops the gradient MMA of head h runs while the SIMT warps
 // work on the scores of head h+1: the producer issues S_{h+1} before dQ_h/dK_h;
 // the warps write the next ds tile once that MMA has read the current one and
@@ -99,7 +106,7 @@ __device__ __forceinline__ void drain_row(uint32_t taddr, __nv_bfloat16 *dst, fl
 
 // --------------------------------------------------------------------------- query side
 enum : int { kQBarLd = 0, kQBarQ = 2, kQBarK = 3, kQBarXFull = 5, kQBarXFree = 6, kQBarDs = 7, kQBarDqFull = 8,
-             kQBarDqFree = 10, kQBarPmap = 12, kQNumBars = 13 };
+             kQBarDqFree = 10, kQBarPmap = 12, kQBarDsRead = 13, kQNumBars = 14 };
 
 // Copy `bytes` bytes of global memory to shared memory: a bulk copy of the 16-byte
 // multiple (completing on `bar`) and plain copies of the rest.  The caller's arrive on
@@ -138,11 +145,12 @@ struct QSideLayout {
     }
 };
 
-template <int D, int MAXC, bool SEG = false, bool DSB = false>
+template <int D, int MAXC, bool SEG = false, bool DSB = false, bool DST = false>
 __global__ void __launch_bounds__(kThreads, 1)
 bwd_query_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__ CUtensorMap map_k,
                  const __grid_constant__ CUtensorMap map_v, const __grid_constant__ CUtensorMap map_do,
-                 const BwdArgs a) {
+                 const __grid_constant__ CUtensorMap map_ds, const BwdArgs a) {
+    static_assert(!(DSB && DST) && !(SEG && (DSB || DST)), "one hand-off per instantiation");
     extern __shared__ uint8_t smem_raw[];
     uint8_t *sm = (uint8_t *)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
     const Shape &s = a.s;
@@ -155,7 +163,11 @@ bwd_query_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int64_t t0 = (int64_t)blockIdx.x * BM;
-    const int64_t kbase = SEG ? t0 - a.seg.shift - (W - 1) : t0 - (W - 1);
+    // DST: the key tile starts BM keys before the block, so that the key blocks of the
+    // key side are whole 64-column-aligned column ranges of the ds tile; row i's window
+    // then starts at column i + off
+    const int off = DST ? BM - (W - 1) : 0;
+    const int64_t kbase = SEG ? t0 - a.seg.shift - (W - 1) : t0 - (W - 1) - off;
     const bool do_p1 = !SEG || a.seg.mode != kQSegFarPart2;   // phase 1 (E, dP band, dg)
     const bool do_dq = !SEG || a.seg.mode != kQSegFarPart1;   // ds and dQ
     const int ph0 = do_p1 ? H : 0;                            // X-buffer phases before phase 2
@@ -163,10 +175,10 @@ bwd_query_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
     validate_seqlens(s);
     if (threadIdx.x == 0) {
         for (int i = 0; i < kQNumBars; ++i) {
-            const bool many = (i == kQBarXFree || i == kQBarDs || i == kQBarDqFree || i == kQBarDqFree + 1);
+            const bool many = (i == kQBarXFree || i == kQBarDs || i == kQBarDqFree || i == kQBarDqFree + 1);   // 384
             ptx::mbar_init(&bars[i], many ? kComputeThreads : 1);
         }
-        *abort_flag = 0;
+        init_ctl(abort_flag, s.wait_ns);
         ptx::fence_mbar_init();
     }
     if (warp == 0) {
@@ -223,6 +235,22 @@ bwd_query_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
                     }
                 }
                 ptx::mma_commit(&bars[kQBarDqFull + b]);
+                if constexpr (DST) {
+                    // the ds tile (its first BM rows, 64-column boxes) to the workspace; the
+                    // compute warps rewrite it for the next head once the store has read it
+                    // (ds_released, after the producer's refills)
+                    if (ok) {
+                        for (int cb = 0; cb < span; cb += 64)
+                            ptx::tma_store_3d(&map_ds, cb, (int)t0, h, sm + L.rd + (cb >> 6) * 16384);
+                    }
+                    ptx::bulk_commit();
+                }
+            };
+            auto ds_released = [&]() {
+                if constexpr (DST) {
+                    ptx::bulk_wait_read();
+                    ptx::mbar_arrive(&bars[kQBarDsRead]);
+                }
             };
 
             // the CTA's pmap rows (one contiguous [BM][W] run) into the upper half of the ds
@@ -295,7 +323,9 @@ bwd_query_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
                                : s_done))
                         issue_k(h + 1);
                 }
+                if (h >= 1 && do_dq) ds_released();   // after the refills: they must not wait on it
             }
+            if constexpr (DST) ptx::bulk_wait_all();   // the ds tiles have reached global memory
         }
         __syncwarp();
     } else {
@@ -318,10 +348,22 @@ bwd_query_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
                 chi = (int)(t - kbase);
             }
         }
-        const Band bd = make_band(q, split, BM, W, span);
+        const Band bd = make_band(q, split, BM, W, span, off);
         const uint32_t lane_base = (uint32_t)(32 * q) << 16;
         const uint32_t x_cols = tmem + lane_base;
         const float sl2 = s.scale * kLog2e;
+        // g (phase 1), lse and c (phase 2) of this row are read once per head.  A first
+        // read that misses L2 costs microseconds while every CTA streams its tiles, so the
+        // rows are brought into L2 now and each head's value is loaded one head ahead.
+        if (valid && split == 0) {
+            ptx::prefetch_l2(a.g + t * H);
+            ptx::prefetch_l2(a.g + t * H + H - 1);
+            ptx::prefetch_l2(a.lse + t * H);
+            ptx::prefetch_l2(a.lse + t * H + H - 1);
+            ptx::prefetch_l2(a.c + t * H);
+            ptx::prefetch_l2(a.c + t * H + H - 1);
+        }
+        float g_next = (valid && do_p1) ? __ldg(a.g + t * H) : 0.f;
         // column c is in this row's window iff (unsigned)(c - win_lo) <= win_n (never for a row
         // with an empty window)
         const uint32_t win_lo = (chi >= clo) ? (uint32_t)clo : ~0u;
@@ -335,7 +377,7 @@ bwd_query_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
             dsrow = (uint16_t *)a.dsb + (kbase + c_first) * kDsbRow + (i + W - 1 - c_first);
         }
 
-        // P(t, c) = pmap[t][c - i] on this thread's band, from the CTA's pmap rows staged by
+        // P(t, c) = pmap[t][c - i - off] on this thread's band, from the CTA's pmap rows staged by
         // the producer; zero outside the window.  Kept in registers (bf16 pairs) for all heads.
         // A segment reads its columns of the row from global memory.
         uint32_t pvp[MAXC][4];
@@ -355,7 +397,7 @@ bwd_query_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
                 }
             }
         } else {
-            const uint16_t *prow = (const uint16_t *)(sm + L.rd + 32768) + i * W - i;
+            const uint16_t *prow = (const uint16_t *)(sm + L.rd + 32768) + i * W - i - off;
             wait_bar(&bars[kQBarPmap], 0, abort_flag);
 #pragma unroll
             for (int cc = 0; cc < MAXC; ++cc) {
@@ -395,9 +437,10 @@ bwd_query_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
         // unmasked: outside the window it only ever meets p = 0 (and the key side reads
         // the band inside the window only); P is zero there, so dg needs no mask either.
         for (int h = 0; h < (do_p1 ? H : 0); ++h) {
+            const float gh = g_next;
+            if (h + 1 < H) g_next = valid ? __ldg(a.g + t * H + h + 1) : 0.f;
             wait_bar(&bars[kQBarXFull], (uint32_t)h & 1, abort_flag);
             ptx::tc_fence_after();
-            const float gh = valid ? __ldg(a.g + t * H + h) : 0.f;
             float dga = 0.f, dgb = 0.f;
             constexpr int G = 3;
 #pragma unroll
@@ -464,7 +507,7 @@ bwd_query_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
                     }
                 }
             }
-        } else if constexpr (!DSB) {   // (with the ds band the key side needs no dP)
+        } else if constexpr (!DSB && !DST) {   // (with the ds band or tiles the key side needs no dP)
             float *stage = (float *)(sm + L.rd);
             if (i < BM) {
 #pragma unroll
@@ -488,6 +531,8 @@ bwd_query_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
         // copy reads it while head 0's scores are processed, and it is reused from head 0's
         // ds tile on (columns outside this quarter's band zeroed once).
         uint8_t *dtile = sm + L.rd;
+        float lse_next = valid ? __ldg(a.lse + t * H) : 0.f;   // head 0's values, loaded ahead
+        float c_next = valid ? __ldg(a.c + t * H) : 0.f;
         auto drain_dq = [&](int h) {
             const int b = h & 1;
             wait_bar(&bars[kQBarDqFull + b], (uint32_t)(h >> 1) & 1, abort_flag);
@@ -504,9 +549,14 @@ bwd_query_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
         for (int h = 0; h <= (do_dq ? H : H - 1); ++h) {   // h == H only drains dQ_{H-1}
             if (h < H) {
                 const uint32_t ph = (uint32_t)(ph0 + h);
+                const float lse2 = lse_next * kLog2e;
+                const float ch = c_next;
+                if (h + 1 < H) {
+                    lse_next = valid ? __ldg(a.lse + t * H + h + 1) : 0.f;
+                    c_next = valid ? __ldg(a.c + t * H + h + 1) : 0.f;
+                }
                 wait_bar(&bars[kQBarXFull], ph & 1, abort_flag);
                 ptx::tc_fence_after();
-                const float lse2 = valid ? __ldg(a.lse + t * H + h) * kLog2e : 0.f;
                 // p_h and dc_h, the band of S_h in two TMEM round trips
                 float dca = 0.f, dcb = 0.f;   // two independent chains
                 uint32_t pp[MAXC][4];   // p_h as packed bf16 pairs
@@ -558,13 +608,13 @@ bwd_query_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
                     if (split == 0 && valid) a.dc[t * H + h] = dch;
                 }
                 if (!do_dq) continue;   // the first far-segment launch stops at dc
-                const float ch = valid ? __ldg(a.c + t * H + h) : 0.f;
                 // the previous head's dQ MMA has been running meanwhile; once it has completed the
                 // ds tile is free for this head (its accumulator is drained after the tile is handed on)
                 if (h >= 1) {
                     wait_bar(&bars[kQBarDqFull + ((h - 1) & 1)], (uint32_t)((h - 1) >> 1) & 1, abort_flag);
+                    if constexpr (DST) wait_bar(&bars[kQBarDsRead], (uint32_t)(h - 1) & 1, abort_flag);
                 } else {
-                    if (!SEG && !DSB && threadIdx.x == 0) ptx::bulk_wait_read();   // the band copy has left the region
+                    if (!SEG && !DSB && !DST && threadIdx.x == 0) ptx::bulk_wait_read();   // the band copy has left the region
                     compute_sync();
                     zero_outside_band(dtile, i, split, bd, span);
                 }
@@ -664,7 +714,7 @@ bwd_key_seg_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_const
                                i == kKBarAccFree + 1 || i == kKBarXFree || i == kKBarDs);
             ptx::mbar_init(&bars[i], many ? kComputeThreads : 1);
         }
-        *abort_flag = 0;
+        init_ctl(abort_flag, s.wait_ns);
         ptx::fence_mbar_init();
     }
     if (warp == 0) {
@@ -1075,7 +1125,7 @@ bwd_key_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant_
                                i == kDBarAccFree + 1 || i == kDBarDs || i == kDBarRowsRead);
             ptx::mbar_init(&bars[i], many ? kComputeThreads : 1);
         }
-        *abort_flag = 0;
+        init_ctl(abort_flag, s.wait_ns);
         ptx::fence_mbar_init();
     }
     if (warp == 0) {
@@ -1290,6 +1340,254 @@ bwd_key_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant_
             }
             if (h >= 1) drain(H + h - 1, a.dk, h - 1, s.scale);   // overlaps the dK_h MMA
         }
+    }
+
+    ptx::tc_fence_before();
+    __syncthreads();
+    if (warp == 0) {
+        ptx::tc_fence_after();
+        ptx::tmem_dealloc(tmem, 512);
+    }
+}
+
+// --------------------------------------------------------------------------- key side, ds tiles
+// Key block [j0, j0 + BK) with BK the query side's BM; the queries that see its keys are
+// t in [j0, j0 + 2 BK) (W - 1 <= BK): the rows of this block's ds tile and of the next
+// block's.  In a query block's tile, column c is key t0 - BM + c, so the key block's keys
+// are columns BK .. 2 BK - 1 of its own block's tile and columns 0 .. BK - 1 of the next
+// block's: whole 64-column boxes for TMA.
+//   phase 1, per head: scale the dO_h rows by g_h in smem; MMA dV_h = P^T gdO_h with
+//            A = the P tile [span queries x 128 keys] (MN-major), built once from pmap.
+//   phase 2, per head: four TMA boxes land ds_h(t, j) for the block's keys as a
+//            [span queries x 128 keys] tile, which is A = ds^T_h (MN-major) as it is;
+//            MMA dK_h = ds^T_h Q_h, drained while the next head's product runs.
+// The compute warps build the P tile, scale dO and drain; they never touch ds.
+enum : int { kTBarLd = 0, kTBarScaled = 2, kTBarPt = 4, kTBarAccFull = 5, kTBarAccFree = 7, kTBarDs = 9,
+             kTBarPmap = 11, kTNumBars = 12 };
+
+template <int D>
+struct TSideLayout {
+    uint32_t tile_a;   // P tile or ds^T tile: 2 boxes of 64 key columns x span rows
+    uint32_t tile_s;   // dO or Q tile over the query span: D/64 boxes of span rows x 128 B
+    uint32_t ra0, ra1, rb0, rb1, bars, bytes;
+    __host__ __device__ TSideLayout(int span) {
+        tile_a = 2u * (uint32_t)span * 128;
+        tile_s = (uint32_t)(D / 64) * span * 128;
+        ra0 = 0;                  // P tile (phase 1) / ds^T of odd heads (phase 2)
+        ra1 = ra0 + tile_a;       // pmap rows of the query span (start) / ds^T of even heads
+        rb0 = ra1 + tile_a;       // dO buffer 0 (phase 1) / Q buffer 0 (phase 2)
+        rb1 = rb0 + tile_s;       // dO buffer 1 / Q buffer 1
+        bars = rb1 + tile_s;
+        bytes = bars + 512;
+    }
+};
+
+template <int D>
+__global__ void __launch_bounds__(kThreads, 1)
+bwd_key_dst_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__ CUtensorMap map_do,
+                   const __grid_constant__ CUtensorMap map_ds, const BwdArgs a) {
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *sm = (uint8_t *)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
+    const Shape &s = a.s;
+    const int H = s.H, W = s.W, BK = a.BM, span = a.span;   // span = 2 BK
+    const TSideLayout<D> L(span);
+    uint64_t *bars = (uint64_t *)(sm + L.bars);
+    uint32_t *tmem_slot = (uint32_t *)(bars + 32);
+    volatile int *abort_flag = (volatile int *)(tmem_slot + 1);
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int64_t j0 = (int64_t)blockIdx.x * BK;
+
+    if (threadIdx.x == 0) {
+        for (int i = 0; i < kTNumBars; ++i) {
+            const bool many = (i == kTBarScaled || i == kTBarScaled + 1 || i == kTBarPt || i == kTBarAccFree ||
+                               i == kTBarAccFree + 1);
+            ptx::mbar_init(&bars[i], many ? kComputeThreads : 1);
+        }
+        init_ctl(abort_flag, s.wait_ns);
+        ptx::fence_mbar_init();
+    }
+    if (warp == 0) {
+        ptx::tmem_alloc(tmem_slot, 512);
+        ptx::tmem_relinquish();
+    }
+    ptx::tc_fence_before();
+    __syncthreads();
+    ptx::tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+
+    if (warp >= kProducerWarp) {
+        regs_producer();
+        if (warp == kProducerWarp && lane == 0) {
+            // load sequence idx = 0 .. 2H-1 into buffers idx & 1: dO_idx for idx < H, Q_{idx-H} after
+            auto issue_ld = [&](int idx) {
+                const int b = idx & 1;
+                uint8_t *dst = sm + (b ? L.rb1 : L.rb0);
+                const CUtensorMap *map = idx < H ? &map_do : &map_q;
+                const int h = idx < H ? idx : idx - H;
+                ptx::mbar_arrive_expect_tx(&bars[kTBarLd + b], L.tile_s);
+                for (int kb = 0; kb < D / 64; ++kb)
+                    ptx::tma_load_2d(dst + kb * span * 128, map, h * D + kb * 64, (int)j0, &bars[kTBarLd + b]);
+            };
+            // ds^T_h: this block's tile, columns BK + 64 c (its rows -> tile rows 0 .. BK-1), and
+            // the next block's, columns 64 c (-> tile rows BK .. 2 BK - 1); even heads into ra1,
+            // odd heads into ra0.  Rows past N and columns past span arrive as zeros.
+            auto issue_ds = [&](int h) {
+                uint8_t *dst = sm + ((h & 1) ? L.ra0 : L.ra1);
+                uint64_t *bar = &bars[kTBarDs + (h & 1)];
+                ptx::mbar_arrive_expect_tx(bar, 4u * (uint32_t)BK * 128);
+                for (int c = 0; c < 2; ++c) {
+                    ptx::tma_load_3d(dst + c * span * 128, &map_ds, BK + 64 * c, (int)j0, h, bar);
+                    ptx::tma_load_3d(dst + c * span * 128 + BK * 128, &map_ds, 64 * c, (int)(j0 + BK), h, bar);
+                }
+            };
+            const uint32_t id_acc = ptx::idesc_bf16_f32(128, D, 1, 1);   // A and B MN-major
+            // accumulator product idx (dV_idx for idx < H, dK_{idx-H} after) into TMEM buffer idx & 1:
+            // A = the [span x 128] tile at abase, B = load buffer idx & 1 (g-scaled dO or Q)
+            auto mma_acc = [&](int idx, uint32_t abase, bool ok) {
+                const int b = idx & 1;
+                const uint32_t n = (uint32_t)(idx >> 1);
+                if (idx >= 2) ok = wait_bar(&bars[kTBarAccFree + b], (n - 1) & 1, abort_flag) && ok;
+                ptx::tc_fence_after();
+                if (ok) {
+                    const uint32_t ba = ptx::smem_u32(sm + (b ? L.rb1 : L.rb0));
+                    for (int k = 0; k < span / 16; ++k) {
+                        const uint64_t ad = ptx::smem_desc_sw128(abase + k * 2048, span * 128, 1024);
+                        const uint64_t bd2 = ptx::smem_desc_sw128(ba + k * 2048, span * 128, 1024);
+                        ptx::mma_bf16(tmem + 256 + 128 * b, ad, bd2, id_acc, k > 0);
+                    }
+                }
+                ptx::mma_commit(&bars[kTBarAccFull + b]);
+            };
+            // pmap rows j0 .. j0 + span - 1 (one contiguous run) into ra1; dO_0, dO_1 (or Q_0)
+            stage_in(sm + L.ra1, a.pmap + j0 * W, (uint32_t)(min((int64_t)span, s.N - j0) * W * 2),
+                     &bars[kTBarPmap]);
+            issue_ld(0);
+            issue_ld(1);   // dO_1, or Q_0 when H == 1 (there are 2H >= 2 loads)
+            // ---- phase 1: dV_h = P^T (g_h dO_h)
+            const bool pt_ok = wait_bar(&bars[kTBarPt], 0, abort_flag);   // P tile built, staging consumed
+            if (pt_ok) issue_ds(0);
+            const uint32_t pa = ptx::smem_u32(sm + L.ra0);
+            for (int h = 0; h < H; ++h) {
+                const int idx = h, b = idx & 1;
+                const uint32_t n = (uint32_t)(idx >> 1);
+                const bool ok = wait_bar(&bars[kTBarScaled + b], n & 1, abort_flag) && pt_ok;
+                mma_acc(idx, pa, ok);
+                if (wait_bar(&bars[kTBarAccFull + b], n & 1, abort_flag)) {
+                    if (idx + 2 < 2 * H) issue_ld(idx + 2);
+                    if (h == H - 1 && H >= 2) issue_ds(1);   // every dV MMA has read the P tile
+                }
+            }
+            // ---- phase 2: dK_h = ds^T_h Q_h
+            for (int h = 0; h < H; ++h) {
+                const int idx = H + h, b = idx & 1;
+                const uint32_t n = (uint32_t)(idx >> 1);
+                bool ok = wait_bar(&bars[kTBarDs + (h & 1)], (uint32_t)(h >> 1) & 1, abort_flag);
+                ok = wait_bar(&bars[kTBarLd + b], n & 1, abort_flag) && ok;   // Q_h
+                mma_acc(idx, ptx::smem_u32(sm + ((h & 1) ? L.ra0 : L.ra1)), ok);
+                if (wait_bar(&bars[kTBarAccFull + b], n & 1, abort_flag)) {   // operands read
+                    if (h + 2 < H) issue_ds(h + 2);
+                    if (idx + 2 < 2 * H) issue_ld(idx + 2);
+                }
+            }
+        }
+        __syncwarp();
+    } else {
+        regs_compute();
+        // ---------------------------------------------------------------- compute warps
+        const int tid = threadIdx.x;   // 0 .. 383
+        const int q = warp & 3, split = warp >> 2;
+        const int i = 32 * q + lane;                 // key row of the accumulators
+        const int64_t j = j0 + i;
+        const bool validk = (i < BK) && (j < s.N);
+        const uint32_t lane_base = (uint32_t)(32 * q) << 16;
+
+        // ---- P tile: element (r, c) = P(j0 + r, j0 + c) = pmap[j0 + r][c - r + W - 1] for key
+        // columns c < BK inside row r's window, else 0.  MN-major, 128-byte swizzle: column c
+        // is in box c / 64, 16-byte chunk (c % 64) / 8 of row r, swizzled with r & 7.  Each
+        // unit is one chunk: 8 consecutive keys of one query row, one 16-byte store.  The
+        // lanes of a warp take consecutive rows of one chunk column: their staged reads are
+        // W - 1 elements apart (spread over the banks) and their stores fill whole 128-byte
+        // rows.
+        wait_bar(&bars[kTBarPmap], 0, abort_flag);
+        {
+            const uint16_t *stage = (const uint16_t *)(sm + L.ra1);
+            const int rows_q = (int)min((int64_t)span, s.N - j0);   // staged query rows
+            uint8_t *ptile = sm + L.ra0;
+            for (int u = tid; u < span * 16; u += kComputeThreads) {
+                const int k = u / span, r = u - k * span;
+                uint32_t w[4];
+#pragma unroll
+                for (int e = 0; e < 8; e += 2) {
+                    const int c0 = k * 8 + e;
+                    const uint32_t x0 = (uint32_t)(c0 - r + W - 1), x1 = x0 + 1;   // pmap columns
+                    const bool row_ok = r < rows_q;
+                    const uint32_t v0 = (row_ok && c0 < BK && x0 < (uint32_t)W) ? stage[r * W + (int)x0] : 0u;
+                    const uint32_t v1 = (row_ok && c0 + 1 < BK && x1 < (uint32_t)W) ? stage[r * W + (int)x1] : 0u;
+                    w[e >> 1] = v0 | (v1 << 16);
+                }
+                *(uint4 *)(ptile + (k >> 3) * (span * 128) + r * 128 + (((k & 7) ^ (r & 7)) << 4)) =
+                    make_uint4(w[0], w[1], w[2], w[3]);
+            }
+        }
+        ptx::fence_proxy_async_smem();
+        ptx::mbar_arrive(&bars[kTBarPt]);
+
+        // Scale the rows of dO_h (buffer h & 1) by g[t, h] in place.  Eight threads
+        // share one 128-byte row (one 16-byte chunk each), so every quarter warp
+        // touches one row: no bank conflicts.  The g values of a thread's rows are
+        // fetched together, before the wait for the tile.
+        constexpr int kRowsPerPass = kComputeThreads / 8;
+        constexpr int kPasses = (256 + kRowsPerPass - 1) / kRowsPerPass;
+        auto scale_do = [&](int h) {
+            const int b = h & 1;
+            float gv[kPasses];
+#pragma unroll
+            for (int it = 0; it < kPasses; ++it) {
+                const int r = (tid >> 3) + it * kRowsPerPass;
+                gv[it] = (r < span && j0 + r < s.N) ? __ldg(a.g + (j0 + r) * H + h) : 0.f;
+            }
+            wait_bar(&bars[kTBarLd + b], (uint32_t)(h >> 1) & 1, abort_flag);
+            uint8_t *tile = sm + (b ? L.rb1 : L.rb0);
+#pragma unroll
+            for (int kb = 0; kb < D / 64; ++kb) {
+#pragma unroll
+                for (int it = 0; it < kPasses; ++it) {
+                    const int r = (tid >> 3) + it * kRowsPerPass;
+                    if (r < span) {
+                        uint4 *p = (uint4 *)(tile + kb * span * 128 + r * 128) + (tid & 7);
+                        uint4 v = *p;
+                        uint32_t *u = &v.x;
+#pragma unroll
+                        for (int e = 0; e < 4; ++e) {
+                            const float f0 = __uint_as_float(u[e] << 16) * gv[it];
+                            const float f1 = __uint_as_float(u[e] & 0xFFFF0000u) * gv[it];
+                            u[e] = pack_bf16x2(f0, f1);
+                        }
+                        *p = v;
+                    }
+                }
+            }
+            ptx::fence_proxy_async_smem();
+            ptx::mbar_arrive(&bars[kTBarScaled + b]);
+        };
+        auto drain = [&](int idx, __nv_bfloat16 *out, int h, float mult) {
+            const int b = idx & 1;
+            wait_bar(&bars[kTBarAccFull + b], (uint32_t)(idx >> 1) & 1, abort_flag);
+            ptx::tc_fence_after();
+            drain_row<D>(tmem + lane_base + 256 + 128 * b, out + (j * H + h) * D, mult, validk, split,
+                         ((uintptr_t)out & 31) == 0);
+            ptx::tc_fence_before();
+            ptx::mbar_arrive(&bars[kTBarAccFree + b]);
+        };
+
+        // ---- phase 1: dV (scaling dO_h runs ahead of draining dV_{h-1}; one copy of each)
+        for (int h = 0; h <= H; ++h) {
+            if (h < H) scale_do(h);
+            if (h >= 1) drain(h - 1, a.dv, h - 1, 1.f);
+        }
+        // ---- phase 2: dK, each head drained while the next head's product runs
+        for (int h = 0; h < H; ++h) drain(H + h, a.dk, h, s.scale);
     }
 
     ptx::tc_fence_before();

@@ -36,7 +36,7 @@ __device__ __forceinline__ void regs_producer() {
 __device__ __forceinline__ void regs_compute() {
     asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kRegsCompute));
 }
-constexpr uint32_t kWaitNs = 2000000000u;   // a legitimate wait lasts microseconds
+constexpr uint32_t kWaitNs = 2000000000u;   // default limit; a legitimate wait lasts microseconds
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kLn2 = 0.6931471805599453f;
 
@@ -44,6 +44,14 @@ __device__ __forceinline__ float ex2(float x) {
     float y;
     asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
     return y;
+}
+
+// Per-CTA control words in shared memory: ctl[0] is the abort flag, ctl[1] the
+// wait limit in nanoseconds (copied from Shape::wait_ns by the thread that
+// initialises the mbarriers).
+__device__ __forceinline__ void init_ctl(volatile int *ctl, uint32_t wait_ns) {
+    ctl[0] = 0;
+    ctl[1] = (int)wait_ns;
 }
 
 // Bounded wait on an mbarrier phase.  After the first timeout anywhere in the
@@ -60,7 +68,7 @@ __device__ __forceinline__ bool wait_bar(uint64_t *bar, uint32_t parity, volatil
         if (ptx::mbar_try_wait(bar, parity)) return true;
         if ((n & 63) == 0) {
             if (n == 64) t0 = ptx::globaltimer_lo();
-            if (*abort_flag || ptx::globaltimer_lo() - t0 > kWaitNs) break;
+            if (*abort_flag || ptx::globaltimer_lo() - t0 > (uint32_t)abort_flag[1]) break;
         }
     }
     *abort_flag = 1;   // after a timeout anywhere in the CTA every later wait returns at once
@@ -101,9 +109,11 @@ __device__ __forceinline__ uint32_t sw128_offset(int row, int col) {
 }
 
 // Column band of TMEM lane quarter q in a [128 x span] score tile whose column
-// c holds key kbase + c (kbase = block start - (W - 1)): rows 32q .. 32q+31
-// (those below `rows`) need columns [32q, 32q + rows_q - 1 + W - 1].  Split in
-// 8-column chunks between the kSplits warps of the quarter.
+// c holds key kbase + c, with kbase = block start - (W - 1) - off: row i's window
+// is columns [i + off, i + off + W - 1], so rows 32q .. 32q+31 (those below `rows`)
+// need columns [32q + off, 32q + off + rows_q - 1 + W - 1].  The band starts at
+// the 8-column boundary at or before that and is split in 8-column chunks between
+// the kSplits warps of the quarter.
 struct Band {
     int cb;      // first column of the quarter's band
     int nch;     // chunks of 8 columns in the band
@@ -111,14 +121,14 @@ struct Band {
     int mync;    // chunks in this thread's part
 };
 
-__device__ __forceinline__ Band make_band(int q, int split, int rows, int W, int span) {
+__device__ __forceinline__ Band make_band(int q, int split, int rows, int W, int span, int off = 0) {
     Band b;
-    b.cb = 32 * q;
+    b.cb = (32 * q + off) & ~7;
     const int rows_q = min(32, rows - 32 * q);
     if (rows_q <= 0) {
         b.nch = 0;
     } else {
-        int ce = b.cb + rows_q - 1 + W;          // one past the last column used
+        int ce = 32 * q + off + rows_q - 1 + W;  // one past the last column used
         ce = (ce + 7) & ~7;
         if (ce > span) ce = span;
         b.nch = (ce - b.cb) >> 3;

@@ -101,7 +101,7 @@ fwd_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__ CU
                 cnt = kComputeThreads;
             ptx::mbar_init(&bars[i], cnt);
         }
-        *abort_flag = 0;
+        init_ctl(abort_flag, s.wait_ns);
         ptx::fence_mbar_init();
     }
     if (warp == 0) {
@@ -142,7 +142,10 @@ fwd_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__ CU
             const uint32_t id_pv = ptx::idesc_bf16_f32(128, D, 0, 1);
 
             // ---- phase 1: S_h = Q_h K_h^T into the single S buffer (TMEM columns 0..)
-            for (int h = 0; h < H && h < 2; ++h) issue_qk(h);
+            // (test hook: with s.inject the first CTA never issues head 0's loads, so the
+            // wait for them runs out and the CTA takes the abort path; nothing is in flight)
+            for (int h = 0; h < H && h < 2; ++h)
+                if (!(h == 0 && s.inject && blockIdx.x == 0)) issue_qk(h);
             for (int h = 0; h < H; ++h) {
                 const int b = h & 1;
                 bool ok = wait_bar(&bars[kBarQK + b], (uint32_t)(h >> 1) & 1, abort_flag);
@@ -217,6 +220,17 @@ fwd_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__ CU
 
         const uint32_t s_cols = tmem + lane_base;          // S_h, columns [0, span)
 
+        // c (phase 1) and g (epilogue) of this row are read once per head.  A first read
+        // that misses L2 costs microseconds while every CTA streams its tiles, so the rows
+        // are brought into L2 now and each head's value is loaded one head ahead.
+        if (valid && split == 0) {
+            ptx::prefetch_l2(a.c + t * H);
+            ptx::prefetch_l2(a.c + t * H + H - 1);
+            ptx::prefetch_l2(a.g + t * H);
+            ptx::prefetch_l2(a.g + t * H + H - 1);
+        }
+        float c_next = valid ? __ldg(a.c + t * H) : 0.f;
+
         // composed map of this thread's band, accumulated over heads in registers
         float P[MAXC][8];
 #pragma unroll
@@ -229,6 +243,8 @@ fwd_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__ CU
         const uint32_t span_n = (chi >= clo) ? (uint32_t)(chi - clo) : 0u;
 
         for (int h = 0; h < H; ++h) {
+            const float ch = c_next;
+            if (h + 1 < H) c_next = valid ? __ldg(a.c + t * H + h + 1) : 0.f;
             wait_bar(&bars[kBarSFull], (uint32_t)h & 1, abort_flag);
             ptx::tc_fence_after();
             // pull this thread's band of S_h into registers with one wait
@@ -267,7 +283,7 @@ fwd_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__ CU
             if constexpr (SEG) {
                 if (a.seg.mode == kFwdSegFarApply) {   // p_h = 2^(s log2e - lse log2e), whole window's LSE
                     const float lref = valid ? __ldg(a.lse + t * H + h) * kLog2e : 0.f;
-                    const float coef = valid ? __ldg(a.c + t * H + h) : 0.f;
+                    const float coef = ch;
 #pragma unroll
                     for (int cc = 0; cc < MAXC; ++cc)
                         if (cc < bd.mync)
@@ -321,7 +337,7 @@ fwd_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__ CU
                 // near segment: the whole window's normalizer, log2(2^l2 + 2^lfar2)
                 const float hi = fmaxf(l2, lfar2), lo = fminf(l2, lfar2);
                 const float lw2 = (lo == -INFINITY) ? hi : hi + __log2f(1.f + ex2(lo - hi));
-                const float coef = (valid && any) ? __ldg(a.c + t * H + h) * ex2(mref - lw2) : 0.f;
+                const float coef = (valid && any) ? ch * ex2(mref - lw2) : 0.f;
 #pragma unroll
                 for (int cc = 0; cc < MAXC; ++cc)
                     if (cc < bd.mync)
@@ -330,7 +346,7 @@ fwd_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__ CU
                 if (split == 0 && valid) a.lse[t * H + h] = lw2 * kLn2;
                 continue;
             }
-            const float coef = (valid && any) ? __ldg(a.c + t * H + h) * ex2(mref - m) / Z : 0.f;
+            const float coef = (valid && any) ? ch * ex2(mref - m) / Z : 0.f;
 #pragma unroll
             for (int cc = 0; cc < MAXC; ++cc)
                 if (cc < bd.mync)
@@ -340,6 +356,7 @@ fwd_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__ CU
         }
 
         if (!stats_only) {   // phase 2 (the segmented LSE launch stops here)
+            float g_next = valid ? __ldg(a.g + t * H) : 0.f;   // head 0's scale, loaded ahead
             // the far segment adds to o: bring the rows it reads into L2 two heads ahead
             const bool o_add = SEG && a.seg.mode == kFwdSegFarApply && valid;
             if (o_add)
@@ -424,9 +441,10 @@ fwd_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__ CU
                 const int b = h & 1;
                 const uint32_t n = (uint32_t)(h >> 1);
                 if (o_add && h + 2 < H) prefetch_drain_row<D>(a.o + (t * H + h + 2) * D, split);
+                const float gh = g_next;
+                if (h + 1 < H) g_next = valid ? __ldg(a.g + t * H + h + 1) : 0.f;
                 wait_bar(&bars[kBarUFull + b], n & 1, abort_flag);
                 ptx::tc_fence_after();
-                const float gh = valid ? __ldg(a.g + t * H + h) : 0.f;
                 uint32_t ur[kMaxC16][16];
 #pragma unroll
                 for (int c = 0; c < kMaxC16; ++c)

@@ -69,6 +69,22 @@ inline cudaError_t make_map(CUtensorMap *m, const void *ptr, int64_t N, int H, i
     return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
 }
 
+// 3-D view [H][N][cols] of the ds tiles in the workspace (bf16, row stride cols): boxes of 64
+// columns x box_rows rows x 1 head, 128-byte swizzle.  Loads outside the tensor read zeros;
+// stores outside it are dropped.
+inline cudaError_t make_map_ds(CUtensorMap *m, const void *ptr, int64_t N, int H, int cols, int box_rows) {
+    EncodeTiledFn enc = encode_fn();
+    if (!enc) return cudaErrorNotSupported;
+    cuuint64_t dims[3] = {(cuuint64_t)cols, (cuuint64_t)N, (cuuint64_t)H};
+    cuuint64_t strides[2] = {(cuuint64_t)cols * 2, (cuuint64_t)N * cols * 2};
+    cuuint32_t box[3] = {64, (cuuint32_t)box_rows, 1};
+    cuuint32_t es[3] = {1, 1, 1};
+    CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(ptr), dims, strides, box, es,
+                     CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                     CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
+}
+
 inline int sm_count() {
     int dev = 0, n = 148;
     if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
@@ -191,15 +207,16 @@ inline cudaError_t fwd(const Shape &s, const void *q, const void *k, const void 
     return e;
 }
 
-template <int D, int MAXC, bool SEG = false, bool DSB = false>
+template <int D, int MAXC, bool SEG = false, bool DSB = false, bool DST = false>
 inline cudaError_t launch_bwd_query(const CUtensorMap &mq, const CUtensorMap &mk, const CUtensorMap &mv,
-                                    const CUtensorMap &mdo, const BwdArgs &a, cudaStream_t st) {
-    auto kern = bwd_query_kernel<D, MAXC, SEG, DSB>;
+                                    const CUtensorMap &mdo, const CUtensorMap &mds, const BwdArgs &a,
+                                    cudaStream_t st) {
+    auto kern = bwd_query_kernel<D, MAXC, SEG, DSB, DST>;
     const uint32_t smem = QSideLayout<D>(a.span).bytes + 1024;
     cudaError_t e = set_smem(kern, smem);
     if (e != cudaSuccess) return e;
     const unsigned grid = (unsigned)((a.s.N + a.BM - 1) / a.BM);
-    kern<<<grid, kThreads, smem, st>>>(mq, mk, mv, mdo, a);
+    kern<<<grid, kThreads, smem, st>>>(mq, mk, mv, mdo, mds, a);
     return cudaGetLastError();
 }
 
@@ -229,6 +246,18 @@ inline cudaError_t launch_bwd_key_dsb(const CUtensorMap &mq, const CUtensorMap &
     return cudaGetLastError();
 }
 
+template <int D>
+inline cudaError_t launch_bwd_key_dst(const CUtensorMap &mq, const CUtensorMap &mdo, const CUtensorMap &mds,
+                                      const BwdArgs &a, cudaStream_t st) {
+    auto kern = bwd_key_dst_kernel<D>;
+    const uint32_t smem = TSideLayout<D>(a.span).bytes + 1024;
+    cudaError_t e = set_smem(kern, smem);
+    if (e != cudaSuccess) return e;
+    const unsigned grid = (unsigned)((a.s.N + a.BM - 1) / a.BM);
+    kern<<<grid, kThreads, smem, st>>>(mq, mdo, mds, a);
+    return cudaGetLastError();
+}
+
 #define DC_TC_MAXC_SWITCH(maxc, CALL)        \
     switch (maxc) {                          \
         case 3: { constexpr int MC = 3; return CALL; }   \
@@ -248,11 +277,48 @@ inline BwdArgs bwd_args(const Shape &s) {
 // Bytes of the key-major ds band [H][N][kDsbRow] bf16 the query side hands to the key side.
 inline size_t dsb_bytes(const Shape &s) { return (size_t)s.H * (size_t)s.N * (size_t)kDsbRow * 2; }
 
+// The ds tile hand-off: query blocks (and key blocks) of kDstBlock tokens, key tiles of
+// 2 kDstBlock columns starting kDstBlock keys before the block, tiles [H][N][2 kDstBlock]
+// bf16 in the workspace.  It covers windows with W - 1 <= kDstBlock; below kDstMinWindow
+// the wider key tile (2 kDstBlock instead of BM + W - 1 columns) costs more than the ds
+// band's stores and de-skew (measured: W = 32 and 64 run slower, W = 112 faster).
+constexpr int kDstBlock = 112;
+constexpr int kDstMinWindow = 97;
+inline bool dst_shape(const Shape &s) {
+    return !segmented(s) && s.W - 1 <= kDstBlock && s.W >= kDstMinWindow;
+}
+inline size_t dst_bytes(const Shape &s) { return (size_t)s.H * (size_t)s.N * (size_t)(2 * kDstBlock) * 2; }
+inline bool use_dst(const Shape &s, size_t workspace_bytes) {
+    if (!dst_shape(s) || workspace_bytes < dst_bytes(s)) return false;
+    const uint32_t need = (s.d == 128 ? TSideLayout<128>(2 * kDstBlock).bytes : TSideLayout<64>(2 * kDstBlock).bytes)
+                          + 1024;
+    return need <= 227u * 1024 && s.W * 2 * kDstBlock * 2 <= (int)TSideLayout<64>(2 * kDstBlock).tile_a;
+}
+// Register-array width for the DST band: row i's window is columns [i + off, i + off + W - 1]
+// with off = kDstBlock - (W - 1), so a lane quarter's band runs from the 8-column boundary at
+// or below 32q + off to 32q + off + 31 + W (make_band with that offset).
+inline int dst_maxc(int W) {
+    const int off = kDstBlock - (W - 1);
+    const int nch = (((off + 31 + W) + 7) / 8 * 8 - (off & ~7)) / 8;
+    const int need = (nch + kSplits - 1) / kSplits;
+    if (need <= 3) return 3;
+    if (need <= 4) return 4;
+    if (need <= 6) return 6;
+    return 7;
+}
+inline BwdArgs dst_args(const Shape &s) {
+    BwdArgs a = {};
+    a.s = s;
+    a.BM = kDstBlock;
+    a.span = 2 * kDstBlock;
+    return a;
+}
+
 // The backward pair that passes ds through the band (instead of the key side recomputing
 // it from S^T and the dP band) runs when the window is one piece, the workspace holds the
 // band and the key side's shared-memory layout fits (pmap staging rows before the ds rows).
 inline bool use_dsb(const Shape &s, size_t workspace_bytes) {
-    if (segmented(s) || workspace_bytes < dsb_bytes(s)) return false;
+    if (segmented(s) || workspace_bytes < dsb_bytes(s) || use_dst(s, workspace_bytes)) return false;
     const BwdArgs a = bwd_args(s);
     const bool fits128 = [&] {
         const DSideLayout<128> L(a.span, s.W, a.BM, kDsbRow);
@@ -296,8 +362,8 @@ inline cudaError_t bwd_query_segmented(const Shape &s, const void *q, const void
         a.dg = dg;
         a.band = band;
         const CUtensorMap &kk = mk[step[0]], &vv = mv[step[0]];
-        e = (s.d == 64) ? launch_bwd_query<64, 7, true>(mq, kk, vv, mdo, a, st)
-                        : launch_bwd_query<128, 7, true>(mq, kk, vv, mdo, a, st);
+        e = (s.d == 64) ? launch_bwd_query<64, 7, true>(mq, kk, vv, mdo, mq, a, st)
+                        : launch_bwd_query<128, 7, true>(mq, kk, vv, mdo, mq, a, st);
         if (e != cudaSuccess) return e;
         ++*launches;
     }
@@ -309,8 +375,9 @@ inline cudaError_t bwd_query(const Shape &s, const void *q, const void *k, const
                              float *dg, void *workspace, size_t workspace_bytes, cudaStream_t st, int32_t *launches) {
     float *band = (float *)workspace;
     if (segmented(s)) return bwd_query_segmented(s, q, k, v, c, g, dO, lse, pmap, dq, dc_, dg, band, st, launches);
+    const bool dst = use_dst(s, workspace_bytes);
     const bool dsb = use_dsb(s, workspace_bytes);
-    BwdArgs a = bwd_args(s);
+    BwdArgs a = dst ? dst_args(s) : bwd_args(s);
     if (dsb) a.dsb = (__nv_bfloat16 *)workspace;
     a.c = c;
     a.g = g;
@@ -320,23 +387,30 @@ inline cudaError_t bwd_query(const Shape &s, const void *q, const void *k, const
     a.dc = dc_;
     a.dg = dg;
     a.band = band;
-    CUtensorMap mq, mk, mv, mdo;
+    CUtensorMap mq, mk, mv, mdo, mds;
     cudaError_t e = make_map(&mq, q, s.N, s.H, s.d, 128);
     if (e == cudaSuccess) e = make_map(&mk, k, s.N, s.H, s.d, a.span);
     if (e == cudaSuccess) e = make_map(&mv, v, s.N, s.H, s.d, a.span);
     if (e == cudaSuccess) e = make_map(&mdo, dO, s.N, s.H, s.d, 128);
+    if (e == cudaSuccess) e = dst ? make_map_ds(&mds, workspace, s.N, s.H, a.span, a.BM) : make_map(&mds, q, s.N, s.H, s.d, 128);
     if (e != cudaSuccess) return e;
     e = [&]() -> cudaError_t {
+        if (dst) {
+            if (s.d == 64) {
+                DC_TC_MAXC_SWITCH(dst_maxc(s.W), (launch_bwd_query<64, MC, false, false, true>(mq, mk, mv, mdo, mds, a, st)));
+            }
+            DC_TC_MAXC_SWITCH(dst_maxc(s.W), (launch_bwd_query<128, MC, false, false, true>(mq, mk, mv, mdo, mds, a, st)));
+        }
         if (dsb) {
             if (s.d == 64) {
-                DC_TC_MAXC_SWITCH(maxc_for(s.W), (launch_bwd_query<64, MC, false, true>(mq, mk, mv, mdo, a, st)));
+                DC_TC_MAXC_SWITCH(maxc_for(s.W), (launch_bwd_query<64, MC, false, true>(mq, mk, mv, mdo, mds, a, st)));
             }
-            DC_TC_MAXC_SWITCH(maxc_for(s.W), (launch_bwd_query<128, MC, false, true>(mq, mk, mv, mdo, a, st)));
+            DC_TC_MAXC_SWITCH(maxc_for(s.W), (launch_bwd_query<128, MC, false, true>(mq, mk, mv, mdo, mds, a, st)));
         }
         if (s.d == 64) {
-            DC_TC_MAXC_SWITCH(maxc_for(s.W), (launch_bwd_query<64, MC>(mq, mk, mv, mdo, a, st)));
+            DC_TC_MAXC_SWITCH(maxc_for(s.W), (launch_bwd_query<64, MC>(mq, mk, mv, mdo, mds, a, st)));
         }
-        DC_TC_MAXC_SWITCH(maxc_for(s.W), (launch_bwd_query<128, MC>(mq, mk, mv, mdo, a, st)));
+        DC_TC_MAXC_SWITCH(maxc_for(s.W), (launch_bwd_query<128, MC>(mq, mk, mv, mdo, mds, a, st)));
     }();
     if (e == cudaSuccess) ++*launches;
     return e;
@@ -383,6 +457,21 @@ inline cudaError_t bwd_key(const Shape &s, const void *q, const void *k, const f
                            size_t workspace_bytes, void *dk, void *dv, cudaStream_t st, int32_t *launches) {
     const float *band = (const float *)workspace;
     if (segmented(s)) return bwd_key_segmented(s, q, k, c, g, dO, lse, pmap, dc_, band, dk, dv, st, launches);
+    if (use_dst(s, workspace_bytes)) {   // ds from the query side's tiles, by TMA
+        BwdArgs a = dst_args(s);
+        a.pmap = (const __nv_bfloat16 *)pmap;
+        a.g = g;
+        a.dk = (__nv_bfloat16 *)dk;
+        a.dv = (__nv_bfloat16 *)dv;
+        CUtensorMap mq, mdo, mds;
+        cudaError_t e = make_map(&mq, q, s.N, s.H, s.d, a.span);
+        if (e == cudaSuccess) e = make_map(&mdo, dO, s.N, s.H, s.d, a.span);
+        if (e == cudaSuccess) e = make_map_ds(&mds, workspace, s.N, s.H, a.span, a.BM);
+        if (e != cudaSuccess) return e;
+        e = (s.d == 64) ? launch_bwd_key_dst<64>(mq, mdo, mds, a, st) : launch_bwd_key_dst<128>(mq, mdo, mds, a, st);
+        if (e == cudaSuccess) ++*launches;
+        return e;
+    }
     BwdArgs a = bwd_args(s);
     if (use_dsb(s, workspace_bytes)) {   // ds from the query side's band
         a.pmap = (const __nv_bfloat16 *)pmap;

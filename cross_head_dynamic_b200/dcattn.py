@@ -24,7 +24,8 @@ DC_DEVERR_TIMEOUT = 0x2
 
 EXPORTED = ("dc_attn_fwd", "dc_attn_bwd_workspace_size", "dc_attn_bwd_query", "dc_attn_bwd_key",
             "dc_attn_bwd", "dc_attn_resolve_impl", "dc_attn_device_status", "dc_attn_status_string",
-            "dc_attn_last_launch_count", "dc_attn_bwd_noalloc", "dc_attn_halo_add")
+            "dc_attn_last_launch_count", "dc_attn_bwd_noalloc", "dc_attn_halo_add", "dc_attn_set_wait_limit",
+            "dc_attn_inject_missing_load")
 
 
 class DCAttnError(RuntimeError):
@@ -76,6 +77,10 @@ def load_library(path: str = LIB_PATH):
     lib.dc_attn_last_launch_count.restype = ctypes.c_int32
     lib.dc_attn_halo_add.argtypes = [vp, vp, ctypes.c_int64, ctypes.c_int32, vp]
     lib.dc_attn_halo_add.restype = st
+    lib.dc_attn_set_wait_limit.argtypes = [ctypes.c_uint32]
+    lib.dc_attn_set_wait_limit.restype = st
+    lib.dc_attn_inject_missing_load.argtypes = []
+    lib.dc_attn_inject_missing_load.restype = st
     _lib = lib
     return lib
 
@@ -269,3 +274,13 @@ def dc_attn_halo_add(dst, src, stream=None):
                                            dt, _stream_handle(stream))
     _check("dc_attn_halo_add", code)
     return dst
+
+
+def dc_attn_set_wait_limit(ns: int = 0):
+    """Limit (nanoseconds) of the tcgen05 kernels' bounded waits for later calls; 0 = default 2 s."""
+    _check("dc_attn_set_wait_limit", load_library().dc_attn_set_wait_limit(int(ns)))
+
+
+def dc_attn_inject_missing_load():
+    """Test hook: the next one-piece tcgen05 forward leaves out its first CTA's head-0 loads."""
+    _check("dc_attn_inject_missing_load", load_library().dc_attn_inject_missing_load())

@@ -150,8 +150,12 @@ dc_status_t dc_attn_bwd(const dc_attn_params *params,
  * so the ds band is used when it fits).
  * - Returns DC_ERR_UNSUPPORTED, before any launch, when the dP band needs more
  *   than that: N * W * 4 bytes > 32 MiB (e.g. N = 65536 tokens at W = 128).
- * - The first call on each device looks up the array's device address with
- *   that device current; make that first call before any stream capture.
+ * - The array's device address is looked up (with the calling thread's
+ *   current device) on every call made outside stream capture, so a
+ *   cudaDeviceReset between two calls does no harm.  A call made while its
+ *   stream is being captured reuses the address that the last uncaptured call
+ *   on that device found: make one uncaptured call on each device before any
+ *   capture, and do not replay a captured graph after a cudaDeviceReset.
  * - Every call on a device shares the one array.  Calls whose kernels overlap
  *   on the GPU (different streams, or different host threads, without
  *   ordering between them) race on it and give undefined results; serialise
@@ -188,6 +192,31 @@ const char *dc_attn_status_string(dc_status_t status);
 /* Number of kernel launches the last successful call on this host thread made
  * (used to report launches per step). */
 int32_t dc_attn_last_launch_count(void);
+
+/* Failure-detection hooks (no counterpart on the page; they exist so that the
+ * bounded waits can be tested without a GPU fault).
+ *
+ * Every wait of a tcgen05 kernel on one of its own pipeline stages (a tile
+ * load, a tensor-core product, a hand-over between its warps) gives up after
+ * a time limit: the CTA then raises DC_DEVERR_TIMEOUT in the device status
+ * word, skips the rest of its work without issuing further loads or products,
+ * and exits normally, so the context stays usable and the host learns of it
+ * through dc_attn_device_status().
+ *
+ * dc_attn_set_wait_limit: limit in nanoseconds for kernels launched by later
+ * calls from any host thread; 0 restores the default of 2 s.  Values below
+ * 100000 (0.1 ms) return DC_ERR_INVALID_ARG.  A legitimate wait lasts
+ * microseconds, so a limit of a few milliseconds still never fires in
+ * normal operation.
+ *
+ * dc_attn_inject_missing_load: the next dc_attn_fwd call (from any host
+ * thread) that runs the one-piece tcgen05 forward leaves out the first
+ * CTA's head-0 Q/K tile loads, so that CTA's wait for them runs out.  The
+ * load is never issued, so nothing is in flight when the CTA exits.  That
+ * call completes after about one wait limit, its outputs are undefined, and
+ * the status word gets DC_DEVERR_TIMEOUT.  One-shot. */
+dc_status_t dc_attn_set_wait_limit(uint32_t ns);
+dc_status_t dc_attn_inject_missing_load(void);
 
 #ifdef __cplusplus
 }

@@ -140,3 +140,10 @@ def test_binding_refuses_cpu_tensors():
     with pytest.raises(ValueError):
         dcattn.dc_attn_fwd(q, q, q, torch.zeros(4, 1), torch.zeros(4, 1), torch.tensor([0, 4], dtype=torch.int32),
                            4, 1.0)
+
+
+def test_wait_limit_hook_validates_on_the_host(lib):
+    assert lib.dc_attn_set_wait_limit(50) == dcattn.DC_ERR_INVALID_ARG      # below 0.1 ms
+    assert lib.dc_attn_set_wait_limit(99999) == dcattn.DC_ERR_INVALID_ARG
+    assert lib.dc_attn_set_wait_limit(5_000_000) == dcattn.DC_OK
+    assert lib.dc_attn_set_wait_limit(0) == dcattn.DC_OK                    # back to the default
