@@ -23,6 +23,9 @@ struct Shape {
     int W;
     float scale;
     const int32_t *cu;
+    int64_t sq;         // elements between consecutive tokens of q, k, v (>= H * d)
+    int64_t sdq;        // ... of dq, dk, dv
+    int64_t so;         // ... of o (forward) and dO (backward)
     uint32_t wait_ns;   // limit of every bounded wait in the tcgen05 kernels (nanoseconds)
     int inject;         // test hook: the tcgen05 forward's first CTA leaves out its first Q/K load
 };

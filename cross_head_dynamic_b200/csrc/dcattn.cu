@@ -53,6 +53,16 @@ dc_status_t check_params(const dc_attn_params *p, Checked *out) {
     out->s.W = p->window;
     out->s.scale = p->softmax_scale;
     out->s.cu = p->cu_seqlens;
+    // row strides: 0 = contiguous; else at least one token's H * d elements and 16-byte rows
+    const int64_t row = (int64_t)p->num_heads * p->head_dim;
+    const int64_t esize = p->dtype == DC_F32 ? 4 : 2;
+    const int64_t strides[3] = {p->stride_qkv, p->stride_dqkv, p->stride_o};
+    int64_t *dst[3] = {&out->s.sq, &out->s.sdq, &out->s.so};
+    for (int i = 0; i < 3; ++i) {
+        const int64_t st = strides[i] == 0 ? row : strides[i];
+        if (st < row || (st * esize) % 16 != 0 || st > ((int64_t)1 << 40) / esize) return DC_ERR_INVALID_ARG;
+        *dst[i] = st;
+    }
     out->s.wait_ns = g_wait_ns.load(std::memory_order_relaxed);
     out->s.inject = 0;
     out->dtype = p->dtype;

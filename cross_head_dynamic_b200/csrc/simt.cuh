@@ -69,7 +69,7 @@ __global__ void fwd_kernel(Shape s, const T *__restrict__ q, const T *__restrict
     float *Pw = ls + kMaxHeads;
     float *tile = Pw + W;
 
-    for (int i = lane; i < H * d; i += 32) qs[i] = ldf<T>(q + t * H * d + i);
+    for (int i = lane; i < H * d; i += 32) qs[i] = ldf<T>(q + t * s.sq + i);
     __syncwarp();
     const int64_t lo = window_lo(s, t);
     const int n = (int)(t - lo + 1);
@@ -78,8 +78,7 @@ __global__ void fwd_kernel(Shape s, const T *__restrict__ q, const T *__restrict
         float m = -INFINITY, z = 0.f;
         for (int base = 0; base < n; base += 32) {
             const int cnt = min(32, n - base);
-            const float x = s.scale * dot_rows32<T, DPL>(qs + h * d, k + ((lo + base) * H + h) * d, (int64_t)H * d,
-                                                         cnt, tile);
+            const float x = s.scale * dot_rows32<T, DPL>(qs + h * d, k + (lo + base) * s.sq + h * d, s.sq, cnt, tile);
             if (lane < cnt) {
                 if (x > m) {
                     z = z * expf(m - x) + 1.f;
@@ -103,8 +102,7 @@ __global__ void fwd_kernel(Shape s, const T *__restrict__ q, const T *__restrict
         const int cnt = min(32, n - base);
         float P = 0.f;
         for (int h = 0; h < H; ++h) {
-            const float x = s.scale * dot_rows32<T, DPL>(qs + h * d, k + ((lo + base) * H + h) * d, (int64_t)H * d,
-                                                         cnt, tile);
+            const float x = s.scale * dot_rows32<T, DPL>(qs + h * d, k + (lo + base) * s.sq + h * d, s.sq, cnt, tile);
             P = fmaf(__ldg(c + t * H + h), expf(x - ls[h]), P);
         }
         if (lane < cnt) Pw[base + lane] = P;
@@ -120,13 +118,13 @@ __global__ void fwd_kernel(Shape s, const T *__restrict__ q, const T *__restrict
         for (int i = 0; i < DPL; ++i) acc[i] = 0.f;
         for (int jj = 0; jj < n; ++jj) {
             const float P = Pw[jj];
-            const T *vr = v + ((lo + jj) * H + h) * d;
+            const T *vr = v + (lo + jj) * s.sq + h * d;
 #pragma unroll
             for (int i = 0; i < DPL; ++i) acc[i] = fmaf(P, ldf<T>(vr + lane + 32 * i), acc[i]);
         }
         const float gh = __ldg(g + t * H + h);
 #pragma unroll
-        for (int i = 0; i < DPL; ++i) stf<T>(o + (t * H + h) * d + lane + 32 * i, gh * acc[i]);
+        for (int i = 0; i < DPL; ++i) stf<T>(o + t * s.so + h * d + lane + 32 * i, gh * acc[i]);
     }
 }
 
@@ -156,8 +154,8 @@ __global__ void bwd_query_kernel(Shape s, const T *__restrict__ q, const T *__re
     float *tile = sw + W;
 
     for (int i = lane; i < H * d; i += 32) {
-        qs[i] = ldf<T>(q + t * H * d + i);
-        dos[i] = ldf<T>(dO + t * H * d + i);
+        qs[i] = ldf<T>(q + t * s.sq + i);
+        dos[i] = ldf<T>(dO + t * s.so + i);
     }
     const int64_t lo = window_lo(s, t);
     const int n = (int)(t - lo + 1);
@@ -177,7 +175,7 @@ __global__ void bwd_query_kernel(Shape s, const T *__restrict__ q, const T *__re
 #pragma unroll
         for (int h = 0; h < kMaxHeads; ++h) {
             if (h < H) {
-                const float E = dot_rows32<T, DPL>(dos + h * d, v + ((lo + base) * H + h) * d, (int64_t)H * d, cnt, tile);
+                const float E = dot_rows32<T, DPL>(dos + h * d, v + (lo + base) * s.sq + h * d, s.sq, cnt, tile);
                 dP = fmaf(__ldg(g + t * H + h), E, dP);
                 dgp[h] = fmaf(pj, E, dgp[h]);
             }
@@ -201,8 +199,7 @@ __global__ void bwd_query_kernel(Shape s, const T *__restrict__ q, const T *__re
         float dcp = 0.f;
         for (int base = 0; base < n; base += 32) {
             const int cnt = min(32, n - base);
-            const float x = s.scale * dot_rows32<T, DPL>(qs + h * d, k + ((lo + base) * H + h) * d, (int64_t)H * d,
-                                                         cnt, tile);
+            const float x = s.scale * dot_rows32<T, DPL>(qs + h * d, k + (lo + base) * s.sq + h * d, s.sq, cnt, tile);
             if (lane < cnt) {
                 const float p = expf(x - l);
                 sw[base + lane] = p;
@@ -219,12 +216,12 @@ __global__ void bwd_query_kernel(Shape s, const T *__restrict__ q, const T *__re
         for (int i = 0; i < DPL; ++i) acc[i] = 0.f;
         for (int jj = 0; jj < n; ++jj) {
             const float ds = sw[jj];
-            const T *kr = k + ((lo + jj) * H + h) * d;
+            const T *kr = k + (lo + jj) * s.sq + h * d;
 #pragma unroll
             for (int i = 0; i < DPL; ++i) acc[i] = fmaf(ds, ldf<T>(kr + lane + 32 * i), acc[i]);
         }
 #pragma unroll
-        for (int i = 0; i < DPL; ++i) stf<T>(dq + (t * H + h) * d + lane + 32 * i, s.scale * acc[i]);
+        for (int i = 0; i < DPL; ++i) stf<T>(dq + t * s.sdq + h * d + lane + 32 * i, s.scale * acc[i]);
         __syncwarp();
     }
 }
@@ -247,7 +244,7 @@ __global__ void bwd_key_kernel(Shape s, const T *__restrict__ q, const T *__rest
     if (j >= s.N) return;
     float *ks = smem + (size_t)warp * (H * d + tile_floats(d));
     float *tile = ks + H * d;
-    for (int i = lane; i < H * d; i += 32) ks[i] = ldf<T>(k + j * H * d + i);
+    for (int i = lane; i < H * d; i += 32) ks[i] = ldf<T>(k + j * s.sq + i);
     __syncwarp();
     int64_t hi = j + W - 1;
     const int64_t b = doc_end(s, j);
@@ -261,8 +258,7 @@ __global__ void bwd_key_kernel(Shape s, const T *__restrict__ q, const T *__rest
         for (int base = 0; base < n; base += 32) {
             float ds = 0.f, pg = 0.f;
             const int cnt0 = min(32, n - base);
-            const float x = s.scale * dot_rows32<T, DPL>(ks + h * d, q + ((j + base) * H + h) * d, (int64_t)H * d,
-                                                         cnt0, tile);
+            const float x = s.scale * dot_rows32<T, DPL>(ks + h * d, q + (j + base) * s.sq + h * d, s.sq, cnt0, tile);
             if (base + lane < n) {
                 const int64_t t = j + base + lane;
                 const int64_t w = j - (t - W + 1);
@@ -275,8 +271,8 @@ __global__ void bwd_key_kernel(Shape s, const T *__restrict__ q, const T *__rest
                 const float dsl = __shfl_sync(0xffffffffu, ds, l);
                 const float pgl = __shfl_sync(0xffffffffu, pg, l);
                 const int64_t t = j + base + l;
-                const T *qr = q + (t * H + h) * d;
-                const T *dr = dO + (t * H + h) * d;
+                const T *qr = q + t * s.sq + h * d;
+                const T *dr = dO + t * s.so + h * d;
 #pragma unroll
                 for (int i = 0; i < DPL; ++i) {
                     ak[i] = fmaf(dsl, ldf<T>(qr + lane + 32 * i), ak[i]);
@@ -286,8 +282,8 @@ __global__ void bwd_key_kernel(Shape s, const T *__restrict__ q, const T *__rest
         }
 #pragma unroll
         for (int i = 0; i < DPL; ++i) {
-            stf<T>(dk + (j * H + h) * d + lane + 32 * i, s.scale * ak[i]);
-            stf<T>(dv + (j * H + h) * d + lane + 32 * i, av[i]);
+            stf<T>(dk + j * s.sdq + h * d + lane + 32 * i, s.scale * ak[i]);
+            stf<T>(dv + j * s.sdq + h * d + lane + 32 * i, av[i]);
         }
     }
 }

@@ -364,6 +364,10 @@ bwd_query_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
             ptx::prefetch_l2(a.c + t * H + H - 1);
         }
         float g_next = (valid && do_p1) ? __ldg(a.g + t * H) : 0.f;
+        // head 0's phase-2 values, loaded now: at the start of phase 2 the memory system is
+        // at its busiest and a load issued there can take microseconds
+        float lse_next = valid ? __ldg(a.lse + t * H) : 0.f;
+        float c_next = valid ? __ldg(a.c + t * H) : 0.f;
         // column c is in this row's window iff (unsigned)(c - win_lo) <= win_n (never for a row
         // with an empty window)
         const uint32_t win_lo = (chi >= clo) ? (uint32_t)clo : ~0u;
@@ -531,18 +535,16 @@ bwd_query_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
         // copy reads it while head 0's scores are processed, and it is reused from head 0's
         // ds tile on (columns outside this quarter's band zeroed once).
         uint8_t *dtile = sm + L.rd;
-        float lse_next = valid ? __ldg(a.lse + t * H) : 0.f;   // head 0's values, loaded ahead
-        float c_next = valid ? __ldg(a.c + t * H) : 0.f;
         auto drain_dq = [&](int h) {
             const int b = h & 1;
             wait_bar(&bars[kQBarDqFull + b], (uint32_t)(h >> 1) & 1, abort_flag);
             ptx::tc_fence_after();
             if (SEG && a.seg.mode == kQSegFarPart2)   // adds the far segment's share to dq
-                drain_row<D, true>(tmem + lane_base + 256 + 128 * b, a.dq + (t * H + h) * D, s.scale, valid, split,
-                                   ((uintptr_t)a.dq & 31) == 0);
+                drain_row<D, true>(tmem + lane_base + 256 + 128 * b, a.dq + t * s.sdq + h * D, s.scale, valid, split,
+                                   (((uintptr_t)a.dq | (uintptr_t)(s.sdq * 2)) & 31) == 0);
             else
-                drain_row<D>(tmem + lane_base + 256 + 128 * b, a.dq + (t * H + h) * D, s.scale, valid, split,
-                             ((uintptr_t)a.dq & 31) == 0);
+                drain_row<D>(tmem + lane_base + 256 + 128 * b, a.dq + t * s.sdq + h * D, s.scale, valid, split,
+                             (((uintptr_t)a.dq | (uintptr_t)(s.sdq * 2)) & 31) == 0);
             ptx::tc_fence_before();
             ptx::mbar_arrive(&bars[kQBarDqFree + b]);
         };
@@ -935,11 +937,11 @@ bwd_key_seg_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_const
             wait_bar(&bars[kKBarAccFull + b], (uint32_t)(idx >> 1) & 1, abort_flag);
             ptx::tc_fence_after();
             if (SEG && a.seg.mode == kKSegAdd)   // a later segment adds its share
-                drain_row<D, true>(tmem + lane_base + 256 + 128 * b, out + (j * H + h) * D, mult, validk, split,
-                                   ((uintptr_t)out & 31) == 0);
+                drain_row<D, true>(tmem + lane_base + 256 + 128 * b, out + j * s.sdq + h * D, mult, validk, split,
+                                   (((uintptr_t)out | (uintptr_t)(s.sdq * 2)) & 31) == 0);
             else
-                drain_row<D>(tmem + lane_base + 256 + 128 * b, out + (j * H + h) * D, mult, validk, split,
-                             ((uintptr_t)out & 31) == 0);
+                drain_row<D>(tmem + lane_base + 256 + 128 * b, out + j * s.sdq + h * D, mult, validk, split,
+                             (((uintptr_t)out | (uintptr_t)(s.sdq * 2)) & 31) == 0);
             ptx::tc_fence_before();
             ptx::mbar_arrive(&bars[kKBarAccFree + b]);
         };
@@ -1292,8 +1294,8 @@ bwd_key_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant_
             const int b = idx & 1;
             wait_bar(&bars[kDBarAccFull + b], (uint32_t)(idx >> 1) & 1, abort_flag);
             ptx::tc_fence_after();
-            drain_row<D>(tmem + lane_base + 256 + 128 * b, out + (j * H + h) * D, mult, validk, split,
-                         ((uintptr_t)out & 31) == 0);
+            drain_row<D>(tmem + lane_base + 256 + 128 * b, out + j * s.sdq + h * D, mult, validk, split,
+                         (((uintptr_t)out | (uintptr_t)(s.sdq * 2)) & 31) == 0);
             ptx::tc_fence_before();
             ptx::mbar_arrive(&bars[kDBarAccFree + b]);
         };
@@ -1536,17 +1538,24 @@ bwd_key_dst_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_const
         // Scale the rows of dO_h (buffer h & 1) by g[t, h] in place.  Eight threads
         // share one 128-byte row (one 16-byte chunk each), so every quarter warp
         // touches one row: no bank conflicts.  The g values of a thread's rows are
-        // fetched together, before the wait for the tile.
+        // loaded one head ahead (a load issued just before its use waits on L2).
         constexpr int kRowsPerPass = kComputeThreads / 8;
         constexpr int kPasses = (256 + kRowsPerPass - 1) / kRowsPerPass;
+        float gnext[kPasses];
+        auto load_g = [&](int h) {
+#pragma unroll
+            for (int it = 0; it < kPasses; ++it) {
+                const int r = (tid >> 3) + it * kRowsPerPass;
+                gnext[it] = (h < H && r < span && j0 + r < s.N) ? __ldg(a.g + (j0 + r) * H + h) : 0.f;
+            }
+        };
+        load_g(0);
         auto scale_do = [&](int h) {
             const int b = h & 1;
             float gv[kPasses];
 #pragma unroll
-            for (int it = 0; it < kPasses; ++it) {
-                const int r = (tid >> 3) + it * kRowsPerPass;
-                gv[it] = (r < span && j0 + r < s.N) ? __ldg(a.g + (j0 + r) * H + h) : 0.f;
-            }
+            for (int it = 0; it < kPasses; ++it) gv[it] = gnext[it];
+            load_g(h + 1);
             wait_bar(&bars[kTBarLd + b], (uint32_t)(h >> 1) & 1, abort_flag);
             uint8_t *tile = sm + (b ? L.rb1 : L.rb0);
 #pragma unroll
@@ -1575,8 +1584,8 @@ bwd_key_dst_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_const
             const int b = idx & 1;
             wait_bar(&bars[kTBarAccFull + b], (uint32_t)(idx >> 1) & 1, abort_flag);
             ptx::tc_fence_after();
-            drain_row<D>(tmem + lane_base + 256 + 128 * b, out + (j * H + h) * D, mult, validk, split,
-                         ((uintptr_t)out & 31) == 0);
+            drain_row<D>(tmem + lane_base + 256 + 128 * b, out + j * s.sdq + h * D, mult, validk, split,
+                         (((uintptr_t)out | (uintptr_t)(s.sdq * 2)) & 31) == 0);
             ptx::tc_fence_before();
             ptx::mbar_arrive(&bars[kTBarAccFree + b]);
         };

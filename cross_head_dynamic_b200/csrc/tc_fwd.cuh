@@ -360,7 +360,7 @@ fwd_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__ CU
             // the far segment adds to o: bring the rows it reads into L2 two heads ahead
             const bool o_add = SEG && a.seg.mode == kFwdSegFarApply && valid;
             if (o_add)
-                for (int h = 0; h < H && h < 2; ++h) prefetch_drain_row<D>(a.o + (t * H + h) * D, split);
+                for (int h = 0; h < H && h < 2; ++h) prefetch_drain_row<D>(a.o + t * s.so + h * D, split);
             // ---- P tile (bf16, K-major, swizzled) in smem; zero the columns outside the band
             uint8_t *ptile = sm + L::kP;
             uint32_t Pb[MAXC][4];   // P rounded to bf16 pairs, also the pmap values
@@ -436,11 +436,11 @@ fwd_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__ CU
             int cb16, ce16;
             acc_split(split, D / 16, cb16, ce16);
             constexpr int kMaxC16 = (D / 16 + kSplits - 1) / kSplits;
-            const bool o_aligned32 = ((uintptr_t)a.o & 31) == 0;
+            const bool o_aligned32 = (((uintptr_t)a.o | (uintptr_t)(s.so * 2)) & 31) == 0;
             for (int h = 0; h < H; ++h) {
                 const int b = h & 1;
                 const uint32_t n = (uint32_t)(h >> 1);
-                if (o_add && h + 2 < H) prefetch_drain_row<D>(a.o + (t * H + h + 2) * D, split);
+                if (o_add && h + 2 < H) prefetch_drain_row<D>(a.o + t * s.so + (h + 2) * D, split);
                 const float gh = g_next;
                 if (h + 1 < H) g_next = valid ? __ldg(a.g + t * H + h + 1) : 0.f;
                 wait_bar(&bars[kBarUFull + b], n & 1, abort_flag);
@@ -461,9 +461,9 @@ fwd_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__ CU
                                 w[e] = pack_bf16x2(gh * __uint_as_float(ur[c][2 * e]), gh * __uint_as_float(ur[c][2 * e + 1]));
                             if constexpr (SEG) {   // later segments add their share to o
                                 if (a.seg.mode == kFwdSegFarApply)
-                                    add_bf16x16(w, a.o + (t * H + h) * D + (cb16 + c) * 16, gh, ur[c]);
+                                    add_bf16x16(w, a.o + t * s.so + h * D + (cb16 + c) * 16, gh, ur[c]);
                             }
-                            ptx::st_global_32b(a.o + (t * H + h) * D + (cb16 + c) * 16, w, o_aligned32);
+                            ptx::st_global_32b(a.o + t * s.so + h * D + (cb16 + c) * 16, w, o_aligned32);
                         }
                     }
                 }

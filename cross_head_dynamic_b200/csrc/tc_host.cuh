@@ -54,13 +54,14 @@ inline EncodeTiledFn encode_fn() {
     return fn;
 }
 
-// 2-D view [N rows][H*d bf16] of a [N][H][d] tensor; boxes of 64 columns x box_rows
+// 2-D view [N rows][H*d bf16] of a [N][H][d] tensor whose consecutive tokens are `stride`
+// elements apart (H * d when contiguous; a multiple of 8); boxes of 64 columns x box_rows
 // rows, 128-byte swizzle, zero fill outside the tensor.
-inline cudaError_t make_map(CUtensorMap *m, const void *ptr, int64_t N, int H, int d, int box_rows) {
+inline cudaError_t make_map(CUtensorMap *m, const void *ptr, int64_t N, int H, int d, int64_t stride, int box_rows) {
     EncodeTiledFn enc = encode_fn();
     if (!enc) return cudaErrorNotSupported;
     cuuint64_t dims[2] = {(cuuint64_t)H * d, (cuuint64_t)N};
-    cuuint64_t strides[1] = {(cuuint64_t)H * d * 2};
+    cuuint64_t strides[1] = {(cuuint64_t)stride * 2};
     cuuint32_t box[2] = {64, (cuuint32_t)box_rows};
     cuuint32_t es[2] = {1, 1};
     CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(ptr), dims, strides, box, es,
@@ -157,12 +158,12 @@ inline cudaError_t fwd_segmented(const Shape &s, const void *q, const void *k, c
     if (!lse) return cudaErrorInvalidValue;
     const int BM = choose_block(s.N, kSegWidth, sm_count());
     CUtensorMap mq, mk[2], mv[2];
-    cudaError_t e = make_map(&mq, q, s.N, s.H, s.d, 128);
+    cudaError_t e = make_map(&mq, q, s.N, s.H, s.d, s.sq, 128);
     for (int sk = 0; sk < 2 && e == cudaSuccess; ++sk) {
         Seg sg;
         const int span = round16(BM + seg_shape(s, sk, 0, &sg).W - 1);
-        e = make_map(&mk[sk], k, s.N, s.H, s.d, span);
-        if (e == cudaSuccess) e = make_map(&mv[sk], v, s.N, s.H, s.d, span);
+        e = make_map(&mk[sk], k, s.N, s.H, s.d, s.sq, span);
+        if (e == cudaSuccess) e = make_map(&mv[sk], v, s.N, s.H, s.d, s.sq, span);
     }
     if (e != cudaSuccess) return e;
     const int order[3][2] = {{1, kFwdSegStats}, {0, kFwdSegNear}, {1, kFwdSegFarApply}};
@@ -197,9 +198,9 @@ inline cudaError_t fwd(const Shape &s, const void *q, const void *k, const void 
     a.lse = lse;
     a.pmap = (__nv_bfloat16 *)pmap;
     CUtensorMap mq, mk, mv;
-    cudaError_t e = make_map(&mq, q, s.N, s.H, s.d, 128);
-    if (e == cudaSuccess) e = make_map(&mk, k, s.N, s.H, s.d, a.span);
-    if (e == cudaSuccess) e = make_map(&mv, v, s.N, s.H, s.d, a.span);
+    cudaError_t e = make_map(&mq, q, s.N, s.H, s.d, s.sq, 128);
+    if (e == cudaSuccess) e = make_map(&mk, k, s.N, s.H, s.d, s.sq, a.span);
+    if (e == cudaSuccess) e = make_map(&mv, v, s.N, s.H, s.d, s.sq, a.span);
     if (e != cudaSuccess) return e;
     const int maxc = maxc_for(s.W);
     e = (s.d == 64) ? launch_fwd_d<64>(maxc, mq, mk, mv, a, st) : launch_fwd_d<128>(maxc, mq, mk, mv, a, st);
@@ -338,13 +339,13 @@ inline cudaError_t bwd_query_segmented(const Shape &s, const void *q, const void
                                        float *dc_, float *dg, float *band, cudaStream_t st, int32_t *launches) {
     const int BM = choose_block(s.N, kSegWidth, sm_count(), kBwdMaxSpan);
     CUtensorMap mq, mdo, mk[2], mv[2];
-    cudaError_t e = make_map(&mq, q, s.N, s.H, s.d, 128);
-    if (e == cudaSuccess) e = make_map(&mdo, dO, s.N, s.H, s.d, 128);
+    cudaError_t e = make_map(&mq, q, s.N, s.H, s.d, s.sq, 128);
+    if (e == cudaSuccess) e = make_map(&mdo, dO, s.N, s.H, s.d, s.so, 128);
     for (int sk = 0; sk < 2 && e == cudaSuccess; ++sk) {
         Seg sg;
         const int span = round16(BM + seg_shape(s, sk, 0, &sg).W - 1);
-        e = make_map(&mk[sk], k, s.N, s.H, s.d, span);
-        if (e == cudaSuccess) e = make_map(&mv[sk], v, s.N, s.H, s.d, span);
+        e = make_map(&mk[sk], k, s.N, s.H, s.d, s.sq, span);
+        if (e == cudaSuccess) e = make_map(&mv[sk], v, s.N, s.H, s.d, s.sq, span);
     }
     if (e != cudaSuccess) return e;
     const int order[3][2] = {{1, kQSegFarPart1}, {0, kQSegNear}, {1, kQSegFarPart2}};
@@ -388,11 +389,11 @@ inline cudaError_t bwd_query(const Shape &s, const void *q, const void *k, const
     a.dg = dg;
     a.band = band;
     CUtensorMap mq, mk, mv, mdo, mds;
-    cudaError_t e = make_map(&mq, q, s.N, s.H, s.d, 128);
-    if (e == cudaSuccess) e = make_map(&mk, k, s.N, s.H, s.d, a.span);
-    if (e == cudaSuccess) e = make_map(&mv, v, s.N, s.H, s.d, a.span);
-    if (e == cudaSuccess) e = make_map(&mdo, dO, s.N, s.H, s.d, 128);
-    if (e == cudaSuccess) e = dst ? make_map_ds(&mds, workspace, s.N, s.H, a.span, a.BM) : make_map(&mds, q, s.N, s.H, s.d, 128);
+    cudaError_t e = make_map(&mq, q, s.N, s.H, s.d, s.sq, 128);
+    if (e == cudaSuccess) e = make_map(&mk, k, s.N, s.H, s.d, s.sq, a.span);
+    if (e == cudaSuccess) e = make_map(&mv, v, s.N, s.H, s.d, s.sq, a.span);
+    if (e == cudaSuccess) e = make_map(&mdo, dO, s.N, s.H, s.d, s.so, 128);
+    if (e == cudaSuccess) e = dst ? make_map_ds(&mds, workspace, s.N, s.H, a.span, a.BM) : make_map(&mds, q, s.N, s.H, s.d, s.sq, 128);
     if (e != cudaSuccess) return e;
     e = [&]() -> cudaError_t {
         if (dst) {
@@ -422,12 +423,12 @@ inline cudaError_t bwd_key_segmented(const Shape &s, const void *q, const void *
                                      const float *band, void *dk, void *dv, cudaStream_t st, int32_t *launches) {
     const int BK = choose_block(s.N, kSegWidth, sm_count(), kBwdMaxSpan);
     CUtensorMap mk, mq[2], mdo[2];
-    cudaError_t e = make_map(&mk, k, s.N, s.H, s.d, 128);
+    cudaError_t e = make_map(&mk, k, s.N, s.H, s.d, s.sq, 128);
     for (int sk = 0; sk < 2 && e == cudaSuccess; ++sk) {
         Seg sg;
         const int span = round16(BK + seg_shape(s, sk, 0, &sg).W - 1);
-        e = make_map(&mq[sk], q, s.N, s.H, s.d, span);
-        if (e == cudaSuccess) e = make_map(&mdo[sk], dO, s.N, s.H, s.d, span);
+        e = make_map(&mq[sk], q, s.N, s.H, s.d, s.sq, span);
+        if (e == cudaSuccess) e = make_map(&mdo[sk], dO, s.N, s.H, s.d, s.so, span);
     }
     if (e != cudaSuccess) return e;
     const int order[2][2] = {{0, kKSegWrite}, {1, kKSegAdd}};
@@ -464,8 +465,8 @@ inline cudaError_t bwd_key(const Shape &s, const void *q, const void *k, const f
         a.dk = (__nv_bfloat16 *)dk;
         a.dv = (__nv_bfloat16 *)dv;
         CUtensorMap mq, mdo, mds;
-        cudaError_t e = make_map(&mq, q, s.N, s.H, s.d, a.span);
-        if (e == cudaSuccess) e = make_map(&mdo, dO, s.N, s.H, s.d, a.span);
+        cudaError_t e = make_map(&mq, q, s.N, s.H, s.d, s.sq, a.span);
+        if (e == cudaSuccess) e = make_map(&mdo, dO, s.N, s.H, s.d, s.so, a.span);
         if (e == cudaSuccess) e = make_map_ds(&mds, workspace, s.N, s.H, a.span, a.BM);
         if (e != cudaSuccess) return e;
         e = (s.d == 64) ? launch_bwd_key_dst<64>(mq, mdo, mds, a, st) : launch_bwd_key_dst<128>(mq, mdo, mds, a, st);
@@ -480,8 +481,8 @@ inline cudaError_t bwd_key(const Shape &s, const void *q, const void *k, const f
         a.dk = (__nv_bfloat16 *)dk;
         a.dv = (__nv_bfloat16 *)dv;
         CUtensorMap mq, mdo;
-        cudaError_t e = make_map(&mq, q, s.N, s.H, s.d, a.span);
-        if (e == cudaSuccess) e = make_map(&mdo, dO, s.N, s.H, s.d, a.span);
+        cudaError_t e = make_map(&mq, q, s.N, s.H, s.d, s.sq, a.span);
+        if (e == cudaSuccess) e = make_map(&mdo, dO, s.N, s.H, s.d, s.so, a.span);
         if (e != cudaSuccess) return e;
         e = [&]() -> cudaError_t {
             if (s.d == 64) {
@@ -501,9 +502,9 @@ inline cudaError_t bwd_key(const Shape &s, const void *q, const void *k, const f
     a.dk = (__nv_bfloat16 *)dk;
     a.dv = (__nv_bfloat16 *)dv;
     CUtensorMap mq, mk, mdo;
-    cudaError_t e = make_map(&mq, q, s.N, s.H, s.d, a.span);
-    if (e == cudaSuccess) e = make_map(&mk, k, s.N, s.H, s.d, 128);
-    if (e == cudaSuccess) e = make_map(&mdo, dO, s.N, s.H, s.d, a.span);
+    cudaError_t e = make_map(&mq, q, s.N, s.H, s.d, s.sq, a.span);
+    if (e == cudaSuccess) e = make_map(&mk, k, s.N, s.H, s.d, s.sq, 128);
+    if (e == cudaSuccess) e = make_map(&mdo, dO, s.N, s.H, s.d, s.so, a.span);
     if (e != cudaSuccess) return e;
     e = [&]() -> cudaError_t {
         if (s.d == 64) {

@@ -38,7 +38,8 @@ class Params(ctypes.Structure):
     _fields_ = [("dtype", ctypes.c_int32), ("impl", ctypes.c_int32), ("total_tokens", ctypes.c_int64),
                 ("num_docs", ctypes.c_int32), ("num_heads", ctypes.c_int32), ("head_dim", ctypes.c_int32),
                 ("window", ctypes.c_int32), ("softmax_scale", ctypes.c_float), ("reserved", ctypes.c_int32),
-                ("cu_seqlens", ctypes.c_void_p)]
+                ("cu_seqlens", ctypes.c_void_p), ("stride_qkv", ctypes.c_int64), ("stride_dqkv", ctypes.c_int64),
+                ("stride_o", ctypes.c_int64)]
 
 
 _lib = None
@@ -96,16 +97,29 @@ def _stream_handle(stream) -> int:
     return s.cuda_stream
 
 
-def _dev(x: torch.Tensor, name: str, dtype=None):
+def _dev(x: torch.Tensor, name: str, dtype=None, rows: bool = False):
+    """Device pointer of x.  With rows=True, x is [N, H, d] with each token's H * d
+    elements contiguous (tokens may be further apart: a view of a fused tensor)."""
     if not isinstance(x, torch.Tensor):
         raise TypeError(f"{name} must be a torch tensor")
     if not x.is_cuda:
         raise ValueError(f"{name} must be a CUDA tensor (libdcattn has no CPU path)")
-    if not x.is_contiguous():
+    if rows:
+        if x.dim() != 3 or x.stride(2) != 1 or x.stride(1) != x.shape[2]:
+            raise ValueError(f"{name} must be [N, H, d] with each token's H * d elements contiguous")
+    elif not x.is_contiguous():
         raise ValueError(f"{name} must be contiguous")
     if dtype is not None and x.dtype != dtype:
         raise TypeError(f"{name} must be {dtype}, got {x.dtype}")
     return x.data_ptr()
+
+
+def _row_stride(name: str, *xs) -> int:
+    """The common token stride of the [N, H, d] tensors xs (None entries ignored)."""
+    st = {int(x.stride(0)) for x in xs if x is not None and x.shape[0] > 1}
+    if len(st) > 1:
+        raise ValueError(f"{name} must share one token stride, got {sorted(st)}")
+    return st.pop() if st else 0
 
 
 def _opt(x, name, dtype=None):
@@ -113,7 +127,7 @@ def _opt(x, name, dtype=None):
 
 
 def make_params(q: torch.Tensor, cu_seqlens: torch.Tensor, window: int, scale: float,
-                impl: str = "auto") -> Params:
+                impl: str = "auto", stride_qkv: int = 0, stride_dqkv: int = 0, stride_o: int = 0) -> Params:
     if q.dim() != 3:
         raise ValueError("q must be [N, H, d]")
     N, H, d = q.shape
@@ -125,7 +139,8 @@ def make_params(q: torch.Tensor, cu_seqlens: torch.Tensor, window: int, scale: f
         raise TypeError(f"unsupported dtype {q.dtype}")
     return Params(dtype=dt, impl=IMPLS[impl], total_tokens=N, num_docs=cu_seqlens.numel() - 1,
                   num_heads=H, head_dim=d, window=int(window), softmax_scale=float(scale), reserved=0,
-                  cu_seqlens=_dev(cu_seqlens, "cu_seqlens", torch.int32))
+                  cu_seqlens=_dev(cu_seqlens, "cu_seqlens", torch.int32), stride_qkv=stride_qkv,
+                  stride_dqkv=stride_dqkv, stride_o=stride_o)
 
 
 def dc_attn_resolve_impl(q, cu_seqlens, window, scale, impl="auto") -> str:
@@ -140,18 +155,19 @@ def dc_attn_fwd(q, k, v, c, g, cu_seqlens, window: int, scale: float, *, o=None,
                 need_backward: bool = True, impl: str = "auto", stream=None):
     """Forward pass; returns (o, lse, pmap).  lse/pmap are None when need_backward
     is False and none were passed in."""
-    p = make_params(q, cu_seqlens, window, scale, impl)
     N, H, d = q.shape
     if o is None:
-        o = torch.empty_like(q)
+        o = torch.empty(q.shape, device=q.device, dtype=q.dtype)
+    p = make_params(q, cu_seqlens, window, scale, impl, stride_qkv=_row_stride("q, k, v", q, k, v),
+                    stride_o=_row_stride("o", o))
     if need_backward:
         if lse is None:
             lse = torch.empty(N, H, device=q.device, dtype=torch.float32)
         if pmap is None:
             pmap = torch.empty(N, int(window), device=q.device, dtype=q.dtype)
     code = load_library().dc_attn_fwd(
-        ctypes.byref(p), _dev(q, "q", q.dtype), _dev(k, "k", q.dtype), _dev(v, "v", q.dtype),
-        _dev(c, "c", torch.float32), _dev(g, "g", torch.float32), _dev(o, "o", q.dtype),
+        ctypes.byref(p), _dev(q, "q", q.dtype, True), _dev(k, "k", q.dtype, True), _dev(v, "v", q.dtype, True),
+        _dev(c, "c", torch.float32), _dev(g, "g", torch.float32), _dev(o, "o", q.dtype, True),
         _opt(lse, "lse", torch.float32), _opt(pmap, "pmap", q.dtype), _stream_handle(stream))
     _check("dc_attn_fwd", code)
     return o, lse, pmap
@@ -172,16 +188,17 @@ def _workspace(q, cu_seqlens, window, scale, impl, workspace):
 def dc_attn_bwd_query(q, k, v, c, g, dO, lse, pmap, cu_seqlens, window, scale, *, dq=None, dc=None,
                       dg=None, workspace=None, impl="auto", stream=None):
     """Query side of the backward; returns (dq, dc, dg, workspace)."""
-    p = make_params(q, cu_seqlens, window, scale, impl)
     N, H, d = q.shape
-    dq = torch.empty_like(q) if dq is None else dq
+    dq = torch.empty(q.shape, device=q.device, dtype=q.dtype) if dq is None else dq
     dc = torch.empty(N, H, device=q.device, dtype=torch.float32) if dc is None else dc
     dg = torch.empty(N, H, device=q.device, dtype=torch.float32) if dg is None else dg
+    p = make_params(q, cu_seqlens, window, scale, impl, stride_qkv=_row_stride("q, k, v", q, k, v),
+                    stride_dqkv=_row_stride("dq", dq), stride_o=_row_stride("dO", dO))
     workspace = _workspace(q, cu_seqlens, window, scale, impl, workspace)
     code = load_library().dc_attn_bwd_query(
-        ctypes.byref(p), _dev(q, "q", q.dtype), _dev(k, "k", q.dtype), _dev(v, "v", q.dtype),
-        _dev(c, "c", torch.float32), _dev(g, "g", torch.float32), _dev(dO, "dO", q.dtype),
-        _dev(lse, "lse", torch.float32), _dev(pmap, "pmap", q.dtype), _dev(dq, "dq", q.dtype),
+        ctypes.byref(p), _dev(q, "q", q.dtype, True), _dev(k, "k", q.dtype, True), _dev(v, "v", q.dtype, True),
+        _dev(c, "c", torch.float32), _dev(g, "g", torch.float32), _dev(dO, "dO", q.dtype, True),
+        _dev(lse, "lse", torch.float32), _dev(pmap, "pmap", q.dtype), _dev(dq, "dq", q.dtype, True),
         _dev(dc, "dc", torch.float32), _dev(dg, "dg", torch.float32), _dev(workspace, "workspace"),
         workspace.numel() * workspace.element_size(), _stream_handle(stream))
     _check("dc_attn_bwd_query", code)
@@ -191,14 +208,15 @@ def dc_attn_bwd_query(q, k, v, c, g, dO, lse, pmap, cu_seqlens, window, scale, *
 def dc_attn_bwd_key(q, k, c, g, dO, lse, pmap, dc, workspace, cu_seqlens, window, scale, *, dk=None, dv=None,
                     impl="auto", stream=None):
     """Key side of the backward (after dc_attn_bwd_query); returns (dk, dv)."""
-    p = make_params(q, cu_seqlens, window, scale, impl)
-    dk = torch.empty_like(q) if dk is None else dk
-    dv = torch.empty_like(q) if dv is None else dv
+    dk = torch.empty(q.shape, device=q.device, dtype=q.dtype) if dk is None else dk
+    dv = torch.empty(q.shape, device=q.device, dtype=q.dtype) if dv is None else dv
+    p = make_params(q, cu_seqlens, window, scale, impl, stride_qkv=_row_stride("q, k", q, k),
+                    stride_dqkv=_row_stride("dk, dv", dk, dv), stride_o=_row_stride("dO", dO))
     code = load_library().dc_attn_bwd_key(
-        ctypes.byref(p), _dev(q, "q", q.dtype), _dev(k, "k", q.dtype), _dev(c, "c", torch.float32),
-        _dev(g, "g", torch.float32), _dev(dO, "dO", q.dtype), _dev(lse, "lse", torch.float32),
-        _dev(pmap, "pmap", q.dtype), _dev(dc, "dc", torch.float32), _dev(dk, "dk", q.dtype),
-        _dev(dv, "dv", q.dtype), _dev(workspace, "workspace"), workspace.numel() * workspace.element_size(),
+        ctypes.byref(p), _dev(q, "q", q.dtype, True), _dev(k, "k", q.dtype, True), _dev(c, "c", torch.float32),
+        _dev(g, "g", torch.float32), _dev(dO, "dO", q.dtype, True), _dev(lse, "lse", torch.float32),
+        _dev(pmap, "pmap", q.dtype), _dev(dc, "dc", torch.float32), _dev(dk, "dk", q.dtype, True),
+        _dev(dv, "dv", q.dtype, True), _dev(workspace, "workspace"), workspace.numel() * workspace.element_size(),
         _stream_handle(stream))
     _check("dc_attn_bwd_key", code)
     return dk, dv
@@ -207,19 +225,20 @@ def dc_attn_bwd_key(q, k, c, g, dO, lse, pmap, dc, workspace, cu_seqlens, window
 def dc_attn_bwd(q, k, v, c, g, dO, lse, pmap, cu_seqlens, window, scale, *, dq=None, dk=None, dv=None,
                 dc=None, dg=None, workspace=None, impl="auto", stream=None):
     """Full backward; returns (dq, dk, dv, dc, dg)."""
-    p = make_params(q, cu_seqlens, window, scale, impl)
     N, H, d = q.shape
-    dq = torch.empty_like(q) if dq is None else dq
-    dk = torch.empty_like(q) if dk is None else dk
-    dv = torch.empty_like(q) if dv is None else dv
+    dq = torch.empty(q.shape, device=q.device, dtype=q.dtype) if dq is None else dq
+    dk = torch.empty(q.shape, device=q.device, dtype=q.dtype) if dk is None else dk
+    dv = torch.empty(q.shape, device=q.device, dtype=q.dtype) if dv is None else dv
+    p = make_params(q, cu_seqlens, window, scale, impl, stride_qkv=_row_stride("q, k, v", q, k, v),
+                    stride_dqkv=_row_stride("dq, dk, dv", dq, dk, dv), stride_o=_row_stride("dO", dO))
     dc = torch.empty(N, H, device=q.device, dtype=torch.float32) if dc is None else dc
     dg = torch.empty(N, H, device=q.device, dtype=torch.float32) if dg is None else dg
     workspace = _workspace(q, cu_seqlens, window, scale, impl, workspace)
     code = load_library().dc_attn_bwd(
-        ctypes.byref(p), _dev(q, "q", q.dtype), _dev(k, "k", q.dtype), _dev(v, "v", q.dtype),
-        _dev(c, "c", torch.float32), _dev(g, "g", torch.float32), _dev(dO, "dO", q.dtype),
-        _dev(lse, "lse", torch.float32), _dev(pmap, "pmap", q.dtype), _dev(dq, "dq", q.dtype),
-        _dev(dk, "dk", q.dtype), _dev(dv, "dv", q.dtype), _dev(dc, "dc", torch.float32),
+        ctypes.byref(p), _dev(q, "q", q.dtype, True), _dev(k, "k", q.dtype, True), _dev(v, "v", q.dtype, True),
+        _dev(c, "c", torch.float32), _dev(g, "g", torch.float32), _dev(dO, "dO", q.dtype, True),
+        _dev(lse, "lse", torch.float32), _dev(pmap, "pmap", q.dtype), _dev(dq, "dq", q.dtype, True),
+        _dev(dk, "dk", q.dtype, True), _dev(dv, "dv", q.dtype, True), _dev(dc, "dc", torch.float32),
         _dev(dg, "dg", torch.float32), _dev(workspace, "workspace"),
         workspace.numel() * workspace.element_size(), _stream_handle(stream))
     _check("dc_attn_bwd", code)
@@ -234,18 +253,19 @@ def dc_attn_bwd_noalloc(q, k, v, c, g, dO, lse, pmap, cu_seqlens, window, scale,
     32 MiB scratch array serves as the workspace, so N * W * 4 must not exceed
     32 MiB; overlapping calls on one device race on that array.  Returns
     (dq, dk, dv, dc, dg)."""
-    p = make_params(q, cu_seqlens, window, scale, impl)
     N, H, d = q.shape
-    dq = torch.empty_like(q) if dq is None else dq
-    dk = torch.empty_like(q) if dk is None else dk
-    dv = torch.empty_like(q) if dv is None else dv
+    dq = torch.empty(q.shape, device=q.device, dtype=q.dtype) if dq is None else dq
+    dk = torch.empty(q.shape, device=q.device, dtype=q.dtype) if dk is None else dk
+    dv = torch.empty(q.shape, device=q.device, dtype=q.dtype) if dv is None else dv
+    p = make_params(q, cu_seqlens, window, scale, impl, stride_qkv=_row_stride("q, k, v", q, k, v),
+                    stride_dqkv=_row_stride("dq, dk, dv", dq, dk, dv), stride_o=_row_stride("dO", dO))
     dc = torch.empty(N, H, device=q.device, dtype=torch.float32) if dc is None else dc
     dg = torch.empty(N, H, device=q.device, dtype=torch.float32) if dg is None else dg
     code = load_library().dc_attn_bwd_noalloc(
-        ctypes.byref(p), _dev(q, "q", q.dtype), _dev(k, "k", q.dtype), _dev(v, "v", q.dtype),
-        _dev(c, "c", torch.float32), _dev(g, "g", torch.float32), _dev(dO, "dO", q.dtype),
-        _dev(lse, "lse", torch.float32), _dev(pmap, "pmap", q.dtype), _dev(dq, "dq", q.dtype),
-        _dev(dk, "dk", q.dtype), _dev(dv, "dv", q.dtype), _dev(dc, "dc", torch.float32),
+        ctypes.byref(p), _dev(q, "q", q.dtype, True), _dev(k, "k", q.dtype, True), _dev(v, "v", q.dtype, True),
+        _dev(c, "c", torch.float32), _dev(g, "g", torch.float32), _dev(dO, "dO", q.dtype, True),
+        _dev(lse, "lse", torch.float32), _dev(pmap, "pmap", q.dtype), _dev(dq, "dq", q.dtype, True),
+        _dev(dk, "dk", q.dtype, True), _dev(dv, "dv", q.dtype, True), _dev(dc, "dc", torch.float32),
         _dev(dg, "dg", torch.float32), _stream_handle(stream))
     _check("dc_attn_bwd_noalloc", code)
     return dq, dk, dv, dc, dg

@@ -19,7 +19,12 @@
  * - Tokens are packed: N = total_tokens rows, documents given by cu_seqlens
  *   (device, int32, num_docs + 1 entries, 0 = cu[0] <= ... <= cu[num_docs] = N;
  *   empty documents are allowed).  No key of another document is ever used.
- * - q, k, v, o, dO, dq, dk, dv: contiguous [N][H][d] in `dtype` (fp32 or bf16).
+ * - q, k, v, o, dO, dq, dk, dv: [N][H][d] in `dtype` (fp32 or bf16), each token's
+ *   H * d elements contiguous, consecutive tokens `stride` elements apart:
+ *   stride_qkv for q, k, v; stride_dqkv for dq, dk, dv; stride_o for o (forward)
+ *   and dO (backward).  A stride of 0 means H * d (contiguous tensors).  The
+ *   strides let q, k, v be views of one fused projection [N][3][H][d] (stride
+ *   3 * H * d) and dq, dk, dv be written straight into its gradient.
  *   c, g, lse, dc, dg: contiguous [N][H] fp32.
  *   pmap: contiguous [N][W] in `dtype`; pmap[t][w] = P(t, t-W+1+w), 0 outside
  *   window(t).  It is the one composed map per token (the H per-head maps are
@@ -82,6 +87,11 @@ typedef struct {
     float softmax_scale;        /* sigma, usually 1/sqrt(d); 1 when q is pre-scaled        */
     int32_t reserved;           /* must be 0                                              */
     const int32_t *cu_seqlens;  /* device pointer, num_docs + 1 entries                   */
+    int64_t stride_qkv;         /* elements between tokens of q, k, v; 0 = H * d          */
+    int64_t stride_dqkv;        /* ... of dq, dk, dv; 0 = H * d                           */
+    int64_t stride_o;           /* ... of o and dO; 0 = H * d                             */
+    /* A nonzero stride must be >= H * d and a multiple of 16 bytes (8 bf16 or 4 fp32
+     * elements), else DC_ERR_INVALID_ARG. */
 } dc_attn_params;
 
 /* Forward pass.

@@ -147,3 +147,19 @@ def test_wait_limit_hook_validates_on_the_host(lib):
     assert lib.dc_attn_set_wait_limit(99999) == dcattn.DC_ERR_INVALID_ARG
     assert lib.dc_attn_set_wait_limit(5_000_000) == dcattn.DC_OK
     assert lib.dc_attn_set_wait_limit(0) == dcattn.DC_OK                    # back to the default
+
+
+@pytest.mark.parametrize("field", ["stride_qkv", "stride_dqkv", "stride_o"])
+@pytest.mark.parametrize("value", [767, 772, -768])
+def test_rejects_bad_row_strides(lib, field, value):
+    """A row stride below H * d (768 here), or one that is not a multiple of 16 bytes, is
+    refused on the host before anything runs."""
+    p = _params(**{field: value})
+    assert _fwd(lib, p) == dcattn.DC_ERR_INVALID_ARG
+
+
+def test_accepts_fused_projection_strides(lib):
+    """3 * H * d (q, k, v as views of one [N][3][H][d] projection) passes the host checks; the
+    call then stops at the device pointers, which are not real (N = 0 would skip them)."""
+    p = _params(stride_qkv=3 * 768, stride_dqkv=3 * 768, stride_o=2 * 768, total_tokens=0)
+    assert _fwd(lib, p) == dcattn.DC_OK
