@@ -57,6 +57,52 @@ def algorithmic_bytes_per_token(H: int, d: int, e: int = 2) -> dict:
     }
 
 
+NOMINAL_HBM_GBS = 8000.0        # the ~8 TB/s HBM3e figure the target is stated against
+NOMINAL_BF16_TFLOPS = 2250.0    # dense bf16 tensor peak
+
+
+def window_lengths(cu_seqlens, W: int):
+    """Per-token window length min(W, position in document + 1), as a float64 array."""
+    import numpy as np
+    cu = [int(x) for x in cu_seqlens]
+    out = []
+    for a, b in zip(cu[:-1], cu[1:]):
+        out.append(np.minimum(np.arange(1, b - a + 1, dtype=np.float64), W))
+    return np.concatenate(out) if out else np.zeros(0)
+
+
+def algorithmic_flops(H: int, d: int, weff_sum: float) -> dict:
+    """Window FLOPs (only valid (query, key) pairs count): the forward's two products
+    (scores, P.V) are 4 H d per pair; the query side's three (score recompute, E, dQ) 6 H d;
+    the key side's two (dV, dK) 4 H d; the step 14 H d."""
+    return {"fwd": 4 * H * d * weff_sum, "bwd_query": 6 * H * d * weff_sum,
+            "bwd_key": 4 * H * d * weff_sum, "step": 14 * H * d * weff_sum}
+
+
+def roofline(bytes_: float, flops: float, seconds: float, hbm_gbs: float, tflops: float) -> dict:
+    """The slower of the two limits (bytes at HBM bandwidth, FLOPs at the bf16 tensor peak)
+    is the bound; achieved and peak are given in that limit's unit."""
+    t_mem = bytes_ / (hbm_gbs * 1e9)
+    t_tc = flops / (tflops * 1e12)
+    if t_mem >= t_tc:
+        return {"bound": "hbm", "achieved": bytes_ / seconds / 1e9, "peak": hbm_gbs, "unit": "GB/s",
+                "frac": t_mem / seconds, "t_hbm_us": t_mem * 1e6, "t_tensor_us": t_tc * 1e6}
+    return {"bound": "tensor", "achieved": flops / seconds / 1e12, "peak": tflops, "unit": "TFLOP/s",
+            "frac": t_tc / seconds, "t_hbm_us": t_mem * 1e6, "t_tensor_us": t_tc * 1e6}
+
+
+def step_dram_bytes(tokens: int):
+    """Sum over the step's kernels of the committed ncu DRAM bytes (read + write), scaled to
+    `tokens`; None unless every kernel's capture matches its current source."""
+    tot = 0.0
+    for k in KERNEL_SOURCES:
+        t = measured_traffic(k, tokens)
+        if t is None:
+            return None
+        tot += t
+    return tot
+
+
 def source_hash(paths) -> str:
     """SHA-1 of the kernel sources' code: comments and whitespace are dropped, so a
     comment edit keeps a DRAM-traffic capture valid while any code change voids it."""
@@ -196,6 +242,44 @@ def oracle_sample_rate(cfg, rows: int, reps: int = 1):
     return rows * cfg.seqlen * reps / dt, oracle.num_threads(), dt
 
 
+_ORACLE_SNIPPET = r'''
+import json, sys, time
+sys.path.insert(0, {root!r})
+import oracle
+from cross_head_dynamic_b200.inputs import CONFIGS, generate
+oracle.build()
+cfg = CONFIGS[{name!r}]
+x = generate(cfg.replace(batch=1) if cfg.docs == "rows" else cfg)
+n = {tokens}
+cu = [int(c) for c in x["cu_seqlens"]]
+docs = [c for c in cu if c <= n]
+if docs[-1] < n:
+    docs.append(n)
+cut = lambda t: t[:n]
+t = time.perf_counter()
+oracle.forward(cut(x["q"]), cut(x["k"]), cut(x["v"]), cut(x["c"]), cut(x["g"]), docs, x["window"], x["scale"])
+oracle.backward(cut(x["q"]), cut(x["k"]), cut(x["v"]), cut(x["c"]), cut(x["g"]), cut(x["dO"]), docs, x["window"],
+                x["scale"])
+dt = time.perf_counter() - t
+print(json.dumps({{"tokens_per_s": n / dt, "seconds": dt, "threads": oracle.num_threads()}}))
+'''
+
+
+def oracle_sample_subprocess(name: str, tokens: int, threads: int = 0):
+    """fp64 oracle fwd+bwd on the first `tokens` tokens of workload `name` (its first batch row;
+    the documents cut at that point), in a fresh process (OMP_NUM_THREADS=threads when > 0).
+    Returns the parsed JSON result, or None if the sample could not run."""
+    env = dict(os.environ)
+    if threads > 0:
+        env["OMP_NUM_THREADS"] = str(threads)
+    code = _ORACLE_SNIPPET.format(root=ROOT, name=name, tokens=int(tokens))
+    try:
+        res = subprocess.run([sys.executable, "-c", code], env=env, capture_output=True, text=True, timeout=600)
+        return json.loads(res.stdout.strip().splitlines()[-1])
+    except (subprocess.SubprocessError, ValueError, IndexError):
+        return None
+
+
 def config_block(cfg, n_gpus):
     return {"workload": f"{WORKLOAD}: B{cfg.batch} x T{cfg.seqlen}, H{cfg.heads} x d{cfg.head_dim}, "
                         f"W{cfg.window}, one document per row, bf16 q/k/v/dO, fp32 c/g",
@@ -246,6 +330,7 @@ def run_sweep(args):
     dev = torch.device("cuda", 0)
     peaks = json.load(open(PEAKS_FILE)) if os.path.exists(PEAKS_FILE) else {}
     hbm = peaks.get("hbm_gbs") or 6650.0
+    tflops = peaks.get("bf16_tflops_sustained") or 1400.0
     for name, cfg in CONFIGS.items():
         if args.workload and name not in args.workload:
             continue
@@ -303,12 +388,12 @@ def run_sweep(args):
         ms = a.elapsed_time(b) / args.steps
         e = 4 if cfg.dtype == "f32" else 2
         per_tok = (11 * H * d * e + 24 * H) if cfg.backward else (4 * H * d * e + 8 * H)
-        gbs = per_tok * N / (ms * 1e-3) / 1e9
+        flops = algorithmic_flops(H, d, float(window_lengths(host["cu_seqlens"], W).sum()))
+        rl = roofline(per_tok * N, flops["step"] if cfg.backward else flops["fwd"], ms * 1e-3, hbm, tflops)
         print(json.dumps({"workload": name, "pass": "fwd+bwd" if cfg.backward else "fwd", "kernels": impl,
                           "tokens": N, "heads": H, "head_dim": d, "window": W, "dtype": cfg.dtype,
                           "docs": cfg.docs, "ms_per_step": ms, "tokens_per_s": N / (ms * 1e-3),
-                          "roofline": {"bound": "hbm", "achieved": gbs, "peak": hbm, "unit": "GB/s",
-                                       "frac": gbs / hbm, "algorithmic_bytes_per_token": per_tok}}), flush=True)
+                          "roofline": dict(rl, algorithmic_bytes_per_token=per_tok)}), flush=True)
         del graphs, sets
         torch.cuda.empty_cache()
     return 0
@@ -428,10 +513,45 @@ def main():
         step(sets[it % N_SETS], evs[it])
     torch.cuda.synchronize()
     names = ("fwd", "bwd_query", "bwd_key")
-    per_kernel = {n: sum(ev[j].elapsed_time(ev[j + 1]) for ev in evs) / args.steps
-                  for j, n in enumerate(names)}   # ms per launch
+    per_kernel_eager = {n: sum(ev[j].elapsed_time(ev[j + 1]) for ev in evs) / args.steps
+                        for j, n in enumerate(names)}   # ms per launch
     split_ms_step = evs[0][0].elapsed_time(evs[-1][3]) / args.steps
     value, ms_step = replica_throughput(N, total_ms, args.steps, world)
+
+    # Per-kernel time without launch gaps: each kernel alone, one CUDA graph per input set
+    # holding 4 launches of it, replayed back to back and timed with CUDA events on the
+    # launching stream (the kernels that surround it in a step are absent, so the cache state
+    # differs slightly from the step's).
+    kernel_calls = {
+        "fwd": lambda x: dcattn.dc_attn_fwd(x["q"], x["k"], x["v"], x["c"], x["g"], x["cu_seqlens"], W, scale,
+                                            o=x["o"], lse=x["lse"], pmap=x["pmap"]),
+        "bwd_query": lambda x: dcattn.dc_attn_bwd_query(x["q"], x["k"], x["v"], x["c"], x["g"], x["dO"], x["lse"],
+                                                        x["pmap"], x["cu_seqlens"], W, scale, dq=x["dq"], dc=x["dc"],
+                                                        dg=x["dg"], workspace=x["ws"]),
+        "bwd_key": lambda x: dcattn.dc_attn_bwd_key(x["q"], x["k"], x["c"], x["g"], x["dO"], x["lse"], x["pmap"],
+                                                    x["dc"], x["ws"], x["cu_seqlens"], W, scale, dk=x["dk"],
+                                                    dv=x["dv"]),
+    }
+    per_kernel = {}
+    reps_per_graph, kernel_replays = 4, max(8, min(args.steps, 40))
+    for kname, call in kernel_calls.items():
+        kg = []
+        for x in sets:
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g):
+                for _ in range(reps_per_graph):
+                    call(x)
+            kg.append(g)
+        for it in range(N_SETS):
+            kg[it].replay()
+        ka, kb = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        ka.record(stream)
+        for it in range(kernel_replays):
+            kg[it % N_SETS].replay()
+        kb.record(stream)
+        torch.cuda.synchronize()
+        per_kernel[kname] = ka.elapsed_time(kb) / (kernel_replays * reps_per_graph)
+        del kg
 
     clocks = sampler.summary(t_wall0, t_wall1)
     clock_note = "sampled during the timed region"
@@ -508,22 +628,43 @@ def main():
            "note": "dc_attn_* calls; inputs uploaded and outputs read back every step on copy streams "
                    "that overlap neighbouring steps"}
 
-    # roofline of the dominant kernel (HBM-bound path) against the measured copy bandwidth
+    # rooflines: the slower of (algorithmic bytes at the measured HBM copy bandwidth) and
+    # (window FLOPs at the measured bf16 tensor peak); the dominant kernel and the whole step
     peaks = json.load(open(PEAKS_FILE)) if os.path.exists(PEAKS_FILE) else {}
     hbm = peaks.get("hbm_gbs")
     peak_note = "of measured" if hbm else "of fallback"
     hbm = hbm or 6650.0
+    # the kernels run back to back for many steps: the sustained GEMM figure applies
+    tflops = peaks.get("bf16_tflops_sustained") or (1400.0 if not peaks else peaks.get("bf16_tflops"))
     abytes = algorithmic_bytes_per_token(H, d)
+    weff = float(window_lengths(host["cu_seqlens"], W).sum())
+    aflops = algorithmic_flops(H, d, weff)
     dom = max(per_kernel, key=per_kernel.get)
-    achieved = abytes[dom] * N / (per_kernel[dom] * 1e-3) / 1e9
+    rl = roofline(abytes[dom] * N, aflops[dom], per_kernel[dom] * 1e-3, hbm, tflops)
     traffic = measured_traffic(dom, N)
-    step_gbs = abytes["step"] * N / (ms_step * 1e-3) / 1e9
+    step_rl = roofline(abytes["step"] * N, aflops["step"], ms_step * 1e-3, hbm, tflops)
+    step_rl_nominal = roofline(abytes["step"] * N, aflops["step"], ms_step * 1e-3, NOMINAL_HBM_GBS,
+                               NOMINAL_BF16_TFLOPS)
+    step_dram = step_dram_bytes(N)
 
     cpu = None
     if rank == 0 and not args.no_cpu_baseline:
         rate, cores, dt = oracle_sample_rate(cfg, rows=cfg.batch)
         cpu = {"value": rate, "unit": UNIT, "cores": cores, "kind": "oracle",
                "sample": f"one fwd+bwd of all {cfg.total_tokens} tokens of the workload in fp64 ({dt:.1f} s)"}
+        # the same oracle on one thread, and on samples of the packed varlen batch and of the
+        # widest-window sweep point (their first 4096 tokens, documents cut there)
+        extra = {}
+        one = oracle_sample_subprocess(WORKLOAD, 2048, threads=1)
+        if one:
+            extra["one_thread"] = {"value": one["tokens_per_s"], "unit": UNIT, "cores": 1,
+                                   "sample": "fwd+bwd of the first 2048 tokens (one batch row) of the workload"}
+        for wname in ("varlen", "sweep_W256_H6_d128"):
+            r = oracle_sample_subprocess(wname, 4096)
+            if r:
+                extra[wname] = {"value": r["tokens_per_s"], "unit": UNIT, "cores": r["threads"],
+                                "sample": f"fwd+bwd of the first 4096 tokens of {wname}"}
+        cpu["other_samples"] = extra
 
     if rank == 0:
         line = {
@@ -532,16 +673,22 @@ def main():
             "vs_baseline": None, "dtype": "bf16", "data": "synthetic", "impl": "dcattn", "kernels": impl,
             "config": config_block(cfg, world),
             "timing": (f"value: {args.steps} back-to-back replays of one CUDA graph per input set (one graph = "
-                       f"one fwd+bwd step, {launches_per_step} kernels); kernel_ms: a second pass of the same "
-                       f"{args.steps} steps launched directly with CUDA events between the kernels "
-                       f"({split_ms_step * 1e3:.1f} us per step there)"),
-            "roofline": {"bound": "hbm", "kernel": dom, "achieved": achieved, "peak": hbm, "unit": "GB/s",
-                         "frac": achieved / hbm, "peak_source": peak_note, "traffic": traffic,
-                         "algorithmic_bytes_per_launch": abytes[dom] * N},
-            "step_roofline": {"achieved": step_gbs, "peak": hbm, "unit": "GB/s", "frac": step_gbs / hbm,
-                              "algorithmic_bytes_per_step": abytes["step"] * N,
-                              "roofline_tokens_per_s": hbm * 1e9 / abytes["step"]},
+                       f"one fwd+bwd step, {launches_per_step} kernels), CUDA events on the launching stream; "
+                       f"kernel_ms: each kernel alone, {reps_per_graph} launches per graph, {kernel_replays} "
+                       f"replays; kernel_ms_eager: a pass of the {args.steps} steps launched directly with "
+                       f"CUDA events between the kernels ({split_ms_step * 1e3:.1f} us per step there)"),
+            "roofline": dict(rl, kernel=dom, peak_source=peak_note, traffic=traffic,
+                             algorithmic_bytes_per_launch=abytes[dom] * N,
+                             algorithmic_flops_per_launch=aflops[dom]),
+            "step_roofline": dict(step_rl, peak_source=peak_note,
+                                  frac_nominal_peaks=step_rl_nominal["frac"],
+                                  nominal_peaks={"hbm_gbs": NOMINAL_HBM_GBS, "bf16_tflops": NOMINAL_BF16_TFLOPS},
+                                  algorithmic_bytes_per_step=abytes["step"] * N,
+                                  algorithmic_flops_per_step=aflops["step"],
+                                  dram_bytes_per_step_ncu=step_dram,
+                                  roofline_tokens_per_s=hbm * 1e9 / abytes["step"]),
             "kernel_ms": per_kernel,
+            "kernel_ms_eager": per_kernel_eager,
             "cpu_baseline": cpu,
             "e2e": e2e,
             "gpu_launches": gpu_launches,
