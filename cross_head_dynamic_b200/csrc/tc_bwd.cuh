@@ -76,6 +76,34 @@ enum : int { kQSegFarPart1 = 1, kQSegNear = 2, kQSegFarPart2 = 3 };
 // Segmented key side: the first segment writes dk and dv, the next one adds to them.
 enum : int { kKSegWrite = 1, kKSegAdd = 2 };
 
+// Drain this split's 16-column chunks of one row of a [128 x D] fp32 accumulator with one
+// TMEM round trip for all of them (for kernels with registers to spare).
+template <int D>
+__device__ __forceinline__ void drain_row_once(uint32_t taddr, __nv_bfloat16 *dst, float mult, bool store, int split,
+                                               bool aligned32) {
+    int cb16, ce16;
+    acc_split(split, D / 16, cb16, ce16);
+    constexpr int kMaxC16 = (D / 16 + kSplits - 1) / kSplits;
+    uint32_t r[kMaxC16][16];
+#pragma unroll
+    for (int c = 0; c < kMaxC16; ++c)
+        if (cb16 + c < ce16) ptx::tmem_ld16_issue(taddr + (cb16 + c) * 16, r[c]);
+    ptx::tmem_wait_ld();
+#pragma unroll
+    for (int c = 0; c < kMaxC16; ++c) {
+        if (cb16 + c < ce16) {
+            ptx::reg_fence16(r[c]);
+            if (store) {
+                uint32_t w[8];
+#pragma unroll
+                for (int e = 0; e < 8; ++e)
+                    w[e] = pack_bf16x2(mult * __uint_as_float(r[c][2 * e]), mult * __uint_as_float(r[c][2 * e + 1]));
+                ptx::st_global_32b(dst + (cb16 + c) * 16, w, aligned32);
+            }
+        }
+    }
+}
+
 // Drain this split's 16-column chunks of one row of a [128 x D] fp32 accumulator
 // (row base address taddr, output row dst): scale, round to bf16, store when `store`
 // (full 32-byte sectors; aligned32 says whether the output buffer allows 256-bit stores).
@@ -1584,8 +1612,8 @@ bwd_key_dst_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_const
             const int b = idx & 1;
             wait_bar(&bars[kTBarAccFull + b], (uint32_t)(idx >> 1) & 1, abort_flag);
             ptx::tc_fence_after();
-            drain_row<D>(tmem + lane_base + 256 + 128 * b, out + j * s.sdq + h * D, mult, validk, split,
-                         (((uintptr_t)out | (uintptr_t)(s.sdq * 2)) & 31) == 0);
+            drain_row_once<D>(tmem + lane_base + 256 + 128 * b, out + j * s.sdq + h * D, mult, validk, split,
+                              (((uintptr_t)out | (uintptr_t)(s.sdq * 2)) & 31) == 0);
             ptx::tc_fence_before();
             ptx::mbar_arrive(&bars[kTBarAccFree + b]);
         };
