@@ -171,3 +171,22 @@ def random_problem(seed: int, doc_lens, heads: int, head_dim: int, window: int,
     return dict(q=q, k=k, v=v, c=c, g=g, dO=dO,
                 cu_seqlens=torch.from_numpy(cu.astype(np.int32)), window=window,
                 scale=(1.0 / math.sqrt(head_dim)) if scale is None else scale)
+
+
+def cg_problem(seed: int, n_tokens: int, model_dim: int, heads: int, dtype: str = "bf16") -> dict:
+    """Seeded inputs for the producer of c and g (random numbers only): x [N, D] ~ N(0,1)
+    in `dtype` (bf16 rounded from fp32, or fp32); w [D, 2H] fp32 ~ N(0, 0.25 / D), so that
+    the projected c has a standard deviation near 0.5; b [2H] fp32 with the c half ~ N(0, 0.1)
+    and the g half 1 + N(0, 0.1); dc, dg [N, H] fp32 ~ N(0, 1).  Draw order: x, w, b, dc, dg."""
+    gen = torch.Generator().manual_seed(seed)
+    x = torch.randn(n_tokens, model_dim, generator=gen)
+    w = torch.randn(model_dim, 2 * heads, generator=gen) * math.sqrt(0.25 / model_dim)
+    b = torch.randn(2 * heads, generator=gen) * 0.1
+    b[heads:] += 1.0
+    dc = torch.randn(n_tokens, heads, generator=gen)
+    dg = torch.randn(n_tokens, heads, generator=gen)
+    if dtype == "bf16":
+        x = x.to(torch.bfloat16)
+    elif dtype != "f32":
+        raise ValueError(f"unknown dtype {dtype!r}")
+    return dict(x=x, w=w, b=b, dc=dc, dg=dg)

@@ -20,16 +20,18 @@ import numpy as np
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
 _SRC = os.path.join(_HERE, "dc_oracle.c")
+_SRC_CG = os.path.join(_HERE, "cg_oracle.c")
 _LIB = os.path.join(_HERE, "libdcoracle.so")
 _lib = None
 
 
 def build(force: bool = False) -> str:
-    """Compile dc_oracle.c into libdcoracle.so next to it (gcc, -O2, OpenMP)."""
-    if force or not os.path.exists(_LIB) or os.path.getmtime(_LIB) < os.path.getmtime(_SRC):
+    """Compile dc_oracle.c and cg_oracle.c into libdcoracle.so next to them (gcc, -O2, OpenMP)."""
+    newest = max(os.path.getmtime(_SRC), os.path.getmtime(_SRC_CG))
+    if force or not os.path.exists(_LIB) or os.path.getmtime(_LIB) < newest:
         tmp = _LIB + f".tmp{os.getpid()}"
         subprocess.check_call(["gcc", "-O2", "-fopenmp", "-fPIC", "-shared", "-std=c99",
-                               "-o", tmp, _SRC, "-lm"])
+                               "-o", tmp, _SRC, _SRC_CG, "-lm"])
         os.replace(tmp, _LIB)
     return _LIB
 
@@ -48,6 +50,10 @@ def _load():
         lib.dc_oracle_bwd.restype = ctypes.c_int
         lib.dc_oracle_num_threads.argtypes = []
         lib.dc_oracle_num_threads.restype = ctypes.c_int
+        lib.dc_oracle_cg_fwd.argtypes = [ctypes.c_int64, ctypes.c_int, ctypes.c_int] + [d] * 5
+        lib.dc_oracle_cg_fwd.restype = ctypes.c_int
+        lib.dc_oracle_cg_bwd.argtypes = [ctypes.c_int64, ctypes.c_int, ctypes.c_int] + [d] * 7
+        lib.dc_oracle_cg_bwd.restype = ctypes.c_int
         _lib = lib
     return _lib
 
@@ -109,3 +115,34 @@ def backward(q, k, v, c, g, dO, cu_seqlens, window: int, scale: float):
     if rc != 0:
         raise ValueError(f"dc_oracle_bwd rejected its arguments (rc={rc})")
     return dq, dk, dv, dc, dg
+
+
+def cg_forward(x, w, b):
+    """The assumed producer of c and g (see cg_oracle.c): x [N, D], w [D, 2H], b [2H].
+    Returns (c [N, H], g [N, H]) as float64 numpy arrays."""
+    x, w, b = map(_f64, (x, w, b))
+    N, D = x.shape
+    H = w.shape[1] // 2
+    if w.shape != (D, 2 * H) or b.shape != (2 * H,):
+        raise ValueError("cg_forward: w must be [D, 2H] and b [2H]")
+    c = np.empty((N, H))
+    g = np.empty((N, H))
+    rc = _load().dc_oracle_cg_fwd(N, D, H, _ptr(x), _ptr(w), _ptr(b), _ptr(c), _ptr(g))
+    if rc != 0:
+        raise ValueError(f"dc_oracle_cg_fwd rejected its arguments (rc={rc})")
+    return c, g
+
+
+def cg_backward(x, w, dc, dg):
+    """Gradients of cg_forward for dL/dc = dc, dL/dg = dg.  Returns (dx [N, D], dw [D, 2H],
+    db [2H]) as float64 numpy arrays."""
+    x, w, dc, dg = map(_f64, (x, w, dc, dg))
+    N, D = x.shape
+    H = w.shape[1] // 2
+    dx = np.empty((N, D))
+    dw = np.empty((D, 2 * H))
+    db = np.empty(2 * H)
+    rc = _load().dc_oracle_cg_bwd(N, D, H, _ptr(x), _ptr(w), _ptr(dc), _ptr(dg), _ptr(dx), _ptr(dw), _ptr(db))
+    if rc != 0:
+        raise ValueError(f"dc_oracle_cg_bwd rejected its arguments (rc={rc})")
+    return dx, dw, db
