@@ -13,6 +13,7 @@
 #include "common.cuh"
 #include "simt.cuh"
 #include "tc_host.cuh"
+#include "cg.cuh"
 
 namespace {
 
@@ -405,6 +406,134 @@ dc_status_t dc_attn_bwd_noalloc(const dc_attn_params *params, const void *q, con
     // pass reads it, so nothing left in the array by an earlier call is read.
     return dc_attn_bwd(params, q, k, v, c, g, dO, lse, pmap, dq, dk, dv, dc_, dg, scratch,
                        DC_NOALLOC_SCRATCH_BYTES, stream);
+}
+
+}  // extern "C"
+
+// --------------------------------------------------------------------------
+// Producer of c and g (assumed per-token affine form; kernels in cg.cuh).
+// --------------------------------------------------------------------------
+
+namespace {
+
+dc_status_t check_cg(const dc_cg_params *p, dc::cg::CgShape *s) {
+    if (!p) return DC_ERR_INVALID_ARG;
+    if (p->dtype != DC_F32 && p->dtype != DC_BF16) return DC_ERR_INVALID_ARG;
+    if (p->num_tokens < 0 || p->model_dim < 2 || (p->model_dim & 1) || p->num_heads < 1) return DC_ERR_INVALID_ARG;
+    const int64_t D = p->model_dim;
+    const int64_t sx = p->stride_x ? p->stride_x : D, sdx = p->stride_dx ? p->stride_dx : D;
+    if (sx < D || sdx < D || (sx & 1) || (sdx & 1)) return DC_ERR_INVALID_ARG;
+    if (p->num_heads > 16 || dc::cg::weight_smem_bytes(p->model_dim, p->num_heads) > dc::cg::kMaxWeightSmem)
+        return DC_ERR_UNSUPPORTED;
+    s->N = p->num_tokens;
+    s->D = p->model_dim;
+    s->H = p->num_heads;
+    s->sx = sx;
+    s->sdx = sdx;
+    return DC_OK;
+}
+
+// Blocks of 8 warps for `groups` warp-sized work items: at most two resident blocks per SM.
+unsigned cg_grid(int64_t groups) {
+    const int64_t want = (groups + 7) / 8;
+    return (unsigned)(want < 1 ? 1 : want > 2 * 148 ? 2 * 148 : want);
+}
+
+template <int OUT, typename T>
+cudaError_t cg_fwd_launch(const dc::cg::CgShape &s, const void *x, const float *w, const float *b, float *c, float *g,
+                          cudaStream_t st) {
+    constexpr int TPW = dc::cg::tokens_per_warp(OUT);
+    auto kern = dc::cg::cg_fwd_kernel<T, OUT>;
+    const size_t smem = sizeof(float) * (size_t)OUT * s.D;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    kern<<<cg_grid((s.N + TPW - 1) / TPW), dc::cg::kThreads, smem, st>>>(s, (const T *)x, w, b, c, g);
+    ++t_launches;
+    return cudaGetLastError();
+}
+
+template <int OUT, typename T>
+cudaError_t cg_bwd_launch(const dc::cg::CgShape &s, const void *x, const float *w, const float *dc_, const float *dg,
+                          void *dx, float *dw, float *db, float *part, int blocks, cudaStream_t st) {
+    constexpr int TPW = dc::cg::tokens_per_warp(OUT);
+    if (s.N > 0) {
+        auto kdx = dc::cg::cg_bwd_dx_kernel<T, OUT>;
+        const size_t smem = sizeof(float) * (size_t)OUT * s.D;
+        cudaError_t e = cudaFuncSetAttribute(kdx, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        if (e != cudaSuccess) return e;
+        kdx<<<cg_grid((s.N + TPW - 1) / TPW), dc::cg::kThreads, smem, st>>>(s, w, dc_, dg, (T *)dx);
+        ++t_launches;
+        const int64_t span = (s.N + blocks - 1) / blocks;
+        dc::cg::cg_bwd_dw_partial_kernel<T, OUT><<<blocks, dc::cg::kThreads, 0, st>>>(s, span, (const T *)x, dc_, dg,
+                                                                                     part);
+        ++t_launches;
+    }
+    const int64_t n = dc::cg::record_floats(s.D, s.H);
+    dc::cg::cg_bwd_dw_reduce_kernel<<<(unsigned)((n + 31) / 32), dc::cg::kThreads, 0, st>>>(s, blocks, part, dw, db);
+    ++t_launches;
+    return cudaGetLastError();
+}
+
+template <typename F>
+cudaError_t cg_dispatch(int H, int dtype, F &&f) {
+    switch (dc::cg::out_pad(2 * H)) {
+        case 8: return dtype == DC_F32 ? f.template operator()<8, float>() : f.template operator()<8, __nv_bfloat16>();
+        case 12: return dtype == DC_F32 ? f.template operator()<12, float>() : f.template operator()<12, __nv_bfloat16>();
+        case 16: return dtype == DC_F32 ? f.template operator()<16, float>() : f.template operator()<16, __nv_bfloat16>();
+        case 24: return dtype == DC_F32 ? f.template operator()<24, float>() : f.template operator()<24, __nv_bfloat16>();
+        default: return dtype == DC_F32 ? f.template operator()<32, float>() : f.template operator()<32, __nv_bfloat16>();
+    }
+}
+
+size_t cg_ws_need(const dc::cg::CgShape &s) {
+    if (s.N == 0) return 0;
+    return sizeof(float) * (size_t)dc::cg::partial_blocks(s.N) * (size_t)dc::cg::record_floats(s.D, s.H);
+}
+
+}  // namespace
+
+extern "C" {
+
+dc_status_t dc_attn_cg_fwd(const dc_cg_params *params, const void *x, const float *weight, const float *bias,
+                           float *c, float *g, void *stream) {
+    dc::cg::CgShape s;
+    dc_status_t r = check_cg(params, &s);
+    if (r != DC_OK) return r;
+    t_launches = 0;
+    if (s.N == 0) return DC_OK;
+    r = ptrs_ok({x, weight, bias, c, g}, {});
+    if (r != DC_OK) return r;
+    cudaStream_t st = (cudaStream_t)stream;
+    return cuda_status(cg_dispatch(s.H, params->dtype, [&]<int OUT, typename T>() {
+        return cg_fwd_launch<OUT, T>(s, x, weight, bias, c, g, st);
+    }));
+}
+
+size_t dc_attn_cg_bwd_workspace_size(const dc_cg_params *params) {
+    dc::cg::CgShape s;
+    if (check_cg(params, &s) != DC_OK) return 0;
+    return cg_ws_need(s);
+}
+
+dc_status_t dc_attn_cg_bwd(const dc_cg_params *params, const void *x, const float *weight, const float *dc_,
+                           const float *dg, void *dx, float *dweight, float *dbias, void *workspace,
+                           size_t workspace_bytes, void *stream) {
+    dc::cg::CgShape s;
+    dc_status_t r = check_cg(params, &s);
+    if (r != DC_OK) return r;
+    t_launches = 0;
+    r = ptrs_ok({dweight, dbias}, {});
+    if (r != DC_OK) return r;
+    if (s.N > 0) {
+        r = ptrs_ok({x, weight, dc_, dg, dx, workspace}, {});
+        if (r != DC_OK) return r;
+        if (workspace_bytes < cg_ws_need(s)) return DC_ERR_INVALID_ARG;
+    }
+    const int blocks = s.N > 0 ? dc::cg::partial_blocks(s.N) : 0;
+    cudaStream_t st = (cudaStream_t)stream;
+    return cuda_status(cg_dispatch(s.H, params->dtype, [&]<int OUT, typename T>() {
+        return cg_bwd_launch<OUT, T>(s, x, weight, dc_, dg, dx, dweight, dbias, (float *)workspace, blocks, st);
+    }));
 }
 
 }  // extern "C"

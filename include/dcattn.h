@@ -228,6 +228,61 @@ int32_t dc_attn_last_launch_count(void);
 dc_status_t dc_attn_set_wait_limit(uint32_t ns);
 dc_status_t dc_attn_inject_missing_load(void);
 
+/* ------------------------------------------------------------------------
+ * Producer of c and g.
+ *
+ * The page's DCMHA paragraph says only that the heads' combination is decided
+ * dynamically from the current input; it gives no formula.  These entry
+ * points implement the plainest reading, an ASSUMED form: per-token affine maps
+ * of the layer's hidden state x [N][D], with no nonlinearity.  For token t,
+ * head h < H and weight [2H][D] (row o produces output o, the layout of a
+ * linear layer's weight), bias [2H]:
+ *
+ *   c[t,h] = bias[h]     + sum_k x[t,k] * weight[h][k]
+ *   g[t,h] = bias[H + h] + sum_k x[t,k] * weight[H + h][k]
+ *
+ * The sums are taken in fp32 (x converted from `dtype`); c, g feed
+ * dc_attn_fwd directly.  Shapes: x, dx [N][D] in `dtype`, consecutive tokens
+ * stride_x / stride_dx elements apart (0 = D); weight, dweight [2H][D] fp32
+ * contiguous; bias, dbias [2H] fp32; c, g, dc, dg [N][H] fp32 contiguous.
+ * Limits: D even; strides even and >= D; 1 <= H <= 16 (larger H returns
+ * DC_ERR_UNSUPPORTED), and the weight padded to 8, 12, 16, 24 or 32 rows must
+ * fit 200 KB of shared memory (e.g. D <= 4266 at H = 6, D <= 1600 at H = 16;
+ * beyond that DC_ERR_UNSUPPORTED).  Pointers: device, 16-byte aligned,
+ * caller-owned; asynchronous on `stream`; outputs overwritten.
+ * ------------------------------------------------------------------------ */
+typedef struct {
+    int32_t dtype;        /* dc_dtype_t of x and dx                                   */
+    int32_t model_dim;    /* D                                                        */
+    int32_t num_heads;    /* H                                                        */
+    int32_t reserved;     /* set to 0                                                 */
+    int64_t num_tokens;   /* N >= 0                                                   */
+    int64_t stride_x;     /* elements between tokens of x (0 = D)                     */
+    int64_t stride_dx;    /* elements between tokens of dx (0 = D)                    */
+} dc_cg_params;
+
+/* c, g from x.  N = 0 launches nothing. */
+dc_status_t dc_attn_cg_fwd(const dc_cg_params *params, const void *x, const float *weight, const float *bias,
+                           float *c, float *g, void *stream);
+
+/* Bytes of workspace dc_attn_cg_bwd needs (0 when N = 0 or the params are
+ * invalid): one fp32 partial record of dweight and dbias per block of tokens. */
+size_t dc_attn_cg_bwd_workspace_size(const dc_cg_params *params);
+
+/* Gradients for dL/dc = dc, dL/dg = dg, writing e[t] = (dc[t,:], dg[t,:]):
+ *
+ *   dx[t,k]       = sum_o e[t,o] * weight[o][k]
+ *   dweight[o][k] = sum_t e[t,o] * x[t,k]        dbias[o] = sum_t e[t,o]
+ *
+ * dweight and dbias are summed over fixed token ranges and then over the
+ * ranges in a fixed order: the result is bitwise reproducible for a given N.
+ * With N = 0 only dweight and dbias are written (zeros) and the other pointers
+ * may be NULL.  workspace_bytes below dc_attn_cg_bwd_workspace_size returns
+ * DC_ERR_INVALID_ARG. */
+dc_status_t dc_attn_cg_bwd(const dc_cg_params *params, const void *x, const float *weight, const float *dc,
+                           const float *dg, void *dx, float *dweight, float *dbias, void *workspace,
+                           size_t workspace_bytes, void *stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -163,3 +163,55 @@ def test_accepts_fused_projection_strides(lib):
     call then stops at the device pointers, which are not real (N = 0 would skip them)."""
     p = _params(stride_qkv=3 * 768, stride_dqkv=3 * 768, stride_o=2 * 768, total_tokens=0)
     assert _fwd(lib, p) == dcattn.DC_OK
+
+
+def _cg(**kw):
+    base = dict(dtype=dcattn.DC_BF16, model_dim=768, num_heads=6, reserved=0, num_tokens=1000, stride_x=0,
+                stride_dx=0)
+    base.update(kw)
+    return dcattn.CgParams(**base)
+
+
+@pytest.mark.parametrize("kw, expect", [
+    (dict(dtype=7), dcattn.DC_ERR_INVALID_ARG),
+    (dict(model_dim=767), dcattn.DC_ERR_INVALID_ARG),      # D must be even
+    (dict(model_dim=0), dcattn.DC_ERR_INVALID_ARG),
+    (dict(num_heads=0), dcattn.DC_ERR_INVALID_ARG),
+    (dict(num_tokens=-1), dcattn.DC_ERR_INVALID_ARG),
+    (dict(stride_x=770 + 1), dcattn.DC_ERR_INVALID_ARG),   # odd stride
+    (dict(stride_x=766), dcattn.DC_ERR_INVALID_ARG),       # below D
+    (dict(stride_dx=-768), dcattn.DC_ERR_INVALID_ARG),
+    (dict(num_heads=17), dcattn.DC_ERR_UNSUPPORTED),
+    (dict(model_dim=4268), dcattn.DC_ERR_UNSUPPORTED),     # 12 weight rows of 4268 floats > 200 KB
+    (dict(num_heads=16, model_dim=1602), dcattn.DC_ERR_UNSUPPORTED),
+])
+def test_cg_bad_params_rejected_on_host(lib, kw, expect):
+    p = _cg(**kw)
+    a = 0x4000
+    assert lib.dc_attn_cg_fwd(ctypes.byref(p), a, a, a, a, a, None) == expect
+    assert lib.dc_attn_cg_bwd(ctypes.byref(p), a, a, a, a, a, a, a, a, 1 << 30, None) == expect
+    assert lib.dc_attn_cg_bwd_workspace_size(ctypes.byref(p)) == 0
+
+
+def test_cg_limits_accepted(lib):
+    """The largest shapes inside the limits pass the host checks (N = 0: nothing runs)."""
+    for D, H in ((4266, 6), (1600, 16), (2, 1), (6400, 4)):
+        p = _cg(model_dim=D, num_heads=H, num_tokens=0)
+        assert lib.dc_attn_cg_fwd(ctypes.byref(p), 0, 0, 0, 0, 0, None) == dcattn.DC_OK, (D, H)
+
+
+def test_cg_workspace_and_pointer_checks(lib):
+    p = _cg()
+    need = lib.dc_attn_cg_bwd_workspace_size(ctypes.byref(p))
+    assert need == 4 * 16 * (12 * 768 + 12)            # ceil(1000 / 64) records of dweight + dbias
+    p_big = _cg(num_tokens=10 ** 7)
+    assert lib.dc_attn_cg_bwd_workspace_size(ctypes.byref(p_big)) == 4 * 296 * (12 * 768 + 12)
+    a = 0x4000
+    assert lib.dc_attn_cg_bwd(ctypes.byref(p), a, a, a, a, a, a, a, a, need - 1, None) == dcattn.DC_ERR_INVALID_ARG
+    assert lib.dc_attn_cg_fwd(ctypes.byref(p), a + 8, a, a, a, a, None) == dcattn.DC_ERR_INVALID_ARG
+    assert lib.dc_attn_cg_fwd(ctypes.byref(p), a, a, a, 0, a, None) == dcattn.DC_ERR_INVALID_ARG
+    p0 = _cg(num_tokens=0)
+    assert lib.dc_attn_cg_bwd_workspace_size(ctypes.byref(p0)) == 0
+    assert lib.dc_attn_cg_fwd(ctypes.byref(p0), 0, 0, 0, 0, 0, None) == dcattn.DC_OK
+    # N = 0 still writes dweight and dbias (zeros), so those two must be valid
+    assert lib.dc_attn_cg_bwd(ctypes.byref(p0), 0, 0, 0, 0, 0, 0, 0, 0, 0, None) == dcattn.DC_ERR_INVALID_ARG

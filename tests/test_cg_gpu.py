@@ -1,0 +1,152 @@
+"""GPU parity of the c/g producer (dc_attn_cg_fwd, dc_attn_cg_bwd) against the fp64 oracle.
+
+Tolerances come from the arithmetic: every output is a sum of products taken in fp32
+(x converted exactly from bf16), so its error is at most gamma_n * sum |terms| with
+gamma_n = n * 2^-24 / (1 - n * 2^-24) and n the longest chain of additions.  The
+kernels' chains: forward D/64 pair steps + a 5-level warp tree; dx 2H terms; dweight
+and dbias at most 64 tokens per partial record, the records added in strided order (at
+most blocks / 8 + 8 additions).  The oracle run on |x|, |w|, |e| gives sum |terms|.
+A bf16 dx adds its own rounding, 2^-9 of the value.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from cross_head_dynamic_b200 import dcattn
+from cross_head_dynamic_b200.inputs import cg_problem
+
+pytestmark = pytest.mark.gpu
+
+U = 2.0 ** -24
+
+
+def gamma(n):
+    return n * U / (1 - n * U)
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _setup():
+    oracle.build()
+    dcattn.load_library()
+
+
+def _to_np(t):
+    return t.detach().double().cpu().numpy()
+
+
+def _run(p, dtype):
+    dev = "cuda"
+    x = p["x"].to(dev)
+    w = p["w"].to(dev).t().contiguous()      # weight [2H][D]
+    b = p["b"].to(dev)
+    dc, dg = p["dc"].to(dev), p["dg"].to(dev)
+    c, g = dcattn.dc_attn_cg_fwd(x, w, b)
+    dx, dw, db = dcattn.dc_attn_cg_bwd(x, w, dc, dg)
+    torch.cuda.synchronize()
+    return c, g, dx, dw, db
+
+
+def _check(p, outs, dtype):
+    c, g, dx, dw, db = (_to_np(t) for t in outs)
+    x, w, b = _to_np(p["x"]), _to_np(p["w"]), _to_np(p["b"])
+    dcn, dgn = _to_np(p["dc"]), _to_np(p["dg"])
+    N, D = x.shape
+    H = dcn.shape[1]
+    rc, rg = oracle.cg_forward(x, w, b)
+    mc, mg = oracle.cg_forward(np.abs(x), np.abs(w), np.abs(b))
+    tf = gamma(D // 64 + 8)
+    assert np.all(np.abs(c - rc) <= tf * mc + 1e-30), np.abs(c - rc).max()
+    assert np.all(np.abs(g - rg) <= tf * mg + 1e-30), np.abs(g - rg).max()
+    rdx, rdw, rdb = oracle.cg_backward(x, w, dcn, dgn)
+    mdx, mdw, mdb = oracle.cg_backward(np.abs(x), np.abs(w), np.abs(dcn), np.abs(dgn))
+    tol_dx = gamma(2 * H + 2) * mdx + (2.0 ** -8 * np.abs(rdx) if dtype == "bf16" else 0) + 1e-30
+    assert np.all(np.abs(dx - rdx) <= tol_dx), np.abs(dx - rdx).max()
+    blocks = min(max((N + 63) // 64, 1), 296)
+    tw = gamma(64 + blocks // 8 + 9)
+    assert np.all(np.abs(dw.T - rdw) <= tw * mdw + 1e-30), np.abs(dw.T - rdw).max()
+    assert np.all(np.abs(db - rdb) <= tw * mdb + 1e-30), np.abs(db - rdb).max()
+
+
+@pytest.mark.parametrize("N, D, H, dtype", [
+    (4096, 768, 6, "bf16"),      # GPT-2 small width, several blocks and a full grid
+    (1000, 768, 6, "f32"),
+    (333, 64, 1, "bf16"),        # 2H = 2 padded to 8, D below one 64-element pass
+    (77, 130, 3, "f32"),         # ragged D (not a multiple of 64), ragged N
+    (517, 256, 16, "bf16"),      # 2H = 32, two tokens per warp
+    (129, 512, 12, "bf16"),      # 2H = 24
+    (640, 96, 8, "f32"),         # 2H = 16
+    (5, 2, 4, "bf16"),           # D = 2: one pair, most lanes idle
+    (1, 768, 6, "bf16"),         # one token
+    (65, 768, 5, "bf16"),        # 2H = 10 padded to 12; one record boundary crossed
+])
+def test_cg_parity(N, D, H, dtype):
+    p = cg_problem(100 + N + D + H, N, D, H, dtype)
+    _check(p, _run(p, dtype), dtype)
+
+
+def test_cg_gpt2_full_size():
+    """The GPT-2 training shape: 16384 tokens (8 x 2048), D = 768, H = 6, every output."""
+    p = cg_problem(7, 16384, 768, 6, "bf16")
+    _check(p, _run(p, "bf16"), "bf16")
+
+
+def test_cg_backward_is_deterministic():
+    p = cg_problem(8, 20000, 768, 6, "bf16")
+    a = _run(p, "bf16")
+    b = _run(p, "bf16")
+    for u, v in zip(a, b):
+        assert torch.equal(u, v)
+
+
+def test_cg_zero_tokens_writes_zero_gradients():
+    dev = "cuda"
+    x = torch.empty(0, 64, device=dev, dtype=torch.bfloat16)
+    w = torch.randn(8, 64, device=dev)
+    dw = torch.full((8, 64), 7.0, device=dev)
+    db = torch.full((8,), 7.0, device=dev)
+    e = torch.empty(0, 4, device=dev)
+    c, g = dcattn.dc_attn_cg_fwd(x, w, torch.zeros(8, device=dev))
+    assert c.shape == (0, 4)
+    dx, dw, db = dcattn.dc_attn_cg_bwd(x, w, e, e, dweight=dw, dbias=db)
+    torch.cuda.synchronize()
+    assert not dw.any() and not db.any()
+
+
+def test_cg_strided_rows():
+    """x a column slice of a wider hidden-state buffer, dx written into a wider buffer:
+    results equal those of contiguous tensors, and the gap columns stay untouched."""
+    p = cg_problem(9, 700, 256, 6, "bf16")
+    dev = "cuda"
+    base = torch.randn(700, 256 + 10, device=dev).to(torch.bfloat16)
+    base[:, 8:264] = p["x"].to(dev)          # 16-byte aligned start; rows 532 bytes apart
+    xs = base[:, 8:264]
+    w = p["w"].to(dev).t().contiguous()
+    b = p["b"].to(dev)
+    dc, dg = p["dc"].to(dev), p["dg"].to(dev)
+    dxbuf = torch.full((700, 256 + 16), 3.0, device=dev, dtype=torch.bfloat16)
+    c, g = dcattn.dc_attn_cg_fwd(xs, w, b)
+    dx, dw, db = dcattn.dc_attn_cg_bwd(xs, w, dc, dg, dx=dxbuf[:, 8:264])
+    ref = _run(p, "bf16")
+    torch.cuda.synchronize()
+    for u, v in zip((c, g, dxbuf[:, 8:264], dw, db), ref):
+        assert torch.equal(u, v)
+    assert bool((dxbuf[:, :8] == 3).all()) and bool((dxbuf[:, 264:] == 3).all())
+
+
+def test_cg_feeds_the_attention_forward():
+    """x -> (c, g) -> windowed attention, against the oracle chain in fp64."""
+    N, D, H, d, W = 600, 256, 4, 64, 112
+    p = cg_problem(10, N, D, H, "bf16")
+    dev = "cuda"
+    gen = torch.Generator().manual_seed(11)
+    q, k, v = (torch.randn(N, H, d, generator=gen).to(torch.bfloat16) for _ in range(3))
+    cu = torch.tensor([0, 250, 600], dtype=torch.int32)
+    c, g = dcattn.dc_attn_cg_fwd(p["x"].to(dev), p["w"].to(dev).t().contiguous(), p["b"].to(dev))
+    scale = d ** -0.5
+    o, _, _ = dcattn.dc_attn_fwd(q.to(dev), k.to(dev), v.to(dev), c, g, cu.to(dev), W, scale)
+    torch.cuda.synchronize()
+    rc, rg = oracle.cg_forward(_to_np(p["x"]), _to_np(p["w"]), _to_np(p["b"]))
+    ro = oracle.forward(_to_np(q), _to_np(k), _to_np(v), rc, rg, cu.numpy(), W, scale)[0]
+    err = np.abs(_to_np(o) - ro)
+    assert err.max() <= 0.02 * np.abs(ro).max(), err.max()
