@@ -423,8 +423,10 @@ dc_status_t check_cg(const dc_cg_params *p, dc::cg::CgShape *s) {
     const int64_t D = p->model_dim;
     const int64_t sx = p->stride_x ? p->stride_x : D, sdx = p->stride_dx ? p->stride_dx : D;
     if (sx < D || sdx < D || (sx & 1) || (sdx & 1)) return DC_ERR_INVALID_ARG;
-    if (p->num_heads > 16 || dc::cg::weight_smem_bytes(p->model_dim, p->num_heads) > dc::cg::kMaxWeightSmem)
-        return DC_ERR_UNSUPPORTED;
+    if (p->num_heads > 16) return DC_ERR_UNSUPPORTED;
+    const size_t smem = p->dtype == DC_F32 ? dc::cg::fwd_smem_bytes<float>(p->model_dim, p->num_heads)
+                                           : dc::cg::fwd_smem_bytes<__nv_bfloat16>(p->model_dim, p->num_heads);
+    if (smem > dc::cg::kMaxSmem) return DC_ERR_UNSUPPORTED;
     s->N = p->num_tokens;
     s->D = p->model_dim;
     s->H = p->num_heads;
@@ -439,15 +441,22 @@ unsigned cg_grid(int64_t groups) {
     return (unsigned)(want < 1 ? 1 : want > 2 * 148 ? 2 * 148 : want);
 }
 
+// 16-byte copies when every row of x starts on a 16-byte boundary and spans whole 16-byte units.
+template <typename T>
+int cg_vec16(const dc::cg::CgShape &s, const void *x) {
+    return (uintptr_t)x % 16 == 0 && (s.sx * (int64_t)sizeof(T)) % 16 == 0 && (s.D * sizeof(T)) % 16 == 0;
+}
+
 template <int OUT, typename T>
 cudaError_t cg_fwd_launch(const dc::cg::CgShape &s, const void *x, const float *w, const float *b, float *c, float *g,
                           cudaStream_t st) {
     constexpr int TPW = dc::cg::tokens_per_warp(OUT);
     auto kern = dc::cg::cg_fwd_kernel<T, OUT>;
-    const size_t smem = sizeof(float) * (size_t)OUT * s.D;
+    const size_t smem = dc::cg::fwd_smem_bytes<T>(s.D, s.H);
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
-    kern<<<cg_grid((s.N + TPW - 1) / TPW), dc::cg::kThreads, smem, st>>>(s, (const T *)x, w, b, c, g);
+    kern<<<cg_grid((s.N + TPW - 1) / TPW), dc::cg::kThreads, smem, st>>>(s, (const T *)x, w, b, c, g,
+                                                                        cg_vec16<T>(s, x));
     ++t_launches;
     return cudaGetLastError();
 }
@@ -458,18 +467,23 @@ cudaError_t cg_bwd_launch(const dc::cg::CgShape &s, const void *x, const float *
     constexpr int TPW = dc::cg::tokens_per_warp(OUT);
     if (s.N > 0) {
         auto kdx = dc::cg::cg_bwd_dx_kernel<T, OUT>;
-        const size_t smem = sizeof(float) * (size_t)OUT * s.D;
+        const size_t smem = dc::cg::weight_smem_bytes(s.D, s.H);
         cudaError_t e = cudaFuncSetAttribute(kdx, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
         if (e != cudaSuccess) return e;
         kdx<<<cg_grid((s.N + TPW - 1) / TPW), dc::cg::kThreads, smem, st>>>(s, w, dc_, dg, (T *)dx);
         ++t_launches;
+        auto kdw = dc::cg::cg_bwd_dw_partial_kernel<T, OUT>;
+        const int chunk = dc::cg::dw_chunk(s.D, s.H, sizeof(T));
+        const size_t dsmem = dc::cg::dw_smem_bytes(s.D, s.H, sizeof(T));
+        e = cudaFuncSetAttribute(kdw, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)dsmem);
+        if (e != cudaSuccess) return e;
         const int64_t span = (s.N + blocks - 1) / blocks;
-        dc::cg::cg_bwd_dw_partial_kernel<T, OUT><<<blocks, dc::cg::kThreads, 0, st>>>(s, span, (const T *)x, dc_, dg,
-                                                                                     part);
+        kdw<<<blocks, dc::cg::kDwThreads, dsmem, st>>>(s, span, chunk, (const T *)x, dc_, dg, part, cg_vec16<T>(s, x));
         ++t_launches;
     }
     const int64_t n = dc::cg::record_floats(s.D, s.H);
-    dc::cg::cg_bwd_dw_reduce_kernel<<<(unsigned)((n + 31) / 32), dc::cg::kThreads, 0, st>>>(s, blocks, part, dw, db);
+    dc::cg::cg_bwd_dw_reduce_kernel<<<(unsigned)((n + 31) / 32), dc::cg::kReduceThreads, 0, st>>>(s, blocks, part, dw,
+                                                                                                db);
     ++t_launches;
     return cudaGetLastError();
 }

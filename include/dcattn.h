@@ -246,9 +246,11 @@ dc_status_t dc_attn_inject_missing_load(void);
  * stride_x / stride_dx elements apart (0 = D); weight, dweight [2H][D] fp32
  * contiguous; bias, dbias [2H] fp32; c, g, dc, dg [N][H] fp32 contiguous.
  * Limits: D even; strides even and >= D; 1 <= H <= 16 (larger H returns
- * DC_ERR_UNSUPPORTED), and the weight padded to 8, 12, 16, 24 or 32 rows must
- * fit 200 KB of shared memory (e.g. D <= 4266 at H = 6, D <= 1600 at H = 16;
- * beyond that DC_ERR_UNSUPPORTED).  Pointers: device, 16-byte aligned,
+ * DC_ERR_UNSUPPORTED).  The forward keeps in shared memory the weight padded
+ * to OUT rows (OUT = 8, 12, 16, 24 or 32, the first >= 2H; 4 * (OUT + 2) * D
+ * bytes) and 8 warps x 6 stages x 64/OUT tokens x 64 elements of x; the two
+ * must fit 227 KB, else DC_ERR_UNSUPPORTED (D <= 3602 at H = 6 in bf16, 3052
+ * in fp32; D <= 1618 at H = 16 in bf16).  Pointers: device, 16-byte aligned,
  * caller-owned; asynchronous on `stream`; outputs overwritten.
  * ------------------------------------------------------------------------ */
 typedef struct {

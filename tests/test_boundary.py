@@ -182,8 +182,9 @@ def _cg(**kw):
     (dict(stride_x=766), dcattn.DC_ERR_INVALID_ARG),       # below D
     (dict(stride_dx=-768), dcattn.DC_ERR_INVALID_ARG),
     (dict(num_heads=17), dcattn.DC_ERR_UNSUPPORTED),
-    (dict(model_dim=4268), dcattn.DC_ERR_UNSUPPORTED),     # 12 weight rows of 4268 floats > 200 KB
-    (dict(num_heads=16, model_dim=1602), dcattn.DC_ERR_UNSUPPORTED),
+    (dict(model_dim=3604), dcattn.DC_ERR_UNSUPPORTED),     # weight + x stages above 227 KB
+    (dict(model_dim=3054, dtype=dcattn.DC_F32), dcattn.DC_ERR_UNSUPPORTED),
+    (dict(num_heads=16, model_dim=1620), dcattn.DC_ERR_UNSUPPORTED),
 ])
 def test_cg_bad_params_rejected_on_host(lib, kw, expect):
     p = _cg(**kw)
@@ -195,9 +196,10 @@ def test_cg_bad_params_rejected_on_host(lib, kw, expect):
 
 def test_cg_limits_accepted(lib):
     """The largest shapes inside the limits pass the host checks (N = 0: nothing runs)."""
-    for D, H in ((4266, 6), (1600, 16), (2, 1), (6400, 4)):
-        p = _cg(model_dim=D, num_heads=H, num_tokens=0)
-        assert lib.dc_attn_cg_fwd(ctypes.byref(p), 0, 0, 0, 0, 0, None) == dcattn.DC_OK, (D, H)
+    for D, H, dt in ((3602, 6, dcattn.DC_BF16), (3052, 6, dcattn.DC_F32), (1618, 16, dcattn.DC_BF16), (2, 1, 0),
+                     (4582, 4, dcattn.DC_BF16)):
+        p = _cg(model_dim=D, num_heads=H, num_tokens=0, dtype=dt)
+        assert lib.dc_attn_cg_fwd(ctypes.byref(p), 0, 0, 0, 0, 0, None) == dcattn.DC_OK, (D, H, dt)
 
 
 def test_cg_workspace_and_pointer_checks(lib):
@@ -205,7 +207,7 @@ def test_cg_workspace_and_pointer_checks(lib):
     need = lib.dc_attn_cg_bwd_workspace_size(ctypes.byref(p))
     assert need == 4 * 16 * (12 * 768 + 12)            # ceil(1000 / 64) records of dweight + dbias
     p_big = _cg(num_tokens=10 ** 7)
-    assert lib.dc_attn_cg_bwd_workspace_size(ctypes.byref(p_big)) == 4 * 296 * (12 * 768 + 12)
+    assert lib.dc_attn_cg_bwd_workspace_size(ctypes.byref(p_big)) == 4 * 148 * (12 * 768 + 12)
     a = 0x4000
     assert lib.dc_attn_cg_bwd(ctypes.byref(p), a, a, a, a, a, a, a, a, need - 1, None) == dcattn.DC_ERR_INVALID_ARG
     assert lib.dc_attn_cg_fwd(ctypes.byref(p), a + 8, a, a, a, a, None) == dcattn.DC_ERR_INVALID_ARG
