@@ -11,16 +11,15 @@
 //   dx[t,k] = sum_o e[t,o] weight[o][k],  dweight[o][k] = sum_t e[t,o] x[t,k],  dbias[o] = sum_t e[t,o]
 //
 // The map reads x once (1.5 KB per token at D = 768 in bf16) and does 2H FMAs per element
-// of x: at 2H = 12 the FMA issue of the CUDA cores and the HBM stream take about the same
-// time, so the kernels are written to spend few instructions per FMA.  They use the
-// packed fma.rn.f32x2 of sm_100 (two IEEE fp32 FMAs, each rounded to nearest, so the
-// result is that of two scalar FMAs in the same order), keep the weight in shared memory
-// and move x through shared memory with asynchronous copies.
+// of x, an fp32 FMA count on the CUDA cores that takes about as long as the HBM stream at
+// 2H = 12, so the kernels spend few instructions per FMA: they use the packed fma.rn.f32x2
+// of sm_100 (two IEEE fp32 FMAs, each rounded to nearest, so the result is that of two
+// scalar FMAs in the same order) on pairs of adjacent columns, with the weight in shared
+// memory read as broadcasts.  The forward and dx give each lane whole tokens (no
+// reduction across lanes); dweight gives each thread column pairs and walks the tokens.
 //
 // Outputs are padded to OUT in {8, 12, 16, 24, 32} (>= 2H; padded weight rows and padded
-// entries of e are zero).  The weight sits in shared memory as pair-rows: pair-row p holds
-// weight[0..OUT-1][2p] then weight[0..OUT-1][2p + 1], padded to kWRow(OUT) floats so that
-// the 32 lanes' 16-byte reads of consecutive pair-rows hit distinct banks.
+// entries of e are zero).
 //
 // dweight and dbias are reduced deterministically: each block of the partial kernel sums
 // a fixed token range into its own record of the workspace; the reduce kernel adds the
@@ -33,12 +32,11 @@
 namespace dc {
 namespace cg {
 
-constexpr int kThreads = 256;             // forward and dx blocks: 8 warps
+constexpr int kThreads = 256;             // forward and dx blocks: 8 warps, one per column slice
 constexpr int kDwThreads = 384;           // dweight partial blocks: 12 warps
 __host__ __device__ constexpr int dw_units(int OUT) { return OUT <= 12 ? 2 : 1; }   // column pairs per thread, per pass
 constexpr size_t kMaxSmem = 227 * 1024;   // dynamic shared memory a block may have
 constexpr size_t kDwStageBudget = 100 * 1024;   // one of the dweight kernel's two stages
-constexpr int kStages = 6;                // depth of each warp's ring of x stages in the forward
 constexpr int kReduceThreads = 512;
 
 struct CgShape {
@@ -50,19 +48,6 @@ struct CgShape {
 };
 
 __host__ __device__ constexpr int out_pad(int H2) { return H2 <= 8 ? 8 : H2 <= 12 ? 12 : H2 <= 16 ? 16 : H2 <= 24 ? 24 : 32; }
-__host__ __device__ constexpr int tokens_per_warp(int OUT) { return 64 / OUT; }
-__host__ __device__ constexpr int kWRow(int OUT) { return 2 * OUT + 4; }
-__host__ __device__ inline size_t weight_smem_bytes(int D, int H) {
-    return sizeof(float) * (size_t)(D / 2) * kWRow(out_pad(2 * H));
-}
-
-// Shared memory of the forward: the weight, then per warp kStages stages of TPW x 64
-// elements of x.
-template <typename T>
-__host__ __device__ inline size_t fwd_smem_bytes(int D, int H) {
-    const int OUT = out_pad(2 * H);
-    return weight_smem_bytes(D, H) + sizeof(T) * (size_t)(kThreads / 32) * kStages * tokens_per_warp(OUT) * 64;
-}
 
 // Tokens per stage of the dweight kernel, and its shared memory (two stages of x rows
 // and of e rows stored as broadcast pairs (e, e)).
@@ -87,17 +72,6 @@ inline int partial_blocks(int64_t N) {
     return (int)(want < 1 ? 1 : want > kMaxPartials ? kMaxPartials : want);
 }
 __host__ __device__ inline int64_t record_floats(int D, int H) { return (int64_t)2 * H * D + 2 * H; }
-
-template <typename T> __device__ __forceinline__ float2 ld2(const T *p);
-template <> __device__ __forceinline__ float2 ld2<float>(const float *p) { return *reinterpret_cast<const float2 *>(p); }
-template <> __device__ __forceinline__ float2 ld2<__nv_bfloat16>(const __nv_bfloat16 *p) {
-    return __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(p));
-}
-template <typename T> __device__ __forceinline__ void st2(T *p, float2 v);
-template <> __device__ __forceinline__ void st2<float>(float *p, float2 v) { *reinterpret_cast<float2 *>(p) = v; }
-template <> __device__ __forceinline__ void st2<__nv_bfloat16>(__nv_bfloat16 *p, float2 v) {
-    *reinterpret_cast<__nv_bfloat162 *>(p) = __floats2bfloat162_rn(v.x, v.y);
-}
 
 // Packed pairs of fp32 live in 64-bit registers (low half first), so that the register
 // allocator keeps each pair in an aligned register pair and the packed FMA needs no moves.
@@ -126,13 +100,6 @@ template <> __device__ __forceinline__ f2reg ldpair<__nv_bfloat16>(const __nv_bf
     const unsigned w = *reinterpret_cast<const unsigned *>(p);
     return pack2(__uint_as_float(w << 16), __uint_as_float(w & 0xffff0000u));
 }
-// The two elements of a pair, each broadcast to both halves.
-__device__ __forceinline__ void split_bcast(f2reg v, f2reg &lo, f2reg &hi) {
-    const float2 f = unpack2(v);
-    lo = pack2(f.x, f.x);
-    hi = pack2(f.y, f.y);
-}
-
 // Asynchronous global -> shared copies (cp.async; completion per thread, by group).
 __device__ __forceinline__ void cp_async16(void *dst, const void *src) {
     const unsigned d = (unsigned)__cvta_generic_to_shared(dst);
@@ -146,263 +113,279 @@ __device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commi
 template <int N>
 __device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;\n" ::"n"(N) : "memory"); }
 
-// weight [2H][D] into the pair-row layout, as 4-byte asynchronous copies (rows 2H..OUT-1
-// zero), committed as one group.  Reads are coalesced along k.
+// ---------------------------------------------------------------------------------------
+// Forward and dx: one lane per token.  A block's 8 warps split the D columns into 8 slices
+// (slice_cols each, a multiple of the item width); a tile is the 32 * TPL tokens of one
+// block, lane l holding tokens l, l + 32 (TPL = 2, or 1 when OUT > 12).  An item is 32
+// bytes of each of the lane's rows (16 bf16 or 8 fp32 columns).  The weight sits in shared
+// memory as column pairs, wp[p * OUT + o] = (weight[o][2p], weight[o][2p + 1]); every lane of
+// a warp reads the same entry (a broadcast).
+// ---------------------------------------------------------------------------------------
+
+__host__ __device__ constexpr int tok_per_lane(int OUT) { return OUT <= 12 ? 2 : 1; }
+__host__ __device__ constexpr int tile_tokens(int OUT) { return 32 * tok_per_lane(OUT); }
+__host__ __device__ inline int slice_cols(int D, int esize) {
+    const int ic = 32 / esize;               // item width in columns
+    const int per = (D + 7) / 8;
+    return (per + ic - 1) / ic * ic;
+}
+__host__ __device__ inline size_t wp_bytes(int D, int H) { return sizeof(float) * (size_t)D * out_pad(2 * H); }
+// Forward: the weight pairs, then the 8 slices' partial sums of one tile [8][OUT][tile].
+__host__ __device__ inline size_t fwd_smem_bytes(int D, int H) {
+    const int OUT = out_pad(2 * H);
+    return wp_bytes(D, H) + sizeof(float) * 8 * (size_t)OUT * tile_tokens(OUT);
+}
+
+// weight [2H][D] into the column-pair layout (outputs 2H..OUT-1 zero); the caller
+// synchronizes the block before use.
 template <int OUT>
-__device__ __forceinline__ void stage_weight(const CgShape &s, const float *__restrict__ weight, float *ws) {
-    constexpr int WR = kWRow(OUT);
-#pragma unroll 1
-    for (int o = 0; o < OUT; ++o) {
-        const float *src = weight + (int64_t)o * s.D;
-        for (int k = threadIdx.x; k < s.D; k += blockDim.x) {
-            float *dst = ws + (k >> 1) * WR + (k & 1) * OUT + o;
-            if (o < 2 * s.H)
-                cp_async4(dst, src + k);
-            else
-                *dst = 0.f;
-        }
-    }
-    cp_async_commit();
-}
-
-// One reduce-scatter step over the warp: lanes that differ in bit HALF/2 exchange halves
-// of their first 2 * HALF slots; each keeps the sum of one half in slots [0, HALF).
-template <int HALF>
-__device__ __forceinline__ void rs_step(float (&v)[64], int lane) {
-    const bool up = (lane & (HALF / 2)) != 0;
+__device__ __forceinline__ void stage_weight_pairs(const CgShape &s, const float *__restrict__ weight, f2reg *wp) {
+    const int H2 = 2 * s.H;
+    if ((s.D & 3) == 0) {
+        const int q4 = s.D / 4;
 #pragma unroll
-    for (int i = 0; i < HALF; ++i) {
-        const float keep = up ? v[i + HALF] : v[i];
-        const float send = up ? v[i] : v[i + HALF];
-        v[i] = keep + __shfl_xor_sync(0xffffffffu, send, HALF / 2);
-    }
-}
-// After the five steps lane l holds in v[0], v[1] the warp-wide sums of slots 2l, 2l + 1
-// (the halves kept are chosen by the lane's bits from the highest down, so the slot
-// index of v[j] is 2 * l + j).  62 shuffles for 64 sums.
-__device__ __forceinline__ void reduce_scatter64(float (&v)[64], int lane) {
-    rs_step<32>(v, lane);
-    rs_step<16>(v, lane);
-    rs_step<8>(v, lane);
-    rs_step<4>(v, lane);
-    rs_step<2>(v, lane);
-}
-
-// Elements [k0, k0 + 64) of TPW consecutive x rows (rows past N zero-filled) into one ring
-// stage [TPW][64].  vec16: every row start is 16-byte aligned and D * sizeof(T) is a
-// multiple of 16, so 16-byte copies cover the rows exactly; otherwise 4-byte copies.
-template <typename T, int TPW>
-__device__ __forceinline__ void copy_stage(const CgShape &s, const T *__restrict__ x, int64_t t0, int k0, T *st,
-                                           int lane, bool vec16) {
-    const int kn = s.D - k0 < 64 ? s.D - k0 : 64;
-    if (vec16) {
-        constexpr int E = 16 / (int)sizeof(T);
-        constexpr int CPR = 64 / E;   // 16-byte chunks per stage row (a power of two)
-#pragma unroll
-        for (int c = 0; c < (TPW * CPR + 31) / 32; ++c) {
-            const int i = lane + 32 * c;
-            const int j = i / CPR, q = i % CPR;
-            if (i < TPW * CPR && q * E < kn) {
-                T *dst = st + j * 64 + q * E;
-                if (t0 + j < s.N)
-                    cp_async16(dst, x + (t0 + j) * s.sx + k0 + q * E);
-                else
-                    *reinterpret_cast<float4 *>(dst) = make_float4(0.f, 0.f, 0.f, 0.f);
+        for (int o = 0; o < OUT; ++o)
+            for (int q = threadIdx.x; q < q4; q += blockDim.x) {
+                const float4 v = o < H2 ? __ldg(reinterpret_cast<const float4 *>(weight + (int64_t)o * s.D) + q)
+                                        : make_float4(0.f, 0.f, 0.f, 0.f);
+                wp[2 * q * OUT + o] = pack2(v.x, v.y);
+                wp[(2 * q + 1) * OUT + o] = pack2(v.z, v.w);
             }
+    } else {
+#pragma unroll
+        for (int o = 0; o < OUT; ++o)
+            for (int q = threadIdx.x; q < s.D / 2; q += blockDim.x) {
+                const float2 v = o < H2 ? __ldg(reinterpret_cast<const float2 *>(weight + (int64_t)o * s.D) + q)
+                                        : make_float2(0.f, 0.f);
+                wp[q * OUT + o] = pack2(v.x, v.y);
+            }
+    }
+}
+
+// 32 bytes of row `row` from column k0 into r[0..7] (zero where t >= N or past column D).
+// vec16: the row start is 16-byte aligned and D is a whole number of 16-byte units.
+template <typename T>
+__device__ __forceinline__ void load_item(const T *__restrict__ row, bool valid, int k0, int D, bool vec16,
+                                          uint32_t (&r)[8]) {
+    constexpr int E16 = 16 / (int)sizeof(T), E4 = 4 / (int)sizeof(T);
+    if (vec16) {
+#pragma unroll
+        for (int c = 0; c < 2; ++c) {
+            uint4 v = make_uint4(0u, 0u, 0u, 0u);
+            if (valid && k0 + c * E16 < D) v = __ldg(reinterpret_cast<const uint4 *>(row + k0 + c * E16));
+            r[4 * c] = v.x;
+            r[4 * c + 1] = v.y;
+            r[4 * c + 2] = v.z;
+            r[4 * c + 3] = v.w;
         }
     } else {
-        constexpr int E = 4 / (int)sizeof(T);
-        constexpr int CPR = 64 / E;   // 4-byte chunks per stage row
 #pragma unroll
-        for (int c = 0; c < (TPW * CPR + 31) / 32; ++c) {
-            const int i = lane + 32 * c;
-            const int j = i / CPR, q = i % CPR;
-            if (i < TPW * CPR && q * E < kn) {
-                T *dst = st + j * 64 + q * E;
-                if (t0 + j < s.N)
-                    cp_async4(dst, x + (t0 + j) * s.sx + k0 + q * E);
-                else
-                    *reinterpret_cast<uint32_t *>(dst) = 0u;
-            }
-        }
+        for (int c = 0; c < 8; ++c)
+            r[c] = (valid && k0 + c * E4 < D) ? __ldg(reinterpret_cast<const uint32_t *>(row + k0 + c * E4)) : 0u;
     }
 }
 
-// c, g.  Work item = (group of TPW tokens, k-step of 64 elements); each warp walks its
-// items (its groups grid-strided, each group's k-steps in order) with kStages - 1 items'
-// copies in flight.  Lane l of k-step s takes the column pair k = 64 s + 2 l: for each
-// token j and output pair (2q, 2q + 1) one packed FMA per column.  Slot j * OUT + o of the
-// partial sums is token t0 + j, output o; a reduce-scatter over the warp ends a group.
+// Column pair kp of an item as packed fp32 (x[2kp], x[2kp + 1]).
+template <typename T> __device__ __forceinline__ f2reg item_pair(const uint32_t (&r)[8], int kp);
+template <> __device__ __forceinline__ f2reg item_pair<__nv_bfloat16>(const uint32_t (&r)[8], int kp) {
+    return pack2(__uint_as_float(r[kp] << 16), __uint_as_float(r[kp] & 0xffff0000u));
+}
+template <> __device__ __forceinline__ f2reg item_pair<float>(const uint32_t (&r)[8], int kp) {
+    return pack2(__uint_as_float(r[2 * kp]), __uint_as_float(r[2 * kp + 1]));
+}
+
+// c, g.  Warp w accumulates, for each of its lane's tokens and each output o, the packed
+// pair (sum over its slice's even columns, sum over its odd columns) of x * weight: one
+// packed FMA per (token, output, column pair).  At the end of a tile the 8 slices' sums
+// (even + odd) meet in shared memory and are added in slice order, then the bias.  The
+// lanes' rows stream from global memory two items ahead of the arithmetic.
 template <typename T, int OUT>
 __global__ void __launch_bounds__(kThreads, 2) cg_fwd_kernel(CgShape s, const T *__restrict__ x,
                                                             const float *__restrict__ weight,
                                                             const float *__restrict__ bias, float *__restrict__ c,
                                                             float *__restrict__ g, int vec16) {
-    constexpr int TPW = tokens_per_warp(OUT);
-    constexpr int STAGE = TPW * 64;
-    constexpr int WR = kWRow(OUT);
+    constexpr int TPL = tok_per_lane(OUT);
+    constexpr int TT = tile_tokens(OUT);
+    constexpr int KP = 16 / (int)sizeof(T);   // column pairs per item
     extern __shared__ __align__(16) unsigned char smem[];
-    float *ws = reinterpret_cast<float *>(smem);
+    f2reg *wp = reinterpret_cast<f2reg *>(smem);
+    float *red = reinterpret_cast<float *>(smem + wp_bytes(s.D, s.H));   // [8][OUT][TT]
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    T *ring = reinterpret_cast<T *>(smem + weight_smem_bytes(s.D, s.H)) + warp * kStages * STAGE;
-    const int ksn = (s.D + 63) / 64;
-    const int64_t ngroups = (s.N + TPW - 1) / TPW;
-    const int64_t wid = (int64_t)blockIdx.x * (kThreads / 32) + warp, nwarps = (int64_t)gridDim.x * (kThreads / 32);
-    const int64_t items = wid < ngroups ? (ngroups - wid + nwarps - 1) / nwarps * ksn : 0;
-    const int64_t tstep = nwarps * TPW;
-    // issue cursor: item, its group's first token, its k-step, its ring stage
-    int64_t iss = 0, iss_t0 = wid * TPW;
-    int iss_ks = 0, iss_st = 0;
-    auto issue = [&]() {
-        if (iss < items) copy_stage<T, TPW>(s, x, iss_t0, iss_ks * 64, ring + iss_st * STAGE, lane, vec16 != 0);
-        cp_async_commit();   // one group per item, empty past the end, so the counts stay uniform
-        ++iss;
-        iss_st = iss_st + 1 == kStages ? 0 : iss_st + 1;
-        if (++iss_ks == ksn) {
-            iss_ks = 0;
-            iss_t0 += tstep;
-        }
-    };
-    stage_weight<OUT>(s, weight, ws);
-#pragma unroll 1
-    for (int i = 0; i < kStages - 1; ++i) issue();
-    cp_async_wait<kStages - 1>();   // the weight group (the oldest) has landed
-    __syncthreads();
-    const int H2 = 2 * s.H;
-    // acc2[j * OUT/2 + q] = partial sums of (output 2q, output 2q + 1) for token j
-    f2reg acc2[32];
-#pragma unroll
-    for (int i = 0; i < 32; ++i) acc2[i] = 0ull;
-    int64_t t0 = wid * TPW;
-    int ks = 0, st_i = 0;
-#pragma unroll 1
-    for (int64_t it = 0; it < items; ++it) {
-        issue();
-        cp_async_wait<kStages - 1>();   // item `it` has landed (this lane's copies) ...
-        __syncwarp();                   // ... and every lane's
-        const T *st = ring + st_i * STAGE;
-        const int p = ks * 32 + lane;   // column pair
-        if (2 * p < s.D) {
-            // (weight[2q][2p], weight[2q+1][2p]) for q < OUT/2, then the same for column 2p + 1
-            const ulonglong2 *w2 = reinterpret_cast<const ulonglong2 *>(ws + p * WR);
-            f2reg wv[OUT];
-#pragma unroll
-            for (int i = 0; i < OUT / 2; ++i) {
-                const ulonglong2 t = w2[i];
-                wv[2 * i] = t.x;
-                wv[2 * i + 1] = t.y;
-            }
-#pragma unroll
-            for (int j = 0; j < TPW; ++j) {
-                f2reg xa, xb;
-                split_bcast(ldpair<T>(st + j * 64 + 2 * lane), xa, xb);
-#pragma unroll
-                for (int q = 0; q < OUT / 2; ++q) acc2[j * (OUT / 2) + q] = ffma2(xa, wv[q], acc2[j * (OUT / 2) + q]);
-#pragma unroll
-                for (int q = 0; q < OUT / 2; ++q)
-                    acc2[j * (OUT / 2) + q] = ffma2(xb, wv[OUT / 2 + q], acc2[j * (OUT / 2) + q]);
-            }
-        }
-        __syncwarp();   // the stage is free for the copy issued next iteration
-        st_i = st_i + 1 == kStages ? 0 : st_i + 1;
-        if (++ks == ksn) {
-            float acc[64];
-#pragma unroll
-            for (int i = 0; i < 32; ++i) {
-                const float2 v = unpack2(acc2[i]);
-                acc[2 * i] = v.x;
-                acc[2 * i + 1] = v.y;
-                acc2[i] = 0ull;
-            }
-            reduce_scatter64(acc, lane);
-#pragma unroll
-            for (int jj = 0; jj < 2; ++jj) {
-                const int slot = 2 * lane + jj;
-                const int j = slot / OUT, o = slot - j * OUT;
-                const int64_t t = t0 + j;
-                if (j < TPW && o < H2 && t < s.N) {
-                    const float r = acc[jj] + __ldg(bias + o);
-                    if (o < s.H)
-                        c[t * s.H + o] = r;
-                    else
-                        g[t * s.H + o - s.H] = r;
-                }
-            }
-            ks = 0;
-            t0 += tstep;
-        }
-    }
-    cp_async_wait<0>();
-}
+    const int sc = slice_cols(s.D, (int)sizeof(T));
+    const int nit = sc / (32 / (int)sizeof(T));
+    const int kbase = warp * sc;
+    const int64_t ntiles = (s.N + TT - 1) / TT;
+    const int64_t items = (int64_t)blockIdx.x < ntiles ? (ntiles - blockIdx.x + gridDim.x - 1) / gridDim.x * nit : 0;
+    stage_weight_pairs<OUT>(s, weight, wp);
 
-// dx for TPW tokens per warp at a time.  e of the group's tokens is held as output pairs
-// (e[2q], e[2q + 1]); lane l of k-step s takes the column pair k = 64 s + 2 l and forms
-// for each token one packed FMA per output pair and column, then adds the two halves.
-// The TPW * H values of dc (and of dg) a group needs are contiguous; lane l loads entry l
-// of each, one group ahead, and the warp reads them by shuffle.
-template <typename T, int OUT>
-__global__ void __launch_bounds__(kThreads) cg_bwd_dx_kernel(CgShape s, const float *__restrict__ weight,
-                                                            const float *__restrict__ dc,
-                                                            const float *__restrict__ dg, T *__restrict__ dx) {
-    constexpr int TPW = tokens_per_warp(OUT);
-    constexpr int WR = kWRow(OUT);
-    extern __shared__ __align__(16) unsigned char smem[];
-    float *ws = reinterpret_cast<float *>(smem);
-    stage_weight<OUT>(s, weight, ws);
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int64_t step = (int64_t)gridDim.x * (kThreads / 32) * TPW;
-    auto load_e = [&](int64_t t0, float &a, float &b) {
-        const int64_t i = t0 * s.H + lane;
-        const bool have = t0 < s.N && lane < TPW * s.H && i < s.N * s.H;
-        a = have ? __ldg(dc + i) : 0.f;
-        b = have ? __ldg(dg + i) : 0.f;
+    // item i -> (tile, step): tiles blockIdx.x, +gridDim.x, ...; steps 0..nit-1
+    auto load = [&](int64_t i, uint32_t (&r)[TPL][8]) {
+        const int64_t ti = i / nit;
+        const int st = (int)(i - ti * nit);
+        const int64_t t0 = ((int64_t)blockIdx.x + ti * gridDim.x) * TT + lane;
+        const int k0 = kbase + st * (32 / (int)sizeof(T));
+#pragma unroll
+        for (int j = 0; j < TPL; ++j) {
+            const int64_t t = t0 + 32 * j;
+            const bool valid = i < items && t < s.N;
+            load_item<T>(x + (valid ? t : 0) * s.sx, valid, k0, s.D, vec16 != 0, r[j]);
+        }
     };
-    int64_t t0 = ((int64_t)blockIdx.x * (kThreads / 32) + warp) * TPW;
-    float na, nb;
-    load_e(t0, na, nb);
-    cp_async_wait<0>();
-    __syncthreads();
-#pragma unroll 1
-    for (; t0 < s.N; t0 += step) {
-        const float a = na, b = nb;
-        load_e(t0 + step, na, nb);
-        float e[TPW][OUT];
+    f2reg acc[TPL][OUT];
 #pragma unroll
-        for (int j = 0; j < TPW; ++j)
+    for (int j = 0; j < TPL; ++j)
 #pragma unroll
-            for (int o = 0; o < OUT; ++o) {
-                // Source lanes are warp-uniform; entries past 2H are zero.
-                const int src = j * s.H + (o < s.H ? o : o - s.H);
-                const float va = __shfl_sync(0xffffffffu, a, src & 31);
-                const float vb = __shfl_sync(0xffffffffu, b, src & 31);
-                e[j][o] = o < s.H ? va : (o < 2 * s.H ? vb : 0.f);
-            }
-        f2reg e2[TPW][OUT / 2];   // (e[2q], e[2q + 1])
+        for (int o = 0; o < OUT; ++o) acc[j][o] = 0ull;
+    const int H2 = 2 * s.H;
+
+    auto step = [&](int64_t i, uint32_t (&r)[TPL][8]) {
+        const int64_t ti = i / nit;
+        const int st = (int)(i - ti * nit);
+        const int k0 = kbase + st * (32 / (int)sizeof(T));
 #pragma unroll
-        for (int j = 0; j < TPW; ++j)
+        for (int kp = 0; kp < KP; ++kp) {
+            if (k0 + 2 * kp < s.D) {   // warp-uniform
+                const ulonglong2 *w2 = reinterpret_cast<const ulonglong2 *>(wp + ((k0 >> 1) + kp) * OUT);
+                f2reg xp[TPL];
 #pragma unroll
-            for (int q = 0; q < OUT / 2; ++q) e2[j][q] = pack2(e[j][2 * q], e[j][2 * q + 1]);
-        const int nrows = (int)(s.N - t0 < TPW ? s.N - t0 : TPW);
-#pragma unroll 1
-        for (int p = lane; 2 * p < s.D; p += 32) {
-            const ulonglong2 *w2 = reinterpret_cast<const ulonglong2 *>(ws + p * WR);
-            f2reg wv[OUT];
-#pragma unroll
-            for (int i = 0; i < OUT / 2; ++i) {
-                const ulonglong2 t = w2[i];
-                wv[2 * i] = t.x;
-                wv[2 * i + 1] = t.y;
-            }
-#pragma unroll
-            for (int j = 0; j < TPW; ++j) {
-                f2reg a0 = 0ull, a1 = 0ull;
+                for (int j = 0; j < TPL; ++j) xp[j] = item_pair<T>(r[j], kp);
 #pragma unroll
                 for (int q = 0; q < OUT / 2; ++q) {
-                    a0 = ffma2(e2[j][q], wv[q], a0);
-                    a1 = ffma2(e2[j][q], wv[OUT / 2 + q], a1);
+                    const ulonglong2 wv = w2[q];
+#pragma unroll
+                    for (int j = 0; j < TPL; ++j) {
+                        acc[j][2 * q] = ffma2(xp[j], wv.x, acc[j][2 * q]);
+                        acc[j][2 * q + 1] = ffma2(xp[j], wv.y, acc[j][2 * q + 1]);
+                    }
                 }
-                const float2 r0 = unpack2(a0), r1 = unpack2(a1);
-                if (j < nrows) st2<T>(dx + (t0 + j) * s.sdx + 2 * p, make_float2(r0.x + r0.y, r1.x + r1.y));
+            }
+        }
+        load(i + 2, r);   // this buffer's next item
+        if (st == nit - 1) {   // the tile is done: every warp of the block reaches this together
+#pragma unroll
+            for (int j = 0; j < TPL; ++j)
+#pragma unroll
+                for (int o = 0; o < OUT; ++o) {
+                    const float2 v = unpack2(acc[j][o]);
+                    red[(warp * OUT + o) * TT + lane + 32 * j] = v.x + v.y;
+                    acc[j][o] = 0ull;
+                }
+            __syncthreads();
+            const int64_t tb = ((int64_t)blockIdx.x + ti * gridDim.x) * TT;
+            for (int e = threadIdx.x; e < TT * H2; e += kThreads) {
+                const int tok = e / H2, o = e - tok * H2;
+                float sum = red[o * TT + tok];
+#pragma unroll
+                for (int w = 1; w < 8; ++w) sum += red[(w * OUT + o) * TT + tok];
+                const int64_t t = tb + tok;
+                if (t < s.N) {
+                    const float v = sum + __ldg(bias + o);
+                    if (o < s.H)
+                        c[t * s.H + o] = v;
+                    else
+                        g[t * s.H + o - s.H] = v;
+                }
+            }
+            __syncthreads();   // red is free for the next tile
+        }
+    };
+
+    uint32_t r0[TPL][8], r1[TPL][8];
+    load(0, r0);
+    load(1, r1);
+    __syncthreads();   // the weight pairs are staged
+#pragma unroll 1
+    for (int64_t i = 0; i < items; i += 2) {
+        step(i, r0);
+        if (i + 1 < items) step(i + 1, r1);
+    }
+}
+
+// dx.  Lane per token as in the forward; for each of its tokens a lane holds e as broadcast
+// pairs (e[o], e[o]) and forms each column pair of dx as one chain of packed FMAs over the
+// outputs o in order: (dx[2p], dx[2p + 1]) = sum_o (e[o], e[o]) * (weight[o][2p], weight[o][2p + 1]).
+template <typename T, int OUT>
+__global__ void __launch_bounds__(kThreads, 2) cg_bwd_dx_kernel(CgShape s, const float *__restrict__ weight,
+                                                               const float *__restrict__ dc,
+                                                               const float *__restrict__ dg, T *__restrict__ dx,
+                                                               int vec16) {
+    constexpr int TPL = tok_per_lane(OUT);
+    constexpr int TT = tile_tokens(OUT);
+    constexpr int KP = 16 / (int)sizeof(T);
+    constexpr int E16 = 16 / (int)sizeof(T), E4 = 4 / (int)sizeof(T);
+    extern __shared__ __align__(16) unsigned char smem[];
+    f2reg *wp = reinterpret_cast<f2reg *>(smem);
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int sc = slice_cols(s.D, (int)sizeof(T));
+    const int nit = sc / (32 / (int)sizeof(T));
+    const int kbase = warp * sc;
+    const int64_t ntiles = (s.N + TT - 1) / TT;
+    stage_weight_pairs<OUT>(s, weight, wp);
+    __syncthreads();
+    const int H2 = 2 * s.H;
+#pragma unroll 1
+    for (int64_t tile = blockIdx.x; tile < ntiles; tile += gridDim.x) {
+        f2reg eb[TPL][OUT];
+#pragma unroll
+        for (int j = 0; j < TPL; ++j) {
+            const int64_t t = tile * TT + lane + 32 * j;
+#pragma unroll
+            for (int o = 0; o < OUT; ++o) {
+                float e = 0.f;
+                if (t < s.N && o < H2) e = o < s.H ? __ldg(dc + t * s.H + o) : __ldg(dg + t * s.H + o - s.H);
+                eb[j][o] = pack2(e, e);
+            }
+        }
+#pragma unroll 1
+        for (int st = 0; st < nit; ++st) {
+            const int k0 = kbase + st * (32 / (int)sizeof(T));
+            uint32_t out[TPL][8];
+#pragma unroll
+            for (int kp = 0; kp < KP; ++kp) {
+                f2reg rr[TPL];
+#pragma unroll
+                for (int j = 0; j < TPL; ++j) rr[j] = 0ull;
+                if (k0 + 2 * kp < s.D) {   // warp-uniform
+                    const ulonglong2 *w2 = reinterpret_cast<const ulonglong2 *>(wp + ((k0 >> 1) + kp) * OUT);
+#pragma unroll
+                    for (int q = 0; q < OUT / 2; ++q) {
+                        const ulonglong2 wv = w2[q];
+#pragma unroll
+                        for (int j = 0; j < TPL; ++j) {
+                            rr[j] = ffma2(eb[j][2 * q], wv.x, rr[j]);
+                            rr[j] = ffma2(eb[j][2 * q + 1], wv.y, rr[j]);
+                        }
+                    }
+                }
+#pragma unroll
+                for (int j = 0; j < TPL; ++j) {
+                    const float2 v = unpack2(rr[j]);
+                    if constexpr (sizeof(T) == 2) {
+                        const __nv_bfloat162 b2 = __floats2bfloat162_rn(v.x, v.y);
+                        out[j][kp] = *reinterpret_cast<const uint32_t *>(&b2);
+                    } else {
+                        out[j][2 * kp] = __float_as_uint(v.x);
+                        out[j][2 * kp + 1] = __float_as_uint(v.y);
+                    }
+                }
+            }
+#pragma unroll
+            for (int j = 0; j < TPL; ++j) {
+                const int64_t t = tile * TT + lane + 32 * j;
+                if (t < s.N) {
+                    T *row = dx + t * s.sdx;
+                    if (vec16) {
+#pragma unroll
+                        for (int c = 0; c < 2; ++c)
+                            if (k0 + c * E16 < s.D)
+                                *reinterpret_cast<uint4 *>(row + k0 + c * E16) =
+                                    make_uint4(out[j][4 * c], out[j][4 * c + 1], out[j][4 * c + 2], out[j][4 * c + 3]);
+                    } else {
+#pragma unroll
+                        for (int c = 0; c < 8; ++c)
+                            if (k0 + c * E4 < s.D) *reinterpret_cast<uint32_t *>(row + k0 + c * E4) = out[j][c];
+                    }
+                }
             }
         }
     }
@@ -443,19 +426,16 @@ __global__ void __launch_bounds__(kDwThreads) cg_bwd_dw_partial_kernel(CgShape s
             const int nt = rows_of(ci);
             T *xd = xs(ci & 1);
             float2 *ed = es(ci & 1);
-            if (vec16) {
-                constexpr int E = 16 / (int)sizeof(T);
-                const int cpr = s.D / E;
-                for (int i = tid; i < nt * cpr; i += kDwThreads) {
-                    const int r = i / cpr, q = i - r * cpr;
-                    cp_async16(xd + r * s.D + q * E, x + (tc + r) * s.sx + q * E);
-                }
-            } else {
-                constexpr int E = 4 / (int)sizeof(T);
-                const int cpr = s.D / E;
-                for (int i = tid; i < nt * cpr; i += kDwThreads) {
-                    const int r = i / cpr, q = i - r * cpr;
-                    cp_async4(xd + r * s.D + q * E, x + (tc + r) * s.sx + q * E);
+            const int warp = tid >> 5, lane = tid & 31;
+            for (int r = warp; r < nt; r += kDwThreads / 32) {
+                const T *src = x + (tc + r) * s.sx;
+                T *dst = xd + r * s.D;
+                if (vec16) {
+                    constexpr int E = 16 / (int)sizeof(T);
+                    for (int q = lane; q < s.D / E; q += 32) cp_async16(dst + q * E, src + q * E);
+                } else {
+                    constexpr int E = 4 / (int)sizeof(T);
+                    for (int q = lane; q < s.D / E; q += 32) cp_async4(dst + q * E, src + q * E);
                 }
             }
             for (int i = tid; i < chunk * OUT; i += kDwThreads) {

@@ -424,9 +424,8 @@ dc_status_t check_cg(const dc_cg_params *p, dc::cg::CgShape *s) {
     const int64_t sx = p->stride_x ? p->stride_x : D, sdx = p->stride_dx ? p->stride_dx : D;
     if (sx < D || sdx < D || (sx & 1) || (sdx & 1)) return DC_ERR_INVALID_ARG;
     if (p->num_heads > 16) return DC_ERR_UNSUPPORTED;
-    const size_t smem = p->dtype == DC_F32 ? dc::cg::fwd_smem_bytes<float>(p->model_dim, p->num_heads)
-                                           : dc::cg::fwd_smem_bytes<__nv_bfloat16>(p->model_dim, p->num_heads);
-    if (smem > dc::cg::kMaxSmem) return DC_ERR_UNSUPPORTED;
+    // the forward keeps the weight and one tile's partial sums in shared memory
+    if (dc::cg::fwd_smem_bytes(p->model_dim, p->num_heads) > dc::cg::kMaxSmem) return DC_ERR_UNSUPPORTED;
     s->N = p->num_tokens;
     s->D = p->model_dim;
     s->H = p->num_heads;
@@ -435,28 +434,37 @@ dc_status_t check_cg(const dc_cg_params *p, dc::cg::CgShape *s) {
     return DC_OK;
 }
 
-// Blocks of 8 warps for `groups` warp-sized work items: at most two resident blocks per SM.
-unsigned cg_grid(int64_t groups) {
-    const int64_t want = (groups + 7) / 8;
-    return (unsigned)(want < 1 ? 1 : want > 2 * 148 ? 2 * 148 : want);
+// 16-byte accesses when every row starts on a 16-byte boundary and spans whole 16-byte units.
+template <typename T>
+int cg_vec16(int64_t stride, int D, const void *base) {
+    return (uintptr_t)base % 16 == 0 && (stride * (int64_t)sizeof(T)) % 16 == 0 && (D * sizeof(T)) % 16 == 0;
 }
 
-// 16-byte copies when every row of x starts on a 16-byte boundary and spans whole 16-byte units.
-template <typename T>
-int cg_vec16(const dc::cg::CgShape &s, const void *x) {
-    return (uintptr_t)x % 16 == 0 && (s.sx * (int64_t)sizeof(T)) % 16 == 0 && (s.D * sizeof(T)) % 16 == 0;
+template <typename K>
+cudaError_t cg_tile_grid(K kern, size_t smem, int64_t tiles, unsigned *grid) {
+    int per_sm = 0;
+    cudaError_t e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, dc::cg::kThreads, smem);
+    if (e != cudaSuccess) return e;
+    int sms = 0, dev = 0;
+    e = cudaGetDevice(&dev);
+    if (e == cudaSuccess) e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    if (e != cudaSuccess) return e;
+    const int64_t resident = (int64_t)sms * (per_sm > 0 ? per_sm : 1);
+    *grid = (unsigned)(tiles < resident ? tiles : resident);
+    return cudaSuccess;
 }
 
 template <int OUT, typename T>
 cudaError_t cg_fwd_launch(const dc::cg::CgShape &s, const void *x, const float *w, const float *b, float *c, float *g,
                           cudaStream_t st) {
-    constexpr int TPW = dc::cg::tokens_per_warp(OUT);
     auto kern = dc::cg::cg_fwd_kernel<T, OUT>;
-    const size_t smem = dc::cg::fwd_smem_bytes<T>(s.D, s.H);
+    const size_t smem = dc::cg::fwd_smem_bytes(s.D, s.H);
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
-    kern<<<cg_grid((s.N + TPW - 1) / TPW), dc::cg::kThreads, smem, st>>>(s, (const T *)x, w, b, c, g,
-                                                                        cg_vec16<T>(s, x));
+    unsigned grid = 0;
+    e = cg_tile_grid(kern, smem, (s.N + dc::cg::tile_tokens(OUT) - 1) / dc::cg::tile_tokens(OUT), &grid);
+    if (e != cudaSuccess) return e;
+    kern<<<grid, dc::cg::kThreads, smem, st>>>(s, (const T *)x, w, b, c, g, cg_vec16<T>(s.sx, s.D, x));
     ++t_launches;
     return cudaGetLastError();
 }
@@ -464,13 +472,15 @@ cudaError_t cg_fwd_launch(const dc::cg::CgShape &s, const void *x, const float *
 template <int OUT, typename T>
 cudaError_t cg_bwd_launch(const dc::cg::CgShape &s, const void *x, const float *w, const float *dc_, const float *dg,
                           void *dx, float *dw, float *db, float *part, int blocks, cudaStream_t st) {
-    constexpr int TPW = dc::cg::tokens_per_warp(OUT);
     if (s.N > 0) {
         auto kdx = dc::cg::cg_bwd_dx_kernel<T, OUT>;
-        const size_t smem = dc::cg::weight_smem_bytes(s.D, s.H);
+        const size_t smem = dc::cg::wp_bytes(s.D, s.H);
         cudaError_t e = cudaFuncSetAttribute(kdx, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
         if (e != cudaSuccess) return e;
-        kdx<<<cg_grid((s.N + TPW - 1) / TPW), dc::cg::kThreads, smem, st>>>(s, w, dc_, dg, (T *)dx);
+        unsigned grid = 0;
+        e = cg_tile_grid(kdx, smem, (s.N + dc::cg::tile_tokens(OUT) - 1) / dc::cg::tile_tokens(OUT), &grid);
+        if (e != cudaSuccess) return e;
+        kdx<<<grid, dc::cg::kThreads, smem, st>>>(s, w, dc_, dg, (T *)dx, cg_vec16<T>(s.sdx, s.D, dx));
         ++t_launches;
         auto kdw = dc::cg::cg_bwd_dw_partial_kernel<T, OUT>;
         const int chunk = dc::cg::dw_chunk(s.D, s.H, sizeof(T));
@@ -478,7 +488,8 @@ cudaError_t cg_bwd_launch(const dc::cg::CgShape &s, const void *x, const float *
         e = cudaFuncSetAttribute(kdw, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)dsmem);
         if (e != cudaSuccess) return e;
         const int64_t span = (s.N + blocks - 1) / blocks;
-        kdw<<<blocks, dc::cg::kDwThreads, dsmem, st>>>(s, span, chunk, (const T *)x, dc_, dg, part, cg_vec16<T>(s, x));
+        kdw<<<blocks, dc::cg::kDwThreads, dsmem, st>>>(s, span, chunk, (const T *)x, dc_, dg, part,
+                                                     cg_vec16<T>(s.sx, s.D, x));
         ++t_launches;
     }
     const int64_t n = dc::cg::record_floats(s.D, s.H);

@@ -247,10 +247,10 @@ dc_status_t dc_attn_inject_missing_load(void);
  * contiguous; bias, dbias [2H] fp32; c, g, dc, dg [N][H] fp32 contiguous.
  * Limits: D even; strides even and >= D; 1 <= H <= 16 (larger H returns
  * DC_ERR_UNSUPPORTED).  The forward keeps in shared memory the weight padded
- * to OUT rows (OUT = 8, 12, 16, 24 or 32, the first >= 2H; 4 * (OUT + 2) * D
- * bytes) and 8 warps x 6 stages x 64/OUT tokens x 64 elements of x; the two
- * must fit 227 KB, else DC_ERR_UNSUPPORTED (D <= 3602 at H = 6 in bf16, 3052
- * in fp32; D <= 1618 at H = 16 in bf16).  Pointers: device, 16-byte aligned,
+ * to OUT rows (OUT = 8, 12, 16, 24 or 32, the first >= 2H; 4 * OUT * D bytes)
+ * and the 8 column slices' partial sums of 64 tokens (32 when OUT > 12); the
+ * two must fit 227 KB, else DC_ERR_UNSUPPORTED (D <= 4330 at H = 6, D <= 1560
+ * at H = 16, either dtype).  Pointers: device, 16-byte aligned,
  * caller-owned; asynchronous on `stream`; outputs overwritten.
  * ------------------------------------------------------------------------ */
 typedef struct {

@@ -182,9 +182,9 @@ def _cg(**kw):
     (dict(stride_x=766), dcattn.DC_ERR_INVALID_ARG),       # below D
     (dict(stride_dx=-768), dcattn.DC_ERR_INVALID_ARG),
     (dict(num_heads=17), dcattn.DC_ERR_UNSUPPORTED),
-    (dict(model_dim=3604), dcattn.DC_ERR_UNSUPPORTED),     # weight + x stages above 227 KB
-    (dict(model_dim=3054, dtype=dcattn.DC_F32), dcattn.DC_ERR_UNSUPPORTED),
-    (dict(num_heads=16, model_dim=1620), dcattn.DC_ERR_UNSUPPORTED),
+    (dict(model_dim=4332), dcattn.DC_ERR_UNSUPPORTED),     # weight + partial sums above 227 KB
+    (dict(model_dim=4332, dtype=dcattn.DC_F32), dcattn.DC_ERR_UNSUPPORTED),
+    (dict(num_heads=16, model_dim=1562), dcattn.DC_ERR_UNSUPPORTED),
 ])
 def test_cg_bad_params_rejected_on_host(lib, kw, expect):
     p = _cg(**kw)
@@ -196,8 +196,8 @@ def test_cg_bad_params_rejected_on_host(lib, kw, expect):
 
 def test_cg_limits_accepted(lib):
     """The largest shapes inside the limits pass the host checks (N = 0: nothing runs)."""
-    for D, H, dt in ((3602, 6, dcattn.DC_BF16), (3052, 6, dcattn.DC_F32), (1618, 16, dcattn.DC_BF16), (2, 1, 0),
-                     (4582, 4, dcattn.DC_BF16)):
+    for D, H, dt in ((4330, 6, dcattn.DC_BF16), (4330, 6, dcattn.DC_F32), (1560, 16, dcattn.DC_BF16), (2, 1, 0),
+                     (6752, 4, dcattn.DC_BF16), (3376, 8, dcattn.DC_BF16)):
         p = _cg(model_dim=D, num_heads=H, num_tokens=0, dtype=dt)
         assert lib.dc_attn_cg_fwd(ctypes.byref(p), 0, 0, 0, 0, 0, None) == dcattn.DC_OK, (D, H, dt)
 
