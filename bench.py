@@ -399,6 +399,73 @@ def run_sweep(args):
     return 0
 
 
+# The producer of c and g (assumed per-token affine form), measured beside the headline
+# step at the GPT-2 width: x [N][768] bf16 -> c, g [N][6] fp32, and its backward.
+CG_SHAPE = (16384, 768, 6)
+CG_SETS = 6                                  # rotating x sets: 6 x 25 MB, larger than L2
+
+
+def cg_measure(dev, hbm_gbs: float, peak_note: str) -> dict:
+    """Graph-timed forward and backward of the c/g producer; rooflines from algorithmic
+    bytes (x read once, c and g written; backward: x and e read, dx written, dweight and
+    dbias written; the partial-sum records in the workspace are not algorithmic)."""
+    from cross_head_dynamic_b200 import dcattn
+    from cross_head_dynamic_b200.inputs import cg_problem
+    N, D, H = CG_SHAPE
+    sets = []
+    for i in range(CG_SETS):
+        p = cg_problem(1000 + i, N, D, H, "bf16")
+        x = {k: v.to(dev) for k, v in p.items()}
+        x["wt"] = x["w"].t().contiguous()
+        x["c"], x["gg"] = torch.empty(N, H, device=dev), torch.empty(N, H, device=dev)
+        x["dx"], x["dw"], x["db"] = torch.empty_like(x["x"]), torch.empty_like(x["wt"]), torch.empty_like(x["b"])
+        x["ws"] = torch.empty(dcattn.dc_attn_cg_bwd_workspace_size(x["x"], H), device=dev, dtype=torch.uint8)
+        sets.append(x)
+    calls = {
+        "fwd": lambda x: dcattn.dc_attn_cg_fwd(x["x"], x["wt"], x["b"], c=x["c"], g=x["gg"]),
+        "bwd": lambda x: dcattn.dc_attn_cg_bwd(x["x"], x["wt"], x["dc"], x["dg"], dx=x["dx"], dweight=x["dw"],
+                                               dbias=x["db"], workspace=x["ws"]),
+    }
+    launches = {}
+    out = {}
+    stream = torch.cuda.current_stream()
+    for name, call in calls.items():
+        call(sets[0])
+        launches[name] = dcattn.dc_attn_last_launch_count()
+        graphs = []
+        for x in sets:
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g):
+                call(x)
+            graphs.append(g)
+        for it in range(2 * CG_SETS):
+            graphs[it % CG_SETS].replay()
+        reps = 60
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        for it in range(reps):
+            graphs[it % CG_SETS].replay()
+        b.record(stream)
+        torch.cuda.synchronize()
+        out[name] = a.elapsed_time(b) / reps * 1e3   # us per call
+        del graphs
+    if dcattn.dc_attn_device_status() != 0:
+        raise RuntimeError("device status word reports an error after the c/g producer")
+    xb, eb = N * D * 2, N * 2 * H * 4
+    fwd_bytes = xb + eb + 2 * H * D * 4
+    bwd_bytes = 2 * xb + eb + 2 * H * D * 4 + 2 * H * 4
+    flops = 2.0 * N * D * 2 * H
+    res = {"workload": f"x [{N}][{D}] bf16, H = {H} (c, g fp32); {CG_SETS} rotating input sets (> L2)",
+           "form": "assumed per-token affine map (the pages give no formula)"}
+    for name, nbytes, nflops in (("fwd", fwd_bytes, flops), ("bwd", bwd_bytes, 2 * flops)):
+        t = out[name] * 1e-6
+        res[name] = {"us": out[name], "launches": launches[name], "algorithmic_bytes": nbytes,
+                     "fp32_flops": nflops,
+                     "roofline": {"bound": "hbm", "achieved": nbytes / t / 1e9, "peak": hbm_gbs, "unit": "GB/s",
+                                  "frac": nbytes / t / 1e9 / hbm_gbs, "peak_source": peak_note}}
+    return res
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -406,6 +473,7 @@ def main():
     ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--impl", choices=["dcattn", "reference"], default="dcattn")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-next-rows", action="store_true", help="skip the c/g producer measurement")
     ap.add_argument("--sweep", action="store_true",
                     help="one JSON line per workload of the inputs module instead of the headline line")
     ap.add_argument("--workload", action="append", choices=list(CONFIGS),
@@ -647,6 +715,8 @@ def main():
                                NOMINAL_BF16_TFLOPS)
     step_dram = step_dram_bytes(N)
 
+    cg = cg_measure(dev, hbm, peak_note) if not args.no_next_rows else None
+
     cpu = None
     if rank == 0 and not args.no_cpu_baseline:
         rate, cores, dt = oracle_sample_rate(cfg, rows=cfg.batch)
@@ -690,6 +760,7 @@ def main():
             "kernel_ms": per_kernel,
             "kernel_ms_eager": per_kernel_eager,
             "cpu_baseline": cpu,
+            "next_rows": {"cg_producer": cg},
             "e2e": e2e,
             "gpu_launches": gpu_launches,
             "clocks": dict(clocks or {}, note=clock_note),

@@ -14,6 +14,7 @@
 #include "simt.cuh"
 #include "tc_host.cuh"
 #include "cg.cuh"
+#include "cg_tc.cuh"
 
 namespace {
 
@@ -423,6 +424,7 @@ dc_status_t check_cg(const dc_cg_params *p, dc::cg::CgShape *s) {
     const int64_t D = p->model_dim;
     const int64_t sx = p->stride_x ? p->stride_x : D, sdx = p->stride_dx ? p->stride_dx : D;
     if (sx < D || sdx < D || (sx & 1) || (sdx & 1)) return DC_ERR_INVALID_ARG;
+    if (p->impl != DC_IMPL_AUTO && p->impl != DC_IMPL_SIMT && p->impl != DC_IMPL_TCGEN05) return DC_ERR_INVALID_ARG;
     if (p->num_heads > 16) return DC_ERR_UNSUPPORTED;
     // the forward keeps the weight and one tile's partial sums in shared memory
     if (dc::cg::fwd_smem_bytes(p->model_dim, p->num_heads) > dc::cg::kMaxSmem) return DC_ERR_UNSUPPORTED;
@@ -432,6 +434,57 @@ dc_status_t check_cg(const dc_cg_params *p, dc::cg::CgShape *s) {
     s->sx = sx;
     s->sdx = sdx;
     return DC_OK;
+}
+
+// Kernel family of the c/g forward: tcgen05 for bf16 x whose rows TMA can address (row
+// stride a multiple of 16 bytes), at least one full 128-token tile and 64 columns, and whose
+// weight splits fit shared memory; SIMT otherwise.  -1: TCGEN05 asked for but not possible.
+int cg_fwd_impl(const dc_cg_params *p, const dc::cg::CgShape &s) {
+    const bool tc_ok = p->dtype == DC_BF16 && (s.sx * 2) % 16 == 0 && s.N >= dc::cg::kTcTile && s.D >= 64 &&
+                       dc::cg::tc_stages(s.D, s.H, dc::cg::kMaxSmem) >= 2;
+    if (p->impl == DC_IMPL_SIMT) return DC_IMPL_SIMT;
+    if (p->impl == DC_IMPL_TCGEN05) return tc_ok ? DC_IMPL_TCGEN05 : -1;
+    return tc_ok ? DC_IMPL_TCGEN05 : DC_IMPL_SIMT;
+}
+
+// Kernel family of dx: tcgen05 for bf16 with 2H <= 16, dx rows on 16-byte boundaries and the
+// weight splits within shared memory; SIMT otherwise.  -1: TCGEN05 asked for but not possible.
+int cg_dx_impl(const dc_cg_params *p, const dc::cg::CgShape &s) {
+    const bool tc_ok = p->dtype == DC_BF16 && 2 * s.H <= 16 && s.sdx % 8 == 0 &&
+                       dc::cg::dx_tc_smem_bytes(s.D) <= dc::cg::kMaxSmem;
+    if (p->impl == DC_IMPL_SIMT) return DC_IMPL_SIMT;
+    if (p->impl == DC_IMPL_TCGEN05) return tc_ok ? DC_IMPL_TCGEN05 : -1;
+    return tc_ok ? DC_IMPL_TCGEN05 : DC_IMPL_SIMT;
+}
+
+cudaError_t cg_dx_tc_launch(const dc::cg::CgShape &s, const float *w, const float *dc_, const float *dg, void *dx,
+                            cudaStream_t st) {
+    const size_t smem = dc::cg::dx_tc_smem_bytes(s.D);
+    cudaError_t e = cudaFuncSetAttribute(dc::cg::cg_bwd_dx_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)smem);
+    if (e != cudaSuccess) return e;
+    const unsigned grid = (unsigned)((s.N + dc::cg::kTcTile - 1) / dc::cg::kTcTile);
+    dc::cg::cg_bwd_dx_tc_kernel<<<grid, dc::cg::kDxThreads, smem, st>>>(s, w, dc_, dg, (__nv_bfloat16 *)dx,
+                                                                         g_wait_ns.load(std::memory_order_relaxed));
+    ++t_launches;
+    return cudaGetLastError();
+}
+
+template <int R>
+cudaError_t cg_fwd_tc_launch(const dc::cg::CgShape &s, const void *x, const float *w, const float *b, float *c,
+                             float *g, cudaStream_t st) {
+    CUtensorMap m;
+    cudaError_t e = dc::tc::make_map(&m, x, s.N, 1, s.D, s.sx, dc::cg::kTcTile);
+    if (e != cudaSuccess) return e;
+    auto kern = dc::cg::cg_fwd_tc_kernel<R>;
+    const int nst = dc::cg::tc_stages(s.D, s.H, dc::cg::kMaxSmem);
+    const size_t smem = dc::cg::tc_smem_bytes(s.D, s.H, nst);
+    e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    const unsigned grid = (unsigned)((s.N + dc::cg::kTcTile - 1) / dc::cg::kTcTile);
+    kern<<<grid, dc::cg::kTcThreads, smem, st>>>(m, s, w, b, c, g, nst, g_wait_ns.load(std::memory_order_relaxed));
+    ++t_launches;
+    return cudaGetLastError();
 }
 
 // 16-byte accesses when every row starts on a 16-byte boundary and spans whole 16-byte units.
@@ -471,8 +524,11 @@ cudaError_t cg_fwd_launch(const dc::cg::CgShape &s, const void *x, const float *
 
 template <int OUT, typename T>
 cudaError_t cg_bwd_launch(const dc::cg::CgShape &s, const void *x, const float *w, const float *dc_, const float *dg,
-                          void *dx, float *dw, float *db, float *part, int blocks, cudaStream_t st) {
-    if (s.N > 0) {
+                          void *dx, float *dw, float *db, float *part, int blocks, bool dx_tc, cudaStream_t st) {
+    if (s.N > 0 && dx_tc) {
+        cudaError_t e = cg_dx_tc_launch(s, w, dc_, dg, dx, st);
+        if (e != cudaSuccess) return e;
+    } else if (s.N > 0) {
         auto kdx = dc::cg::cg_bwd_dx_kernel<T, OUT>;
         const size_t smem = dc::cg::wp_bytes(s.D, s.H);
         cudaError_t e = cudaFuncSetAttribute(kdx, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
@@ -482,10 +538,12 @@ cudaError_t cg_bwd_launch(const dc::cg::CgShape &s, const void *x, const float *
         if (e != cudaSuccess) return e;
         kdx<<<grid, dc::cg::kThreads, smem, st>>>(s, w, dc_, dg, (T *)dx, cg_vec16<T>(s.sdx, s.D, dx));
         ++t_launches;
+    }
+    if (s.N > 0) {
         auto kdw = dc::cg::cg_bwd_dw_partial_kernel<T, OUT>;
         const int chunk = dc::cg::dw_chunk(s.D, s.H, sizeof(T));
         const size_t dsmem = dc::cg::dw_smem_bytes(s.D, s.H, sizeof(T));
-        e = cudaFuncSetAttribute(kdw, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)dsmem);
+        cudaError_t e = cudaFuncSetAttribute(kdw, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)dsmem);
         if (e != cudaSuccess) return e;
         const int64_t span = (s.N + blocks - 1) / blocks;
         kdw<<<blocks, dc::cg::kDwThreads, dsmem, st>>>(s, span, chunk, (const T *)x, dc_, dg, part,
@@ -528,10 +586,21 @@ dc_status_t dc_attn_cg_fwd(const dc_cg_params *params, const void *x, const floa
     if (s.N == 0) return DC_OK;
     r = ptrs_ok({x, weight, bias, c, g}, {});
     if (r != DC_OK) return r;
+    const int impl = cg_fwd_impl(params, s);
+    if (impl < 0) return DC_ERR_UNSUPPORTED;
     cudaStream_t st = (cudaStream_t)stream;
+    if (impl == DC_IMPL_TCGEN05)
+        return cuda_status(dc::cg::tc_rows_per_split(s.H) == 16 ? cg_fwd_tc_launch<16>(s, x, weight, bias, c, g, st)
+                                                                : cg_fwd_tc_launch<32>(s, x, weight, bias, c, g, st));
     return cuda_status(cg_dispatch(s.H, params->dtype, [&]<int OUT, typename T>() {
         return cg_fwd_launch<OUT, T>(s, x, weight, bias, c, g, st);
     }));
+}
+
+int32_t dc_attn_cg_resolve_impl(const dc_cg_params *params) {
+    dc::cg::CgShape s;
+    if (check_cg(params, &s) != DC_OK) return -1;
+    return cg_fwd_impl(params, s);
 }
 
 size_t dc_attn_cg_bwd_workspace_size(const dc_cg_params *params) {
@@ -555,9 +624,12 @@ dc_status_t dc_attn_cg_bwd(const dc_cg_params *params, const void *x, const floa
         if (workspace_bytes < cg_ws_need(s)) return DC_ERR_INVALID_ARG;
     }
     const int blocks = s.N > 0 ? dc::cg::partial_blocks(s.N) : 0;
+    const int dx_impl = cg_dx_impl(params, s);
+    if (dx_impl < 0) return DC_ERR_UNSUPPORTED;
     cudaStream_t st = (cudaStream_t)stream;
     return cuda_status(cg_dispatch(s.H, params->dtype, [&]<int OUT, typename T>() {
-        return cg_bwd_launch<OUT, T>(s, x, weight, dc_, dg, dx, dweight, dbias, (float *)workspace, blocks, st);
+        return cg_bwd_launch<OUT, T>(s, x, weight, dc_, dg, dx, dweight, dbias, (float *)workspace, blocks,
+                                     dx_impl == DC_IMPL_TCGEN05, st);
     }));
 }
 

@@ -257,21 +257,37 @@ typedef struct {
     int32_t dtype;        /* dc_dtype_t of x and dx                                   */
     int32_t model_dim;    /* D                                                        */
     int32_t num_heads;    /* H                                                        */
-    int32_t reserved;     /* set to 0                                                 */
+    int32_t impl;         /* dc_impl_t for the forward and for dx                     */
     int64_t num_tokens;   /* N >= 0                                                   */
     int64_t stride_x;     /* elements between tokens of x (0 = D)                     */
     int64_t stride_dx;    /* elements between tokens of dx (0 = D)                    */
 } dc_cg_params;
 
-/* c, g from x.  N = 0 launches nothing. */
+/* c, g from x.  N = 0 launches nothing.
+ * Two kernel families.  SIMT: CUDA-core fp32 FMAs in a fixed order.  TCGEN05 (bf16 x
+ * only, row stride a multiple of 8 elements, N >= 128, D >= 64, and the weight splits
+ * below within shared memory: D <= 2048 at H <= 8, D <= 1024 at H <= 16): tensor-core
+ * products of x with the three bf16 terms hi + mid + lo of the weight, whose sum is the
+ * fp32 weight to within 2^-24 of each element, accumulated in fp32 by the tensor core
+ * (its accumulation order and rounding are the hardware's).  AUTO takes TCGEN05 when
+ * possible; TCGEN05 where it is not possible returns DC_ERR_UNSUPPORTED. */
 dc_status_t dc_attn_cg_fwd(const dc_cg_params *params, const void *x, const float *weight, const float *bias,
                            float *c, float *g, void *stream);
+
+/* Which family the forward resolves to (DC_IMPL_SIMT or DC_IMPL_TCGEN05), or -1 if the
+ * params are invalid or ask for TCGEN05 where it is not possible. */
+int32_t dc_attn_cg_resolve_impl(const dc_cg_params *params);
 
 /* Bytes of workspace dc_attn_cg_bwd needs (0 when N = 0 or the params are
  * invalid): one fp32 partial record of dweight and dbias per block of tokens. */
 size_t dc_attn_cg_bwd_workspace_size(const dc_cg_params *params);
 
-/* Gradients for dL/dc = dc, dL/dg = dg, writing e[t] = (dc[t,:], dg[t,:]):
+/* Gradients for dL/dc = dc, dL/dg = dg, writing e[t] = (dc[t,:], dg[t,:]).
+ * dx runs on tcgen05 for bf16 with 2H <= 16, a dx row stride that is a multiple of 8
+ * elements and D <= 1024 (AUTO; TCGEN05 elsewhere returns DC_ERR_UNSUPPORTED): products
+ * of the bf16 splits of e and of the weight, six of the nine pairs, whose sum is e * w to
+ * within 2^-23 |e w|, accumulated by the tensor core; SIMT otherwise.  dweight and dbias
+ * always run on the CUDA cores:
  *
  *   dx[t,k]       = sum_o e[t,o] * weight[o][k]
  *   dweight[o][k] = sum_t e[t,o] * x[t,k]        dbias[o] = sum_t e[t,o]

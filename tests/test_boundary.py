@@ -166,7 +166,7 @@ def test_accepts_fused_projection_strides(lib):
 
 
 def _cg(**kw):
-    base = dict(dtype=dcattn.DC_BF16, model_dim=768, num_heads=6, reserved=0, num_tokens=1000, stride_x=0,
+    base = dict(dtype=dcattn.DC_BF16, model_dim=768, num_heads=6, impl=0, num_tokens=1000, stride_x=0,
                 stride_dx=0)
     base.update(kw)
     return dcattn.CgParams(**base)
@@ -185,6 +185,7 @@ def _cg(**kw):
     (dict(model_dim=4332), dcattn.DC_ERR_UNSUPPORTED),     # weight + partial sums above 227 KB
     (dict(model_dim=4332, dtype=dcattn.DC_F32), dcattn.DC_ERR_UNSUPPORTED),
     (dict(num_heads=16, model_dim=1562), dcattn.DC_ERR_UNSUPPORTED),
+    (dict(impl=3), dcattn.DC_ERR_INVALID_ARG),
 ])
 def test_cg_bad_params_rejected_on_host(lib, kw, expect):
     p = _cg(**kw)
@@ -217,3 +218,21 @@ def test_cg_workspace_and_pointer_checks(lib):
     assert lib.dc_attn_cg_fwd(ctypes.byref(p0), 0, 0, 0, 0, 0, None) == dcattn.DC_OK
     # N = 0 still writes dweight and dbias (zeros), so those two must be valid
     assert lib.dc_attn_cg_bwd(ctypes.byref(p0), 0, 0, 0, 0, 0, 0, 0, 0, 0, None) == dcattn.DC_ERR_INVALID_ARG
+
+
+def test_cg_resolve_impl(lib):
+    """bf16 x with TMA-addressable rows, a full 128-token tile, D >= 64 and the weight splits
+    within shared memory runs on tcgen05; everything else on SIMT; forcing tcgen05 where it
+    is not possible is refused."""
+    tc, simt = dcattn.IMPLS["tcgen05"], dcattn.IMPLS["simt"]
+    for kw, want in ((dict(), tc), (dict(dtype=dcattn.DC_F32), simt), (dict(num_tokens=127), simt),
+                     (dict(stride_x=770), simt), (dict(stride_x=776), tc), (dict(model_dim=62), simt),
+                     (dict(model_dim=2048, num_heads=8), tc), (dict(model_dim=2050, num_heads=8), simt),
+                     (dict(model_dim=1024, num_heads=16), tc), (dict(model_dim=1026, num_heads=16), simt),
+                     (dict(impl=simt), simt), (dict(impl=tc, dtype=dcattn.DC_F32), -1), (dict(impl=tc), tc),
+                     (dict(impl=7), -1)):
+        p = _cg(**kw)
+        assert lib.dc_attn_cg_resolve_impl(ctypes.byref(p)) == want, kw
+    p = _cg(impl=tc, dtype=dcattn.DC_F32)
+    a = 0x4000
+    assert lib.dc_attn_cg_fwd(ctypes.byref(p), a, a, a, a, a, None) == dcattn.DC_ERR_UNSUPPORTED

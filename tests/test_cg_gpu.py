@@ -36,19 +36,51 @@ def _to_np(t):
     return t.detach().double().cpu().numpy()
 
 
-def _run(p, dtype):
+def _run(p, dtype, impl="auto", dx_impl=None):
     dev = "cuda"
     x = p["x"].to(dev)
     w = p["w"].to(dev).t().contiguous()      # weight [2H][D]
     b = p["b"].to(dev)
     dc, dg = p["dc"].to(dev), p["dg"].to(dev)
-    c, g = dcattn.dc_attn_cg_fwd(x, w, b)
-    dx, dw, db = dcattn.dc_attn_cg_bwd(x, w, dc, dg)
+    c, g = dcattn.dc_attn_cg_fwd(x, w, b, impl=impl)
+    dx, dw, db = dcattn.dc_attn_cg_bwd(x, w, dc, dg, impl=dx_impl or _dx_impl(p, impl))
     torch.cuda.synchronize()
     return c, g, dx, dw, db
 
 
-def _check(p, outs, dtype):
+def _dx_on_tc(p):
+    """The conditions under which AUTO runs dx on tcgen05 (contiguous dx)."""
+    N, D = p["x"].shape
+    H = p["dc"].shape[1]
+    return p["x"].dtype == torch.bfloat16 and 2 * H <= 16 and D % 8 == 0 and D <= 1024
+
+
+def _dx_impl(p, fwd_impl):
+    """dx follows the forward's choice where tcgen05 is possible for it, else SIMT."""
+    return "tcgen05" if fwd_impl != "simt" and _dx_on_tc(p) else "simt"
+
+
+def _fwd_tolerance(D, fwd_impl):
+    """Relative to the sum of |terms|.  SIMT: fp32 FMAs in the kernel's order.  tcgen05: the
+    products with the bf16 weight terms are exact and the terms sum to the weight within
+    2^-24; the tensor core's fp32 accumulation is not specified to round to nearest, so each
+    of its ceil(D/16) accumulation steps is allowed 2 units in the last place (2^-22) of the
+    sum of |terms|, plus the epilogue's three additions and the bias."""
+    if fwd_impl == "simt":
+        return gamma(D // 16 + 18)
+    return (-(-D // 16) + 2) * 2.0 ** -22 + 2.0 ** -24 + gamma(4)
+
+
+def _dx_tolerance(H, dx_impl):
+    """Relative to the sum of |terms|, before the bf16 rounding of dx.  SIMT: 2H fp32 FMAs
+    in order.  tcgen05: six of the nine products of the bf16 splits of e and the weight,
+    2^-23 of |e w| left out, accumulated by the tensor core in 6 steps of 16 (2^-22 each)."""
+    if dx_impl == "simt":
+        return gamma(2 * H + 2)
+    return 8 * 2.0 ** -22 + 2.0 ** -23
+
+
+def _check(p, outs, dtype, fwd_impl="simt", dx_impl=None):
     c, g, dx, dw, db = (_to_np(t) for t in outs)
     x, w, b = _to_np(p["x"]), _to_np(p["w"]), _to_np(p["b"])
     dcn, dgn = _to_np(p["dc"]), _to_np(p["dg"])
@@ -56,12 +88,12 @@ def _check(p, outs, dtype):
     H = dcn.shape[1]
     rc, rg = oracle.cg_forward(x, w, b)
     mc, mg = oracle.cg_forward(np.abs(x), np.abs(w), np.abs(b))
-    tf = gamma(D // 16 + 18)
+    tf = _fwd_tolerance(D, fwd_impl)
     assert np.all(np.abs(c - rc) <= tf * mc + 1e-30), np.abs(c - rc).max()
     assert np.all(np.abs(g - rg) <= tf * mg + 1e-30), np.abs(g - rg).max()
     rdx, rdw, rdb = oracle.cg_backward(x, w, dcn, dgn)
     mdx, mdw, mdb = oracle.cg_backward(np.abs(x), np.abs(w), np.abs(dcn), np.abs(dgn))
-    tol_dx = gamma(2 * H + 2) * mdx + (2.0 ** -8 * np.abs(rdx) if dtype == "bf16" else 0) + 1e-30
+    tol_dx = _dx_tolerance(H, dx_impl or _dx_impl(p, fwd_impl)) * mdx + (2.0 ** -8 * np.abs(rdx) if dtype == "bf16" else 0) + 1e-30
     assert np.all(np.abs(dx - rdx) <= tol_dx), np.abs(dx - rdx).max()
     blocks = min(max((N + 63) // 64, 1), 148)
     span = -(-N // blocks)
@@ -84,13 +116,46 @@ def _check(p, outs, dtype):
 ])
 def test_cg_parity(N, D, H, dtype):
     p = cg_problem(100 + N + D + H, N, D, H, dtype)
-    _check(p, _run(p, dtype), dtype)
+    impls = ["simt"]
+    if dcattn.dc_attn_cg_resolve_impl(p["x"].cuda(), H) == "tcgen05":
+        impls.append("tcgen05")
+    for impl in impls:
+        _check(p, _run(p, dtype, impl), dtype, impl)
+
+
+@pytest.mark.parametrize("N, D, H", [
+    (128, 64, 1),        # one tile, one 64-column block
+    (300, 200, 6),       # ragged tile and a ragged column block (zero-filled by TMA)
+    (1000, 2048, 8),     # widest weight that fits at 2H = 16 (a 2-stage x ring)
+    (777, 1024, 16),     # 32 outputs per split, widest that fits
+    (513, 768, 16),      # 32 outputs per split, a 5-stage ring
+    (4099, 768, 6),      # GPT-2 width, ragged last tile
+    (256, 768, 3),       # 2H = 6 padded to 16 per split
+])
+def test_cg_forward_tcgen05(N, D, H):
+    p = cg_problem(200 + N + D + H, N, D, H, "bf16")
+    assert dcattn.dc_attn_cg_resolve_impl(p["x"].cuda(), H) == "tcgen05"
+    _check(p, _run(p, "bf16", "tcgen05"), "bf16", "tcgen05")
+
+
+@pytest.mark.parametrize("N, D, H", [
+    (128, 64, 1),        # one tile, one 64-column chunk
+    (300, 200, 6),       # ragged tile, D not a multiple of 16 (last columns stored singly)
+    (1000, 1024, 8),     # widest weight that fits, four 256-column chunks
+    (4099, 768, 6),      # GPT-2 width, three chunks alternating the two TMEM buffers
+    (65, 328, 4),        # fewer tokens than a tile; a 64-column last chunk (5 blocks)
+])
+def test_cg_dx_tcgen05(N, D, H):
+    p = cg_problem(300 + N + D + H, N, D, H, "bf16")
+    _check(p, _run(p, "bf16", "simt", "tcgen05"), "bf16", "simt", "tcgen05")
 
 
 def test_cg_gpt2_full_size():
-    """The GPT-2 training shape: 16384 tokens (8 x 2048), D = 768, H = 6, every output."""
+    """The GPT-2 training shape: 16384 tokens (8 x 2048), D = 768, H = 6, every output, on
+    both forward families."""
     p = cg_problem(7, 16384, 768, 6, "bf16")
-    _check(p, _run(p, "bf16"), "bf16")
+    for impl in ("simt", "tcgen05"):
+        _check(p, _run(p, "bf16", impl), "bf16", impl)
 
 
 def test_cg_backward_is_deterministic():
@@ -115,9 +180,11 @@ def test_cg_zero_tokens_writes_zero_gradients():
     assert not dw.any() and not db.any()
 
 
-def test_cg_strided_rows():
+@pytest.mark.parametrize("dx_impl", ["simt", "tcgen05"])
+def test_cg_strided_rows(dx_impl):
     """x a column slice of a wider hidden-state buffer, dx written into a wider buffer:
-    results equal those of contiguous tensors, and the gap columns stay untouched."""
+    results equal those of contiguous tensors on the same kernel families, and the gap
+    columns stay untouched."""
     p = cg_problem(9, 700, 256, 6, "bf16")
     dev = "cuda"
     base = torch.randn(700, 256 + 10, device=dev).to(torch.bfloat16)
@@ -127,9 +194,11 @@ def test_cg_strided_rows():
     b = p["b"].to(dev)
     dc, dg = p["dc"].to(dev), p["dg"].to(dev)
     dxbuf = torch.full((700, 256 + 16), 3.0, device=dev, dtype=torch.bfloat16)
-    c, g = dcattn.dc_attn_cg_fwd(xs, w, b)
-    dx, dw, db = dcattn.dc_attn_cg_bwd(xs, w, dc, dg, dx=dxbuf[:, 8:264])
-    ref = _run(p, "bf16")
+    fwd_impl = dcattn.dc_attn_cg_resolve_impl(xs, 6)     # rows 532 bytes apart: no TMA, SIMT
+    assert fwd_impl == "simt"
+    c, g = dcattn.dc_attn_cg_fwd(xs, w, b, impl=fwd_impl)
+    dx, dw, db = dcattn.dc_attn_cg_bwd(xs, w, dc, dg, dx=dxbuf[:, 8:264], impl=dx_impl)
+    ref = _run(p, "bf16", fwd_impl, dx_impl)
     torch.cuda.synchronize()
     for u, v in zip((c, g, dxbuf[:, 8:264], dw, db), ref):
         assert torch.equal(u, v)
