@@ -405,7 +405,7 @@ CG_SHAPE = (16384, 768, 6)
 CG_SETS = 6                                  # rotating x sets: 6 x 25 MB, larger than L2
 
 
-def cg_measure(dev, hbm_gbs: float, peak_note: str) -> dict:
+def cg_measure(dev, hbm_gbs: float, peak_note: str, reps: int = 60) -> dict:
     """Graph-timed forward and backward of the c/g producer; rooflines from algorithmic
     bytes (x read once, c and g written; backward: x and e read, dx written, dweight and
     dbias written; the partial-sum records in the workspace are not algorithmic)."""
@@ -429,9 +429,10 @@ def cg_measure(dev, hbm_gbs: float, peak_note: str) -> dict:
     launches = {}
     out = {}
     stream = torch.cuda.current_stream()
-    for name, call in calls.items():
+    for name, call in calls.items():   # one direct call of each first: fwd, then the backward's kernels
         call(sets[0])
         launches[name] = dcattn.dc_attn_last_launch_count()
+    for name, call in calls.items():
         graphs = []
         for x in sets:
             g = torch.cuda.CUDAGraph()
@@ -440,7 +441,6 @@ def cg_measure(dev, hbm_gbs: float, peak_note: str) -> dict:
             graphs.append(g)
         for it in range(2 * CG_SETS):
             graphs[it % CG_SETS].replay()
-        reps = 60
         a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         a.record(stream)
         for it in range(reps):
@@ -474,6 +474,8 @@ def main():
     ap.add_argument("--impl", choices=["dcattn", "reference"], default="dcattn")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-next-rows", action="store_true", help="skip the c/g producer measurement")
+    ap.add_argument("--cg-only", action="store_true",
+                    help="only the c/g producer measurement (--steps graph replays per pass)")
     ap.add_argument("--sweep", action="store_true",
                     help="one JSON line per workload of the inputs module instead of the headline line")
     ap.add_argument("--workload", action="append", choices=list(CONFIGS),
@@ -485,6 +487,17 @@ def main():
         return run_reference(args)
     if args.sweep:
         return run_sweep(args)
+    if args.cg_only:
+        from cross_head_dynamic_b200 import build, dcattn
+        torch.cuda.set_device(0)
+        build.build()
+        dcattn.load_library()
+        peaks = json.load(open(PEAKS_FILE)) if os.path.exists(PEAKS_FILE) else {}
+        hbm = peaks.get("hbm_gbs")
+        note = "of measured" if hbm else "of fallback"
+        print(json.dumps({"next_rows": {"cg_producer": cg_measure(torch.device("cuda", 0), hbm or 6650.0, note,
+                                                                  reps=max(args.steps, 4))}}), flush=True)
+        return 0
 
     from cross_head_dynamic_b200 import build, dcattn
     world, rank, local = dist_setup(args.gpus)

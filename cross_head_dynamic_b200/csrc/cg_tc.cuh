@@ -50,7 +50,7 @@ inline size_t tc_smem_bytes(int D, int H, int stages) { return kTcFixed + (size_
 // Work item = (output o < R, 8-column chunk); each writes one 16-byte chunk in each split.
 // A thread loads the weights of kBatch items before converting any, so their L2 round
 // trips overlap.
-constexpr int kBatch = 8;
+constexpr int kBatch = 10;   // 16 outputs x 96 chunks (D = 768) over 160 threads in one round
 
 __device__ __forceinline__ void split3(float v, uint32_t &h, uint32_t &m, uint32_t &l) {
     const __nv_bfloat16 hb = __float2bfloat16_rn(v);
@@ -425,6 +425,225 @@ cg_bwd_dx_tc_kernel(CgShape s, const float *__restrict__ weight, const float *__
     ptx::tc_fence_before();
     __syncthreads();
     if (warp == 4) {
+        ptx::tc_fence_after();
+        ptx::tmem_dealloc(tmem, 512);
+    }
+}
+
+// ---------------------------------------------------------------------------------------
+// dweight on the tensor cores (bf16 x, 2H <= 16): the CTA of partial record b sums its token
+// range [b * span, (b + 1) * span) as D[m][k] = sum_t A[t][m] x[t][k] with m = split * 16 + o,
+// A[t][m] the bf16 split `split` of e[t][o] (rows m >= 48 zero), so that every product is exact
+// and dweight's partial is D[o] + D[16 + o] + D[32 + o], added in that order.  A and x are
+// MN-major operands (x straight from TMA in [64 tokens][64 columns] boxes); the columns go in
+// groups of up to 256 into two alternating TMEM buffers, each group over all the range's
+// 64-token chunks.  Warps 0-1 read TMEM rows 0-63 and write the record, warps 2-3 build the A
+// stages, warp 4 issues the TMA loads, warp 5 the MMAs.  dbias's partial is the plain fp32 sum
+// of e over the range (threads o < 2H of warp 0, tokens in order).  The record is that of the
+// CUDA-core kernel, so the same reduce kernel adds the records.
+// ---------------------------------------------------------------------------------------
+
+constexpr int kDwTcThreads = 192;
+constexpr int kDwTcStages = 3;
+constexpr int kDwTcChunk = 64;                         // tokens per A / x stage (K)
+constexpr int kDwTcXBytes = 4 * 64 * 128;              // 4 column blocks of [64 tokens][128 B]
+constexpr int kDwTcABytes = 2 * 64 * 128;              // M blocks 0 (e splits) and 1 (zero)
+constexpr int kDwTcStageBytes = kDwTcXBytes + kDwTcABytes;
+constexpr int kDwTcXRow = 257;                        // floats per exchange row (odd: rows hit distinct banks)
+constexpr size_t kDwTcSmem = 1024 + (size_t)kDwTcStages * kDwTcStageBytes + 32 * kDwTcXRow * 4 + 64 * 17 * 4 + 256;
+
+__global__ void __launch_bounds__(kDwTcThreads, 1)
+cg_bwd_dw_tc_kernel(const __grid_constant__ CUtensorMap map_x, CgShape s, int64_t span, const float *__restrict__ dc,
+                    const float *__restrict__ dg, float *__restrict__ part, uint32_t wait_ns) {
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *sm = (uint8_t *)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
+    // rows 0-15: split 2 of outputs 0-15; rows 16-31: split 0 + split 1 (one column group)
+    float *xchg = (float *)(sm + kDwTcStages * kDwTcStageBytes);
+    float *dbpart = xchg + 32 * kDwTcXRow;   // [64 A-builder threads][17]: their sums of e per output
+    uint64_t *bars = (uint64_t *)(((uintptr_t)(dbpart + 64 * 17) + 7) & ~(uintptr_t)7);
+    uint64_t *full = bars, *aready = bars + kDwTcStages, *empty = bars + 2 * kDwTcStages;
+    uint64_t *accfull = bars + 3 * kDwTcStages, *tfree = accfull + 2;
+    uint32_t *tmem_slot = (uint32_t *)(tfree + 2);
+    volatile int *abort_flag = (volatile int *)(tmem_slot + 1);
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int H2 = 2 * s.H;
+    const int64_t ta = (int64_t)blockIdx.x * span;
+    const int64_t tb = ta + span < s.N ? ta + span : s.N;
+    const int nch = tb > ta ? (int)((tb - ta + kDwTcChunk - 1) / kDwTcChunk) : 0;
+    const int nblk = (s.D + 63) / 64;
+    const int ngr = (nblk + 3) / 4;
+    const int items = ngr * nch;
+    float *rec = part + (int64_t)blockIdx.x * record_floats(s.D, s.H);
+
+    if (threadIdx.x == 0) {
+        for (int i = 0; i < kDwTcStages; ++i) {
+            ptx::mbar_init(&full[i], 1);
+            ptx::mbar_init(&aready[i], 64);
+            ptx::mbar_init(&empty[i], 1);
+        }
+        for (int i = 0; i < 2; ++i) {
+            ptx::mbar_init(&accfull[i], 1);
+            ptx::mbar_init(&tfree[i], 64);
+        }
+        tc::init_ctl(abort_flag, wait_ns);
+        ptx::fence_mbar_init();
+    }
+    if (warp == 5) {
+        ptx::tmem_alloc(tmem_slot, 512);
+        ptx::tmem_relinquish();
+    }
+    // M block 1 of every A stage stays zero
+    for (int i = threadIdx.x; i < kDwTcStages * 64 * 128 / 16; i += kDwTcThreads) {
+        const int st = i / (64 * 128 / 16), r = i - st * (64 * 128 / 16);
+        *reinterpret_cast<uint4 *>(sm + st * kDwTcStageBytes + kDwTcXBytes + 64 * 128 + r * 16) = make_uint4(0u, 0u, 0u, 0u);
+    }
+    ptx::fence_proxy_async_smem();
+    ptx::tc_fence_before();
+    __syncthreads();
+    ptx::tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+    auto group_blocks = [&](int g) { return nblk - 4 * g < 4 ? nblk - 4 * g : 4; };
+
+    if (warp == 4) {
+        if (lane == 0) {
+            ptx::prefetch_tensormap(&map_x);
+            for (int i = 0; i < items; ++i) {
+                const int st = i % kDwTcStages, g = i / nch, ch = i - g * nch;
+                if (i >= kDwTcStages && !tc::wait_bar(&empty[st], (uint32_t)((i / kDwTcStages - 1) & 1), abort_flag)) break;
+                const int nb = group_blocks(g);
+                ptx::mbar_arrive_expect_tx(&full[st], (uint32_t)nb * 8192);
+                for (int b = 0; b < nb; ++b)
+                    ptx::tma_load_2d(sm + st * kDwTcStageBytes + b * 8192, &map_x, (4 * g + b) * 64,
+                                     (int)(ta + (int64_t)ch * kDwTcChunk), &full[st]);
+            }
+        }
+    } else if (warp == 2 || warp == 3) {
+        // A stages: thread r builds token row r of the chunk (64 M values, 128 bytes); during the
+        // first column group it also sums its tokens' e per output (for dbias)
+        const int r = threadIdx.x - 64;
+        float dbacc[16];
+#pragma unroll
+        for (int o = 0; o < 16; ++o) dbacc[o] = 0.f;
+        for (int i = 0; i < items; ++i) {
+            const int st = i % kDwTcStages, g = i / nch, ch = i - g * nch;
+            if (i >= kDwTcStages && !tc::wait_bar(&empty[st], (uint32_t)((i / kDwTcStages - 1) & 1), abort_flag)) break;
+            const int64_t t = ta + (int64_t)ch * kDwTcChunk + r;
+            uint32_t w[3][8];
+#pragma unroll
+            for (int q = 0; q < 8; ++q) {
+                float e0 = 0.f, e1 = 0.f;
+                const int o0 = 2 * q, o1 = 2 * q + 1;
+                if (t < tb) {
+                    if (o0 < H2) e0 = o0 < s.H ? __ldg(dc + t * s.H + o0) : __ldg(dg + t * s.H + o0 - s.H);
+                    if (o1 < H2) e1 = o1 < s.H ? __ldg(dc + t * s.H + o1) : __ldg(dg + t * s.H + o1 - s.H);
+                }
+                if (g == 0) {
+                    dbacc[o0] += e0;
+                    dbacc[o1] += e1;
+                }
+                uint32_t h0, m0, l0, h1, m1, l1;
+                split3(e0, h0, m0, l0);
+                split3(e1, h1, m1, l1);
+                w[0][q] = h0 | (h1 << 16);
+                w[1][q] = m0 | (m1 << 16);
+                w[2][q] = l0 | (l1 << 16);
+            }
+            uint8_t *arow = sm + st * kDwTcStageBytes + kDwTcXBytes + r * 128;
+#pragma unroll
+            for (int c = 0; c < 8; ++c) {   // 16-byte chunk c holds m = 8c .. 8c + 7
+                const int sp = c >> 1, half = c & 1;
+                uint4 v = make_uint4(0u, 0u, 0u, 0u);
+                if (sp < 3) v = make_uint4(w[sp][4 * half], w[sp][4 * half + 1], w[sp][4 * half + 2], w[sp][4 * half + 3]);
+                *reinterpret_cast<uint4 *>(arow + ((c ^ (r & 7)) << 4)) = v;
+            }
+            ptx::fence_proxy_async_smem();
+            ptx::mbar_arrive(&aready[st]);
+        }
+#pragma unroll
+        for (int o = 0; o < 16; ++o) dbpart[r * 17 + o] = dbacc[o];
+        tc::named_sync(2, 128);   // warps 0-3: the dbias sums are in dbpart
+    } else if (warp == 5) {
+        if (lane == 0) {
+            bool ok = true;
+            for (int i = 0; i < items && ok; ++i) {
+                const int st = i % kDwTcStages, g = i / nch, ch = i - g * nch;
+                const int b = g & 1;
+                if (ch == 0 && g >= 2) {
+                    ok = tc::wait_bar(&tfree[b], (uint32_t)((g / 2 - 1) & 1), abort_flag);
+                    if (!ok) break;
+                }
+                ok = tc::wait_bar(&full[st], (uint32_t)((i / kDwTcStages) & 1), abort_flag) &&
+                     tc::wait_bar(&aready[st], (uint32_t)((i / kDwTcStages) & 1), abort_flag);
+                if (!ok) break;
+                ptx::tc_fence_after();
+                const uint32_t xa = ptx::smem_u32(sm + st * kDwTcStageBytes);
+                const uint32_t aa = xa + kDwTcXBytes;
+                const uint32_t idesc = ptx::idesc_bf16_f32(128, group_blocks(g) * 64, 1, 1);
+#pragma unroll
+                for (int k = 0; k < kDwTcChunk / 16; ++k) {
+                    const uint64_t ad = ptx::smem_desc_sw128(aa + k * 2048, 64 * 128, 1024);
+                    const uint64_t bd = ptx::smem_desc_sw128(xa + k * 2048, 8192, 1024);
+                    ptx::mma_bf16(tmem + b * 256, ad, bd, idesc, (ch | k) != 0);
+                }
+                ptx::mma_commit(&empty[st]);
+                if (ch == nch - 1) ptx::mma_commit(&accfull[b]);
+            }
+        }
+    } else {
+        // warps 0-1: TMEM rows 0-63 (warp 0: split 0 in lanes 0-15, split 1 in 16-31; warp 1:
+        // split 2 in lanes 0-15)
+        const uint32_t lane_base = (uint32_t)(warp * 32) << 16;
+        const int tid64 = threadIdx.x;   // 0..63
+        volatile int *verdict = abort_flag + 2;
+        // One decision for both warps (the flag may be set by other warps at any time): thread
+        // 0 copies it between two barriers of the 64 threads.
+        auto collective_abort = [&]() {
+            tc::named_sync(1, 64);
+            if (tid64 == 0) *verdict = *abort_flag;
+            tc::named_sync(1, 64);
+            return *verdict != 0;
+        };
+        for (int g = 0; g < ngr && nch > 0; ++g) {
+            const int b = g & 1;
+            (void)tc::wait_bar(&accfull[b], (uint32_t)((g / 2) & 1), abort_flag);
+            ptx::tc_fence_after();
+            if (collective_abort()) break;
+            const int ncols = group_blocks(g) * 64;
+            for (int c16 = 0; c16 < ncols / 16; ++c16) {
+                uint32_t r[16];
+                ptx::tmem_ld16_issue(tmem + b * 256 + lane_base + c16 * 16, r);
+                ptx::tmem_wait_ld();
+                ptx::reg_fence16(r);
+#pragma unroll
+                for (int e = 0; e < 16; ++e) {
+                    const float own = __uint_as_float(r[e]);
+                    const float up = __shfl_down_sync(0xffffffffu, own, 16);   // warp 0: split 1 of the same output
+                    if (lane < 16) xchg[(warp == 0 ? 16 + lane : lane) * kDwTcXRow + c16 * 16 + e] = warp == 0 ? own + up : own;
+                }
+            }
+            ptx::tc_fence_before();
+            ptx::mbar_arrive(&tfree[b]);   // TMEM buffer b may be overwritten
+            tc::named_sync(1, 64);         // the group's sums are in xchg
+            for (int o = 0; o < H2; ++o) {
+                float *dst = rec + (int64_t)o * s.D + g * 256;
+                for (int c = tid64; c < ncols && g * 256 + c < s.D; c += 64)
+                    dst[c] = xchg[(16 + o) * kDwTcXRow + c] + xchg[o * kDwTcXRow + c];   // (split 0 + split 1) + split 2
+            }
+            tc::named_sync(1, 64);   // xchg is free for the next group
+        }
+        tc::named_sync(2, 128);   // warps 0-3: the A builders' dbias sums are in dbpart
+        if (nch == 0) {   // an empty range: zero record
+            for (int64_t i = tid64; i < record_floats(s.D, s.H); i += 64) rec[i] = 0.f;
+        } else if (tid64 < H2) {
+            // dbias: the 64 builder threads' sums (each over its tokens in order), added in order
+            float acc = dbpart[tid64];
+            for (int i = 1; i < 64; ++i) acc += dbpart[i * 17 + tid64];
+            rec[(int64_t)H2 * s.D + tid64] = acc;
+        }
+    }
+    ptx::tc_fence_before();
+    __syncthreads();
+    if (warp == 5) {
         ptx::tc_fence_after();
         ptx::tmem_dealloc(tmem, 512);
     }

@@ -457,6 +457,30 @@ int cg_dx_impl(const dc_cg_params *p, const dc::cg::CgShape &s) {
     return tc_ok ? DC_IMPL_TCGEN05 : DC_IMPL_SIMT;
 }
 
+// Kernel family of the dweight partial sums: tcgen05 on request for bf16 with 2H <= 16 and x
+// rows that TMA can address (N >= 64 tokens, D >= 64); AUTO keeps the CUDA-core kernel, which
+// measured faster at the GPT-2 width (22.0 against 23.9 us for 16384 x 768 tokens).
+int cg_dw_impl(const dc_cg_params *p, const dc::cg::CgShape &s) {
+    const bool tc_ok = p->dtype == DC_BF16 && 2 * s.H <= 16 && (s.sx * 2) % 16 == 0 && s.N >= 64 && s.D >= 64;
+    if (p->impl == DC_IMPL_TCGEN05) return tc_ok ? DC_IMPL_TCGEN05 : -1;
+    return DC_IMPL_SIMT;
+}
+
+cudaError_t cg_dw_tc_launch(const dc::cg::CgShape &s, const void *x, const float *dc_, const float *dg, float *part,
+                            int blocks, cudaStream_t st) {
+    CUtensorMap m;
+    cudaError_t e = dc::tc::make_map(&m, x, s.N, 1, s.D, s.sx, dc::cg::kDwTcChunk);
+    if (e != cudaSuccess) return e;
+    e = cudaFuncSetAttribute(dc::cg::cg_bwd_dw_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)dc::cg::kDwTcSmem);
+    if (e != cudaSuccess) return e;
+    const int64_t span = (s.N + blocks - 1) / blocks;
+    dc::cg::cg_bwd_dw_tc_kernel<<<blocks, dc::cg::kDwTcThreads, dc::cg::kDwTcSmem, st>>>(
+        m, s, span, dc_, dg, part, g_wait_ns.load(std::memory_order_relaxed));
+    ++t_launches;
+    return cudaGetLastError();
+}
+
 cudaError_t cg_dx_tc_launch(const dc::cg::CgShape &s, const float *w, const float *dc_, const float *dg, void *dx,
                             cudaStream_t st) {
     const size_t smem = dc::cg::dx_tc_smem_bytes(s.D);
@@ -524,7 +548,8 @@ cudaError_t cg_fwd_launch(const dc::cg::CgShape &s, const void *x, const float *
 
 template <int OUT, typename T>
 cudaError_t cg_bwd_launch(const dc::cg::CgShape &s, const void *x, const float *w, const float *dc_, const float *dg,
-                          void *dx, float *dw, float *db, float *part, int blocks, bool dx_tc, cudaStream_t st) {
+                          void *dx, float *dw, float *db, float *part, int blocks, bool dx_tc, bool dw_tc,
+                          cudaStream_t st) {
     if (s.N > 0 && dx_tc) {
         cudaError_t e = cg_dx_tc_launch(s, w, dc_, dg, dx, st);
         if (e != cudaSuccess) return e;
@@ -539,7 +564,10 @@ cudaError_t cg_bwd_launch(const dc::cg::CgShape &s, const void *x, const float *
         kdx<<<grid, dc::cg::kThreads, smem, st>>>(s, w, dc_, dg, (T *)dx, cg_vec16<T>(s.sdx, s.D, dx));
         ++t_launches;
     }
-    if (s.N > 0) {
+    if (s.N > 0 && dw_tc) {
+        cudaError_t e = cg_dw_tc_launch(s, x, dc_, dg, part, blocks, st);
+        if (e != cudaSuccess) return e;
+    } else if (s.N > 0) {
         auto kdw = dc::cg::cg_bwd_dw_partial_kernel<T, OUT>;
         const int chunk = dc::cg::dw_chunk(s.D, s.H, sizeof(T));
         const size_t dsmem = dc::cg::dw_smem_bytes(s.D, s.H, sizeof(T));
@@ -624,12 +652,12 @@ dc_status_t dc_attn_cg_bwd(const dc_cg_params *params, const void *x, const floa
         if (workspace_bytes < cg_ws_need(s)) return DC_ERR_INVALID_ARG;
     }
     const int blocks = s.N > 0 ? dc::cg::partial_blocks(s.N) : 0;
-    const int dx_impl = cg_dx_impl(params, s);
-    if (dx_impl < 0) return DC_ERR_UNSUPPORTED;
+    const int dx_impl = cg_dx_impl(params, s), dw_impl = cg_dw_impl(params, s);
+    if (dx_impl < 0 || dw_impl < 0) return DC_ERR_UNSUPPORTED;
     cudaStream_t st = (cudaStream_t)stream;
     return cuda_status(cg_dispatch(s.H, params->dtype, [&]<int OUT, typename T>() {
         return cg_bwd_launch<OUT, T>(s, x, weight, dc_, dg, dx, dweight, dbias, (float *)workspace, blocks,
-                                     dx_impl == DC_IMPL_TCGEN05, st);
+                                     dx_impl == DC_IMPL_TCGEN05, dw_impl == DC_IMPL_TCGEN05, st);
     }));
 }
 

@@ -286,8 +286,13 @@ size_t dc_attn_cg_bwd_workspace_size(const dc_cg_params *params);
  * dx runs on tcgen05 for bf16 with 2H <= 16, a dx row stride that is a multiple of 8
  * elements and D <= 1024 (AUTO; TCGEN05 elsewhere returns DC_ERR_UNSUPPORTED): products
  * of the bf16 splits of e and of the weight, six of the nine pairs, whose sum is e * w to
- * within 2^-23 |e w|, accumulated by the tensor core; SIMT otherwise.  dweight and dbias
- * always run on the CUDA cores:
+ * within 2^-23 |e w|, accumulated by the tensor core; SIMT otherwise.  The partial sums
+ * of dweight run on the CUDA cores under AUTO and SIMT; TCGEN05 moves them to the tensor
+ * cores (bf16 with 2H <= 16, x rows that TMA can address (row stride a multiple of 8
+ * elements), N >= 64 and D >= 64): products of x with the bf16 splits of e (exact),
+ * accumulated by the tensor core over each block's tokens.  dbias and the final sum over
+ * blocks are fp32 on the CUDA cores.  TCGEN05 requires both dx and dweight to be possible
+ * on the tensor cores:
  *
  *   dx[t,k]       = sum_o e[t,o] * weight[o][k]
  *   dweight[o][k] = sum_t e[t,o] * x[t,k]        dbias[o] = sum_t e[t,o]

@@ -55,9 +55,27 @@ def _dx_on_tc(p):
     return p["x"].dtype == torch.bfloat16 and 2 * H <= 16 and D % 8 == 0 and D <= 1024
 
 
+def _dw_on_tc(p):
+    """The conditions under which AUTO runs the dweight partial sums on tcgen05 (contiguous x)."""
+    N, D = p["x"].shape
+    H = p["dc"].shape[1]
+    return p["x"].dtype == torch.bfloat16 and 2 * H <= 16 and D % 8 == 0 and N >= 64 and D >= 64
+
+
 def _dx_impl(p, fwd_impl):
-    """dx follows the forward's choice where tcgen05 is possible for it, else SIMT."""
-    return "tcgen05" if fwd_impl != "simt" and _dx_on_tc(p) else "simt"
+    """The backward's impl argument: AUTO (each kernel on tcgen05 where it can) unless the
+    forward was asked to run SIMT."""
+    return "simt" if fwd_impl == "simt" else "auto"
+
+
+def _families(p, bwd_impl):
+    """(dx family, dweight family) that a backward call with `bwd_impl` runs: AUTO takes
+    tcgen05 for dx where possible and keeps dweight on the CUDA cores; TCGEN05 both."""
+    if bwd_impl == "simt":
+        return "simt", "simt"
+    if bwd_impl == "tcgen05":
+        return "tcgen05", "tcgen05"
+    return ("tcgen05" if _dx_on_tc(p) else "simt"), "simt"
 
 
 def _fwd_tolerance(D, fwd_impl):
@@ -80,6 +98,25 @@ def _dx_tolerance(H, dx_impl):
     return 8 * 2.0 ** -22 + 2.0 ** -23
 
 
+def _dw_tolerance(N, blocks, dw_impl):
+    """dweight, relative to the sum of |terms|.  SIMT: the tokens of one record in order, then
+    the records (16 strided sums, then those 16).  tcgen05: exact products of x with the bf16
+    splits of e (2^-24 left out), the tensor core's accumulation over ceil(span / 16) steps,
+    the epilogue's two additions, then the same record sums."""
+    span = -(-N // blocks)
+    reduce = gamma(blocks // 16 + 18)
+    if dw_impl == "simt":
+        return gamma(span + blocks // 16 + 18)
+    return (-(-span // 16) + 2) * 2.0 ** -22 + 2.0 ** -24 + gamma(2) + reduce
+
+
+def _db_tolerance(N, blocks, dw_impl):
+    span = -(-N // blocks)
+    if dw_impl == "simt":
+        return gamma(span + blocks // 16 + 18)
+    return gamma(span // 64 + 66 + blocks // 16 + 18)   # 64 strided sums, then those 64, then the records
+
+
 def _check(p, outs, dtype, fwd_impl="simt", dx_impl=None):
     c, g, dx, dw, db = (_to_np(t) for t in outs)
     x, w, b = _to_np(p["x"]), _to_np(p["w"]), _to_np(p["b"])
@@ -93,13 +130,13 @@ def _check(p, outs, dtype, fwd_impl="simt", dx_impl=None):
     assert np.all(np.abs(g - rg) <= tf * mg + 1e-30), np.abs(g - rg).max()
     rdx, rdw, rdb = oracle.cg_backward(x, w, dcn, dgn)
     mdx, mdw, mdb = oracle.cg_backward(np.abs(x), np.abs(w), np.abs(dcn), np.abs(dgn))
-    tol_dx = _dx_tolerance(H, dx_impl or _dx_impl(p, fwd_impl)) * mdx + (2.0 ** -8 * np.abs(rdx) if dtype == "bf16" else 0) + 1e-30
+    dx_fam, dw_fam = _families(p, dx_impl or _dx_impl(p, fwd_impl))
+    tol_dx = _dx_tolerance(H, dx_fam) * mdx + (2.0 ** -8 * np.abs(rdx) if dtype == "bf16" else 0) + 1e-30
     assert np.all(np.abs(dx - rdx) <= tol_dx), np.abs(dx - rdx).max()
     blocks = min(max((N + 63) // 64, 1), 148)
-    span = -(-N // blocks)
-    tw = gamma(span + blocks // 16 + 18)
+    tw, tb = _dw_tolerance(N, blocks, dw_fam), _db_tolerance(N, blocks, dw_fam)
     assert np.all(np.abs(dw.T - rdw) <= tw * mdw + 1e-30), np.abs(dw.T - rdw).max()
-    assert np.all(np.abs(db - rdb) <= tw * mdb + 1e-30), np.abs(db - rdb).max()
+    assert np.all(np.abs(db - rdb) <= tb * mdb + 1e-30), np.abs(db - rdb).max()
 
 
 @pytest.mark.parametrize("N, D, H, dtype", [
@@ -145,8 +182,18 @@ def test_cg_forward_tcgen05(N, D, H):
     (4099, 768, 6),      # GPT-2 width, three chunks alternating the two TMEM buffers
     (65, 328, 4),        # fewer tokens than a tile; a 64-column last chunk (5 blocks)
 ])
-def test_cg_dx_tcgen05(N, D, H):
+def test_cg_backward_tcgen05(N, D, H):
+    """dx and the dweight partial sums both on tcgen05 (forced)."""
     p = cg_problem(300 + N + D + H, N, D, H, "bf16")
+    _check(p, _run(p, "bf16", "simt", "tcgen05"), "bf16", "simt", "tcgen05")
+
+
+@pytest.mark.parametrize("N", [64, 8191, 20000, 300000])
+def test_cg_dweight_tcgen05_spans(N):
+    """Token ranges of 1, several and many 64-token chunks per record (the record count is
+    capped at 148), a ragged last chunk, and ranges that end inside a TMA box."""
+    p = cg_problem(400 + N, N, 256, 6, "bf16")
+    assert _dw_on_tc(p)
     _check(p, _run(p, "bf16", "simt", "tcgen05"), "bf16", "simt", "tcgen05")
 
 
@@ -180,25 +227,25 @@ def test_cg_zero_tokens_writes_zero_gradients():
     assert not dw.any() and not db.any()
 
 
-@pytest.mark.parametrize("dx_impl", ["simt", "tcgen05"])
-def test_cg_strided_rows(dx_impl):
+@pytest.mark.parametrize("width, impl", [(266, "simt"), (264, "tcgen05")])
+def test_cg_strided_rows(width, impl):
     """x a column slice of a wider hidden-state buffer, dx written into a wider buffer:
     results equal those of contiguous tensors on the same kernel families, and the gap
-    columns stay untouched."""
+    columns stay untouched.  Rows 532 bytes apart (no TMA): SIMT; 528 bytes apart: every
+    kernel on tcgen05."""
     p = cg_problem(9, 700, 256, 6, "bf16")
     dev = "cuda"
-    base = torch.randn(700, 256 + 10, device=dev).to(torch.bfloat16)
-    base[:, 8:264] = p["x"].to(dev)          # 16-byte aligned start; rows 532 bytes apart
+    base = torch.randn(700, width, device=dev).to(torch.bfloat16)
+    base[:, 8:264] = p["x"].to(dev)          # 16-byte aligned start
     xs = base[:, 8:264]
     w = p["w"].to(dev).t().contiguous()
     b = p["b"].to(dev)
     dc, dg = p["dc"].to(dev), p["dg"].to(dev)
     dxbuf = torch.full((700, 256 + 16), 3.0, device=dev, dtype=torch.bfloat16)
-    fwd_impl = dcattn.dc_attn_cg_resolve_impl(xs, 6)     # rows 532 bytes apart: no TMA, SIMT
-    assert fwd_impl == "simt"
-    c, g = dcattn.dc_attn_cg_fwd(xs, w, b, impl=fwd_impl)
-    dx, dw, db = dcattn.dc_attn_cg_bwd(xs, w, dc, dg, dx=dxbuf[:, 8:264], impl=dx_impl)
-    ref = _run(p, "bf16", fwd_impl, dx_impl)
+    assert dcattn.dc_attn_cg_resolve_impl(xs, 6) == ("simt" if width == 266 else "tcgen05")
+    c, g = dcattn.dc_attn_cg_fwd(xs, w, b, impl=impl)
+    dx, dw, db = dcattn.dc_attn_cg_bwd(xs, w, dc, dg, dx=dxbuf[:, 8:264], impl=impl)
+    ref = _run(p, "bf16", impl, impl)
     torch.cuda.synchronize()
     for u, v in zip((c, g, dxbuf[:, 8:264], dw, db), ref):
         assert torch.equal(u, v)
