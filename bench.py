@@ -420,11 +420,14 @@ def cg_measure(dev, hbm_gbs: float, peak_note: str, reps: int = 60) -> dict:
         x["c"], x["gg"] = torch.empty(N, H, device=dev), torch.empty(N, H, device=dev)
         x["dx"], x["dw"], x["db"] = torch.empty_like(x["x"]), torch.empty_like(x["wt"]), torch.empty_like(x["b"])
         x["ws"] = torch.empty(dcattn.dc_attn_cg_bwd_workspace_size(x["x"], H), device=dev, dtype=torch.uint8)
+        x["img"] = dcattn.dc_attn_cg_prepare(x["wt"])
         sets.append(x)
+    # A training step converts its weight once (prepare) and runs forward and backward on it.
     calls = {
-        "fwd": lambda x: dcattn.dc_attn_cg_fwd(x["x"], x["wt"], x["b"], c=x["c"], g=x["gg"]),
+        "fwd": lambda x: dcattn.dc_attn_cg_fwd(x["x"], x["wt"], x["b"], c=x["c"], g=x["gg"], weight_splits=x["img"]),
         "bwd": lambda x: dcattn.dc_attn_cg_bwd(x["x"], x["wt"], x["dc"], x["dg"], dx=x["dx"], dweight=x["dw"],
-                                               dbias=x["db"], workspace=x["ws"]),
+                                               dbias=x["db"], workspace=x["ws"], weight_splits=x["img"]),
+        "prepare": lambda x: dcattn.dc_attn_cg_prepare(x["wt"], splits=x["img"]),
     }
     launches = {}
     out = {}
@@ -457,6 +460,9 @@ def cg_measure(dev, hbm_gbs: float, peak_note: str, reps: int = 60) -> dict:
     flops = 2.0 * N * D * 2 * H
     res = {"workload": f"x [{N}][{D}] bf16, H = {H} (c, g fp32); {CG_SETS} rotating input sets (> L2)",
            "form": "assumed per-token affine map (the pages give no formula)"}
+    res["prepare"] = {"us": out["prepare"], "launches": launches["prepare"],
+                      "note": "the weight's bf16 splits for the tensor-core kernels, once per weight update"}
+    res["step_us"] = out["prepare"] + out["fwd"] + out["bwd"]
     for name, nbytes, nflops in (("fwd", fwd_bytes, flops), ("bwd", bwd_bytes, 2 * flops)):
         t = out[name] * 1e-6
         res[name] = {"us": out[name], "launches": launches[name], "algorithmic_bytes": nbytes,

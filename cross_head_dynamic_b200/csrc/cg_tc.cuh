@@ -111,8 +111,8 @@ __device__ __forceinline__ void stage_weight_splits(const CgShape &s, const floa
 template <int R>
 __global__ void __launch_bounds__(kTcThreads, 1)
 cg_fwd_tc_kernel(const __grid_constant__ CUtensorMap map_x, CgShape s, const float *__restrict__ weight,
-                 const float *__restrict__ bias, float *__restrict__ c, float *__restrict__ g, int nst,
-                 uint32_t wait_ns) {
+                 const uint8_t *__restrict__ splits, const float *__restrict__ bias, float *__restrict__ c,
+                 float *__restrict__ g, int nst, uint32_t wait_ns) {
     constexpr int NCOL = 3 * R;                  // MMA N
     constexpr uint32_t TMEM_COLS = NCOL <= 64 ? 64 : 128;
     extern __shared__ uint8_t smem_raw[];
@@ -122,6 +122,7 @@ cg_fwd_tc_kernel(const __grid_constant__ CUtensorMap map_x, CgShape s, const flo
     uint8_t *wb = sm + (size_t)nst * 16384;
     uint64_t *bars = (uint64_t *)(wb + (size_t)nkb * NCOL * 128);
     uint64_t *full = bars, *empty = bars + kTcMaxStages, *accfull = bars + 2 * kTcMaxStages;
+    uint64_t *wready = accfull + 1;   // the prepared weight image has landed
     uint32_t *tmem_slot = (uint32_t *)(bars + 2 * kTcMaxStages + 2);
     volatile int *abort_flag = (volatile int *)(tmem_slot + 1);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -131,7 +132,7 @@ cg_fwd_tc_kernel(const __grid_constant__ CUtensorMap map_x, CgShape s, const flo
     // threads meanwhile write the weight splits.
     const int first = nkb < nst ? nkb : nst;
     if (warp == 4 && lane == 0) {
-        for (int i = 0; i < 2 * kTcMaxStages + 1; ++i) ptx::mbar_init(&bars[i], 1);
+        for (int i = 0; i < 2 * kTcMaxStages + 2; ++i) ptx::mbar_init(&bars[i], 1);
         tc::init_ctl(abort_flag, wait_ns);
         ptx::fence_mbar_init();
         ptx::prefetch_tensormap(&map_x);
@@ -139,12 +140,17 @@ cg_fwd_tc_kernel(const __grid_constant__ CUtensorMap map_x, CgShape s, const flo
             ptx::mbar_arrive_expect_tx(&full[kb], 16384);
             ptx::tma_load_2d(xs + kb * 16384, &map_x, kb * 64, (int)t0, &full[kb]);
         }
+        if (splits) {   // the weight image, one bulk copy per 64-column block
+            ptx::mbar_arrive_expect_tx(wready, (uint32_t)(nkb * NCOL * 128));
+            for (int kb = 0; kb < nkb; ++kb)
+                ptx::bulk_load(wb + kb * NCOL * 128, splits + (size_t)kb * NCOL * 128, NCOL * 128, wready);
+        }
     }
     if (warp == 5) {
         ptx::tmem_alloc(tmem_slot, TMEM_COLS);
         ptx::tmem_relinquish();
     }
-    if (warp != 4) {
+    if (warp != 4 && !splits) {
         const int tid = warp < 4 ? threadIdx.x : threadIdx.x - 32;   // warps 0-3 and 5
         stage_weight_splits<R>(s, weight, wb, nkb, tid, kTcThreads - 32);
     }
@@ -166,7 +172,7 @@ cg_fwd_tc_kernel(const __grid_constant__ CUtensorMap map_x, CgShape s, const flo
     } else if (warp == 5) {
         if (lane == 0) {
             const uint32_t idesc = ptx::idesc_bf16_f32(128, NCOL, 0, 0);
-            bool ok = true;
+            bool ok = !splits || tc::wait_bar(wready, 0, abort_flag);
             for (int kb = 0; kb < nkb && ok; ++kb) {
                 const int st = kb % nst;
                 ok = tc::wait_bar(&full[st], (uint32_t)((kb / nst) & 1), abort_flag);
@@ -291,8 +297,9 @@ __device__ __forceinline__ void stage_dx_weight(const CgShape &s, const float *_
 }
 
 __global__ void __launch_bounds__(kDxThreads, 1)
-cg_bwd_dx_tc_kernel(CgShape s, const float *__restrict__ weight, const float *__restrict__ dc,
-                    const float *__restrict__ dg, __nv_bfloat16 *__restrict__ dx, uint32_t wait_ns) {
+cg_bwd_dx_tc_kernel(CgShape s, const float *__restrict__ weight, const uint8_t *__restrict__ splits,
+                    const float *__restrict__ dc, const float *__restrict__ dg, __nv_bfloat16 *__restrict__ dx,
+                    uint32_t wait_ns) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t *sm = (uint8_t *)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
     const int nblk = (s.D + 63) / 64;
@@ -300,8 +307,8 @@ cg_bwd_dx_tc_kernel(CgShape s, const float *__restrict__ weight, const float *__
     uint8_t *as = sm;                 // A: two K blocks of [128 rows][128 bytes]
     uint8_t *wb = sm + 2 * 16384;     // B
     uint64_t *bars = (uint64_t *)(wb + (size_t)nblk * kDxBRow);
-    uint64_t *accfull = bars, *tfree = bars + 2;
-    uint32_t *tmem_slot = (uint32_t *)(bars + 4);
+    uint64_t *accfull = bars, *tfree = bars + 2, *wready = bars + 4;
+    uint32_t *tmem_slot = (uint32_t *)(bars + 5);
     volatile int *abort_flag = (volatile int *)(tmem_slot + 1);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int64_t t0 = (int64_t)blockIdx.x * kTcTile;
@@ -311,8 +318,14 @@ cg_bwd_dx_tc_kernel(CgShape s, const float *__restrict__ weight, const float *__
         ptx::mbar_init(&accfull[1], 1);
         ptx::mbar_init(&tfree[0], 128);
         ptx::mbar_init(&tfree[1], 128);
+        ptx::mbar_init(wready, 1);
         tc::init_ctl(abort_flag, wait_ns);
         ptx::fence_mbar_init();
+        if (splits) {   // the weight image, one bulk copy per 64-column block
+            ptx::mbar_arrive_expect_tx(wready, (uint32_t)(nblk * kDxBRow));
+            for (int kb = 0; kb < nblk; ++kb)
+                ptx::bulk_load(wb + kb * kDxBRow, splits + (size_t)kb * kDxBRow, kDxBRow, wready);
+        }
     }
     if (warp == 4) {
         ptx::tmem_alloc(tmem_slot, 512);
@@ -350,7 +363,7 @@ cg_bwd_dx_tc_kernel(CgShape s, const float *__restrict__ weight, const float *__
             *reinterpret_cast<uint4 *>(as + blk * 16384 + row * 128 + ((c16 ^ (row & 7)) << 4)) = v;
         }
     }
-    stage_dx_weight(s, weight, wb, nblk, threadIdx.x, kDxThreads);
+    if (!splits) stage_dx_weight(s, weight, wb, nblk, threadIdx.x, kDxThreads);
     ptx::fence_proxy_async_smem();
     ptx::tc_fence_before();
     __syncthreads();
@@ -359,7 +372,7 @@ cg_bwd_dx_tc_kernel(CgShape s, const float *__restrict__ weight, const float *__
 
     if (warp == 4) {
         if (lane == 0) {
-            bool ok = true;
+            bool ok = !splits || tc::wait_bar(wready, 0, abort_flag);
             const uint32_t aa = ptx::smem_u32(as), ba = ptx::smem_u32(wb);
             for (int c = 0; c < nch && ok; ++c) {
                 const int b = c & 1;
@@ -647,6 +660,26 @@ cg_bwd_dw_tc_kernel(const __grid_constant__ CUtensorMap map_x, CgShape s, int64_
         ptx::tc_fence_after();
         ptx::tmem_dealloc(tmem, 512);
     }
+}
+
+// ---------------------------------------------------------------------------------------
+// The weight's bf16 split images, written once per weight: the forward's B operand
+// (3R x 128 bytes per 64-column block) followed, when 2H <= 16, by dx's (96 x 128 bytes per
+// block), byte for byte what the kernels otherwise build in shared memory, so results are
+// identical with or without them.
+// ---------------------------------------------------------------------------------------
+__host__ __device__ inline size_t prep_fwd_bytes(int D, int H) { return tc_split_bytes(D, H); }
+__host__ __device__ inline size_t prep_dx_bytes(int D, int H) {
+    return 2 * H <= 16 ? (size_t)kDxBRow * ((D + 63) / 64) : 0;
+}
+
+template <int R>
+__global__ void __launch_bounds__(256) cg_prepare_kernel(CgShape s, const float *__restrict__ weight,
+                                                        uint8_t *__restrict__ img) {
+    const int nkb = (s.D + 63) / 64;
+    const int tid = blockIdx.x * blockDim.x + threadIdx.x, nth = gridDim.x * blockDim.x;
+    stage_weight_splits<R>(s, weight, img, nkb, tid, nth);
+    if (R == 16) stage_dx_weight(s, weight, img + prep_fwd_bytes(s.D, s.H), nkb, tid, nth);
 }
 
 }  // namespace cg

@@ -424,6 +424,7 @@ dc_status_t check_cg(const dc_cg_params *p, dc::cg::CgShape *s) {
     const int64_t D = p->model_dim;
     const int64_t sx = p->stride_x ? p->stride_x : D, sdx = p->stride_dx ? p->stride_dx : D;
     if (sx < D || sdx < D || (sx & 1) || (sdx & 1)) return DC_ERR_INVALID_ARG;
+    if (p->weight_splits && !aligned16(p->weight_splits)) return DC_ERR_INVALID_ARG;
     if (p->impl != DC_IMPL_AUTO && p->impl != DC_IMPL_SIMT && p->impl != DC_IMPL_TCGEN05) return DC_ERR_INVALID_ARG;
     if (p->num_heads > 16) return DC_ERR_UNSUPPORTED;
     // the forward keeps the weight and one tile's partial sums in shared memory
@@ -481,22 +482,23 @@ cudaError_t cg_dw_tc_launch(const dc::cg::CgShape &s, const void *x, const float
     return cudaGetLastError();
 }
 
-cudaError_t cg_dx_tc_launch(const dc::cg::CgShape &s, const float *w, const float *dc_, const float *dg, void *dx,
-                            cudaStream_t st) {
+cudaError_t cg_dx_tc_launch(const dc::cg::CgShape &s, const float *w, const uint8_t *splits, const float *dc_,
+                            const float *dg, void *dx, cudaStream_t st) {
     const size_t smem = dc::cg::dx_tc_smem_bytes(s.D);
     cudaError_t e = cudaFuncSetAttribute(dc::cg::cg_bwd_dx_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          (int)smem);
     if (e != cudaSuccess) return e;
     const unsigned grid = (unsigned)((s.N + dc::cg::kTcTile - 1) / dc::cg::kTcTile);
-    dc::cg::cg_bwd_dx_tc_kernel<<<grid, dc::cg::kDxThreads, smem, st>>>(s, w, dc_, dg, (__nv_bfloat16 *)dx,
-                                                                         g_wait_ns.load(std::memory_order_relaxed));
+    dc::cg::cg_bwd_dx_tc_kernel<<<grid, dc::cg::kDxThreads, smem, st>>>(
+        s, w, splits ? splits + dc::cg::prep_fwd_bytes(s.D, s.H) : nullptr, dc_, dg, (__nv_bfloat16 *)dx,
+        g_wait_ns.load(std::memory_order_relaxed));
     ++t_launches;
     return cudaGetLastError();
 }
 
 template <int R>
-cudaError_t cg_fwd_tc_launch(const dc::cg::CgShape &s, const void *x, const float *w, const float *b, float *c,
-                             float *g, cudaStream_t st) {
+cudaError_t cg_fwd_tc_launch(const dc::cg::CgShape &s, const void *x, const float *w, const uint8_t *splits,
+                             const float *b, float *c, float *g, cudaStream_t st) {
     CUtensorMap m;
     cudaError_t e = dc::tc::make_map(&m, x, s.N, 1, s.D, s.sx, dc::cg::kTcTile);
     if (e != cudaSuccess) return e;
@@ -506,7 +508,8 @@ cudaError_t cg_fwd_tc_launch(const dc::cg::CgShape &s, const void *x, const floa
     e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     const unsigned grid = (unsigned)((s.N + dc::cg::kTcTile - 1) / dc::cg::kTcTile);
-    kern<<<grid, dc::cg::kTcThreads, smem, st>>>(m, s, w, b, c, g, nst, g_wait_ns.load(std::memory_order_relaxed));
+    kern<<<grid, dc::cg::kTcThreads, smem, st>>>(m, s, w, splits, b, c, g, nst,
+                                                  g_wait_ns.load(std::memory_order_relaxed));
     ++t_launches;
     return cudaGetLastError();
 }
@@ -549,9 +552,9 @@ cudaError_t cg_fwd_launch(const dc::cg::CgShape &s, const void *x, const float *
 template <int OUT, typename T>
 cudaError_t cg_bwd_launch(const dc::cg::CgShape &s, const void *x, const float *w, const float *dc_, const float *dg,
                           void *dx, float *dw, float *db, float *part, int blocks, bool dx_tc, bool dw_tc,
-                          cudaStream_t st) {
+                          const uint8_t *splits, cudaStream_t st) {
     if (s.N > 0 && dx_tc) {
-        cudaError_t e = cg_dx_tc_launch(s, w, dc_, dg, dx, st);
+        cudaError_t e = cg_dx_tc_launch(s, w, splits, dc_, dg, dx, st);
         if (e != cudaSuccess) return e;
     } else if (s.N > 0) {
         auto kdx = dc::cg::cg_bwd_dx_kernel<T, OUT>;
@@ -618,8 +621,11 @@ dc_status_t dc_attn_cg_fwd(const dc_cg_params *params, const void *x, const floa
     if (impl < 0) return DC_ERR_UNSUPPORTED;
     cudaStream_t st = (cudaStream_t)stream;
     if (impl == DC_IMPL_TCGEN05)
-        return cuda_status(dc::cg::tc_rows_per_split(s.H) == 16 ? cg_fwd_tc_launch<16>(s, x, weight, bias, c, g, st)
-                                                                : cg_fwd_tc_launch<32>(s, x, weight, bias, c, g, st));
+    {
+        const uint8_t *sp = (const uint8_t *)params->weight_splits;
+        return cuda_status(dc::cg::tc_rows_per_split(s.H) == 16 ? cg_fwd_tc_launch<16>(s, x, weight, sp, bias, c, g, st)
+                                                                : cg_fwd_tc_launch<32>(s, x, weight, sp, bias, c, g, st));
+    }
     return cuda_status(cg_dispatch(s.H, params->dtype, [&]<int OUT, typename T>() {
         return cg_fwd_launch<OUT, T>(s, x, weight, bias, c, g, st);
     }));
@@ -657,8 +663,34 @@ dc_status_t dc_attn_cg_bwd(const dc_cg_params *params, const void *x, const floa
     cudaStream_t st = (cudaStream_t)stream;
     return cuda_status(cg_dispatch(s.H, params->dtype, [&]<int OUT, typename T>() {
         return cg_bwd_launch<OUT, T>(s, x, weight, dc_, dg, dx, dweight, dbias, (float *)workspace, blocks,
-                                     dx_impl == DC_IMPL_TCGEN05, dw_impl == DC_IMPL_TCGEN05, st);
+                                     dx_impl == DC_IMPL_TCGEN05, dw_impl == DC_IMPL_TCGEN05,
+                                     (const uint8_t *)params->weight_splits, st);
     }));
+}
+
+size_t dc_attn_cg_prepare_size(const dc_cg_params *params) {
+    dc::cg::CgShape s;
+    if (check_cg(params, &s) != DC_OK) return 0;
+    return dc::cg::prep_fwd_bytes(s.D, s.H) + dc::cg::prep_dx_bytes(s.D, s.H);
+}
+
+dc_status_t dc_attn_cg_prepare(const dc_cg_params *params, const float *weight, void *splits, void *stream) {
+    dc::cg::CgShape s;
+    dc_status_t r = check_cg(params, &s);
+    if (r != DC_OK) return r;
+    t_launches = 0;
+    r = ptrs_ok({weight, splits}, {});
+    if (r != DC_OK) return r;
+    cudaStream_t st = (cudaStream_t)stream;
+    const int R = dc::cg::tc_rows_per_split(s.H);
+    const int64_t items = (int64_t)R * ((s.D + 63) / 64) * 8;
+    const unsigned blocks = (unsigned)((items + 255) / 256 < 148 ? (items + 255) / 256 : 148);
+    if (R == 16)
+        dc::cg::cg_prepare_kernel<16><<<blocks, 256, 0, st>>>(s, weight, (uint8_t *)splits);
+    else
+        dc::cg::cg_prepare_kernel<32><<<blocks, 256, 0, st>>>(s, weight, (uint8_t *)splits);
+    ++t_launches;
+    return cuda_status(cudaGetLastError());
 }
 
 }  // extern "C"

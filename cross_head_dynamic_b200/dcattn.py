@@ -26,7 +26,7 @@ EXPORTED = ("dc_attn_fwd", "dc_attn_bwd_workspace_size", "dc_attn_bwd_query", "d
             "dc_attn_bwd", "dc_attn_resolve_impl", "dc_attn_device_status", "dc_attn_status_string",
             "dc_attn_last_launch_count", "dc_attn_bwd_noalloc", "dc_attn_halo_add", "dc_attn_set_wait_limit",
             "dc_attn_inject_missing_load", "dc_attn_cg_fwd", "dc_attn_cg_bwd_workspace_size", "dc_attn_cg_bwd",
-            "dc_attn_cg_resolve_impl")
+            "dc_attn_cg_resolve_impl", "dc_attn_cg_prepare_size", "dc_attn_cg_prepare")
 
 
 class DCAttnError(RuntimeError):
@@ -46,7 +46,7 @@ class Params(ctypes.Structure):
 class CgParams(ctypes.Structure):
     _fields_ = [("dtype", ctypes.c_int32), ("model_dim", ctypes.c_int32), ("num_heads", ctypes.c_int32),
                 ("impl", ctypes.c_int32), ("num_tokens", ctypes.c_int64), ("stride_x", ctypes.c_int64),
-                ("stride_dx", ctypes.c_int64)]
+                ("stride_dx", ctypes.c_int64), ("weight_splits", ctypes.c_void_p)]
 
 
 _lib = None
@@ -98,6 +98,10 @@ def load_library(path: str = LIB_PATH):
     lib.dc_attn_cg_bwd.restype = st
     lib.dc_attn_cg_resolve_impl.argtypes = [CP]
     lib.dc_attn_cg_resolve_impl.restype = ctypes.c_int32
+    lib.dc_attn_cg_prepare_size.argtypes = [CP]
+    lib.dc_attn_cg_prepare_size.restype = ctypes.c_size_t
+    lib.dc_attn_cg_prepare.argtypes = [CP, vp, vp, vp]
+    lib.dc_attn_cg_prepare.restype = st
     _lib = lib
     return lib
 
@@ -335,14 +339,32 @@ def _token_rows(x: torch.Tensor, name: str, dtype=None) -> int:
     return int(x.stride(0)) if x.shape[0] > 1 else 0
 
 
-def make_cg_params(x: torch.Tensor, num_heads: int, dx=None, impl: str = "auto") -> CgParams:
+def make_cg_params(x: torch.Tensor, num_heads: int, dx=None, impl: str = "auto", weight_splits=None) -> CgParams:
     dt = {torch.float32: DC_F32, torch.bfloat16: DC_BF16}.get(x.dtype)
     if dt is None:
         raise TypeError(f"unsupported dtype {x.dtype}")
     sx = _token_rows(x, "x")
     sdx = 0 if dx is None else _token_rows(dx, "dx", x.dtype)
     return CgParams(dtype=dt, model_dim=int(x.shape[1]), num_heads=int(num_heads), impl=IMPLS[impl],
-                    num_tokens=int(x.shape[0]), stride_x=sx, stride_dx=sdx)
+                    num_tokens=int(x.shape[0]), stride_x=sx, stride_dx=sdx,
+                    weight_splits=None if weight_splits is None else _dev(weight_splits, "weight_splits"))
+
+
+def dc_attn_cg_prepare(weight, *, splits=None, stream=None):
+    """The weight [2H, D] fp32 as the tensor-core kernels read it (bf16 splits in their
+    shared-memory layout); pass the result as weight_splits= to the producer's calls while
+    the weight is unchanged.  Returns the image (uint8 device tensor)."""
+    H, D = weight.shape[0] // 2, weight.shape[1]
+    probe = torch.empty(0, D, device=weight.device, dtype=torch.bfloat16)
+    p = make_cg_params(probe, H)
+    n = int(load_library().dc_attn_cg_prepare_size(ctypes.byref(p)))
+    if n == 0:
+        raise DCAttnError("dc_attn_cg_prepare_size", DC_ERR_INVALID_ARG, "invalid parameters")
+    splits = torch.empty(n, device=weight.device, dtype=torch.uint8) if splits is None else splits
+    code = load_library().dc_attn_cg_prepare(ctypes.byref(p), _dev(weight, "weight", torch.float32),
+                                             _dev(splits, "splits"), _stream_handle(stream))
+    _check("dc_attn_cg_prepare", code)
+    return splits
 
 
 def dc_attn_cg_resolve_impl(x, num_heads: int, impl: str = "auto") -> str:
@@ -353,14 +375,14 @@ def dc_attn_cg_resolve_impl(x, num_heads: int, impl: str = "auto") -> str:
     return IMPL_NAMES[r]
 
 
-def dc_attn_cg_fwd(x, weight, bias, *, c=None, g=None, impl: str = "auto", stream=None):
+def dc_attn_cg_fwd(x, weight, bias, *, c=None, g=None, impl: str = "auto", weight_splits=None, stream=None):
     """c, g [N, H] fp32 from the hidden state x [N, D] (per-token affine maps; weight
     [2H, D] fp32 in a linear layer's layout, bias [2H] fp32).  Returns (c, g)."""
     H = weight.shape[0] // 2
     N = x.shape[0]
     c = torch.empty(N, H, device=x.device, dtype=torch.float32) if c is None else c
     g = torch.empty(N, H, device=x.device, dtype=torch.float32) if g is None else g
-    p = make_cg_params(x, H, impl=impl)
+    p = make_cg_params(x, H, impl=impl, weight_splits=weight_splits)
     code = load_library().dc_attn_cg_fwd(ctypes.byref(p), x.data_ptr(), _dev(weight, "weight", torch.float32),
                                          _dev(bias, "bias", torch.float32), _dev(c, "c", torch.float32),
                                          _dev(g, "g", torch.float32), _stream_handle(stream))
@@ -374,7 +396,7 @@ def dc_attn_cg_bwd_workspace_size(x, num_heads: int) -> int:
 
 
 def dc_attn_cg_bwd(x, weight, dc, dg, *, dx=None, dweight=None, dbias=None, workspace=None, impl: str = "auto",
-                   stream=None):
+                   weight_splits=None, stream=None):
     """Gradients of the c/g producer for dL/dc = dc, dL/dg = dg.  Returns
     (dx, dweight, dbias); dweight and dbias are bitwise reproducible for a given N.
     `impl` chooses the kernel family of dx."""
@@ -382,7 +404,7 @@ def dc_attn_cg_bwd(x, weight, dc, dg, *, dx=None, dweight=None, dbias=None, work
     dx = torch.empty(x.shape, device=x.device, dtype=x.dtype) if dx is None else dx
     dweight = torch.empty(weight.shape, device=x.device, dtype=torch.float32) if dweight is None else dweight
     dbias = torch.empty(2 * H, device=x.device, dtype=torch.float32) if dbias is None else dbias
-    p = make_cg_params(x, H, dx, impl=impl)
+    p = make_cg_params(x, H, dx, impl=impl, weight_splits=weight_splits)
     if workspace is None:
         workspace = torch.empty(max(dc_attn_cg_bwd_workspace_size(x, H), 16), device=x.device, dtype=torch.uint8)
     code = load_library().dc_attn_cg_bwd(

@@ -261,6 +261,10 @@ typedef struct {
     int64_t num_tokens;   /* N >= 0                                                   */
     int64_t stride_x;     /* elements between tokens of x (0 = D)                     */
     int64_t stride_dx;    /* elements between tokens of dx (0 = D)                    */
+    const void *weight_splits;  /* NULL, or the image dc_attn_cg_prepare wrote for this
+                                 * weight (device, 16-byte aligned): the tcgen05 kernels
+                                 * then copy it instead of converting the weight
+                                 * themselves; results are identical either way         */
 } dc_cg_params;
 
 /* c, g from x.  N = 0 launches nothing.
@@ -277,6 +281,15 @@ dc_status_t dc_attn_cg_fwd(const dc_cg_params *params, const void *x, const floa
 /* Which family the forward resolves to (DC_IMPL_SIMT or DC_IMPL_TCGEN05), or -1 if the
  * params are invalid or ask for TCGEN05 where it is not possible. */
 int32_t dc_attn_cg_resolve_impl(const dc_cg_params *params);
+
+/* The weight in the form the tensor-core kernels read (the bf16 splits, laid out as
+ * their shared-memory operands), for callers that run the producer many times with one
+ * weight (a training step's forward and backward): written once with dc_attn_cg_prepare
+ * and passed as params->weight_splits.  Size in bytes for the params' D and H (dtype,
+ * N and strides do not matter; 0 if the params are invalid).  The image depends only
+ * on the weight's values; after the weight changes it must be prepared again. */
+size_t dc_attn_cg_prepare_size(const dc_cg_params *params);
+dc_status_t dc_attn_cg_prepare(const dc_cg_params *params, const float *weight, void *splits, void *stream);
 
 /* Bytes of workspace dc_attn_cg_bwd needs (0 when N = 0 or the params are
  * invalid): one fp32 partial record of dweight and dbias per block of tokens. */

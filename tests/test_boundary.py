@@ -236,3 +236,17 @@ def test_cg_resolve_impl(lib):
     p = _cg(impl=tc, dtype=dcattn.DC_F32)
     a = 0x4000
     assert lib.dc_attn_cg_fwd(ctypes.byref(p), a, a, a, a, a, None) == dcattn.DC_ERR_UNSUPPORTED
+
+
+def test_cg_prepare_size_and_alignment(lib):
+    """The weight image holds the forward's splits (3 x 16 rows x 128 bytes per 64 columns)
+    and, for 2H <= 16, dx's (96 rows x 128 bytes per 64 columns); a misaligned image
+    pointer is refused on the host."""
+    p = _cg()
+    assert lib.dc_attn_cg_prepare_size(ctypes.byref(p)) == 12 * (48 * 128 + 96 * 128)
+    p16 = _cg(num_heads=16, model_dim=1024)
+    assert lib.dc_attn_cg_prepare_size(ctypes.byref(p16)) == 16 * 96 * 128
+    a = 0x4000
+    pm = _cg(weight_splits=a + 8)
+    assert lib.dc_attn_cg_fwd(ctypes.byref(pm), a, a, a, a, a, None) == dcattn.DC_ERR_INVALID_ARG
+    assert lib.dc_attn_cg_prepare(ctypes.byref(_cg()), a, a + 4, None) == dcattn.DC_ERR_INVALID_ARG

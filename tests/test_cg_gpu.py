@@ -268,3 +268,24 @@ def test_cg_feeds_the_attention_forward():
     ro = oracle.forward(_to_np(q), _to_np(k), _to_np(v), rc, rg, cu.numpy(), W, scale)[0]
     err = np.abs(_to_np(o) - ro)
     assert err.max() <= 0.02 * np.abs(ro).max(), err.max()
+
+
+@pytest.mark.parametrize("N, D, H", [(16384, 768, 6), (300, 200, 6), (777, 1024, 16), (256, 64, 1)])
+def test_cg_prepared_weight_is_bit_identical(N, D, H):
+    """The tensor-core kernels give the same bits whether they convert the weight themselves
+    or copy the image dc_attn_cg_prepare wrote (H = 16: the forward's image only; dx then
+    runs on the CUDA cores and ignores it)."""
+    p = cg_problem(500 + N + D + H, N, D, H, "bf16")
+    dev = "cuda"
+    x, w, b = p["x"].to(dev), p["w"].to(dev).t().contiguous(), p["b"].to(dev)
+    dc, dg = p["dc"].to(dev), p["dg"].to(dev)
+    img = dcattn.dc_attn_cg_prepare(w)
+    for use in (None, img):
+        outs = dcattn.dc_attn_cg_fwd(x, w, b, weight_splits=use) + dcattn.dc_attn_cg_bwd(x, w, dc, dg,
+                                                                                        weight_splits=use)
+        torch.cuda.synchronize()
+        if use is None:
+            ref = [t.clone() for t in outs]
+    for u, v in zip(outs, ref):
+        assert torch.equal(u, v)
+    _check(p, outs, "bf16", "auto")
