@@ -289,3 +289,32 @@ def test_cg_prepared_weight_is_bit_identical(N, D, H):
     for u, v in zip(outs, ref):
         assert torch.equal(u, v)
     _check(p, outs, "bf16", "auto")
+
+
+def test_cg_chain_backward_through_the_attention():
+    """The whole layer chain on the GPU, x -> (c, g) -> windowed attention -> backward ->
+    (dc, dg) -> dx, dweight, dbias, against the same chain in the fp64 oracle (bf16
+    attention: compared relative to each output's largest magnitude)."""
+    N, D, H, d, W = 700, 256, 6, 128, 112
+    p = cg_problem(12, N, D, H, "bf16")
+    dev = "cuda"
+    gen = torch.Generator().manual_seed(13)
+    q, k, v, dO = (torch.randn(N, H, d, generator=gen).to(torch.bfloat16) for _ in range(4))
+    cu = torch.tensor([0, 300, 700], dtype=torch.int32)
+    scale = d ** -0.5
+    x, w, b = p["x"].to(dev), p["w"].to(dev).t().contiguous(), p["b"].to(dev)
+    img = dcattn.dc_attn_cg_prepare(w)
+    c, g = dcattn.dc_attn_cg_fwd(x, w, b, weight_splits=img)
+    qd, kd, vd, dOd, cud = q.to(dev), k.to(dev), v.to(dev), dO.to(dev), cu.to(dev)
+    o, lse, pmap = dcattn.dc_attn_fwd(qd, kd, vd, c, g, cud, W, scale)
+    dq, dk, dv, dcv, dgv = dcattn.dc_attn_bwd(qd, kd, vd, c, g, dOd, lse, pmap, cud, W, scale)
+    dx, dw, db = dcattn.dc_attn_cg_bwd(x, w, dcv, dgv, weight_splits=img)
+    torch.cuda.synchronize()
+    rc, rg = oracle.cg_forward(_to_np(p["x"]), _to_np(p["w"]), _to_np(p["b"]))
+    ro = oracle.forward(_to_np(q), _to_np(k), _to_np(v), rc, rg, cu.numpy(), W, scale)[0]
+    rgrads = oracle.backward(_to_np(q), _to_np(k), _to_np(v), rc, rg, _to_np(dO), cu.numpy(), W, scale)
+    rdx, rdw, rdb = oracle.cg_backward(_to_np(p["x"]), _to_np(p["w"]), rgrads[3], rgrads[4])
+    for name, got, ref in (("o", o, ro), ("dq", dq, rgrads[0]), ("dc", dcv, rgrads[3]), ("dg", dgv, rgrads[4]),
+                           ("dx", dx, rdx), ("dweight", dw.t(), rdw), ("dbias", db, rdb)):
+        err = np.abs(_to_np(got) - ref).max() / np.abs(ref).max()
+        assert err <= 2e-2, (name, err)
