@@ -136,14 +136,14 @@ cg_fwd_tc_kernel(const __grid_constant__ CUtensorMap map_x, CgShape s, const flo
         tc::init_ctl(abort_flag, wait_ns);
         ptx::fence_mbar_init();
         ptx::prefetch_tensormap(&map_x);
-        for (int kb = 0; kb < first; ++kb) {
-            ptx::mbar_arrive_expect_tx(&full[kb], 16384);
-            ptx::tma_load_2d(xs + kb * 16384, &map_x, kb * 64, (int)t0, &full[kb]);
-        }
-        if (splits) {   // the weight image, one bulk copy per 64-column block
+        if (splits) {   // the weight image first (from L2; the MMAs need all of it), one bulk copy per block
             ptx::mbar_arrive_expect_tx(wready, (uint32_t)(nkb * NCOL * 128));
             for (int kb = 0; kb < nkb; ++kb)
                 ptx::bulk_load(wb + kb * NCOL * 128, splits + (size_t)kb * NCOL * 128, NCOL * 128, wready);
+        }
+        for (int kb = 0; kb < first; ++kb) {
+            ptx::mbar_arrive_expect_tx(&full[kb], 16384);
+            ptx::tma_load_2d(xs + kb * 16384, &map_x, kb * 64, (int)t0, &full[kb]);
         }
     }
     if (warp == 5) {
@@ -200,16 +200,21 @@ cg_fwd_tc_kernel(const __grid_constant__ CUtensorMap map_x, CgShape s, const flo
 #pragma unroll
             for (int b = 0; b < NCOL / 16; ++b) ptx::tmem_ld16_issue(base + b * 16, r[b]);
             ptx::tmem_wait_ld();
+            float acc[NCOL];
 #pragma unroll
-            for (int b = 0; b < NCOL / 16; ++b) ptx::reg_fence16(r[b]);
+            for (int b = 0; b < NCOL / 16; ++b) {
+                ptx::reg_fence16(r[b]);
+#pragma unroll
+                for (int e = 0; e < 16; ++e) acc[b * 16 + e] = __uint_as_float(r[b][e]);
+            }
             const int64_t t = t0 + warp * 32 + lane;
             if (t < s.N) {
 #pragma unroll
                 for (int o = 0; o < R; ++o) {
                     if (o < 2 * s.H) {
-                        const float hi = __uint_as_float(r[o / 16][o % 16]);
-                        const float mid = __uint_as_float(r[(R + o) / 16][(R + o) % 16]);
-                        const float lo = __uint_as_float(r[(2 * R + o) / 16][(2 * R + o) % 16]);
+                        const float hi = acc[o];
+                        const float mid = acc[R + o];
+                        const float lo = acc[2 * R + o];
                         const float v = ((hi + mid) + lo) + __ldg(bias + o);
                         if (o < s.H)
                             c[t * s.H + o] = v;
