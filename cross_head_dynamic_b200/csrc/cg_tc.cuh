@@ -238,16 +238,21 @@ cg_fwd_tc_kernel(const __grid_constant__ CUtensorMap map_x, CgShape s, const flo
 // D[128 tokens][k] = A[128][96] . B[96][k], with K = six 16-wide terms pairing the bf16 splits
 // of e and of the weight: (e1, w1), (e1, w2), (e2, w1), (e1, w3), (e3, w1), (e2, w2).  The
 // dropped products (e2 w3, e3 w2, e3 w3) and the two splits' residuals are below 2^-23 of
-// |e w|.  A is K-major (the CTA's threads write each token's row); B is MN-major (row
-// j * 16 + o holds split s(j) of weight[o][.], 64-column blocks of 96 x 128 bytes).  The
+// |e w|.  A is K-major (the CTA's threads write each token's row); B is MN-major: the
+// forward's split image (rows split * 16 + o, 64-column blocks of 48 x 128 bytes), K16 step j
+// pointing at the 16 rows of the weight split it pairs with.  The
 // columns go in chunks of up to 256 (6 MMAs each) into two alternating TMEM buffers, so the
 // epilogue of one chunk (TMEM -> bf16 -> 32-byte stores of each token's row) overlaps the
 // products of the next.
 // ---------------------------------------------------------------------------------------
 
-constexpr int kDxThreads = 160;    // warps 0-3: A rows and epilogue (TMEM lane quarters); warp 4: TMEM, MMAs
+constexpr int kDxThreads = 288;    // warps 0-3: A rows and epilogue; 5-8: epilogue; warp 4: TMEM, MMAs
+constexpr int kDxMaxChunks = 8;    // 256-column chunks: D <= 2048
 constexpr int kDxK = 96;           // six 16-wide terms
-constexpr int kDxBRow = kDxK * 128;   // bytes of one 64-column block of B
+// B in shared memory holds the three splits only, rows split * 16 + o of each 64-column
+// block (the forward's image, byte for byte); K16 step j of the six terms reads the 16 rows
+// of split dx_term_b(j)
+constexpr int kDxBRow = 3 * 16 * 128;   // bytes of one 64-column block of B
 constexpr size_t kDxFixed = 1024 + 2 * 16384 + 256;   // alignment slack, A (two 64-wide K blocks), barriers
 
 inline size_t dx_tc_smem_bytes(int D) { return kDxFixed + (size_t)kDxBRow * ((D + 63) / 64); }
@@ -255,51 +260,6 @@ inline size_t dx_tc_smem_bytes(int D) { return kDxFixed + (size_t)kDxBRow * ((D 
 // split of e or of the weight used by term j (0 = hi, 1 = mid, 2 = lo), for A and for B
 __host__ __device__ constexpr int dx_term_a(int j) { return j == 2 || j == 5 ? 1 : j == 4 ? 2 : 0; }
 __host__ __device__ constexpr int dx_term_b(int j) { return j == 1 || j == 5 ? 1 : j == 3 ? 2 : 0; }
-
-__device__ __forceinline__ void stage_dx_weight(const CgShape &s, const float *__restrict__ weight, uint8_t *wb,
-                                                int nblk, int tid, int nthreads) {
-    const int chunks = nblk * 8;
-    const int total = 16 * chunks;
-    for (int i0 = tid; i0 < total; i0 += nthreads * kBatch) {
-        float2 v[kBatch][4];
-#pragma unroll
-        for (int b = 0; b < kBatch; ++b) {
-            const int i = i0 + b * nthreads;
-            const int o = i / chunks, kc = i - o * chunks;
-#pragma unroll
-            for (int u = 0; u < 4; ++u) {
-                const int k = kc * 8 + 2 * u;
-                v[b][u] = (i < total && o < 2 * s.H && k < s.D)
-                              ? __ldg(reinterpret_cast<const float2 *>(weight + (int64_t)o * s.D + k))
-                              : make_float2(0.f, 0.f);
-            }
-        }
-#pragma unroll
-        for (int b = 0; b < kBatch; ++b) {
-            const int i = i0 + b * nthreads;
-            if (i >= total) break;
-            const int o = i / chunks, kc = i - o * chunks;
-            uint32_t w3[3][4];
-#pragma unroll
-            for (int u = 0; u < 4; ++u) {
-                uint32_t h0, m0, l0, h1, m1, l1;
-                split3(v[b][u].x, h0, m0, l0);
-                split3(v[b][u].y, h1, m1, l1);
-                w3[0][u] = h0 | (h1 << 16);
-                w3[1][u] = m0 | (m1 << 16);
-                w3[2][u] = l0 | (l1 << 16);
-            }
-            const int kb = kc >> 3, c16 = kc & 7;
-#pragma unroll
-            for (int j = 0; j < 6; ++j) {
-                const int r = j * 16 + o;
-                const int sp = dx_term_b(j);
-                *reinterpret_cast<uint4 *>(wb + kb * kDxBRow + r * 128 + ((c16 ^ (r & 7)) << 4)) =
-                    make_uint4(w3[sp][0], w3[sp][1], w3[sp][2], w3[sp][3]);
-            }
-        }
-    }
-}
 
 __global__ void __launch_bounds__(kDxThreads, 1)
 cg_bwd_dx_tc_kernel(CgShape s, const float *__restrict__ weight, const uint8_t *__restrict__ splits,
@@ -312,8 +272,8 @@ cg_bwd_dx_tc_kernel(CgShape s, const float *__restrict__ weight, const uint8_t *
     uint8_t *as = sm;                 // A: two K blocks of [128 rows][128 bytes]
     uint8_t *wb = sm + 2 * 16384;     // B
     uint64_t *bars = (uint64_t *)(wb + (size_t)nblk * kDxBRow);
-    uint64_t *accfull = bars, *tfree = bars + 2, *wready = bars + 4;
-    uint32_t *tmem_slot = (uint32_t *)(bars + 5);
+    uint64_t *accfull = bars, *tfree = bars + 2, *wready = bars + 4;   // wready[chunk]: its blocks of the image
+    uint32_t *tmem_slot = (uint32_t *)(bars + 4 + kDxMaxChunks);
     volatile int *abort_flag = (volatile int *)(tmem_slot + 1);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int64_t t0 = (int64_t)blockIdx.x * kTcTile;
@@ -321,15 +281,18 @@ cg_bwd_dx_tc_kernel(CgShape s, const float *__restrict__ weight, const uint8_t *
     if (threadIdx.x == 0) {
         ptx::mbar_init(&accfull[0], 1);
         ptx::mbar_init(&accfull[1], 1);
-        ptx::mbar_init(&tfree[0], 128);
-        ptx::mbar_init(&tfree[1], 128);
-        ptx::mbar_init(wready, 1);
+        ptx::mbar_init(&tfree[0], 256);
+        ptx::mbar_init(&tfree[1], 256);
+        for (int c = 0; c < kDxMaxChunks; ++c) ptx::mbar_init(&wready[c], 1);
         tc::init_ctl(abort_flag, wait_ns);
         ptx::fence_mbar_init();
-        if (splits) {   // the weight image, one bulk copy per 64-column block
-            ptx::mbar_arrive_expect_tx(wready, (uint32_t)(nblk * kDxBRow));
-            for (int kb = 0; kb < nblk; ++kb)
-                ptx::bulk_load(wb + kb * kDxBRow, splits + (size_t)kb * kDxBRow, kDxBRow, wready);
+        if (splits) {   // the weight image, one bulk copy per 64-column block, chunk by chunk
+            for (int c = 0; c < nch; ++c) {
+                const int nb = nblk - 4 * c < 4 ? nblk - 4 * c : 4;
+                ptx::mbar_arrive_expect_tx(&wready[c], (uint32_t)(nb * kDxBRow));
+                for (int kb = 4 * c; kb < 4 * c + nb; ++kb)
+                    ptx::bulk_load(wb + kb * kDxBRow, splits + (size_t)kb * kDxBRow, kDxBRow, &wready[c]);
+            }
         }
     }
     if (warp == 4) {
@@ -368,7 +331,7 @@ cg_bwd_dx_tc_kernel(CgShape s, const float *__restrict__ weight, const uint8_t *
             *reinterpret_cast<uint4 *>(as + blk * 16384 + row * 128 + ((c16 ^ (row & 7)) << 4)) = v;
         }
     }
-    if (!splits) stage_dx_weight(s, weight, wb, nblk, threadIdx.x, kDxThreads);
+    if (!splits) stage_weight_splits<16>(s, weight, wb, nblk, threadIdx.x, kDxThreads);
     ptx::fence_proxy_async_smem();
     ptx::tc_fence_before();
     __syncthreads();
@@ -377,10 +340,14 @@ cg_bwd_dx_tc_kernel(CgShape s, const float *__restrict__ weight, const uint8_t *
 
     if (warp == 4) {
         if (lane == 0) {
-            bool ok = !splits || tc::wait_bar(wready, 0, abort_flag);
+            bool ok = true;
             const uint32_t aa = ptx::smem_u32(as), ba = ptx::smem_u32(wb);
             for (int c = 0; c < nch && ok; ++c) {
                 const int b = c & 1;
+                if (splits) {
+                    ok = tc::wait_bar(&wready[c], 0, abort_flag);
+                    if (!ok) break;
+                }
                 if (c >= 2) {
                     ok = tc::wait_bar(&tfree[b], (uint32_t)((c / 2 - 1) & 1), abort_flag);
                     if (!ok) break;
@@ -391,14 +358,18 @@ cg_bwd_dx_tc_kernel(CgShape s, const float *__restrict__ weight, const uint8_t *
 #pragma unroll
                 for (int k = 0; k < kDxK / 16; ++k) {
                     const uint64_t ad = ptx::smem_desc_sw128(aa + (k >> 2) * 16384 + (k & 3) * 32, 16, 1024);
-                    const uint64_t bd = ptx::smem_desc_sw128(ba + 4 * c * kDxBRow + k * 2048, kDxBRow, 1024);
+                    const uint64_t bd =
+                        ptx::smem_desc_sw128(ba + 4 * c * kDxBRow + dx_term_b(k) * 16 * 128, kDxBRow, 1024);
                     ptx::mma_bf16(tmem + b * 256, ad, bd, idesc, k != 0);
                 }
                 ptx::mma_commit(&accfull[b]);
             }
         }
     } else {
-        const int64_t t = t0 + warp * 32 + lane;
+        // epilogue: warps 0-3 and 5-8 (warp w reads TMEM lane quarter w % 4); the two sets take
+        // alternate pairs of 16-column groups of each chunk
+        const int qtr = warp & 3, set = warp < 4 ? 0 : 1;
+        const int64_t t = t0 + qtr * 32 + lane;
         __nv_bfloat16 *rowp = dx + (t < s.N ? t : 0) * s.sdx;
         const bool a32 = ((uintptr_t)rowp & 31) == 0;
         for (int c = 0; c < nch; ++c) {
@@ -407,8 +378,8 @@ cg_bwd_dx_tc_kernel(CgShape s, const float *__restrict__ weight, const uint8_t *
             ptx::tc_fence_after();
             if (!ok) break;
             const int ncols = (nblk - 4 * c < 4 ? nblk - 4 * c : 4) * 64;
-            const uint32_t base = tmem + b * 256 + ((uint32_t)(warp * 32) << 16);
-            for (int g16 = 0; g16 < ncols / 16; g16 += 2) {
+            const uint32_t base = tmem + b * 256 + ((uint32_t)(qtr * 32) << 16);
+            for (int g16 = 2 * set; g16 < ncols / 16; g16 += 4) {
                 uint32_t r0[16], r1[16];
                 ptx::tmem_ld16_issue(base + g16 * 16, r0);
                 ptx::tmem_ld16_issue(base + (g16 + 1) * 16, r1);
@@ -668,15 +639,12 @@ cg_bwd_dw_tc_kernel(const __grid_constant__ CUtensorMap map_x, CgShape s, int64_
 }
 
 // ---------------------------------------------------------------------------------------
-// The weight's bf16 split images, written once per weight: the forward's B operand
-// (3R x 128 bytes per 64-column block) followed, when 2H <= 16, by dx's (96 x 128 bytes per
-// block), byte for byte what the kernels otherwise build in shared memory, so results are
-// identical with or without them.
+// The weight's bf16 split image, written once per weight: 3R rows x 128 bytes per 64-column
+// block, byte for byte what the forward (K-major B) and dx (MN-major B, 2H <= 16) otherwise
+// build in shared memory, so results are identical with or without it.
 // ---------------------------------------------------------------------------------------
 __host__ __device__ inline size_t prep_fwd_bytes(int D, int H) { return tc_split_bytes(D, H); }
-__host__ __device__ inline size_t prep_dx_bytes(int D, int H) {
-    return 2 * H <= 16 ? (size_t)kDxBRow * ((D + 63) / 64) : 0;
-}
+
 
 template <int R>
 __global__ void __launch_bounds__(256) cg_prepare_kernel(CgShape s, const float *__restrict__ weight,
@@ -684,7 +652,6 @@ __global__ void __launch_bounds__(256) cg_prepare_kernel(CgShape s, const float 
     const int nkb = (s.D + 63) / 64;
     const int tid = blockIdx.x * blockDim.x + threadIdx.x, nth = gridDim.x * blockDim.x;
     stage_weight_splits<R>(s, weight, img, nkb, tid, nth);
-    if (R == 16) stage_dx_weight(s, weight, img + prep_fwd_bytes(s.D, s.H), nkb, tid, nth);
 }
 
 }  // namespace cg

@@ -490,7 +490,7 @@ cudaError_t cg_dx_tc_launch(const dc::cg::CgShape &s, const float *w, const uint
     if (e != cudaSuccess) return e;
     const unsigned grid = (unsigned)((s.N + dc::cg::kTcTile - 1) / dc::cg::kTcTile);
     dc::cg::cg_bwd_dx_tc_kernel<<<grid, dc::cg::kDxThreads, smem, st>>>(
-        s, w, splits ? splits + dc::cg::prep_fwd_bytes(s.D, s.H) : nullptr, dc_, dg, (__nv_bfloat16 *)dx,
+        s, w, splits, dc_, dg, (__nv_bfloat16 *)dx,
         g_wait_ns.load(std::memory_order_relaxed));
     ++t_launches;
     return cudaGetLastError();
@@ -671,7 +671,7 @@ dc_status_t dc_attn_cg_bwd(const dc_cg_params *params, const void *x, const floa
 size_t dc_attn_cg_prepare_size(const dc_cg_params *params) {
     dc::cg::CgShape s;
     if (check_cg(params, &s) != DC_OK) return 0;
-    return dc::cg::prep_fwd_bytes(s.D, s.H) + dc::cg::prep_dx_bytes(s.D, s.H);
+    return dc::cg::prep_fwd_bytes(s.D, s.H);
 }
 
 dc_status_t dc_attn_cg_prepare(const dc_cg_params *params, const float *weight, void *splits, void *stream) {

@@ -297,7 +297,7 @@ size_t dc_attn_cg_bwd_workspace_size(const dc_cg_params *params);
 
 /* Gradients for dL/dc = dc, dL/dg = dg, writing e[t] = (dc[t,:], dg[t,:]).
  * dx runs on tcgen05 for bf16 with 2H <= 16, a dx row stride that is a multiple of 8
- * elements and D <= 1024 (AUTO; TCGEN05 elsewhere returns DC_ERR_UNSUPPORTED): products
+ * elements and D <= 2048 (AUTO; TCGEN05 elsewhere returns DC_ERR_UNSUPPORTED): products
  * of the bf16 splits of e and of the weight, six of the nine pairs, whose sum is e * w to
  * within 2^-23 |e w|, accumulated by the tensor core; SIMT otherwise.  The partial sums
  * of dweight run on the CUDA cores under AUTO and SIMT; TCGEN05 moves them to the tensor

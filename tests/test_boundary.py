@@ -239,11 +239,11 @@ def test_cg_resolve_impl(lib):
 
 
 def test_cg_prepare_size_and_alignment(lib):
-    """The weight image holds the forward's splits (3 x 16 rows x 128 bytes per 64 columns)
-    and, for 2H <= 16, dx's (96 rows x 128 bytes per 64 columns); a misaligned image
-    pointer is refused on the host."""
+    """The weight image holds the three bf16 splits (3 x R rows x 128 bytes per 64 columns,
+    R = 16 outputs per split for 2H <= 16, else 32), read by the forward and by dx; a
+    misaligned image pointer is refused on the host."""
     p = _cg()
-    assert lib.dc_attn_cg_prepare_size(ctypes.byref(p)) == 12 * (48 * 128 + 96 * 128)
+    assert lib.dc_attn_cg_prepare_size(ctypes.byref(p)) == 12 * 48 * 128
     p16 = _cg(num_heads=16, model_dim=1024)
     assert lib.dc_attn_cg_prepare_size(ctypes.byref(p16)) == 16 * 96 * 128
     a = 0x4000

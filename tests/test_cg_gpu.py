@@ -52,7 +52,7 @@ def _dx_on_tc(p):
     """The conditions under which AUTO runs dx on tcgen05 (contiguous dx)."""
     N, D = p["x"].shape
     H = p["dc"].shape[1]
-    return p["x"].dtype == torch.bfloat16 and 2 * H <= 16 and D % 8 == 0 and D <= 1024
+    return p["x"].dtype == torch.bfloat16 and 2 * H <= 16 and D % 8 == 0 and D <= 2048
 
 
 def _dw_on_tc(p):
@@ -178,7 +178,8 @@ def test_cg_forward_tcgen05(N, D, H):
 @pytest.mark.parametrize("N, D, H", [
     (128, 64, 1),        # one tile, one 64-column chunk
     (300, 200, 6),       # ragged tile, D not a multiple of 16 (last columns stored singly)
-    (1000, 1024, 8),     # widest weight that fits, four 256-column chunks
+    (1000, 1024, 8),     # four 256-column chunks
+    (600, 2048, 8),      # widest weight that fits, eight chunks
     (4099, 768, 6),      # GPT-2 width, three chunks alternating the two TMEM buffers
     (65, 328, 4),        # fewer tokens than a tile; a 64-column last chunk (5 blocks)
 ])
