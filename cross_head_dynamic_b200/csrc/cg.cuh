@@ -12,11 +12,13 @@
 //
 // The map reads x once (1.5 KB per token at D = 768 in bf16) and does 2H FMAs per element
 // of x, an fp32 FMA count on the CUDA cores that takes about as long as the HBM stream at
-// 2H = 12, so the kernels spend few instructions per FMA: they use the packed fma.rn.f32x2
-// of sm_100 (two IEEE fp32 FMAs, each rounded to nearest, so the result is that of two
-// scalar FMAs in the same order) on pairs of adjacent columns, with the weight in shared
-// memory read as broadcasts.  The forward and dx give each lane whole tokens (no
-// reduction across lanes); dweight gives each thread column pairs and walks the tokens.
+// 2H = 12, so the kernels spend few instructions per FMA.  The forward and dx use the
+// packed fma.rn.f32x2 of sm_100 (two IEEE fp32 FMAs, each rounded to nearest, so the result
+// is that of two scalar FMAs in the same order) on pairs of adjacent columns, with the
+// weight in shared memory read as broadcasts, and give each lane whole tokens (no
+// reduction across lanes).  dweight gives each thread column pairs and walks the tokens
+// with scalar FMAs: there the packed form needs each x pair moved into a 64-bit register
+// pair, which cost as many instructions as it saved (measured).
 //
 // Outputs are padded to OUT in {8, 12, 16, 24, 32} (>= 2H; padded weight rows and padded
 // entries of e are zero).
@@ -33,10 +35,12 @@ namespace dc {
 namespace cg {
 
 constexpr int kThreads = 256;             // forward and dx blocks: 8 warps, one per column slice
-constexpr int kDwThreads = 384;           // dweight partial blocks: 12 warps
-__host__ __device__ constexpr int dw_units(int OUT) { return OUT <= 12 ? 2 : 1; }   // column pairs per thread, per pass
+constexpr int kDwThreads = 384;           // dweight partial blocks: 12 warps, two token groups
+constexpr int kDwGroup = kDwThreads / 2;  // threads of one token group
+constexpr int kDwStages = 4;              // dweight token stages in flight
+__host__ __device__ constexpr int dw_ppt(int OUT) { return OUT <= 16 ? 2 : 1; }   // column pairs per thread, per pass
 constexpr size_t kMaxSmem = 227 * 1024;   // dynamic shared memory a block may have
-constexpr size_t kDwStageBudget = 100 * 1024;   // one of the dweight kernel's two stages
+constexpr size_t kDwStageBudget = 48 * 1024;   // one of the dweight kernel's stages
 constexpr int kReduceThreads = 512;
 
 struct CgShape {
@@ -49,19 +53,25 @@ struct CgShape {
 
 __host__ __device__ constexpr int out_pad(int H2) { return H2 <= 8 ? 8 : H2 <= 12 ? 12 : H2 <= 16 ? 16 : H2 <= 24 ? 24 : 32; }
 
-// Tokens per stage of the dweight kernel, and its shared memory (two stages of x rows
-// and of e rows stored as broadcast pairs (e, e)).
+// Tokens per stage of the dweight kernel, and its shared memory: kDwStages stages, each the
+// x rows then the e rows (fp32); after the last stage the same
+// bytes hold one token group's sums for the other ([kDwGroup][pairs per thread][OUT] pairs).
 inline int dw_chunk(int D, int H, size_t esize) {
-    const size_t per_token = esize * (size_t)D + 8 * (size_t)out_pad(2 * H);
+    const size_t per_token = esize * (size_t)D + 4 * (size_t)out_pad(2 * H);
     const size_t c = kDwStageBudget / per_token;
     return (int)(c > 64 ? 64 : c < 1 ? 1 : c);
 }
 __host__ __device__ inline size_t dw_xbytes(int chunk, int D, size_t esize) {
-    return (esize * (size_t)chunk * D + 15) / 16 * 16;   // e stages follow on a 16-byte boundary
+    return (esize * (size_t)chunk * D + 15) / 16 * 16;   // the e rows follow on a 16-byte boundary
+}
+__host__ __device__ inline size_t dw_stage_bytes(int chunk, int D, int OUT, size_t esize) {
+    return dw_xbytes(chunk, D, esize) + 4 * (size_t)chunk * OUT;   // a multiple of 16 (OUT is one of 4)
 }
 inline size_t dw_smem_bytes(int D, int H, size_t esize) {
-    const int chunk = dw_chunk(D, H, esize);
-    return 2 * dw_xbytes(chunk, D, esize) + 2 * sizeof(float) * 2 * (size_t)chunk * out_pad(2 * H);
+    const int OUT = out_pad(2 * H);
+    const size_t stages = kDwStages * dw_stage_bytes(dw_chunk(D, H, esize), D, OUT, esize);
+    const size_t xch = 8 * (size_t)kDwGroup * dw_ppt(OUT) * OUT;
+    return stages > xch ? stages : xch;
 }
 
 // Number of partial records (blocks of the dweight kernel, one wave of one block per SM)
@@ -99,6 +109,24 @@ template <> __device__ __forceinline__ f2reg ldpair<float>(const float *p) { ret
 template <> __device__ __forceinline__ f2reg ldpair<__nv_bfloat16>(const __nv_bfloat16 *p) {
     const unsigned w = *reinterpret_cast<const unsigned *>(p);
     return pack2(__uint_as_float(w << 16), __uint_as_float(w & 0xffff0000u));
+}
+// Shared-memory loads at 32-bit shared addresses (a loop steps the address by a constant
+// instead of recomputing a generic pointer per load).
+template <typename T> __device__ __forceinline__ float2 lds_pair(uint32_t a);
+template <> __device__ __forceinline__ float2 lds_pair<float>(uint32_t a) {
+    float2 v;
+    asm volatile("ld.shared.v2.f32 {%0, %1}, [%2];" : "=f"(v.x), "=f"(v.y) : "r"(a));
+    return v;
+}
+template <> __device__ __forceinline__ float2 lds_pair<__nv_bfloat16>(uint32_t a) {
+    unsigned w;
+    asm volatile("ld.shared.u32 %0, [%1];" : "=r"(w) : "r"(a));
+    return make_float2(__uint_as_float(w << 16), __uint_as_float(w & 0xffff0000u));
+}
+__device__ __forceinline__ float4 lds_f4(uint32_t a) {
+    float4 v;
+    asm volatile("ld.shared.v4.f32 {%0, %1, %2, %3}, [%4];" : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w) : "r"(a));
+    return v;
 }
 // Asynchronous global -> shared copies (cp.async; completion per thread, by group).
 __device__ __forceinline__ void cp_async16(void *dst, const void *src) {
@@ -392,11 +420,17 @@ __global__ void __launch_bounds__(kThreads, 2) cg_bwd_dx_kernel(CgShape s, const
 }
 
 // Partial dweight and dbias of the token range [blockIdx.x * span, +span) into record
-// blockIdx.x of `part`.  Thread i takes the column pairs p = i, i + kDwThreads (dw_units
-// of them per pass over the columns).  Tokens go through shared memory `chunk` at a time,
-// double-buffered with asynchronous copies: the x rows, and e as broadcast pairs (e, e)
-// so that one packed FMA per output adds e[o] * (x[2p], x[2p + 1]).  dbias: the threads
-// o < 2H add the e column o.
+// blockIdx.x of `part`.  The block's two token groups of kDwGroup threads take the even and
+// the odd tokens of every stage; within a group, thread i takes the column pairs
+// i + k * kDwGroup (k < dw_ppt(OUT)) of each pass over the columns (a warp's reads of one
+// row are then consecutive words), so one broadcast read of four e values feeds
+// 4 * 2 * dw_ppt(OUT) scalar FMAs.
+// Tokens go through shared memory `chunk` at a time in a ring of kDwStages stages filled
+// by asynchronous copies (the x rows and the e rows).  At the end of a pass the odd
+// group's sums are added to the even group's in shared memory, in that order.
+// dbias: lane o of warp w adds e column o of the tokens w, w + 12, ... of every stage; the
+// 12 warp sums are then added in warp order.  Every assignment is fixed, so the record is
+// bitwise reproducible.
 template <typename T, int OUT>
 __global__ void __launch_bounds__(kDwThreads) cg_bwd_dw_partial_kernel(CgShape s, int64_t span, int chunk,
                                                                       const T *__restrict__ x,
@@ -404,12 +438,16 @@ __global__ void __launch_bounds__(kDwThreads) cg_bwd_dw_partial_kernel(CgShape s
                                                                       const float *__restrict__ dg,
                                                                       float *__restrict__ part, int vec16) {
     extern __shared__ __align__(16) unsigned char smem[];
+    __shared__ float dbred[kDwThreads / 32][32];
+    constexpr int PPT = dw_ppt(OUT);
+    constexpr int NW = kDwThreads / 32;
     const size_t xbytes = dw_xbytes(chunk, s.D, sizeof(T));
-    const size_t ebytes = sizeof(float2) * (size_t)chunk * OUT;
-    auto xs = [&](int b) { return reinterpret_cast<T *>(smem + b * xbytes); };
-    auto es = [&](int b) { return reinterpret_cast<float2 *>(smem + 2 * xbytes + b * ebytes); };
+    const size_t sbytes = dw_stage_bytes(chunk, s.D, OUT, sizeof(T));
+    auto xs = [&](int b) { return reinterpret_cast<T *>(smem + b * sbytes); };
+    auto es = [&](int b) { return reinterpret_cast<float *>(smem + b * sbytes + xbytes); };
     const int H2 = 2 * s.H;
-    const int tid = threadIdx.x;
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int grp = tid / kDwGroup, tg = tid - grp * kDwGroup;
     const int64_t ta = (int64_t)blockIdx.x * span;
     const int64_t tb = ta + span < s.N ? ta + span : s.N;
     const int64_t ntok = tb > ta ? tb - ta : 0;
@@ -420,14 +458,14 @@ __global__ void __launch_bounds__(kDwThreads) cg_bwd_dw_partial_kernel(CgShape s
         const int64_t left = ntok - (int64_t)ci * chunk;
         return (int)(left < chunk ? left : chunk);
     };
+    // stage ci % kDwStages <- chunk ci (nothing past the last chunk); always one commit group
     auto issue = [&](int ci) {
         if (ci < nchunks) {
             const int64_t tc = ta + (int64_t)ci * chunk;
             const int nt = rows_of(ci);
-            T *xd = xs(ci & 1);
-            float2 *ed = es(ci & 1);
-            const int warp = tid >> 5, lane = tid & 31;
-            for (int r = warp; r < nt; r += kDwThreads / 32) {
+            T *xd = xs(ci % kDwStages);
+            float *ed = es(ci % kDwStages);
+            for (int r = warp; r < nt; r += NW) {
                 const T *src = x + (tc + r) * s.sx;
                 T *dst = xd + r * s.D;
                 if (vec16) {
@@ -440,69 +478,104 @@ __global__ void __launch_bounds__(kDwThreads) cg_bwd_dw_partial_kernel(CgShape s
             }
             for (int i = tid; i < chunk * OUT; i += kDwThreads) {
                 const int r = i / OUT, o = i - r * OUT;
-                float *d2 = reinterpret_cast<float *>(ed + i);
-                if (r < nt && o < H2) {
-                    const float *src = o < s.H ? dc + (tc + r) * s.H + o : dg + (tc + r) * s.H + o - s.H;
-                    cp_async4(d2, src);
-                    cp_async4(d2 + 1, src);
-                } else {
-                    d2[0] = 0.f;
-                    d2[1] = 0.f;
-                }
+                if (r < nt && o < H2)
+                    cp_async4(ed + i, o < s.H ? dc + (tc + r) * s.H + o : dg + (tc + r) * s.H + o - s.H);
+                else
+                    ed[i] = 0.f;
             }
         }
         cp_async_commit();
     };
-    constexpr int UPT = dw_units(OUT);
-    for (int ug = 0; ug < pairs; ug += kDwThreads * UPT) {
-        f2reg acc[UPT][OUT];   // (dweight[o][2p], dweight[o][2p + 1])
+    float dbacc = 0.f;
+    for (int pg = 0; pg < pairs; pg += kDwGroup * PPT) {
+        // this thread's pairs; one past the end reads the last pair (always in bounds) and is not written
+        int pk[PPT];
 #pragma unroll
-        for (int u = 0; u < UPT; ++u)
+        for (int k = 0; k < PPT; ++k) pk[k] = min(pg + tg + k * kDwGroup, pairs - 1);
+        float acc[PPT][OUT][2];   // (dweight[o][2p], dweight[o][2p + 1]) of pair k
 #pragma unroll
-            for (int o = 0; o < OUT; ++o) acc[u][o] = 0ull;
-        float dbacc = 0.f;
-        __syncthreads();   // the previous pass's readers are done with both buffers
-        issue(0);
+        for (int k = 0; k < PPT; ++k)
+#pragma unroll
+            for (int o = 0; o < OUT; ++o) acc[k][o][0] = acc[k][o][1] = 0.f;
+        __syncthreads();   // the previous pass's readers are done with every stage
+        for (int ci = 0; ci < kDwStages - 1; ++ci) issue(ci);
 #pragma unroll 1
         for (int ci = 0; ci < nchunks; ++ci) {
-            issue(ci + 1);
-            cp_async_wait<1>();
+            issue(ci + kDwStages - 1);
+            cp_async_wait<kDwStages - 1>();   // chunk ci has landed (groups complete in order)
             __syncthreads();
             const int nt = rows_of(ci);
-            const T *xc = xs(ci & 1);
-            const float2 *ec = es(ci & 1);
+            const T *xc = xs(ci % kDwStages);
+            const float *ec = es(ci % kDwStages);
+            // shared addresses of this group's first token: its x pairs and its e row
+            uint32_t xa[PPT];
 #pragma unroll
-            for (int u = 0; u < UPT; ++u) {
-                const int p = ug + u * kDwThreads + tid;
-                if (ug + u * kDwThreads < pairs) {   // block-uniform test first, then the thread's
-#pragma unroll 2
-                    for (int r = 0; r < nt; ++r) {
-                        const f2reg xv = p < pairs ? ldpair<T>(xc + r * s.D + 2 * p) : 0ull;
-                        const ulonglong2 *e2 = reinterpret_cast<const ulonglong2 *>(ec + r * OUT);
+            for (int k = 0; k < PPT; ++k)
+                xa[k] = (uint32_t)__cvta_generic_to_shared(xc + grp * s.D + 2 * pk[k]);
+            uint32_t ea = (uint32_t)__cvta_generic_to_shared(ec + grp * OUT);
+            const uint32_t xstep = 2u * (uint32_t)s.D * (uint32_t)sizeof(T);   // two tokens
+#pragma unroll(OUT > 16 ? 1 : 2)
+            for (int r = grp; r < nt; r += 2) {
+                float2 xv[PPT];
 #pragma unroll
-                        for (int o2 = 0; o2 < OUT / 2; ++o2) {
-                            const ulonglong2 ev = e2[o2];   // (e[2 o2], e[2 o2]), (e[2 o2 + 1], e[2 o2 + 1])
-                            acc[u][2 * o2] = ffma2(ev.x, xv, acc[u][2 * o2]);
-                            acc[u][2 * o2 + 1] = ffma2(ev.y, xv, acc[u][2 * o2 + 1]);
+                for (int k = 0; k < PPT; ++k) {
+                    xv[k] = lds_pair<T>(xa[k]);
+                    xa[k] += xstep;
+                }
+#pragma unroll
+                for (int o4 = 0; o4 < OUT / 4; ++o4) {
+                    const float4 ev = lds_f4(ea + 16u * o4);
+                    const float e[4] = {ev.x, ev.y, ev.z, ev.w};
+#pragma unroll
+                    for (int j = 0; j < 4; ++j)
+#pragma unroll
+                        for (int k = 0; k < PPT; ++k) {
+                            acc[k][4 * o4 + j][0] = fmaf(e[j], xv[k].x, acc[k][4 * o4 + j][0]);
+                            acc[k][4 * o4 + j][1] = fmaf(e[j], xv[k].y, acc[k][4 * o4 + j][1]);
+                        }
+                }
+                ea += 2u * OUT * 4u;
+            }
+            if (pg == 0 && lane < H2)
+                for (int r = warp; r < nt; r += NW) dbacc += ec[r * OUT + lane];
+            __syncthreads();   // stage ci % kDwStages is free for chunk ci + kDwStages
+        }
+        cp_async_wait<0>();   // only empty groups can remain
+        __syncthreads();
+        // the odd group's sums to shared memory (the stage bytes, [pair k][output o][thread]),
+        // then the even group adds them
+        float2 *xch = reinterpret_cast<float2 *>(smem);
+        if (grp == 1) {
+#pragma unroll
+            for (int k = 0; k < PPT; ++k)
+#pragma unroll
+                for (int o = 0; o < OUT; ++o) xch[(k * OUT + o) * kDwGroup + tg] = make_float2(acc[k][o][0], acc[k][o][1]);
+        }
+        __syncthreads();
+        if (grp == 0) {
+#pragma unroll
+            for (int k = 0; k < PPT; ++k) {
+                const int p = pg + tg + k * kDwGroup;
+                if (p < pairs) {
+#pragma unroll
+                    for (int o = 0; o < OUT; ++o) {
+                        if (o < H2) {
+                            const float2 b = xch[(k * OUT + o) * kDwGroup + tg];
+                            *reinterpret_cast<float2 *>(rec + (int64_t)o * s.D + 2 * p) =
+                                make_float2(acc[k][o][0] + b.x, acc[k][o][1] + b.y);
                         }
                     }
                 }
             }
-            if (ug == 0 && tid < H2)
-                for (int r = 0; r < nt; ++r) dbacc += ec[r * OUT + tid].x;
-            __syncthreads();   // buffer ci & 1 is free for chunk ci + 2
         }
-        cp_async_wait<0>();
+    }
+    dbred[warp][lane] = dbacc;
+    __syncthreads();
+    if (tid < H2) {
+        float tot = dbred[0][tid];
 #pragma unroll
-        for (int u = 0; u < UPT; ++u) {
-            const int p = ug + u * kDwThreads + tid;
-            if (p < pairs) {
-#pragma unroll
-                for (int o = 0; o < OUT; ++o)
-                    if (o < H2) *reinterpret_cast<f2reg *>(rec + (int64_t)o * s.D + 2 * p) = acc[u][o];
-            }
-        }
-        if (ug == 0 && tid < H2) rec[(int64_t)H2 * s.D + tid] = dbacc;
+        for (int w = 1; w < NW; ++w) tot += dbred[w][tid];
+        rec[(int64_t)H2 * s.D + tid] = tot;
     }
 }
 
