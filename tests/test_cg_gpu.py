@@ -99,8 +99,10 @@ def _dx_tolerance(H, dx_impl):
 
 
 def _dw_tolerance(N, blocks, dw_impl):
-    """dweight, relative to the sum of |terms|.  SIMT: the tokens of one record in order, then
-    the records (16 strided sums, then those 16).  tcgen05: exact products of x with the bf16
+    """dweight, relative to the sum of |terms|.  SIMT: the tokens of one record in two
+    interleaved halves (even and odd tokens), each in order, the halves added, then the
+    records (16 strided sums, then those 16); bounded by the sum of one record's tokens in
+    order.  tcgen05: exact products of x with the bf16
     splits of e (2^-24 left out), the tensor core's accumulation over ceil(span / 16) steps,
     the epilogue's two additions, then the same record sums."""
     span = -(-N // blocks)
@@ -111,6 +113,8 @@ def _dw_tolerance(N, blocks, dw_impl):
 
 
 def _db_tolerance(N, blocks, dw_impl):
+    """dbias.  SIMT: twelve interleaved parts of one record's tokens, each in order, then the
+    twelve and the records; bounded by the sum of the record's tokens in order."""
     span = -(-N // blocks)
     if dw_impl == "simt":
         return gamma(span + blocks // 16 + 18)
@@ -187,6 +191,18 @@ def test_cg_backward_tcgen05(N, D, H):
     """dx and the dweight partial sums both on tcgen05 (forced)."""
     p = cg_problem(300 + N + D + H, N, D, H, "bf16")
     _check(p, _run(p, "bf16", "simt", "tcgen05"), "bf16", "simt", "tcgen05")
+
+
+@pytest.mark.parametrize("N, D, H, dtype", [
+    (100000, 256, 6, "bf16"),    # 676 tokens per record: the 4-stage ring of 64-token stages wraps
+    (30001, 768, 6, "bf16"),     # 203 tokens per record at the GPT-2 width, ragged last stage
+    (20000, 1030, 4, "f32"),     # fp32 x, D % 4 == 2, two passes over the columns
+    (9000, 520, 16, "bf16"),     # 2H = 32 (one column pair per thread), two passes
+])
+def test_cg_dweight_simt_spans(N, D, H, dtype):
+    """The CUDA-core dweight on long token ranges per record (many stages through the ring)."""
+    p = cg_problem(500 + N + D + H, N, D, H, dtype)
+    _check(p, _run(p, dtype, "simt"), dtype, "simt")
 
 
 @pytest.mark.parametrize("N", [64, 8191, 20000, 300000])
