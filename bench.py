@@ -134,36 +134,90 @@ def measured_traffic(kernel: str, tokens: int):
 
 
 class ClockSampler:
-    """nvidia-smi sampling of SM clocks and throttle reasons while the GPU works."""
+    """SM clocks and clock-event reasons while the GPU works.  NVML is polled every 2 ms from a
+    host thread, so that a timed region of a few milliseconds still holds samples; without
+    NVML, nvidia-smi samples every 100 ms.  Both only read the GPU's state."""
 
-    QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
-             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
-             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    REASONS = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
+    SMI_QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+                 "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+                 "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
 
     def __init__(self, device_index: int):
-        self.samples = []
-        self.proc = None
+        self.samples = []   # (time, sm MHz, max sm MHz, active reasons)
         self.dev = device_index
+        self.source = None
+        self.proc = None
+        self._stop = threading.Event()
         self._thread = None
 
     def start(self):
+        if not self._start_nvml():
+            self._start_smi()
+
+    def _start_nvml(self) -> bool:
+        try:
+            import pynvml as nv
+            nv.nvmlInit()
+            props = torch.cuda.get_device_properties(self.dev)
+            if hasattr(props, "pci_bus_id"):
+                bus = f"{getattr(props, 'pci_domain_id', 0):08x}:{props.pci_bus_id:02x}:{props.pci_device_id:02x}.0"
+                h = nv.nvmlDeviceGetHandleByPciBusId(bus)
+            else:
+                h = nv.nvmlDeviceGetHandleByIndex(self.dev)
+            mx = nv.nvmlDeviceGetMaxClockInfo(h, nv.NVML_CLOCK_SM)
+            get_reasons = getattr(nv, "nvmlDeviceGetCurrentClocksEventReasons", None) or \
+                nv.nvmlDeviceGetCurrentClocksThrottleReasons
+            bits = []
+            for name, key in zip(self.REASONS, ("HwSlowdown", "HwThermalSlowdown", "SwThermalSlowdown", "SwPowerCap")):
+                bits.append((name, getattr(nv, "nvmlClocksEventReason" + key, None) or
+                             getattr(nv, "nvmlClocksThrottleReason" + key)))
+            nv.nvmlDeviceGetClockInfo(h, nv.NVML_CLOCK_SM)
+            get_reasons(h)
+        except Exception:
+            return False
+
+        def poll():
+            while not self._stop.is_set():
+                try:
+                    sm = nv.nvmlDeviceGetClockInfo(h, nv.NVML_CLOCK_SM)
+                    r = get_reasons(h)
+                    self.samples.append((time.time(), float(sm), float(mx), {n for n, b in bits if r & b}))
+                except Exception:
+                    pass
+                time.sleep(0.002)
+
+        self.source = "nvml, every 2 ms"
+        self._thread = threading.Thread(target=poll, daemon=True)
+        self._thread.start()
+        return True
+
+    def _start_smi(self):
         try:
             self.proc = subprocess.Popen(
-                ["nvidia-smi", f"--id={self.dev}", f"--query-gpu={self.QUERY}", "--format=csv,noheader,nounits",
+                ["nvidia-smi", f"--id={self.dev}", f"--query-gpu={self.SMI_QUERY}", "--format=csv,noheader,nounits",
                  "-lms", "100"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
         except (OSError, ValueError):
             self.proc = None
             return
-        self._thread = threading.Thread(target=self._read, daemon=True)
+        self.source = "nvidia-smi, every 100 ms"
+        self._thread = threading.Thread(target=self._read_smi, daemon=True)
         self._thread.start()
 
-    def _read(self):
+    def _read_smi(self):
+        def num(x):
+            try:
+                return float(x)
+            except ValueError:
+                return None
         for line in self.proc.stdout:
             parts = [p.strip() for p in line.split(",")]
             if len(parts) >= 9:
-                self.samples.append((time.time(), parts))
+                active = {self.REASONS[k] for k in range(4) if parts[5 + k].lower().startswith("active")}
+                self.samples.append((time.time(), num(parts[1]), num(parts[2]), active))
 
     def stop(self):
+        self._stop.set()
         if self.proc is not None:
             self.proc.terminate()
             try:
@@ -174,20 +228,14 @@ class ClockSampler:
             self._thread.join(timeout=2)
 
     def summary(self, t0: float, t1: float):
-        win = [p for (ts, p) in self.samples if t0 <= ts <= t1]
+        win = [x for x in self.samples if t0 <= x[0] <= t1]
         if not win:
             return None
-        def num(x):
-            try:
-                return float(x)
-            except ValueError:
-                return None
-        sm = [num(p[1]) for p in win if num(p[1]) is not None]
-        mx = [num(p[2]) for p in win if num(p[2]) is not None]
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        reasons = sorted({names[k] for p in win for k in range(4) if p[5 + k].lower().startswith("active")})
+        sm = [x[1] for x in win if x[1] is not None]
+        mx = [x[2] for x in win if x[2] is not None]
+        reasons = sorted(set().union(*(x[3] for x in win)))
         return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(mx) if mx else None,
-                "reasons": reasons, "samples": len(win)}
+                "reasons": reasons, "samples": len(win), "source": self.source}
 
 
 def dist_setup(n_gpus: int):

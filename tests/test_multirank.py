@@ -67,3 +67,21 @@ def test_single_rank_needs_no_process_group():
     value, ms_step = bench.replica_throughput(1000, 40.0, 4, 1)
     assert ms_step == pytest.approx(10.0)
     assert value == pytest.approx(1000 / 10e-3)
+
+
+def test_clock_summary_window_and_reasons():
+    """The clock record keeps only samples inside the timed window: median SM clock, the
+    highest max clock, and the union of the active reasons."""
+    sys.path.insert(0, ROOT)
+    import bench
+    cs = bench.ClockSampler(0)
+    cs.source = "test"
+    cs.samples = [(0.5, 900.0, 1965.0, {"hw_slowdown"}),          # before the window
+                  (1.0, 1950.0, 1965.0, set()),
+                  (1.1, 1900.0, 1965.0, {"sw_power_cap"}),
+                  (1.2, 1935.0, 1965.0, set()),
+                  (3.0, 600.0, 1965.0, {"sw_thermal_slowdown"})]   # after it
+    got = cs.summary(1.0, 2.0)
+    assert got == {"sm_mhz": 1935.0, "sm_max_mhz": 1965.0, "reasons": ["sw_power_cap"], "samples": 3,
+                   "source": "test"}
+    assert cs.summary(5.0, 6.0) is None
