@@ -100,16 +100,17 @@ dc_status_t cuda_status(cudaError_t e) {
 // SIMT launches
 // --------------------------------------------------------------------------
 
+// SIMT kernels: `blocks` CTAs, one warp per work item of a CTA up to 8, fewer when the
+// shape's shared memory needs it.
 template <typename K>
-cudaError_t launch_warps(K kernel, const dc::Shape &s, size_t per_warp, cudaStream_t st, auto &&...args) {
-    int wpb = (int)((96 * 1024) / (per_warp > 0 ? per_warp : 1));
-    if (wpb > 8) wpb = 8;
-    if (wpb < 1) wpb = 1;
-    const size_t smem = per_warp * wpb;
+cudaError_t launch_simt(K kernel, const dc::Shape &s, int64_t blocks, int items, const dc::simt::SimtSmem &m,
+                        cudaStream_t st, auto &&...args) {
+    const int nw = dc::simt::warps_per_cta(items, m);
+    if (nw < 1) return cudaErrorInvalidValue;   // not reached for the shapes check_params admits
+    const size_t smem = m.bytes(nw);
     cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
-    const int64_t blocks = (s.N + wpb - 1) / wpb;
-    kernel<<<(unsigned)blocks, 32 * wpb, smem, st>>>(s, args...);
+    kernel<<<(unsigned)blocks, 32 * nw, smem, st>>>(s, args...);
     ++t_launches;
     return cudaGetLastError();
 }
@@ -117,26 +118,27 @@ cudaError_t launch_warps(K kernel, const dc::Shape &s, size_t per_warp, cudaStre
 template <typename T, int DPL>
 cudaError_t simt_fwd(const dc::Shape &s, const void *q, const void *k, const void *v, const float *c,
                      const float *g, void *o, float *lse, void *pmap, cudaStream_t st) {
-    return launch_warps(dc::simt::fwd_kernel<T, DPL>, s, dc::simt::fwd_smem_per_warp(s.H, s.d, s.W), st,
-                        (const T *)q, (const T *)k, (const T *)v, c, g, (T *)o, lse, (T *)pmap, 1);
+    return launch_simt(dc::simt::fwd_kernel<T, DPL>, s, s.N, s.H, dc::simt::fwd_smem(s.H, s.d, s.W), st,
+                       (const T *)q, (const T *)k, (const T *)v, c, g, (T *)o, lse, (T *)pmap, 1);
 }
 
 template <typename T, int DPL>
 cudaError_t simt_bwd_query(const dc::Shape &s, const void *q, const void *k, const void *v, const float *c,
                            const float *g, const void *dO, const float *lse, const void *pmap, void *dq,
                            float *dc_, float *dg, float *band, cudaStream_t st) {
-    return launch_warps(dc::simt::bwd_query_kernel<T, DPL>, s, dc::simt::bwdq_smem_per_warp(s.H, s.d, s.W), st,
-                        (const T *)q, (const T *)k, (const T *)v, c, g, (const T *)dO, lse, (const T *)pmap,
-                        (T *)dq, dc_, dg, band, 1);
+    return launch_simt(dc::simt::bwd_query_kernel<T, DPL>, s, s.N, s.H, dc::simt::bwdq_smem(s.H, s.d, s.W), st,
+                       (const T *)q, (const T *)k, (const T *)v, c, g, (const T *)dO, lse, (const T *)pmap,
+                       (T *)dq, dc_, dg, band, 1);
 }
 
 template <typename T, int DPL>
 cudaError_t simt_bwd_key(const dc::Shape &s, const void *q, const void *k, const float *c, const float *g,
                          const void *dO, const float *lse, const void *pmap, const float *dc_,
                          const float *band, void *dk, void *dv, cudaStream_t st) {
-    return launch_warps(dc::simt::bwd_key_kernel<T, DPL>, s, dc::simt::bwdk_smem_per_warp(s.H, s.d, s.W), st,
-                        (const T *)q, (const T *)k, c, g, (const T *)dO, lse, (const T *)pmap, dc_, band,
-                        (T *)dk, (T *)dv);
+    const int tk = dc::simt::key_tile(s.N);
+    return launch_simt(dc::simt::bwd_key_kernel<T, DPL>, s, (s.N + tk - 1) / tk, tk * s.H,
+                       dc::simt::bwdk_smem(s.H, s.d, tk), st, tk, (const T *)q, (const T *)k, c, g, (const T *)dO,
+                       lse, (const T *)pmap, dc_, band, (T *)dk, (T *)dv);
 }
 
 // Calls F<T, DPL>::run(args...) for the runtime dtype and d = 32 * DPL.

@@ -1,7 +1,9 @@
 // simt.cuh -- CUDA-core kernels for Lightweight DC attention (fp32 arithmetic).
 //
-// One warp per query token (forward, backward query side) or per key token
-// (backward key side), all heads of that token in the warp.  These kernels
+// One CTA per query token (forward, backward query side) or per key token
+// (backward key side) with one warp per head (up to 8; a warp takes heads w, w + nw, ...
+// when there are more).  The sums over heads (the composed map P, dP) are formed by one
+// warp in head order, so the results do not depend on the warp count.  These kernels
 // cover every supported shape and both storage types; they are the fp32 path
 // (tensor cores cannot meet an fp32 tolerance) and the path for bf16 shapes
 // the tcgen05 kernels do not take.  Arithmetic is fp32 with expf/logf.
@@ -13,17 +15,38 @@ namespace dc {
 namespace simt {
 
 constexpr int kMaxHeads = 16;
+constexpr int kMaxWarps = 8;                    // warps per token (one per head up to 8)
+constexpr size_t kSmemBudget = 200 * 1024;      // a CTA's shared memory at most
 
 // Floats of the per-warp row tile used by dot_rows32 (32 rows of d + 1).
 __host__ __device__ inline size_t tile_floats(int d) { return 32 * ((size_t)d + 1); }
-// Bytes of shared memory one warp needs in each kernel.
-inline size_t fwd_smem_per_warp(int H, int d, int W) {
-    return sizeof(float) * ((size_t)H * d + kMaxHeads + W + tile_floats(d));
+
+// Shared memory of one CTA (one token) with nw warps: a part per token, a part per warp.
+struct SimtSmem {
+    size_t per_token, per_warp;
+    size_t bytes(int nw) const { return sizeof(float) * (per_token + (size_t)nw * per_warp); }
+};
+// Forward: q of every head | lse per head | P over the window | p_h of one 32-key chunk per
+// head | per warp: row tile.
+inline SimtSmem fwd_smem(int H, int d, int W) {
+    return {(size_t)H * d + kMaxHeads + W + 32 * (size_t)H, tile_floats(d)};
 }
-inline size_t bwdq_smem_per_warp(int H, int d, int W) {
-    return sizeof(float) * (2 * (size_t)H * d + 3 * (size_t)W + tile_floats(d));
+// Query side: q and dO of every head | P and dP over the window | E_h of one 32-key chunk
+// per head | per warp: ds over the window, row tile.
+inline SimtSmem bwdq_smem(int H, int d, int W) {
+    return {2 * (size_t)H * d + 2 * (size_t)W + 32 * (size_t)H, (size_t)W + tile_floats(d)};
 }
-inline size_t bwdk_smem_per_warp(int H, int d, int W) { return sizeof(float) * ((size_t)H * d + tile_floats(d)); }
+// Key side with a tile of TK keys: k of every head of each key | per warp: row tile.
+inline SimtSmem bwdk_smem(int H, int d, int TK) { return {(size_t)TK * H * d, tile_floats(d)}; }
+// Keys per CTA of the key side: 4 once there are at least 16 keys per SM, else 1.
+inline int key_tile(int64_t N) { return N >= 16 * 148 ? 4 : 1; }
+// Warps per CTA: one per work item (head, or (head, key) on the key side) up to kMaxWarps,
+// fewer when shared memory runs short (0: not even one warp fits).
+inline int warps_per_cta(int items, const SimtSmem &m) {
+    int nw = items < kMaxWarps ? items : kMaxWarps;
+    while (nw > 0 && m.bytes(nw) > kSmemBudget) --nw;
+    return nw;
+}
 
 // <xs, row(lane)> for up to 32 consecutive rows, row r at rows + r * stride (d = 32 * DPL
 // elements, xs in shared memory).  The rows pass through this warp's tile with coalesced
@@ -50,8 +73,10 @@ __device__ __forceinline__ float dot_rows32(const float *xs, const T *rows, int6
     return acc;
 }
 
-// Forward: lse per head (pass 1), composed map P over the window (pass 2),
-// o_h = g_h * sum_j P(j) v_h(j) (pass 3).
+// Forward: one CTA per query token, warp w takes heads w, w + nw, ...  lse per head
+// (pass 1); the composed map P over the window, 32 keys at a time: every warp writes p_h
+// of its heads, then warp 0 adds c_h p_h in head order (pass 2); o_h = g_h * sum_j P(j)
+// v_h(j) per head (pass 3).
 template <typename T, int DPL>
 __global__ void fwd_kernel(Shape s, const T *__restrict__ q, const T *__restrict__ k,
                            const T *__restrict__ v, const float *__restrict__ c,
@@ -61,20 +86,20 @@ __global__ void fwd_kernel(Shape s, const T *__restrict__ q, const T *__restrict
     extern __shared__ float smem[];
     if (check_seqlens) validate_seqlens(s);
     const int H = s.H, W = s.W;
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int64_t t = (int64_t)blockIdx.x * (blockDim.x >> 5) + warp;
-    if (t >= s.N) return;
-    float *qs = smem + (size_t)warp * (H * d + kMaxHeads + W + tile_floats(d));
+    const int nw = blockDim.x >> 5, warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int64_t t = blockIdx.x;
+    float *qs = smem;
     float *ls = qs + H * d;
     float *Pw = ls + kMaxHeads;
-    float *tile = Pw + W;
+    float *ph = Pw + W;                                     // [H][32]
+    float *tile = ph + 32 * H + (size_t)warp * tile_floats(d);
 
-    for (int i = lane; i < H * d; i += 32) qs[i] = ldf<T>(q + t * s.sq + i);
-    __syncwarp();
+    for (int i = threadIdx.x; i < H * d; i += blockDim.x) qs[i] = ldf<T>(q + t * s.sq + i);
+    __syncthreads();
     const int64_t lo = window_lo(s, t);
     const int n = (int)(t - lo + 1);
 
-    for (int h = 0; h < H; ++h) {
+    for (int h = warp; h < H; h += nw) {
         float m = -INFINITY, z = 0.f;
         for (int base = 0; base < n; base += 32) {
             const int cnt = min(32, n - base);
@@ -97,22 +122,26 @@ __global__ void fwd_kernel(Shape s, const T *__restrict__ q, const T *__restrict
             if (lse) lse[t * H + h] = l;
         }
     }
-    __syncwarp();
+    __syncthreads();
     for (int base = 0; base < n; base += 32) {
         const int cnt = min(32, n - base);
-        float P = 0.f;
-        for (int h = 0; h < H; ++h) {
+        for (int h = warp; h < H; h += nw) {
             const float x = s.scale * dot_rows32<T, DPL>(qs + h * d, k + (lo + base) * s.sq + h * d, s.sq, cnt, tile);
-            P = fmaf(__ldg(c + t * H + h), expf(x - ls[h]), P);
+            ph[h * 32 + lane] = expf(x - ls[h]);
         }
-        if (lane < cnt) Pw[base + lane] = P;
+        __syncthreads();
+        if (warp == 0) {
+            float P = 0.f;
+            for (int h = 0; h < H; ++h) P = fmaf(__ldg(c + t * H + h), ph[h * 32 + lane], P);
+            if (lane < cnt) Pw[base + lane] = P;
+        }
+        __syncthreads();   // Pw written; ph free for the next chunk
     }
-    __syncwarp();
     if (pmap) {
         const int64_t w0 = lo - (t - W + 1);   // band index of key lo
-        for (int w = lane; w < W; w += 32) stf<T>(pmap + t * W + w, (w >= w0) ? Pw[w - w0] : 0.f);
+        for (int w = threadIdx.x; w < W; w += blockDim.x) stf<T>(pmap + t * W + w, (w >= w0) ? Pw[w - w0] : 0.f);
     }
-    for (int h = 0; h < H; ++h) {
+    for (int h = warp; h < H; h += nw) {
         float acc[DPL];
 #pragma unroll
         for (int i = 0; i < DPL; ++i) acc[i] = 0.f;
@@ -128,10 +157,11 @@ __global__ void fwd_kernel(Shape s, const T *__restrict__ q, const T *__restrict
     }
 }
 
-// Backward, query side.  Pass 1 over the window: E_h(j) = <dO_h, v_h(j)>,
-// dP(j) = sum_h g_h E_h(j) (stored to the workspace band), dg_h = sum_j P(j) E_h(j).
-// Pass 2 per head: p_h(j) from lse, dc_h = sum_j dP(j) p_h(j),
-// ds_h(j) = c_h p_h(j) (dP(j) - dc_h), dq_h = sigma sum_j ds_h(j) k_h(j).
+// Backward, query side: one CTA per query token, warp w takes heads w, w + nw, ...
+// Pass 1 over the window, 32 keys at a time: every warp writes E_h(j) = <dO_h, v_h(j)> of its
+// heads and adds P(j) E_h(j) to dg_h; warp 0 then forms dP(j) = sum_h g_h E_h(j) in head order
+// (stored to the workspace band).  Pass 2 per head: p_h(j) from lse, dc_h = sum_j dP(j)
+// p_h(j), ds_h(j) = c_h p_h(j) (dP(j) - dc_h), dq_h = sigma sum_j ds_h(j) k_h(j).
 template <typename T, int DPL>
 __global__ void bwd_query_kernel(Shape s, const T *__restrict__ q, const T *__restrict__ k,
                                  const T *__restrict__ v, const float *__restrict__ c,
@@ -143,58 +173,64 @@ __global__ void bwd_query_kernel(Shape s, const T *__restrict__ q, const T *__re
     extern __shared__ float smem[];
     if (check_seqlens) validate_seqlens(s);
     const int H = s.H, W = s.W;
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int64_t t = (int64_t)blockIdx.x * (blockDim.x >> 5) + warp;
-    if (t >= s.N) return;
-    float *qs = smem + (size_t)warp * (2 * H * d + 3 * W + tile_floats(d));
+    const int nw = blockDim.x >> 5, warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int64_t t = blockIdx.x;
+    float *qs = smem;
     float *dos = qs + H * d;
     float *Pw = dos + H * d;
     float *dPw = Pw + W;
-    float *sw = dPw + W;
+    float *eh = dPw + W;                                    // [H][32]
+    float *sw = eh + 32 * H + (size_t)warp * (W + tile_floats(d));
     float *tile = sw + W;
 
-    for (int i = lane; i < H * d; i += 32) {
+    for (int i = threadIdx.x; i < H * d; i += blockDim.x) {
         qs[i] = ldf<T>(q + t * s.sq + i);
         dos[i] = ldf<T>(dO + t * s.so + i);
     }
     const int64_t lo = window_lo(s, t);
     const int n = (int)(t - lo + 1);
     const int w0 = (int)(lo - (t - W + 1));
-    for (int jj = lane; jj < n; jj += 32) Pw[jj] = ldf<T>(pmap + t * W + w0 + jj);
-    for (int w = lane; w < w0; w += 32) dPband[t * W + w] = 0.f;
-    __syncwarp();
+    for (int jj = threadIdx.x; jj < n; jj += blockDim.x) Pw[jj] = ldf<T>(pmap + t * W + w0 + jj);
+    for (int w = threadIdx.x; w < w0; w += blockDim.x) dPband[t * W + w] = 0.f;
+    __syncthreads();
 
-    float dgp[kMaxHeads];
+    float dgp[kMaxHeads];   // slot u: head warp + u * nw
 #pragma unroll
-    for (int h = 0; h < kMaxHeads; ++h) dgp[h] = 0.f;
+    for (int u = 0; u < kMaxHeads; ++u) dgp[u] = 0.f;
     for (int base = 0; base < n; base += 32) {
         const int cnt = min(32, n - base);
         const int jj = base + lane;
         const float pj = lane < cnt ? Pw[jj] : 0.f;
-        float dP = 0.f;
 #pragma unroll
-        for (int h = 0; h < kMaxHeads; ++h) {
+        for (int u = 0; u < kMaxHeads; ++u) {
+            const int h = warp + u * nw;
             if (h < H) {
                 const float E = dot_rows32<T, DPL>(dos + h * d, v + (lo + base) * s.sq + h * d, s.sq, cnt, tile);
-                dP = fmaf(__ldg(g + t * H + h), E, dP);
-                dgp[h] = fmaf(pj, E, dgp[h]);
+                eh[h * 32 + lane] = E;
+                dgp[u] = fmaf(pj, E, dgp[u]);
             }
         }
-        if (lane < cnt) {
-            dPw[jj] = dP;
-            dPband[t * W + w0 + jj] = dP;
+        __syncthreads();
+        if (warp == 0) {
+            float dP = 0.f;
+            for (int h = 0; h < H; ++h) dP = fmaf(__ldg(g + t * H + h), eh[h * 32 + lane], dP);
+            if (lane < cnt) {
+                dPw[jj] = dP;
+                dPband[t * W + w0 + jj] = dP;
+            }
         }
+        __syncthreads();   // dPw written; eh free for the next chunk
     }
 #pragma unroll
-    for (int h = 0; h < kMaxHeads; ++h) {
+    for (int u = 0; u < kMaxHeads; ++u) {
+        const int h = warp + u * nw;
         if (h < H) {
-            const float x = warp_sum(dgp[h]);
+            const float x = warp_sum(dgp[u]);
             if (lane == 0) dg[t * H + h] = x;
         }
     }
-    __syncwarp();
 
-    for (int h = 0; h < H; ++h) {
+    for (int h = warp; h < H; h += nw) {
         const float l = __ldg(lse + t * H + h);
         float dcp = 0.f;
         for (int base = 0; base < n; base += 32) {
@@ -226,11 +262,15 @@ __global__ void bwd_query_kernel(Shape s, const T *__restrict__ q, const T *__re
     }
 }
 
-// Backward, key side: for key j and the queries t whose window holds it,
-// ds_h(t,j) = c[t,h] p_h(t,j) (dP(t,j) - dc[t,h]) with p_h from lse and dP from
-// the workspace band, dk_h(j) = sigma sum_t ds_h q_h(t), dv_h(j) = sum_t P g_h dO_h(t).
+// Backward, key side: one CTA per tile of TK consecutive key tokens (TK = 4 when there are
+// enough keys, so that the query rows the tile's keys share are reused from L1; else 1);
+// the warps (one per item up to 8) take the (head, key) items h * TK + kk of the tile in
+// turn, so that warps running at the same time share a head and read overlapping query rows.  For key j and the queries
+// t whose window holds it, ds_h(t,j) = c[t,h] p_h(t,j) (dP(t,j) - dc[t,h]) with p_h from lse
+// and dP from the workspace band, dk_h(j) = sigma sum_t ds_h q_h(t),
+// dv_h(j) = sum_t P g_h dO_h(t).
 template <typename T, int DPL>
-__global__ void bwd_key_kernel(Shape s, const T *__restrict__ q, const T *__restrict__ k,
+__global__ void bwd_key_kernel(Shape s, int TK, const T *__restrict__ q, const T *__restrict__ k,
                                const float *__restrict__ c, const float *__restrict__ g,
                                const T *__restrict__ dO, const float *__restrict__ lse,
                                const T *__restrict__ pmap, const float *__restrict__ dc,
@@ -239,26 +279,29 @@ __global__ void bwd_key_kernel(Shape s, const T *__restrict__ q, const T *__rest
     constexpr int d = 32 * DPL;
     extern __shared__ float smem[];
     const int H = s.H, W = s.W;
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int64_t j = (int64_t)blockIdx.x * (blockDim.x >> 5) + warp;
-    if (j >= s.N) return;
-    float *ks = smem + (size_t)warp * (H * d + tile_floats(d));
-    float *tile = ks + H * d;
-    for (int i = lane; i < H * d; i += 32) ks[i] = ldf<T>(k + j * s.sq + i);
-    __syncwarp();
-    int64_t hi = j + W - 1;
-    const int64_t b = doc_end(s, j);
-    if (hi > b - 1) hi = b - 1;
-    const int n = (int)(hi - j + 1);
+    const int nw = blockDim.x >> 5, warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int64_t j0 = (int64_t)blockIdx.x * TK;
+    const int tk = (int)min((int64_t)TK, s.N - j0);   // keys of this tile
+    float *ks = smem;                                 // [TK][H * d]
+    float *tile = ks + (size_t)TK * H * d + (size_t)warp * tile_floats(d);
+    for (int i = threadIdx.x; i < tk * H * d; i += blockDim.x) ks[i] = ldf<T>(k + (j0 + i / (H * d)) * s.sq + i % (H * d));
+    __syncthreads();
 
-    for (int h = 0; h < H; ++h) {
+    for (int item = warp; item < H * tk; item += nw) {
+        const int h = item / tk, kk = item - h * tk;
+        const int64_t j = j0 + kk;
+        const float *kh = ks + (size_t)kk * H * d + h * d;
+        int64_t hi = j + W - 1;
+        const int64_t b = doc_end(s, j);
+        if (hi > b - 1) hi = b - 1;
+        const int n = (int)(hi - j + 1);
         float ak[DPL], av[DPL];
 #pragma unroll
         for (int i = 0; i < DPL; ++i) ak[i] = av[i] = 0.f;
         for (int base = 0; base < n; base += 32) {
             float ds = 0.f, pg = 0.f;
             const int cnt0 = min(32, n - base);
-            const float x = s.scale * dot_rows32<T, DPL>(ks + h * d, q + (j + base) * s.sq + h * d, s.sq, cnt0, tile);
+            const float x = s.scale * dot_rows32<T, DPL>(kh, q + (j + base) * s.sq + h * d, s.sq, cnt0, tile);
             if (base + lane < n) {
                 const int64_t t = j + base + lane;
                 const int64_t w = j - (t - W + 1);
