@@ -119,7 +119,8 @@ template <typename T, int DPL>
 cudaError_t simt_fwd(const dc::Shape &s, const void *q, const void *k, const void *v, const float *c,
                      const float *g, void *o, float *lse, void *pmap, cudaStream_t st) {
     return launch_simt(dc::simt::fwd_kernel<T, DPL>, s, s.N, s.H, dc::simt::fwd_smem(s.H, s.d, s.W), st,
-                       (const T *)q, (const T *)k, (const T *)v, c, g, (T *)o, lse, (T *)pmap, 1);
+                       (int)dc::simt::fwd_keeps_scores(s.H, s.W), (const T *)q, (const T *)k, (const T *)v, c, g,
+                       (T *)o, lse, (T *)pmap, 1);
 }
 
 template <typename T, int DPL>

@@ -27,9 +27,12 @@ struct SimtSmem {
     size_t bytes(int nw) const { return sizeof(float) * (per_token + (size_t)nw * per_warp); }
 };
 // Forward: q of every head | lse per head | P over the window | p_h of one 32-key chunk per
-// head | per warp: row tile.
+// head | the scores of every head over the window when they fit (fwd_keeps_scores) | per
+// warp: row tile.
+inline bool fwd_keeps_scores(int H, int W) { return (size_t)H * W * sizeof(float) <= 64 * 1024; }
 inline SimtSmem fwd_smem(int H, int d, int W) {
-    return {(size_t)H * d + kMaxHeads + W + 32 * (size_t)H, tile_floats(d)};
+    return {(size_t)H * d + kMaxHeads + W + 32 * (size_t)H + (fwd_keeps_scores(H, W) ? (size_t)H * W : 0),
+            tile_floats(d)};
 }
 // Query side: q and dO of every head | P and dP over the window | E_h of one 32-key chunk
 // per head | per warp: ds over the window, row tile.
@@ -76,9 +79,10 @@ __device__ __forceinline__ float dot_rows32(const float *xs, const T *rows, int6
 // Forward: one CTA per query token, warp w takes heads w, w + nw, ...  lse per head
 // (pass 1); the composed map P over the window, 32 keys at a time: every warp writes p_h
 // of its heads, then warp 0 adds c_h p_h in head order (pass 2); o_h = g_h * sum_j P(j)
-// v_h(j) per head (pass 3).
+// v_h(j) per head (pass 3).  With `keep`, pass 1 keeps the scores in shared memory and
+// pass 2 reads them back instead of computing them again (the same values).
 template <typename T, int DPL>
-__global__ void fwd_kernel(Shape s, const T *__restrict__ q, const T *__restrict__ k,
+__global__ void fwd_kernel(Shape s, int keep, const T *__restrict__ q, const T *__restrict__ k,
                            const T *__restrict__ v, const float *__restrict__ c,
                            const float *__restrict__ g, T *__restrict__ o,
                            float *__restrict__ lse, T *__restrict__ pmap, int check_seqlens) {
@@ -92,7 +96,8 @@ __global__ void fwd_kernel(Shape s, const T *__restrict__ q, const T *__restrict
     float *ls = qs + H * d;
     float *Pw = ls + kMaxHeads;
     float *ph = Pw + W;                                     // [H][32]
-    float *tile = ph + 32 * H + (size_t)warp * tile_floats(d);
+    float *sc = ph + 32 * H;                                // [H][W] scores (with keep)
+    float *tile = sc + (keep ? (size_t)H * W : 0) + (size_t)warp * tile_floats(d);
 
     for (int i = threadIdx.x; i < H * d; i += blockDim.x) qs[i] = ldf<T>(q + t * s.sq + i);
     __syncthreads();
@@ -104,6 +109,7 @@ __global__ void fwd_kernel(Shape s, const T *__restrict__ q, const T *__restrict
         for (int base = 0; base < n; base += 32) {
             const int cnt = min(32, n - base);
             const float x = s.scale * dot_rows32<T, DPL>(qs + h * d, k + (lo + base) * s.sq + h * d, s.sq, cnt, tile);
+            if (keep && lane < cnt) sc[h * W + base + lane] = x;
             if (lane < cnt) {
                 if (x > m) {
                     z = z * expf(m - x) + 1.f;
@@ -126,7 +132,9 @@ __global__ void fwd_kernel(Shape s, const T *__restrict__ q, const T *__restrict
     for (int base = 0; base < n; base += 32) {
         const int cnt = min(32, n - base);
         for (int h = warp; h < H; h += nw) {
-            const float x = s.scale * dot_rows32<T, DPL>(qs + h * d, k + (lo + base) * s.sq + h * d, s.sq, cnt, tile);
+            const float x = keep ? (lane < cnt ? sc[h * W + base + lane] : s.scale * 0.f)
+                                 : s.scale * dot_rows32<T, DPL>(qs + h * d, k + (lo + base) * s.sq + h * d, s.sq, cnt,
+                                                                tile);
             ph[h * 32 + lane] = expf(x - ls[h]);
         }
         __syncthreads();
