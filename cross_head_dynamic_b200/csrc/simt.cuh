@@ -153,7 +153,7 @@ __global__ void fwd_kernel(Shape s, int keep, const T *__restrict__ q, const T *
         float acc[DPL];
 #pragma unroll
         for (int i = 0; i < DPL; ++i) acc[i] = 0.f;
-        for (int jj = 0; jj < n; ++jj) {
+        for (int jj = 0; jj < n; ++jj) {   // (unrolling this loop measured slower)
             const float P = Pw[jj];
             const T *vr = v + (lo + jj) * s.sq + h * d;
 #pragma unroll
@@ -258,6 +258,7 @@ __global__ void bwd_query_kernel(Shape s, const T *__restrict__ q, const T *__re
         float acc[DPL];
 #pragma unroll
         for (int i = 0; i < DPL; ++i) acc[i] = 0.f;
+#pragma unroll 8
         for (int jj = 0; jj < n; ++jj) {
             const float ds = sw[jj];
             const T *kr = k + (lo + jj) * s.sq + h * d;
@@ -318,6 +319,7 @@ __global__ void bwd_key_kernel(Shape s, int TK, const T *__restrict__ q, const T
                 pg = ldf<T>(pmap + t * W + w) * __ldg(g + t * H + h);
             }
             const int cnt = min(32, n - base);
+#pragma unroll 8
             for (int l = 0; l < cnt; ++l) {
                 const float dsl = __shfl_sync(0xffffffffu, ds, l);
                 const float pgl = __shfl_sync(0xffffffffu, pg, l);
