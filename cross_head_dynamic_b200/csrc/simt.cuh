@@ -15,15 +15,16 @@ namespace dc {
 namespace simt {
 
 constexpr int kMaxHeads = 16;
-constexpr int kMaxWarps = 8;                    // warps per token (one per head up to 8)
+constexpr int kMaxWarps = 8;                    // warps per CTA (one per work item up to 8)
 constexpr size_t kSmemBudget = 200 * 1024;      // a CTA's shared memory at most
 
 // Floats of the per-warp row tile used by dot_rows32 (32 rows of d + 1).
 __host__ __device__ inline size_t tile_floats(int d) { return 32 * ((size_t)d + 1); }
 
-// Shared memory of one CTA (one token) with nw warps: a part per token, a part per warp.
+// Shared memory of one CTA with nw warps: a part for the CTA's token (or key tile) and a
+// part per warp.
 struct SimtSmem {
-    size_t per_token, per_warp;
+    size_t per_token, per_warp;   // floats
     size_t bytes(int nw) const { return sizeof(float) * (per_token + (size_t)nw * per_warp); }
 };
 // Forward: q of every head | lse per head | P over the window | p_h of one 32-key chunk per
