@@ -102,6 +102,13 @@ EDGE_CASES = [
     ("bf16_w250_h16_d64", [520], 16, 64, 250, "bf16"),
     ("bf16_w256_h1", [1100], 1, 128, 256, "bf16"),
     ("bf16_w256_short", [100, 60], 4, 128, 256, "bf16"),
+    # SIMT kernels: key tiles of 4 consecutive keys (N >= 16 keys per SM) with a ragged last
+    # tile and documents ending inside tiles; a window past the tcgen05 range; a forward
+    # whose scores (H * W floats) do not fit the shared-memory budget and are recomputed
+    ("simt_key_tiles", [1500, 3, 1100], 6, 64, 112, "f32"),
+    ("bf16_simt_key_tiles", [2500, 1, 99], 6, 128, 112, "bf16"),
+    ("w300", [700, 500], 4, 64, 300, "f32"),
+    ("w1100_h16_scores_recomputed", [1200], 16, 32, 1100, "f32"),
 ]
 
 
